@@ -1,0 +1,83 @@
+"""The C-ABI library: it loads, exports every entry point include/gdn2.h
+declares, and rejects bad arguments on the host before anything is launched
+(these calls never reach the GPU, so they run without one)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_gdn2_b200 as g
+from gated_delta_rule_gdn2_b200 import build as gbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "gdn2.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn2_\w+)\s*\(", text)))
+
+
+def test_build_is_current():
+    assert gbuild.build() == g.LIB_PATH
+    assert os.path.exists(g.LIB_PATH)
+
+
+def test_exports_every_declared_symbol():
+    lib = ctypes.CDLL(g.LIB_PATH)
+    syms = declared_symbols()
+    assert len(syms) >= 8
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert set(syms) <= set(g.binding.SIGNATURES)
+
+
+def test_version_and_status_strings():
+    assert g.gdn2_version() == 100
+    for code, name in g.STATUS.items():
+        assert g.gdn2_status_string(code).startswith(name)
+    assert "unknown" in g.gdn2_status_string(-99)
+
+
+def _fwd(**kw):
+    a = dict(q=16, k=16, v=16, log_alpha=16, b=16, w=16, S0=None, o=16, S_T=None, B=1, T=64, H=1,
+             dk=64, dv=64, dtype=g.GDN2_BF16, ws=16, ws_bytes=1 << 30, stream=0)
+    a.update(kw)
+    return g.gdn2_chunk_fwd(a["q"], a["k"], a["v"], a["log_alpha"], a["b"], a["w"], a["S0"], a["o"],
+                            a["S_T"], a["B"], a["T"], a["H"], a["dk"], a["dv"], a["dtype"], a["ws"],
+                            a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dk=96), -2), (dict(dv=32), -2), (dict(dtype=7), -2),
+    (dict(B=-1), -1), (dict(T=-5), -1), (dict(H=-1), -1),
+    (dict(q=None), -1), (dict(o=None), -1), (dict(k=24), -1), (dict(S0=8), -1),
+    (dict(ws=None), -5), (dict(ws_bytes=16), -5),
+])
+def test_chunk_fwd_rejects_bad_arguments(kw, code):
+    assert _fwd(**kw) == code
+
+
+def test_empty_batch_is_a_noop():
+    assert _fwd(B=0, q=None, k=None, v=None, log_alpha=None, b=None, w=None, o=None) == 0
+    assert _fwd(H=0, q=None, k=None, v=None, log_alpha=None, b=None, w=None, o=None) == 0
+
+
+def test_decode_and_bwd_reject_bad_arguments():
+    assert g.gdn2_decode_step(16, 16, 16, 16, 16, 16, None, 16, 1, 1, 64, 64, 0, 0) == -1
+    assert g.gdn2_decode_step(16, 16, 16, 16, 16, 16, 16, 16, 1, 1, 64, 80, 0, 0) == -2
+    assert g.gdn2_decode_step(16, 16, 16, 16, 16, 16, 20, 16, 1, 1, 64, 64, 0, 0) == -1
+    args = [16] * 6 + [None, 16, None] + [16] * 6 + [None]
+    assert g.gdn2_chunk_bwd(*args, 1, 64, 1, 64, 64, 0, None, 0, 0) == -5
+    args[7] = None  # dO
+    assert g.gdn2_chunk_bwd(*args, 1, 64, 1, 64, 64, 0, 16, 1 << 40, 0) == -1
+    assert g.gdn2_chunk_bwd(*([16] * 16), 1, 64, 1, 128, 64, 3, 16, 1 << 40, 0) == -2
+
+
+def test_workspace_sizes():
+    assert g.gdn2_chunk_fwd_workspace(8, 4096, 16, 128, 128, g.GDN2_BF16) == 8 * 16 * 64 * 128 * 4
+    assert g.gdn2_chunk_fwd_workspace(8, 4096, 16, 128, 128, g.GDN2_FP32) == 0
+    assert g.gdn2_chunk_fwd_workspace(0, 4096, 16, 128, 128, g.GDN2_BF16) == 0
+    assert g.gdn2_chunk_bwd_workspace(8, 4096, 16, 128, 128, g.GDN2_BF16) > 0
+    assert g.gdn2_chunk_bwd_workspace(8, 4096, 16, 96, 128, g.GDN2_BF16) == 0
