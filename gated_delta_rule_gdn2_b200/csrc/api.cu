@@ -117,7 +117,8 @@ int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_
     const size_t need = gdn2_chunk_fwd_workspace(B, T, H, dk, dv, dtype);
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return GDN2_ERR_WORKSPACE;
     if (dtype == GDN2_BF16) {
-        ChunkFwdArgs a{q, k, v, log_alpha, b, w, S0, o, S_T, static_cast<float *>(ws), B, T, H};
+        ChunkFwdArgs a{q, k, v, log_alpha, b, w, S0, o, S_T, static_cast<float *>(ws),
+                       (size_t)64 * dk, nullptr, B, T, H};
         return launch_status(launch_chunk_fwd(a, dk, dv, stream));
     }
     // fp32 precision mode: the recurrence token by token in fp32
@@ -141,6 +142,7 @@ int gdn2_decode_step(const void *q, const void *k, const void *v, const void *lo
 size_t gdn2_chunk_bwd_workspace(int B, int T, int H, int dk, int dv, int dtype) {
     if (check_sizes(B, T, H, dk, dv, dtype) != GDN2_OK) return 0;
     if (B == 0 || H == 0 || T == 0) return 0;
+    if (dtype == GDN2_BF16) return chunk_bwd_ws_bytes(B, T, H, dk, dv, nullptr, nullptr);
     return recurrent_bwd_ws_bytes(B, T, H, dk, dv);
 }
 
@@ -161,9 +163,17 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
         return GDN2_ERR_INVALID_ARG;
     const size_t need = gdn2_chunk_bwd_workspace(B, T, H, dk, dv, dtype);
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return GDN2_ERR_WORKSPACE;
+    if (dtype == GDN2_BF16) {
+        size_t stride = 0, sbytes = 0;
+        chunk_bwd_ws_bytes(B, T, H, dk, dv, &stride, &sbytes);
+        ChunkBwdArgs a{q, k, v, log_alpha, b, w, S0, dO, dS_T, dq, dk_, dv_, dlog_alpha, db, dw, dS0, ws,
+                       reinterpret_cast<float *>(static_cast<char *>(ws) + sbytes), stride, B, T, H};
+        return launch_status(launch_chunk_bwd(a, dk, dv, stream));
+    }
+    // fp32 precision mode: reverse-time recurrence token by token in fp32
     RecurrentBwdArgs a{q, k, v, log_alpha, b, w, S0, dO, dS_T, dq, dk_, dv_, dlog_alpha, db, dw,
                        dS0, static_cast<float *>(ws), B, T, H};
-    return launch_status(launch_recurrent_bwd(a, dk, dv, dtype == GDN2_BF16, stream));
+    return launch_status(launch_recurrent_bwd(a, dk, dv, false, stream));
 }
 
 }  // extern "C"

@@ -1,0 +1,457 @@
+// Gate-aware backward (vector-Jacobian product) of the chunk-parallel forward.
+//
+// "Why NVIDIA Gated DeltaNet-2 separates erase and write gates" (axbrief),
+// section "Gated Delta Rule-2: per-channel erase/write split": the backward
+// can no longer use KDA's scalar shortcut, because the distinct diagonal
+// gates on the erase side (b, key axis) and the write side (w, value axis)
+// sit inside every gradient-accumulating inner product.  Here b enters through
+// g = b . k inside the key Gram and the erase term, and w through w . v in
+// the value targets; their gradients are taken inside those products.
+//
+// Two launches.  (1) The forward kernel re-runs with a state output: the bf16
+// state at every chunk boundary goes to the workspace.  (2) This kernel walks
+// each (batch, head) sequence's chunks in reverse order, carrying
+// dSigma = dL/dS(chunk end) in fp32 registers.  For a chunk with start state S,
+// end state Sigma and the forward's quantities (chunk_common.cuh, fast path;
+// Dh = Diag(gam) dSigma):
+//
+//   dU   = M^T dO + Kb Dh                    dM = strict_lower(dO U^T), diag(dO U^T)
+//   nR   = -T^T dU      (= -dRHS)            dA = strict_lower(nR U^T)
+//   dv   = -nR . w,  dw = -nR . v            dKb = U Dh^T + dA^T Gt + dM^T Qt
+//   dQt  = dO S^T + dM Kb                    dGt = nR S^T + dA Kb
+//   dS   = Dh + Qt^T dO + Gt^T nR            (-> dSigma of the previous chunk)
+//   dq = dQt e^{L} + dMd k,  dg = dGt e^{L},  dk = dKb e^{-L} + dMd q + dg . b,
+//   db = dg . k   (dMd = diagonal of dO U^T)
+//   dL_r = dQt.Qt + dGt.Gt - dKb.Kb (+ rowsum(dSigma . Sigma) at the chunk end)
+//   dlog_alpha = reverse cumulative sum of dL within the chunk.
+//
+// A slow chunk (decay beyond e^{-64} inside the chunk) uses Kt = k e^{L_end-L}
+// with Dh = dSigma, and takes the Gram gradients term by term in fp32.
+//
+// Per-CTA fp32 scratch (L, dQt, dGt, dKb, dL and the slow-path partial
+// gradients) lives in the caller's workspace and stays resident in L2.
+#include "chunk_common.cuh"
+#include "launch.h"
+
+namespace gdn2 {
+namespace cbwd {
+
+using namespace chunk;
+
+template <int DK, int DV>
+struct BSmem {
+    static constexpr int TQ = C * DK * 2, TV = C * DV * 2, TS = DK * DV * 2;
+    static constexpr int OQ = 0, OK = TQ, OLA = 2 * TQ, OB = 3 * TQ;
+    static constexpr int OV = 4 * TQ, OW = OV + TV, ODO = OW + TV;
+    static constexpr int OS = ODO + TV, OD = OS + TS;
+    static constexpr int OAT = OD + TS;              // A32 | T32 (2 x 16 KB fp32)
+    static constexpr bool AM_IN_K = (DK == 128);     // dM16 | dA16 in the k slot
+    static constexpr int OAM = OAT + 32768;
+    static constexpr int BYTES = OAM + (AM_IN_K ? 0 : 16384);
+};
+
+template <int DK>
+struct Scratch {
+    static constexpr int TILE = C * DK;
+    static constexpr int LAM = 0, DQT = 1, DGT = 2, DKB = 3, DLAM = 4, PQ = 5, PG = 6, PK = 7, PL = 8;
+    static constexpr int RS = 9 * TILE;              // 2 x DK row sums
+    static constexpr int DMD = 9 * TILE + 2 * DK;    // diagonal of dM (C floats)
+    static constexpr size_t FLOATS = 9 * TILE + 2 * DK + C;
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
+    using L = BSmem<DK, DV>;
+    using SC = Scratch<DK>;
+    constexpr int WR = DK / 4, WC = DV / 2;
+    constexpr int MTS = WR / 16, NTS = WC / 8;
+    constexpr int NTV = DV / 8, NTK = DK / 8;
+    constexpr int P = NTHR / DK, RSEG = C / P;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ IntraShared<DK> sh;
+    __shared__ float s_dpart[P][DK];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+    const int T = a.T, H = a.H;
+    const int nchunks = (T + C - 1) / C;
+
+    ChunkTiles st{reinterpret_cast<bf16 *>(smem + L::OQ), reinterpret_cast<bf16 *>(smem + L::OK),
+                  reinterpret_cast<bf16 *>(smem + L::OLA), reinterpret_cast<bf16 *>(smem + L::OB),
+                  reinterpret_cast<bf16 *>(smem + L::OV), reinterpret_cast<bf16 *>(smem + L::OW)};
+    bf16 *dO16 = reinterpret_cast<bf16 *>(smem + L::ODO);
+    bf16 *S16 = reinterpret_cast<bf16 *>(smem + L::OS);
+    bf16 *D16 = reinterpret_cast<bf16 *>(smem + L::OD);
+    float *A32 = reinterpret_cast<float *>(smem + L::OAT);
+    float *T32 = A32 + C * C;
+    bf16 *T16 = reinterpret_cast<bf16 *>(T32);
+    bf16 *M16 = T16 + C * C;
+    bf16 *W16 = reinterpret_cast<bf16 *>(A32);   // after the solve
+    bf16 *dU16 = reinterpret_cast<bf16 *>(A32);  // after U
+    bf16 *U16 = st.w;                            // w . v went to the v slot
+    bf16 *nR16 = st.v;                           // after Uv
+    bf16 *dM16 = reinterpret_cast<bf16 *>(L::AM_IN_K ? smem + L::OK : smem + L::OAM);
+    bf16 *dA16 = dM16 + C * C;
+
+    float *scr = a.scratch + (size_t)bh * a.scr_stride;
+    float *LAM = scr + SC::LAM * SC::TILE, *DQT = scr + SC::DQT * SC::TILE, *DGT = scr + SC::DGT * SC::TILE;
+    float *DKB = scr + SC::DKB * SC::TILE, *DLAM = scr + SC::DLAM * SC::TILE;
+    float *PQ = scr + SC::PQ * SC::TILE, *PG = scr + SC::PG * SC::TILE, *PK = scr + SC::PK * SC::TILE;
+    float *PL = scr + SC::PL * SC::TILE, *RS = scr + SC::RS, *DMD = scr + SC::DMD;
+    const bf16 *states = static_cast<const bf16 *>(a.states) + (size_t)bh * (nchunks + 1) * DK * DV;
+    const bf16 *gq = static_cast<const bf16 *>(a.q), *gk = static_cast<const bf16 *>(a.k);
+    const bf16 *gb = static_cast<const bf16 *>(a.b), *gv = static_cast<const bf16 *>(a.v);
+    const bf16 *gw = static_cast<const bf16 *>(a.w);
+
+    // dSigma: fp32, same register tiling as the forward's state
+    const int c0 = (warp >> 1) * WR, j0 = (warp & 1) * WC;
+    float dS[MTS][NTS][4];
+#pragma unroll
+    for (int mt = 0; mt < MTS; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NTS; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int c = c0 + 16 * mt + (lane >> 2) + (e >> 1) * 8;
+                const int j = j0 + 8 * nt + 2 * (lane & 3) + (e & 1);
+                dS[mt][nt][e] = a.dS_T ? a.dS_T[(size_t)bh * DK * DV + (size_t)c * DV + j] : 0.f;
+            }
+
+    for (int n = nchunks - 1; n >= 0; --n) {
+        const int Cn = min(C, T - n * C);
+        // ---- loads: six token tiles, dO, the chunk-start state
+        load_token_tile<DK>(st.q, gq, b, h, n, T, H);
+        load_token_tile<DK>(st.k, gk, b, h, n, T, H);
+        load_token_tile<DK>(st.la, static_cast<const bf16 *>(a.log_alpha), b, h, n, T, H);
+        load_token_tile<DK>(st.b, gb, b, h, n, T, H);
+        load_token_tile<DV>(st.v, gv, b, h, n, T, H);
+        load_token_tile<DV>(st.w, gw, b, h, n, T, H);
+        load_token_tile<DV>(dO16, static_cast<const bf16 *>(a.dO), b, h, n, T, H);
+        {
+            const bf16 *src = states + (size_t)n * DK * DV;
+            for (int id = tid; id < DK * DV / 8; id += NTHR) {
+                const int r = id / (DV / 8), ch = id % (DV / 8);
+                cp_async16(S16 + swz<DV>(r, ch * 8), src + (size_t)r * DV + ch * 8, true);
+            }
+        }
+        cp_commit();
+        cp_wait<0>();
+        __syncthreads();
+
+        const bool slow = intra_chunk<DK, DV>(st, A32, T32, sh, LAM, true);
+
+        // ---- Dh = gam . dSigma (fast) or dSigma (slow) as bf16; row sums of
+        // dSigma . Sigma (Sigma = next chunk-boundary state) for dL_end
+        {
+            const bf16 *Snext = states + (size_t)(n + 1) * DK * DV;
+#pragma unroll
+            for (int mt = 0; mt < MTS; ++mt) {
+                const int c = c0 + 16 * mt + (lane >> 2);
+                const float g0 = slow ? 1.f : sh.gamma[c], g1 = slow ? 1.f : sh.gamma[c + 8];
+                float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < NTS; ++nt) {
+                    const int j = j0 + 8 * nt + 2 * (lane & 3);
+                    *reinterpret_cast<uint32_t *>(D16 + swz<DV>(c, j)) =
+                        pack_bf16(g0 * dS[mt][nt][0], g0 * dS[mt][nt][1]);
+                    *reinterpret_cast<uint32_t *>(D16 + swz<DV>(c + 8, j)) =
+                        pack_bf16(g1 * dS[mt][nt][2], g1 * dS[mt][nt][3]);
+                    const __nv_bfloat162 s0 = *reinterpret_cast<const __nv_bfloat162 *>(Snext + (size_t)c * DV + j);
+                    const __nv_bfloat162 s1 =
+                        *reinterpret_cast<const __nv_bfloat162 *>(Snext + (size_t)(c + 8) * DV + j);
+                    r0 += dS[mt][nt][0] * __low2float(s0) + dS[mt][nt][1] * __high2float(s0);
+                    r1 += dS[mt][nt][2] * __low2float(s1) + dS[mt][nt][3] * __high2float(s1);
+                }
+                r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
+                r0 += __shfl_xor_sync(0xffffffffu, r0, 2);
+                r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+                r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
+                if ((lane & 3) == 0) {
+                    RS[(warp & 1) * DK + c] = r0;
+                    RS[(warp & 1) * DK + c + 8] = r1;
+                }
+            }
+        }
+
+        // ---- W = T Gt (warps 4..7, stored negated), Uv = T WV (warps 0..3)
+        constexpr int NTX = NTV > NTK ? NTV : NTK;
+        float accX[1][NTX][4];
+        auto &accV = reinterpret_cast<float(&)[1][NTV][4]>(accX);
+        auto &accK = reinterpret_cast<float(&)[1][NTK][4]>(accX);
+        zero(accX);
+        if (warp < 4) {
+            warp_gemm<1, NTV, true, false, 64, DV>(accV, T16, 16 * warp, st.v, 0, C, lane);
+        } else {
+            warp_gemm<1, NTK, true, false, 64, DK>(accK, T16, 16 * (warp & 3), st.b, 0, C, lane);
+            store_tile_bf16<NTK, DK>(accK, W16, 16 * (warp & 3), lane, -1.f);
+        }
+        __syncthreads();
+        // ---- U = Uv - W S (warps 0..3) into the w slot
+        if (warp < 4) {
+            warp_gemm<1, NTV, true, false, DK, DV>(accV, W16, 16 * warp, S16, 0, DK, lane);
+            store_tile_bf16<NTV, DV>(accV, U16, 16 * warp, lane, 1.f);
+        }
+        __syncthreads();
+
+        // ---- dU = M^T dO + Kh Dh (warps 0..3) ; dM = lower(dO U^T) (warps 4..7)
+        if (warp < 4) {
+            zero(accX);
+            warp_gemm<1, NTV, false, false, 64, DV>(accV, M16, 16 * warp, dO16, 0, C, lane);
+            warp_gemm<1, NTV, true, false, DK, DV>(accV, st.la, 16 * warp, D16, 0, DK, lane);
+            store_tile_bf16<NTV, DV>(accV, dU16, 16 * warp, lane, 1.f);
+        } else {
+            float acc[1][8][4];
+            zero(acc);
+            warp_gemm<1, 8, true, true, DV, DV>(acc, dO16, 16 * (warp & 3), U16, 0, DV, lane);
+            const int r0 = 16 * (warp & 3) + (lane >> 2);
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    // The diagonal of M carries no decay factor (e^{L_r - L_r} = 1):
+                    // its gradient goes straight to dq and dk in fp32 and is kept
+                    // out of the Gram products, where it would cancel in dL.
+                    const int r = r0 + (e >> 1) * 8, i = 8 * nt + 2 * (lane & 3) + (e & 1);
+                    if (i == r) DMD[r] = acc[0][nt][e];
+                    if (i >= r) acc[0][nt][e] = 0.f;
+                }
+            store_tile_bf16<8, 64>(acc, dM16, 16 * (warp & 3), lane, 1.f);
+        }
+        __syncthreads();
+
+        // ---- nR = -T^T dU, dv, dw (warps 0..3) ; dKb(state) = U Dh^T (warps 4..7)
+        if (warp < 4) {
+            zero(accX);
+            warp_gemm<1, NTV, false, false, 64, DV>(accV, T16, 16 * warp, dU16, 0, C, lane);
+            store_tile_bf16<NTV, DV>(accV, nR16, 16 * warp, lane, -1.f);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int r = 16 * warp + (lane >> 2) + 8 * half;
+                if (r < Cn) {
+                    const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV;
+#pragma unroll
+                    for (int nt = 0; nt < NTV; ++nt) {
+                        const int j = 8 * nt + 2 * (lane & 3);
+                        const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162 *>(gv + o + j);
+                        const __nv_bfloat162 w2 = *reinterpret_cast<const __nv_bfloat162 *>(gw + o + j);
+                        const float d0 = accV[0][nt][2 * half], d1 = accV[0][nt][2 * half + 1];
+                        *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dv) + o + j) =
+                            pack_bf16(d0 * __low2float(w2), d1 * __high2float(w2));
+                        *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dw) + o + j) =
+                            pack_bf16(d0 * __low2float(v2), d1 * __high2float(v2));
+                    }
+                }
+            }
+        } else {
+            zero(accX);
+            warp_gemm<1, NTK, true, true, DV, DV>(accK, U16, 16 * (warp & 3), D16, 0, DV, lane);
+            store_tile_f32<NTK>(accK, DKB, DK, 16 * (warp & 3), lane);
+        }
+        __syncthreads();
+
+        // ---- dA = strict_lower(nR U^T) (warps 0..3) ; dQt = dO S^T (warps 4..7)
+        if (warp < 4) {
+            float acc[1][8][4];
+            zero(acc);
+            warp_gemm<1, 8, true, true, DV, DV>(acc, nR16, 16 * warp, U16, 0, DV, lane);
+            const int r0 = 16 * warp + (lane >> 2);
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = r0 + (e >> 1) * 8, i = 8 * nt + 2 * (lane & 3) + (e & 1);
+                    if (i >= r) acc[0][nt][e] = 0.f;
+                }
+            store_tile_bf16<8, 64>(acc, dA16, 16 * warp, lane, 1.f);
+        } else {
+            zero(accX);
+            warp_gemm<1, NTK, true, true, DV, DV>(accK, dO16, 16 * (warp & 3), S16, 0, DV, lane);
+        }
+        __syncthreads();
+
+        // ---- dGt = nR S^T + dA Kb (warps 0..3) ; dQt += dM Kb, dKb += dA^T Gt + dM^T Qt (warps 4..7)
+        if (warp < 4) {
+            zero(accX);
+            warp_gemm<1, NTK, true, true, DV, DV>(accK, nR16, 16 * warp, S16, 0, DV, lane);
+            if (!slow) warp_gemm<1, NTK, true, false, 64, DK>(accK, dA16, 16 * warp, st.la, 0, C, lane);
+            store_tile_f32<NTK>(accK, DGT, DK, 16 * warp, lane);
+        } else {
+            const int m0 = 16 * (warp & 3);
+            if (!slow) warp_gemm<1, NTK, true, false, 64, DK>(accK, dM16, m0, st.la, 0, C, lane);
+            store_tile_f32<NTK>(accK, DQT, DK, m0, lane);
+            if (!slow) {
+                zero(accX);
+                warp_gemm<1, NTK, false, false, 64, DK>(accK, dA16, m0, st.b, 0, C, lane);
+                warp_gemm<1, NTK, false, false, 64, DK>(accK, dM16, m0, st.q, 0, C, lane);
+                const int r = m0 + (lane >> 2);
+#pragma unroll
+                for (int nt = 0; nt < NTK; ++nt) {
+                    const int c = 8 * nt + 2 * (lane & 3);
+                    float2 *p0 = reinterpret_cast<float2 *>(DKB + r * DK + c);
+                    float2 *p1 = reinterpret_cast<float2 *>(DKB + (r + 8) * DK + c);
+                    float2 x0 = *p0, x1 = *p1;
+                    x0.x += accK[0][nt][0]; x0.y += accK[0][nt][1];
+                    x1.x += accK[0][nt][2]; x1.y += accK[0][nt][3];
+                    *p0 = x0;
+                    *p1 = x1;
+                }
+            }
+        }
+
+        // ---- dSigma <- Diag(gam) dSigma + Qt^T dO + Gt^T nR (all warps)
+#pragma unroll
+        for (int mt = 0; mt < MTS; ++mt) {
+            const float g0 = sh.gamma[c0 + 16 * mt + (lane >> 2)], g1 = sh.gamma[c0 + 16 * mt + (lane >> 2) + 8];
+#pragma unroll
+            for (int nt = 0; nt < NTS; ++nt) {
+                dS[mt][nt][0] *= g0; dS[mt][nt][1] *= g0; dS[mt][nt][2] *= g1; dS[mt][nt][3] *= g1;
+            }
+        }
+        warp_gemm<MTS, NTS, false, false, DK, DV>(dS, st.q, c0, dO16, j0, C, lane);
+        warp_gemm<MTS, NTS, false, false, DK, DV>(dS, st.b, c0, nR16, j0, C, lane);
+        __syncthreads();
+
+        // ---- slow chunk: Gram gradients term by term, e^{L_r - L_i} <= 1
+        const int ch = tid % DK, seg = tid / DK;
+        if (slow) {
+            if (seg == 0) {
+                for (int r = 0; r < C; ++r) {
+                    PQ[r * DK + ch] = 0.f; PG[r * DK + ch] = 0.f; PK[r * DK + ch] = 0.f; PL[r * DK + ch] = 0.f;
+                }
+                for (int r = 0; r < Cn; ++r) {
+                    const size_t orr = (((size_t)b * T + n * C + r) * H + h) * DK + ch;
+                    const float qr = __bfloat162float(gq[orr]);
+                    const float gr = __bfloat162float(gb[orr]) * __bfloat162float(gk[orr]);
+                    const float lr = LAM[r * DK + ch];
+                    float pq = 0.f, pg = 0.f, pl = 0.f;
+                    for (int i = 0; i <= r; ++i) {
+                        const size_t oi = (((size_t)b * T + n * C + i) * H + h) * DK + ch;
+                        const float ki = __bfloat162float(gk[oi]);
+                        const float e = __expf(lr - LAM[i * DK + ch]);
+                        const float wA = i < r ? __bfloat162float(dA16[swz<64>(r, i)]) * e : 0.f;
+                        const float wM = __bfloat162float(dM16[swz<64>(r, i)]) * e;
+                        pg += wA * ki;
+                        pq += wM * ki;
+                        const float tk = wA * gr + wM * qr;
+                        PK[i * DK + ch] += tk;
+                        const float tl = tk * ki;
+                        pl += tl;
+                        PL[i * DK + ch] -= tl;
+                    }
+                    PQ[r * DK + ch] += pq;
+                    PG[r * DK + ch] += pg;
+                    PL[r * DK + ch] += pl;
+                }
+            }
+            __syncthreads();
+        }
+
+        // ---- elementwise gradients and the in-chunk reverse cumulative sum
+        {
+            const float lend = LAM[(Cn - 1) * DK + ch];
+            float part = 0.f;
+            for (int r = seg * RSEG; r < (seg + 1) * RSEG; ++r) {
+                if (r >= Cn) break;
+                const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + ch;
+                const float q = __bfloat162float(gq[o]), kk = __bfloat162float(gk[o]);
+                const float bb = __bfloat162float(gb[o]);
+                const float lam = LAM[r * DK + ch];
+                const float e = __expf(lam);
+                const float dqt = DQT[r * DK + ch], dgt = DGT[r * DK + ch], dkb = DKB[r * DK + ch];
+                float dq, dg, dkx, dL;
+                if (!slow) {
+                    const float ie = __expf(-lam);
+                    dq = dqt * e;
+                    dg = dgt * e;
+                    dkx = dkb * ie;
+                    dL = dqt * q * e + dgt * bb * kk * e - dkb * kk * ie;
+                } else {
+                    const float ke = __expf(lend - lam);
+                    dq = dqt * e + PQ[r * DK + ch];
+                    dg = dgt * e + PG[r * DK + ch];
+                    dkx = dkb * ke + PK[r * DK + ch];
+                    dL = dqt * q * e + dgt * bb * kk * e - dkb * kk * ke + PL[r * DK + ch];
+                }
+                const float mdiag = DMD[r];
+                dq += mdiag * kk;
+                dkx += mdiag * q;
+                if (r == Cn - 1) dL += RS[ch] + RS[DK + ch];
+                static_cast<bf16 *>(a.dq)[o] = __float2bfloat16_rn(dq);
+                static_cast<bf16 *>(a.dk)[o] = __float2bfloat16_rn(dkx + dg * bb);
+                static_cast<bf16 *>(a.db)[o] = __float2bfloat16_rn(dg * kk);
+                DLAM[r * DK + ch] = dL;
+                part += dL;
+            }
+            s_dpart[seg][ch] = part;
+            __syncthreads();
+            float acc = 0.f;
+#pragma unroll
+            for (int s = 0; s < P; ++s)
+                if (s > seg) acc += s_dpart[s][ch];
+            for (int r = min(Cn, (seg + 1) * RSEG) - 1; r >= seg * RSEG; --r) {
+                acc += DLAM[r * DK + ch];
+                static_cast<bf16 *>(a.dlog_alpha)[(((size_t)b * T + n * C + r) * H + h) * DK + ch] =
+                    __float2bfloat16_rn(acc);
+            }
+        }
+        __syncthreads();
+    }
+
+    if (a.dS0) {
+#pragma unroll
+        for (int mt = 0; mt < MTS; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NTS; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; e += 2) {
+                    const int c = c0 + 16 * mt + (lane >> 2) + (e >> 1) * 8;
+                    const int j = j0 + 8 * nt + 2 * (lane & 3);
+                    *reinterpret_cast<float2 *>(a.dS0 + (size_t)bh * DK * DV + (size_t)c * DV + j) =
+                        make_float2(dS[mt][nt][e], dS[mt][nt][e + 1]);
+                }
+    }
+}
+
+template <int DK, int DV>
+cudaError_t launch_t(const ChunkBwdArgs &a, cudaStream_t s) {
+    // (1) state pass: the forward with bf16 chunk-boundary states, no output
+    ChunkFwdArgs f{a.q, a.k, a.v, a.log_alpha, a.b, a.w, a.S0, nullptr, nullptr, a.scratch, a.scr_stride,
+                   a.states, a.B, a.T, a.H};
+    cudaError_t e = launch_chunk_fwd(f, DK, DV, s);
+    if (e != cudaSuccess) return e;
+    // (2) reverse chunk pass
+    constexpr int bytes = BSmem<DK, DV>::BYTES;
+    e = cudaFuncSetAttribute(chunk_bwd_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    chunk_bwd_kernel<DK, DV><<<(unsigned)(a.B * a.H), NTHR, bytes, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int DK, int DV>
+size_t ws_t(int B, int T, int H, size_t *scr_stride, size_t *states_bytes) {
+    const size_t nc = (size_t)((T + C - 1) / C);
+    const size_t sb = ((size_t)B * H * (nc + 1) * DK * DV * 2 + 255) / 256 * 256;
+    const size_t stride = (Scratch<DK>::FLOATS + 63) / 64 * 64;
+    if (scr_stride) *scr_stride = stride;
+    if (states_bytes) *states_bytes = sb;
+    return sb + (size_t)B * H * stride * sizeof(float);
+}
+
+}  // namespace cbwd
+
+size_t chunk_bwd_ws_bytes(int B, int T, int H, int dk, int dv, size_t *scr_stride, size_t *states_bytes) {
+    if (dk == 128 && dv == 128) return cbwd::ws_t<128, 128>(B, T, H, scr_stride, states_bytes);
+    if (dk == 128 && dv == 64) return cbwd::ws_t<128, 64>(B, T, H, scr_stride, states_bytes);
+    if (dk == 64 && dv == 128) return cbwd::ws_t<64, 128>(B, T, H, scr_stride, states_bytes);
+    return cbwd::ws_t<64, 64>(B, T, H, scr_stride, states_bytes);
+}
+
+cudaError_t launch_chunk_bwd(const ChunkBwdArgs &a, int dk, int dv, cudaStream_t s) {
+    if (dk == 128 && dv == 128) return cbwd::launch_t<128, 128>(a, s);
+    if (dk == 128 && dv == 64) return cbwd::launch_t<128, 64>(a, s);
+    if (dk == 64 && dv == 128) return cbwd::launch_t<64, 128>(a, s);
+    return cbwd::launch_t<64, 64>(a, s);
+}
+
+}  // namespace gdn2

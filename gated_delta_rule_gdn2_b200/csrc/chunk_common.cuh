@@ -1,0 +1,420 @@
+// Building blocks shared by the chunk-parallel forward and backward kernels:
+// warp-level bf16 tensor-core products over swizzled shared-memory tiles,
+// cp.async tile loads, and the intra-chunk stage (decay prefix, gated and
+// decay-referenced operands, key Gram matrices, the WY solve).
+//
+// Chunk algebra ("Why NVIDIA Gated DeltaNet-2 separates erase and write
+// gates", section "Gated Delta Rule-2: per-channel erase/write split"; WY form
+// from the laonpeople Gated DeltaNet page, parallel-computation section).  For
+// a chunk of C = 64 tokens, L = in-chunk cumulative log-decay, g = b . k:
+//
+//   Gt = g e^{L}, Qt = q e^{L}  (in (0,1]),   Kb = k e^{-L},   gam = e^{L_end}
+//   A = strict_lower([Gt] Kb^T),  M = lower([Qt] Kb^T),  T = (I + A)^{-1}
+//
+// Kb grows with the decay inside the chunk.  A chunk in which a key channel
+// decays by more than e^{-64} ("slow" chunk) forms A and M term by term from
+// e^{L_r - L_i} <= 1 instead and replaces Kb by Kt = k e^{L_end - L} (<= 1).
+#pragma once
+
+#include "common.cuh"
+
+namespace gdn2 {
+namespace chunk {
+
+typedef __nv_bfloat16 bf16;
+constexpr int C = 64;
+constexpr int NTHR = 256;
+constexpr float kSpanGuard = 64.f;  // max in-chunk log-decay span of the fast path
+
+// [rows][D] bf16 tiles: the 16-byte chunk index of a row is XORed with
+// (row & 7) so that ldmatrix row addresses fall in distinct banks.
+template <int D>
+__device__ __forceinline__ int swz(int r, int c) {
+    return r * D + ((((c >> 3) ^ (r & 7))) << 3) + (c & 7);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void ldsm4(uint32_t a, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(a));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t a, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(a));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool ok) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(ok ? 16 : 0));
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+// acc[MT][NT][4] += A[m0 + 16 mt + .., k] * B[k, n0 + 8 nt + ..], k in [0, K).
+// A_KM: A stored [m][k] in a [.][DA] tile, else stored [k][m].
+// B_KM: B stored [n][k] in a [.][DB] tile, else stored [k][n].
+template <int MT, int NT, bool A_KM, bool B_KM, int DA, int DB>
+__device__ __forceinline__ void warp_gemm(float (&acc)[MT][NT][4], const bf16 *A, int m0, const bf16 *B,
+                                          int n0, int K, int lane) {
+    static_assert(NT % 2 == 0, "n tiles come in pairs");
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        uint32_t a[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            if (A_KM) {
+                const int r = m0 + 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int c = k0 + (lane >> 4) * 8;
+                ldsm4(smem_u32(A + swz<DA>(r, c)), a[mt]);
+            } else {
+                const int i = lane >> 3;
+                const int kr = k0 + (lane & 7) + (i >> 1) * 8;
+                const int mc = m0 + 16 * mt + (i & 1) * 8;
+                ldsm4t(smem_u32(A + swz<DA>(kr, mc)), a[mt]);
+            }
+        }
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+            uint32_t b[4];
+            if (B_KM) {
+                const int r = n0 + 16 * np + (lane & 7) + (lane >> 4) * 8;
+                const int c = k0 + ((lane >> 3) & 1) * 8;
+                ldsm4(smem_u32(B + swz<DB>(r, c)), b);
+            } else {
+                const int kr = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int nc = n0 + 16 * np + (lane >> 4) * 8;
+                ldsm4t(smem_u32(B + swz<DB>(kr, nc)), b);
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                mma16816(acc[mt][2 * np], a[mt], b[0], b[1]);
+                mma16816(acc[mt][2 * np + 1], a[mt], b[2], b[3]);
+            }
+        }
+    }
+}
+
+template <int MT, int NT>
+__device__ __forceinline__ void zero(float (&acc)[MT][NT][4]) {
+#pragma unroll
+    for (int i = 0; i < MT; ++i)
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+}
+
+// Writes a 16-row accumulator tile (rows m0.., cols 0..8NT) as bf16 into a
+// swizzled [.][D] tile, scaled by `scale`.
+template <int NT, int D>
+__device__ __forceinline__ void store_tile_bf16(const float (&acc)[1][NT][4], bf16 *dst, int m0, int lane,
+                                                float scale) {
+    const int r = m0 + (lane >> 2);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int c = 8 * nt + 2 * (lane & 3);
+        *reinterpret_cast<uint32_t *>(dst + swz<D>(r, c)) = pack_bf16(scale * acc[0][nt][0], scale * acc[0][nt][1]);
+        *reinterpret_cast<uint32_t *>(dst + swz<D>(r + 8, c)) =
+            pack_bf16(scale * acc[0][nt][2], scale * acc[0][nt][3]);
+    }
+}
+
+// Writes a 16-row accumulator tile as fp32 into a plain row-major [.][ld] array.
+template <int NT>
+__device__ __forceinline__ void store_tile_f32(const float (&acc)[1][NT][4], float *dst, int ld, int m0,
+                                               int lane) {
+    const int r = m0 + (lane >> 2);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int c = 8 * nt + 2 * (lane & 3);
+        *reinterpret_cast<float2 *>(dst + r * ld + c) = make_float2(acc[0][nt][0], acc[0][nt][1]);
+        *reinterpret_cast<float2 *>(dst + (r + 8) * ld + c) = make_float2(acc[0][nt][2], acc[0][nt][3]);
+    }
+}
+
+// cp.async of rows [n*C, n*C + C) of a token tensor [B,T,H,D] (head h of
+// batch b) into a swizzled [C][D] tile; rows past T are zero-filled.
+template <int D>
+__device__ __forceinline__ void load_token_tile(bf16 *dst, const bf16 *src, int b, int h, int n, int T, int H) {
+    constexpr int CPR = D / 8;  // 16-byte chunks per row
+    for (int id = threadIdx.x; id < C * CPR; id += NTHR) {
+        const int r = id / CPR, ch = id % CPR;
+        const int t = n * C + r;
+        const bool ok = t < T;
+        const bf16 *g = src + (ok ? ((((size_t)b * T + t) * H + h) * D + ch * 8) : 0);
+        cp_async16(dst + swz<D>(r, ch * 8), g, ok);
+    }
+}
+
+struct ChunkTiles {
+    bf16 *q, *k, *la, *b, *v, *w;
+};
+
+// Shared-memory scratch of the intra-chunk stage (static, per CTA).
+template <int DK>
+struct IntraShared {
+    float part[NTHR / DK][DK];
+    float gamma[DK];
+    int slow;
+};
+
+// Intra-chunk stage.  On entry the six raw token tiles of the chunk are in
+// shared memory (and visible to all threads).  On exit (all threads, after a
+// barrier):
+//   st.q -> Qt, st.b -> Gt, st.la -> Kb (fast) or Kt (slow), st.v -> w . v;
+//   T16 = bf16 (I + A)^{-1} and M16 = bf16 M (swizzled [64][64]);
+//   sh.gamma = e^{L_end}; returns true for a slow chunk.
+// A32 and T32 are 64x64 fp32 work areas; A32 is free on return, T32 holds
+// T16 and M16.  lam_ws (per-CTA [64][DK] fp32, global) receives L when
+// keep_lam is set and is always used by a slow chunk.
+template <int DK, int DV>
+__device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<DK> &sh, float *lam_ws,
+                            bool keep_lam) {
+    constexpr int P = NTHR / DK;
+    constexpr int RSEG = C / P;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    bf16 *T16 = reinterpret_cast<bf16 *>(T32);
+    bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
+
+    if (tid == 0) sh.slow = 0;
+    // ---- pass 1: per-channel segment sums of log_alpha, and w . v in place of v
+    const int ch = tid % DK, seg = tid / DK;
+    {
+        float part = 0.f;
+        for (int r = seg * RSEG; r < (seg + 1) * RSEG; ++r) part += __bfloat162float(st.la[swz<DK>(r, ch)]);
+        sh.part[seg][ch] = part;
+        for (int id = tid; id < C * DV / 8; id += NTHR) {
+            uint4 wv = reinterpret_cast<const uint4 *>(st.w)[id];
+            uint4 vv = reinterpret_cast<const uint4 *>(st.v)[id];
+            const bf16 *w8 = reinterpret_cast<const bf16 *>(&wv);
+            const bf16 *v8 = reinterpret_cast<const bf16 *>(&vv);
+            uint4 o;
+            uint32_t *o4 = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                o4[e] = pack_bf16(__bfloat162float(w8[2 * e]) * __bfloat162float(v8[2 * e]),
+                                  __bfloat162float(w8[2 * e + 1]) * __bfloat162float(v8[2 * e + 1]));
+            reinterpret_cast<uint4 *>(st.v)[id] = o;
+        }
+    }
+    __syncthreads();
+    float lam0 = 0.f, lam_end = 0.f;
+#pragma unroll
+    for (int s = 0; s < P; ++s) {
+        const float p = sh.part[s][ch];
+        if (s < seg) lam0 += p;
+        lam_end += p;
+    }
+    if (seg == 0) {
+        sh.gamma[ch] = __expf(lam_end);
+        if (-lam_end > kSpanGuard) sh.slow = 1;
+    }
+    __syncthreads();
+    const bool slow = sh.slow != 0;
+
+    float accM[1][8][4];  // M rows of warps 4..7 (lower incl. diagonal)
+    if (!slow) {
+        // ---- pass 2 (fast): Qt, Gt, Kb in place of q, b, log_alpha
+        float lam = lam0;
+        for (int r = seg * RSEG; r < (seg + 1) * RSEG; ++r) {
+            const int o = swz<DK>(r, ch);
+            lam += __bfloat162float(st.la[o]);
+            if (keep_lam) lam_ws[r * DK + ch] = lam;
+            const float e = __expf(lam), ie = __expf(-lam);
+            const float kk = __bfloat162float(st.k[o]);
+            st.q[o] = __float2bfloat16_rn(__bfloat162float(st.q[o]) * e);
+            st.b[o] = __float2bfloat16_rn(__bfloat162float(st.b[o]) * kk * e);
+            st.la[o] = __float2bfloat16_rn(kk * ie);
+        }
+        __syncthreads();
+        // ---- Grams: [Gt; Qt] Kb^T, warp w -> rows 16w..16w+15 of the stacked operand
+        float acc[1][8][4];
+        zero(acc);
+        const bf16 *Aop = warp < 4 ? st.b : st.q;
+        warp_gemm<1, 8, true, true, DK, DK>(acc, Aop, 16 * (warp & 3), st.la, 0, DK, lane);
+        const int r0 = 16 * (warp & 3) + (lane >> 2);
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = r0 + (e >> 1) * 8, i = 8 * nt + 2 * (lane & 3) + (e & 1);
+                if (warp < 4) A32[r * C + i] = i < r ? acc[0][nt][e] : 0.f;
+                else accM[0][nt][e] = i <= r ? acc[0][nt][e] : 0.f;
+            }
+    } else {
+        // ---- slow chunk: exact per-term decays.  L goes to the per-CTA
+        // workspace; raw q, k, b stay in shared memory until A and M exist.
+        float lam = lam0;
+        for (int r = seg * RSEG; r < (seg + 1) * RSEG; ++r) {
+            lam += __bfloat162float(st.la[swz<DK>(r, ch)]);
+            lam_ws[r * DK + ch] = lam;
+        }
+        __syncthreads();
+        float pa[9], pm[9];
+#pragma unroll
+        for (int s = 0; s < 9; ++s) {
+            pa[s] = 0.f;
+            pm[s] = 0.f;
+            const int p = tid + NTHR * s;
+            if (p < C * (C + 1) / 2) {
+                int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+                while ((r + 1) * (r + 2) / 2 <= p) ++r;
+                while (r * (r + 1) / 2 > p) --r;
+                const int i = p - r * (r + 1) / 2;
+                for (int c = 0; c < DK; ++c) {
+                    const float e = __expf(lam_ws[r * DK + c] - lam_ws[i * DK + c]);
+                    const float ki = __bfloat162float(st.k[swz<DK>(i, c)]);
+                    const float kr = __bfloat162float(st.k[swz<DK>(r, c)]);
+                    pa[s] += __bfloat162float(st.b[swz<DK>(r, c)]) * kr * ki * e;
+                    pm[s] += __bfloat162float(st.q[swz<DK>(r, c)]) * ki * e;
+                }
+            }
+        }
+        __syncthreads();
+        // Qt, Gt and Kt = k e^{L_end - L} in place of q, b, log_alpha
+        for (int r = seg * RSEG; r < (seg + 1) * RSEG; ++r) {
+            const int o = swz<DK>(r, ch);
+            const float lr = lam_ws[r * DK + ch];
+            const float e = __expf(lr);
+            const float kk = __bfloat162float(st.k[o]);
+            st.q[o] = __float2bfloat16_rn(__bfloat162float(st.q[o]) * e);
+            st.b[o] = __float2bfloat16_rn(__bfloat162float(st.b[o]) * kk * e);
+            st.la[o] = __float2bfloat16_rn(kk * __expf(lam_end - lr));
+        }
+        __syncthreads();
+        for (int e = tid; e < C * C; e += NTHR) {
+            A32[e] = 0.f;
+            T32[e] = 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int s = 0; s < 9; ++s) {
+            const int p = tid + NTHR * s;
+            if (p < C * (C + 1) / 2) {
+                int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+                while ((r + 1) * (r + 2) / 2 <= p) ++r;
+                while (r * (r + 1) / 2 > p) --r;
+                const int i = p - r * (r + 1) / 2;
+                if (i < r) A32[r * C + i] = pa[s];
+                T32[r * C + i] = pm[s];  // M parked in the T region
+            }
+        }
+        __syncthreads();
+        if (warp >= 4) {
+            const int r0 = 16 * (warp & 3) + (lane >> 2);
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    accM[0][nt][e] = T32[(r0 + (e >> 1) * 8) * C + 8 * nt + 2 * (lane & 3) + (e & 1)];
+        }
+    }
+    __syncthreads();
+
+    // ---- T = (I + A)^{-1}: 16x16 diagonal blocks by substitution, then
+    // off-diagonal blocks level by level: T_RQ = -T_RR sum_J A_RJ T_JQ.
+    if (tid < 64) {
+        const int R = tid >> 4, j = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float v = (r == j) ? 1.f : 0.f;
+            if (r > j) {
+#pragma unroll
+                for (int i = 0; i < r; ++i)
+                    if (i >= j) v -= A32[(16 * R + r) * C + 16 * R + i] * x[i];
+            }
+            x[r] = v;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) T32[(16 * R + r) * C + 16 * R + j] = x[r];
+    } else {
+        for (int e = tid - 64; e < 6 * 256; e += NTHR - 64) {
+            const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            const int R = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+            const int Q = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            T32[(16 * R + r) * C + 16 * Q + c] = 0.f;
+        }
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int lvl = 1; lvl < 4; ++lvl) {
+        const int nb = 4 - lvl;
+        float xv[3];
+#pragma unroll
+        for (int s = 0; s < 3; ++s) {
+            const int e = tid + 256 * s;
+            xv[s] = 0.f;
+            if (s < nb) {
+                const int Q = e >> 8, R = Q + lvl, r = (e >> 4) & 15, c = e & 15;
+                float acc = 0.f;
+                for (int J = Q; J < R; ++J)
+#pragma unroll
+                    for (int m = 0; m < 16; ++m)
+                        acc += A32[(16 * R + r) * C + 16 * J + m] * T32[(16 * J + m) * C + 16 * Q + c];
+                xv[s] = acc;
+            }
+        }
+#pragma unroll
+        for (int s = 0; s < 3; ++s)
+            if (s < nb) {
+                const int e = tid + 256 * s;
+                const int Q = e >> 8, R = Q + lvl, r = (e >> 4) & 15, c = e & 15;
+                T32[(16 * R + r) * C + 16 * Q + c] = xv[s];
+            }
+        __syncthreads();
+#pragma unroll
+        for (int s = 0; s < 3; ++s) {
+            if (s < nb) {
+                const int e = tid + 256 * s;
+                const int Q = e >> 8, R = Q + lvl, r = (e >> 4) & 15, c = e & 15;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    if (m <= r) acc += T32[(16 * R + r) * C + 16 * R + m] * T32[(16 * R + m) * C + 16 * Q + c];
+                xv[s] = -acc;
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int s = 0; s < 3; ++s)
+            if (s < nb) {
+                const int e = tid + 256 * s;
+                const int Q = e >> 8, R = Q + lvl, r = (e >> 4) & 15, c = e & 15;
+                T32[(16 * R + r) * C + 16 * Q + c] = xv[s];
+            }
+        __syncthreads();
+    }
+    // T32 -> T16, M -> M16 (both bf16, swizzled [64][64])
+    {
+        float tv[16];
+#pragma unroll
+        for (int s = 0; s < 16; ++s) tv[s] = T32[tid * 16 + s];
+        __syncthreads();
+        const int r = tid >> 2, cb = (tid & 3) * 16;
+#pragma unroll
+        for (int s = 0; s < 16; s += 2)
+            *reinterpret_cast<uint32_t *>(T16 + swz<64>(r, cb + s)) = pack_bf16(tv[s], tv[s + 1]);
+        if (warp >= 4) store_tile_bf16<8, 64>(accM, M16, 16 * (warp & 3), lane, 1.f);
+    }
+    __syncthreads();
+    return slow;
+}
+
+}  // namespace chunk
+}  // namespace gdn2

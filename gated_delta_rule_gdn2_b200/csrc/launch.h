@@ -26,19 +26,43 @@ struct RecurrentBwdArgs {
     int B, T, H;
 };
 
-// Chunk-parallel tensor-core forward (bf16 tokens).  ws: B*H*64*dk floats,
-// used only by chunks whose in-chunk decay exceeds the fast path's range.
+// Chunk-parallel tensor-core forward (bf16 tokens).  ws: per-CTA fp32
+// scratch of ws_stride floats (>= 64*dk), used by chunks whose in-chunk decay
+// exceeds the fast path's range.  states: optional bf16 [B*H][nchunks+1][dk][dv]
+// output of the state at every chunk boundary (the backward's state pass);
+// o may then be null.
 struct ChunkFwdArgs {
     const void *q, *k, *v, *log_alpha, *b, *w;
     const float *S0;
     void *o;
     float *S_T;
     float *ws;
+    size_t ws_stride;
+    void *states;
     int B, T, H;
 };
 
 cudaError_t launch_chunk_fwd(const ChunkFwdArgs &a, int dk, int dv, cudaStream_t s);
 size_t chunk_fwd_ws_bytes(int B, int H, int dk);
+
+// Chunk-parallel gate-aware backward (bf16 tokens): a state pass (the
+// forward writing bf16 chunk-boundary states to `states`) and a reverse chunk
+// pass.  scratch: per-CTA fp32 work area of scr_stride floats.
+struct ChunkBwdArgs {
+    const void *q, *k, *v, *log_alpha, *b, *w;
+    const float *S0;
+    const void *dO;
+    const float *dS_T;
+    void *dq, *dk, *dv, *dlog_alpha, *db, *dw;
+    float *dS0;
+    void *states;
+    float *scratch;
+    size_t scr_stride;
+    int B, T, H;
+};
+
+cudaError_t launch_chunk_bwd(const ChunkBwdArgs &a, int dk, int dv, cudaStream_t s);
+size_t chunk_bwd_ws_bytes(int B, int T, int H, int dk, int dv, size_t *scr_stride, size_t *states_bytes);
 
 cudaError_t launch_recurrent_fwd(const RecurrentArgs &a, int dk, int dv, bool bf16, cudaStream_t s);
 cudaError_t launch_recurrent_bwd(const RecurrentBwdArgs &a, int dk, int dv, bool bf16, cudaStream_t s);

@@ -98,3 +98,90 @@ def chunk_fwd(q, k, v, la, b, w, S0=None, bf16=False, force_slow=False):
                                                     la[bb, :, h], b[bb, :, h], w[bb, :, h], s0, bf16,
                                                     force_slow)
     return o, ST
+
+
+def chunk_bwd_head(q, k, v, la, b, w, S0, dO, dST, bf16=False, opts=()):
+    """Backward of chunk_fwd_head (fast path only), rounding the tensor-core
+    operands where the CUDA backward rounds them.  Returns dict of gradients."""
+    rd = rnd_bf16 if bf16 else (lambda x: np.asarray(x, dtype=np.float64))
+    out_rd = rd if "fp32_out" not in opts else (lambda x: np.asarray(x, dtype=np.float64))
+    T, dk = q.shape
+    dv = v.shape[1]
+    # forward states at chunk boundaries (bf16 as the state pass stores them)
+    S = np.array(S0, dtype=np.float64)
+    states = [rd(S)]
+    for n0 in range(0, T, C):
+        n1 = min(T, n0 + C)
+        _, S = chunk_fwd_head(q[n0:n1], k[n0:n1], v[n0:n1], la[n0:n1], b[n0:n1], w[n0:n1], S, bf16)
+        states.append(rd(S))
+    g = {n: np.zeros((T, dk)) for n in ("dq", "dk", "dlog_alpha", "db")}
+    g.update({n: np.zeros((T, dv)) for n in ("dv", "dw")})
+    dS = np.zeros((dk, dv)) if dST is None else np.array(dST, dtype=np.float64)
+    nchunks = (T + C - 1) // C
+    for n in range(nchunks - 1, -1, -1):
+        n0, n1 = n * C, min(T, n * C + C)
+        Sn = states[n]
+        Snext = states[n + 1]
+        qc, kc, vc, lac, bc, wc, dOc = (x[n0:n1].astype(np.float64) for x in (q, k, v, la, b, w, dO))
+        L = np.cumsum(lac, axis=0)
+        gg = bc * kc
+        e, ie = np.exp(L), np.exp(-L)
+        Gt, Qt, Kb, WV = rd(gg * e), rd(qc * e), rd(kc * ie), rd(wc * vc)
+        gam = np.exp(L[-1])
+        A = np.tril(Gt @ Kb.T, -1)
+        M = np.tril(Qt @ Kb.T, 0)
+        Tm = rd(np.linalg.inv(np.eye(n1 - n0) + A))
+        Mb = rd(M)
+        W = rd(-(Tm @ Gt))
+        Uv = Tm @ WV
+        U = rd(Uv + W @ Sn)
+        Dh = rd(gam[:, None] * dS)
+        rs = np.sum(dS * Snext, axis=1)
+        dU = rd(Mb.T @ dOc + Kb @ Dh)
+        dRHS = Tm.T @ dU
+        nR = rd(-dRHS)
+        g["dv"][n0:n1] = out_rd(dRHS * wc)
+        g["dw"][n0:n1] = out_rd(dRHS * vc)
+        dKb = U @ Dh.T
+        dMm = np.tril(dOc @ U.T, 0)
+        dAm = np.tril(nR @ U.T, -1)
+        dMdiag = np.diag(dMm).copy()  # the kernel keeps the diagonal out of the Gram products
+        dMm = dMm - np.diag(dMdiag)
+        dMb, dAb = rd(dMm), rd(dAm)
+        dQt = dOc @ Sn.T + dMb @ Kb
+        dGt = nR @ Sn.T + dAb @ Kb
+        dKb = dKb + dAb.T @ Gt + dMb.T @ Qt
+        dS = gam[:, None] * dS + Qt.T @ dOc + Gt.T @ nR
+        dq = dQt * e
+        dg = dGt * e
+        dkk = dKb * ie
+        dL = dQt * qc * e + dGt * gg * e - dKb * kc * ie
+        dq += dMdiag[:, None] * kc
+        dkk += dMdiag[:, None] * qc
+        dL[-1] += rs
+        g["dq"][n0:n1] = out_rd(dq)
+        g["dk"][n0:n1] = out_rd(dkk + dg * bc)
+        g["db"][n0:n1] = out_rd(dg * kc)
+        g["dlog_alpha"][n0:n1] = out_rd(np.cumsum(dL[::-1], axis=0)[::-1])
+    g["dS0"] = dS
+    return g
+
+
+def chunk_bwd(q, k, v, la, b, w, S0, dO, dST=None, bf16=False, opts=()):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    out = {n: np.zeros((B, T, H, dk)) for n in ("dq", "dk", "dlog_alpha", "db")}
+    out.update({n: np.zeros((B, T, H, dv)) for n in ("dv", "dw")})
+    out["dS0"] = np.zeros((B, H, dk, dv))
+    for bb in range(B):
+        for h in range(H):
+            s0 = np.zeros((dk, dv)) if S0 is None else S0[bb, h]
+            dst = None if dST is None else dST[bb, h]
+            r = chunk_bwd_head(q[bb, :, h], k[bb, :, h], v[bb, :, h], la[bb, :, h], b[bb, :, h],
+                               w[bb, :, h], s0, dO[bb, :, h], dst, bf16, opts)
+            for n in out:
+                if n == "dS0":
+                    out[n][bb, h] = r[n]
+                else:
+                    out[n][bb, :, h] = r[n]
+    return out

@@ -46,3 +46,26 @@ def test_bf16_error_budget():
     oe, Se = E.chunk_fwd(*_args(x), bf16=True)
     rel = lambda a, b: np.linalg.norm(a - b) / np.linalg.norm(b)
     assert rel(oe, o) < 5e-3 and rel(Se, S) < 5e-3
+
+
+@pytest.mark.parametrize("T", [1, 64, 150])
+def test_chunk_backward_algebra_exact(T):
+    """The backward's chunk algebra (as the CUDA reverse pass computes it) is
+    the oracle's gradient in fp64."""
+    x = make_inputs(1, T, 2, 64, 64, seed=T, dtype="fp32", with_do=True)
+    rng = np.random.default_rng(T)
+    dST = rng.standard_normal(x["S0"].shape)
+    ref = oracle.bwd(*_args(x), x["dO"], dST)
+    got = E.chunk_bwd(*_args(x), x["dO"], dST)
+    for n in ref:
+        np.testing.assert_allclose(got[n], ref[n], rtol=0, atol=1e-11)
+
+
+def test_chunk_backward_bf16_error_budget():
+    x = make_inputs(1, 512, 1, 128, 128, seed=1004, dtype="bf16", with_do=True)
+    ref = oracle.bwd(*_args(x), x["dO"], None)
+    got = E.chunk_bwd(*_args(x), x["dO"], None, bf16=True)
+    rel = lambda a, b: np.linalg.norm(a - b) / np.linalg.norm(b)
+    for n in ref:
+        assert rel(got[n], ref[n]) < 8e-3, n
+        assert np.max(np.abs(got[n] - ref[n])) < 5e-2, n
