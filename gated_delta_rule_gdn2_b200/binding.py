@@ -32,6 +32,7 @@ SIGNATURES = {
     "gdn2_decode_step": (_I, [_P] * 8 + [_I] * 5 + [_P]),
     "gdn2_chunk_bwd_workspace": (_Z, [_I] * 6),
     "gdn2_chunk_bwd": (_I, [_P] * 16 + [_I] * 6 + [_P, _Z, _P]),
+    "gdn2_chunk_fwd_noalloc": (_I, [_P] * 9 + [_I] * 6 + [_P]),
 }
 
 _lib = None
@@ -106,6 +107,15 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, dk, dv, dtype,
     return load().gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
                                  _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, dtype, _ptr(ws),
                                  ws_bytes, _stream(stream))
+
+
+def gdn2_chunk_fwd_noalloc(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, dk, dv, dtype,
+                           stream=None) -> int:
+    """gdn2_chunk_fwd for callers that cannot allocate: the scratch comes from
+    a fixed 8 MiB array inside the library (see include/gdn2.h)."""
+    return load().gdn2_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                                         _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, dtype,
+                                         _stream(stream))
 
 
 def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o, B, H, dk, dv, dtype, stream=None) -> int:

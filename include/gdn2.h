@@ -108,6 +108,27 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
                    void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * gdn2_chunk_fwd without a caller-provided workspace, for callers that cannot
+ * allocate device memory (no cudaMalloc available to them, or a code path
+ * that must not allocate).  The pages have no counterpart to this call; it is
+ * an interface convenience of this library.
+ *
+ * Arguments, layouts, results and error codes are those of gdn2_chunk_fwd.
+ * The scratch comes from an 8 MiB array in the library's device image, which
+ * every GPU that loads the library holds until the process exits; problems
+ * needing more (B*H*dk > 32768, e.g. B*H > 256 at dk = 128) get
+ * GDN2_ERR_WORKSPACE before anything is launched.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture.  The call itself
+ * allocates nothing.  All calls share the one array and nothing in it needs
+ * to start at zero, but calls that overlap on the GPU (different streams, or
+ * concurrent host threads) race on it: serialise them.
+ */
+int gdn2_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *log_alpha,
+                           const void *b, const void *w, const float *S0, void *o, float *S_T,
+                           int B, int T, int H, int dk, int dv, int dtype, cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of
  * the current device: GDN2_OK, GDN2_ERR_TIMEOUT (a bounded device wait ran
  * out) or GDN2_ERR_CUDA (the stream reported an error).
