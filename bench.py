@@ -33,7 +33,7 @@ B, T, H, D = 8, 4096, 16, 128  # B can be lowered with --batch for profiling cap
 DEC_B, DEC_H = 256, 16
 WORKLOAD = "train fwd+bwd B8 T4096 H16 dk=dv=128 bf16 (prefill shape; decode B256 H16 alongside)"
 METRIC = "GDN-2 chunk fwd+bwd tokens/s & TFLOP/s (H16 dk=dv=128); decode state GB/s"
-# algorithmic work per (token, head), d = 128, C = 64
+# algorithmic work per (token, head), d = 128, C = 64: dense-counted products and bytes read + written once
 FLOP_FWD = 6 * D * D + 10 * 64 * D          # 180,224
 FLOP_BWD = 524288                            # state recompute + reverse pass + intra-chunk grads
 BYTES_FWD = 7 * D * 2                        # q,k,v,log_alpha,b,w in + o out, bf16
@@ -125,9 +125,13 @@ def kernel_traffic(name):
     d = json.load(open(p)).get(name)
     if not d:
         return None
-    src = os.path.join(ROOT, d["source"])
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] if os.path.exists(src) else None
-    return d["bytes_per_launch"] if h == d["source_sha"] else None
+    hs = hashlib.sha256()
+    for f in d["sources"]:
+        p = os.path.join(ROOT, f)
+        if not os.path.exists(p):
+            return None
+        hs.update(open(p, "rb").read())
+    return d["bytes_per_launch"] if hs.hexdigest()[:16] == d["source_sha"] else None
 
 
 # ---------------------------------------------------------------------------
@@ -283,9 +287,10 @@ def run_gpu(args):
     fwd_gbs = (th * BYTES_FWD + 2 * B * H * STATE_BYTES) / (fwd_ms * 1e-3) / 1e9
     bwd_gbs = (th * BYTES_BWD + 2 * B * H * STATE_BYTES) / (bwd_ms * 1e-3) / 1e9
     dom = "bwd" if bwd_ms >= fwd_ms else "fwd"
-    kname = {"fwd": "chunk_fwd_kernel", "bwd": "recurrent_bwd_kernel"}[dom]
+    kname = {"fwd": "chunk_fwd_kernel",
+             "bwd": "gdn2_chunk_bwd (state pass chunk_fwd_kernel + chunk_bwd_kernel)"}[dom]
     achieved = bwd_gbs if dom == "bwd" else fwd_gbs
-    traffic = kernel_traffic(kname)
+    traffic = kernel_traffic("chunk_fwd_kernel" if dom == "fwd" else "chunk_bwd")
     clocks = clk.summary()
     out = {
         "metric": METRIC,
@@ -322,7 +327,7 @@ def run_gpu(args):
                                              / ((fwd_ms if dom == "fwd" else bwd_ms) * 1e-3) / 1e12) / tf_sus},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 3 * args.steps,  # chunk_fwd_kernel, then the backward's state pass + reverse kernel
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -66,11 +66,10 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
     constexpr int WR = DK / 4, WC = DV / 2;
     constexpr int MTS = WR / 16, NTS = WC / 8;
     constexpr int NTV = DV / 8, NTK = DK / 8;
-    constexpr int P = NTHR / DK, RSEG = C / P;
 
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ IntraShared<DK> sh;
-    __shared__ float s_dpart[P][DK];
+    __shared__ float s_dpart[NTHR / (DK / 2)][DK];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
@@ -138,6 +137,27 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
         cp_commit();
         cp_wait<0>();
         __syncthreads();
+        if (n > 0) {
+            // warm L2 with the next chunk of the reverse walk while this one computes
+            const int slot = tid & 63, grp = tid >> 6;
+            if (grp == 0) {
+                prefetch_token_rows_l2<DK>(gq, b, h, n - 1, T, H, slot, 64);
+                prefetch_token_rows_l2<DK>(gk, b, h, n - 1, T, H, slot, 64);
+            } else if (grp == 1) {
+                prefetch_token_rows_l2<DK>(static_cast<const bf16 *>(a.log_alpha), b, h, n - 1, T, H, slot, 64);
+                prefetch_token_rows_l2<DK>(gb, b, h, n - 1, T, H, slot, 64);
+            } else if (grp == 2) {
+                prefetch_token_rows_l2<DV>(gv, b, h, n - 1, T, H, slot, 64);
+                prefetch_token_rows_l2<DV>(gw, b, h, n - 1, T, H, slot, 64);
+            } else {
+                prefetch_token_rows_l2<DV>(static_cast<const bf16 *>(a.dO), b, h, n - 1, T, H, slot, 64);
+                if (slot < 16) {
+                    const bf16 *sp = states + (size_t)(n - 1) * DK * DV + (size_t)slot * (DK * DV / 16);
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(sp), "r"(DK * DV * 2 / 16)
+                                 : "memory");
+                }
+            }
+        }
 
         const bool slow = intra_chunk<DK, DV>(st, A32, T32, sh, LAM, true);
 
@@ -348,51 +368,76 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
         }
 
         // ---- elementwise gradients and the in-chunk reverse cumulative sum
+        // (two key channels per thread, rows split into P2 segments)
         {
-            const float lend = LAM[(Cn - 1) * DK + ch];
-            float part = 0.f;
-            for (int r = seg * RSEG; r < (seg + 1) * RSEG; ++r) {
-                if (r >= Cn) break;
-                const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + ch;
-                const float q = __bfloat162float(gq[o]), kk = __bfloat162float(gk[o]);
-                const float bb = __bfloat162float(gb[o]);
-                const float lam = LAM[r * DK + ch];
-                const float e = __expf(lam);
-                const float dqt = DQT[r * DK + ch], dgt = DGT[r * DK + ch], dkb = DKB[r * DK + ch];
-                float dq, dg, dkx, dL;
-                if (!slow) {
-                    const float ie = __expf(-lam);
-                    dq = dqt * e;
-                    dg = dgt * e;
-                    dkx = dkb * ie;
-                    dL = dqt * q * e + dgt * bb * kk * e - dkb * kk * ie;
-                } else {
-                    const float ke = __expf(lend - lam);
-                    dq = dqt * e + PQ[r * DK + ch];
-                    dg = dgt * e + PG[r * DK + ch];
-                    dkx = dkb * ke + PK[r * DK + ch];
-                    dL = dqt * q * e + dgt * bb * kk * e - dkb * kk * ke + PL[r * DK + ch];
+            constexpr int NP = DK / 2, P2 = NTHR / NP, RS2 = C / P2;
+            const int cp = tid % NP, s2 = tid / NP, c2 = 2 * cp;
+            const float2 lend = *reinterpret_cast<const float2 *>(LAM + (Cn - 1) * DK + c2);
+            const float2 rs0 = *reinterpret_cast<const float2 *>(RS + c2);
+            const float2 rs1 = *reinterpret_cast<const float2 *>(RS + DK + c2);
+            float pa = 0.f, pb = 0.f;
+#pragma unroll 4
+            for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r) {
+                if (r < Cn) {
+                    const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c2;
+                    const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(gq + o));
+                    const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(gk + o));
+                    const float2 bb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(gb + o));
+                    const float2 lam = *reinterpret_cast<const float2 *>(LAM + r * DK + c2);
+                    const float2 dqt = *reinterpret_cast<const float2 *>(DQT + r * DK + c2);
+                    const float2 dgt = *reinterpret_cast<const float2 *>(DGT + r * DK + c2);
+                    const float2 dkb = *reinterpret_cast<const float2 *>(DKB + r * DK + c2);
+                    const float mdiag = DMD[r];
+                    const float ea = __expf(lam.x), eb = __expf(lam.y);
+                    float dqa, dqb, dga, dgb, dka, dkb2, dla, dlb;
+                    if (!slow) {
+                        const float iea = __expf(-lam.x), ieb = __expf(-lam.y);
+                        dqa = dqt.x * ea; dqb = dqt.y * eb;
+                        dga = dgt.x * ea; dgb = dgt.y * eb;
+                        dka = dkb.x * iea; dkb2 = dkb.y * ieb;
+                        dla = dqt.x * q.x * ea + dgt.x * bb.x * kk.x * ea - dkb.x * kk.x * iea;
+                        dlb = dqt.y * q.y * eb + dgt.y * bb.y * kk.y * eb - dkb.y * kk.y * ieb;
+                    } else {
+                        const float kea = __expf(lend.x - lam.x), keb = __expf(lend.y - lam.y);
+                        const float2 pq = *reinterpret_cast<const float2 *>(PQ + r * DK + c2);
+                        const float2 pg = *reinterpret_cast<const float2 *>(PG + r * DK + c2);
+                        const float2 pk = *reinterpret_cast<const float2 *>(PK + r * DK + c2);
+                        const float2 pl = *reinterpret_cast<const float2 *>(PL + r * DK + c2);
+                        dqa = dqt.x * ea + pq.x; dqb = dqt.y * eb + pq.y;
+                        dga = dgt.x * ea + pg.x; dgb = dgt.y * eb + pg.y;
+                        dka = dkb.x * kea + pk.x; dkb2 = dkb.y * keb + pk.y;
+                        dla = dqt.x * q.x * ea + dgt.x * bb.x * kk.x * ea - dkb.x * kk.x * kea + pl.x;
+                        dlb = dqt.y * q.y * eb + dgt.y * bb.y * kk.y * eb - dkb.y * kk.y * keb + pl.y;
+                    }
+                    dqa += mdiag * kk.x; dqb += mdiag * kk.y;
+                    dka += mdiag * q.x; dkb2 += mdiag * q.y;
+                    if (r == Cn - 1) { dla += rs0.x + rs1.x; dlb += rs0.y + rs1.y; }
+                    *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dq) + o) = pack_bf16(dqa, dqb);
+                    *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dk) + o) =
+                        pack_bf16(dka + dga * bb.x, dkb2 + dgb * bb.y);
+                    *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.db) + o) = pack_bf16(dga * kk.x, dgb * kk.y);
+                    *reinterpret_cast<float2 *>(DLAM + r * DK + c2) = make_float2(dla, dlb);
+                    pa += dla;
+                    pb += dlb;
                 }
-                const float mdiag = DMD[r];
-                dq += mdiag * kk;
-                dkx += mdiag * q;
-                if (r == Cn - 1) dL += RS[ch] + RS[DK + ch];
-                static_cast<bf16 *>(a.dq)[o] = __float2bfloat16_rn(dq);
-                static_cast<bf16 *>(a.dk)[o] = __float2bfloat16_rn(dkx + dg * bb);
-                static_cast<bf16 *>(a.db)[o] = __float2bfloat16_rn(dg * kk);
-                DLAM[r * DK + ch] = dL;
-                part += dL;
             }
-            s_dpart[seg][ch] = part;
+            s_dpart[s2][c2] = pa;
+            s_dpart[s2][c2 + 1] = pb;
             __syncthreads();
-            float acc = 0.f;
+            float acca = 0.f, accb = 0.f;
 #pragma unroll
-            for (int s = 0; s < P; ++s)
-                if (s > seg) acc += s_dpart[s][ch];
-            for (int r = min(Cn, (seg + 1) * RSEG) - 1; r >= seg * RSEG; --r) {
-                acc += DLAM[r * DK + ch];
-                static_cast<bf16 *>(a.dlog_alpha)[(((size_t)b * T + n * C + r) * H + h) * DK + ch] =
-                    __float2bfloat16_rn(acc);
+            for (int s = 0; s < P2; ++s)
+                if (s > s2) { acca += s_dpart[s][c2]; accb += s_dpart[s][c2 + 1]; }
+#pragma unroll 4
+            for (int r = (s2 + 1) * RS2 - 1; r >= s2 * RS2; --r) {
+                if (r < Cn) {
+                    const float2 d = *reinterpret_cast<const float2 *>(DLAM + r * DK + c2);
+                    acca += d.x;
+                    accb += d.y;
+                    *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dlog_alpha) +
+                                                  (((size_t)b * T + n * C + r) * H + h) * DK + c2) =
+                        pack_bf16(acca, accb);
+                }
             }
         }
         __syncthreads();

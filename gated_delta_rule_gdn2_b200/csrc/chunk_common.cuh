@@ -161,6 +161,20 @@ __device__ __forceinline__ void load_token_tile(bf16 *dst, const bf16 *src, int 
     }
 }
 
+// L2 prefetch (no shared-memory destination) of rows [n*C, n*C + C) of a
+// token tensor [B,T,H,D], one bulk request per row; thread `slot` of `nslots`.
+template <int D>
+__device__ __forceinline__ void prefetch_token_rows_l2(const bf16 *src, int b, int h, int n, int T, int H, int slot,
+                                                       int nslots) {
+    for (int r = slot; r < C; r += nslots) {
+        const int t = n * C + r;
+        if (t < T) {
+            const bf16 *g = src + (((size_t)b * T + t) * H + h) * D;
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(g), "r"(D * 2) : "memory");
+        }
+    }
+}
+
 struct ChunkTiles {
     bf16 *q, *k, *la, *b, *v, *w;
 };
@@ -168,10 +182,44 @@ struct ChunkTiles {
 // Shared-memory scratch of the intra-chunk stage (static, per CTA).
 template <int DK>
 struct IntraShared {
-    float part[NTHR / DK][DK];
+    float part[NTHR / (DK / 2)][DK];  // segment sums of log_alpha (channel-pair layout)
     float gamma[DK];
     int slow;
 };
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma1688_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// One 16x16 block product on the tensor cores in TF32, operands read from
+// row-major fp32 [.][64] arrays: acc += X[r0.., k0..k0+16) * Y[k0.., c0..c0+16).
+__device__ __forceinline__ void block16_tf32(float (&acc)[2][4], const float *X, int r0, int k0, const float *Y,
+                                             int c0, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < 16; kk += 8) {
+        uint32_t a[4];
+        a[0] = to_tf32(X[(r0 + g) * C + k0 + kk + t]);
+        a[1] = to_tf32(X[(r0 + g + 8) * C + k0 + kk + t]);
+        a[2] = to_tf32(X[(r0 + g) * C + k0 + kk + t + 4]);
+        a[3] = to_tf32(X[(r0 + g + 8) * C + k0 + kk + t + 4]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t b0 = to_tf32(Y[(k0 + kk + t) * C + c0 + 8 * nt + g]);
+            const uint32_t b1 = to_tf32(Y[(k0 + kk + t + 4) * C + c0 + 8 * nt + g]);
+            mma1688_tf32(acc[nt], a, b0, b1);
+        }
+    }
+}
 
 // Intra-chunk stage.  On entry the six raw token tiles of the chunk are in
 // shared memory (and visible to all threads).  On exit (all threads, after a
@@ -185,19 +233,24 @@ struct IntraShared {
 template <int DK, int DV>
 __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<DK> &sh, float *lam_ws,
                             bool keep_lam) {
-    constexpr int P = NTHR / DK;
-    constexpr int RSEG = C / P;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     bf16 *T16 = reinterpret_cast<bf16 *>(T32);
     bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
 
     if (tid == 0) sh.slow = 0;
-    // ---- pass 1: per-channel segment sums of log_alpha, and w . v in place of v
-    const int ch = tid % DK, seg = tid / DK;
+    // ---- pass 1: segment sums of log_alpha per channel pair, and w . v in place of v
+    constexpr int NP = DK / 2, P2 = NTHR / NP, RS2 = C / P2;
+    const int cp = tid % NP, s2 = tid / NP, c2 = 2 * cp;
     {
-        float part = 0.f;
-        for (int r = seg * RSEG; r < (seg + 1) * RSEG; ++r) part += __bfloat162float(st.la[swz<DK>(r, ch)]);
-        sh.part[seg][ch] = part;
+        float pa = 0.f, pb = 0.f;
+#pragma unroll 4
+        for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r) {
+            const float2 l = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.la + swz<DK>(r, c2)));
+            pa += l.x;
+            pb += l.y;
+        }
+        sh.part[s2][c2] = pa;
+        sh.part[s2][c2 + 1] = pb;
         for (int id = tid; id < C * DV / 8; id += NTHR) {
             uint4 wv = reinterpret_cast<const uint4 *>(st.w)[id];
             uint4 vv = reinterpret_cast<const uint4 *>(st.v)[id];
@@ -213,33 +266,40 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
         }
     }
     __syncthreads();
-    float lam0 = 0.f, lam_end = 0.f;
+    float la0 = 0.f, lb0 = 0.f, la_end = 0.f, lb_end = 0.f;
 #pragma unroll
-    for (int s = 0; s < P; ++s) {
-        const float p = sh.part[s][ch];
-        if (s < seg) lam0 += p;
-        lam_end += p;
+    for (int s = 0; s < P2; ++s) {
+        const float pa = sh.part[s][c2], pb = sh.part[s][c2 + 1];
+        if (s < s2) { la0 += pa; lb0 += pb; }
+        la_end += pa;
+        lb_end += pb;
     }
-    if (seg == 0) {
-        sh.gamma[ch] = __expf(lam_end);
-        if (-lam_end > kSpanGuard) sh.slow = 1;
+    if (s2 == 0) {
+        sh.gamma[c2] = __expf(la_end);
+        sh.gamma[c2 + 1] = __expf(lb_end);
+        if (-la_end > kSpanGuard || -lb_end > kSpanGuard) sh.slow = 1;
     }
     __syncthreads();
     const bool slow = sh.slow != 0;
 
     float accM[1][8][4];  // M rows of warps 4..7 (lower incl. diagonal)
     if (!slow) {
-        // ---- pass 2 (fast): Qt, Gt, Kb in place of q, b, log_alpha
-        float lam = lam0;
-        for (int r = seg * RSEG; r < (seg + 1) * RSEG; ++r) {
-            const int o = swz<DK>(r, ch);
-            lam += __bfloat162float(st.la[o]);
-            if (keep_lam) lam_ws[r * DK + ch] = lam;
-            const float e = __expf(lam), ie = __expf(-lam);
-            const float kk = __bfloat162float(st.k[o]);
-            st.q[o] = __float2bfloat16_rn(__bfloat162float(st.q[o]) * e);
-            st.b[o] = __float2bfloat16_rn(__bfloat162float(st.b[o]) * kk * e);
-            st.la[o] = __float2bfloat16_rn(kk * ie);
+        // ---- pass 2 (fast): Qt, Gt, Kb in place of q, b, log_alpha (two channels per thread)
+        float la = la0, lb = lb0;
+#pragma unroll 4
+        for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r) {
+            const int o = swz<DK>(r, c2);
+            const float2 l = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.la + o));
+            const float2 q2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.q + o));
+            const float2 k2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.k + o));
+            const float2 b2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.b + o));
+            la += l.x;
+            lb += l.y;
+            if (keep_lam) *reinterpret_cast<float2 *>(lam_ws + r * DK + c2) = make_float2(la, lb);
+            const float ea = __expf(la), eb = __expf(lb), iea = __expf(-la), ieb = __expf(-lb);
+            *reinterpret_cast<uint32_t *>(st.q + o) = pack_bf16(q2.x * ea, q2.y * eb);
+            *reinterpret_cast<uint32_t *>(st.b + o) = pack_bf16(b2.x * k2.x * ea, b2.y * k2.y * eb);
+            *reinterpret_cast<uint32_t *>(st.la + o) = pack_bf16(k2.x * iea, k2.y * ieb);
         }
         __syncthreads();
         // ---- Grams: [Gt; Qt] Kb^T, warp w -> rows 16w..16w+15 of the stacked operand
@@ -258,11 +318,14 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
             }
     } else {
         // ---- slow chunk: exact per-term decays.  L goes to the per-CTA
-        // workspace; raw q, k, b stay in shared memory until A and M exist.
-        float lam = lam0;
-        for (int r = seg * RSEG; r < (seg + 1) * RSEG; ++r) {
-            lam += __bfloat162float(st.la[swz<DK>(r, ch)]);
-            lam_ws[r * DK + ch] = lam;
+        // workspace (one thread per key channel); raw q, k, b stay in shared
+        // memory until A and M exist.
+        if (tid < DK) {
+            float lam = 0.f;
+            for (int r = 0; r < C; ++r) {
+                lam += __bfloat162float(st.la[swz<DK>(r, tid)]);
+                lam_ws[r * DK + tid] = lam;
+            }
         }
         __syncthreads();
         float pa[9], pm[9];
@@ -287,14 +350,17 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
         }
         __syncthreads();
         // Qt, Gt and Kt = k e^{L_end - L} in place of q, b, log_alpha
-        for (int r = seg * RSEG; r < (seg + 1) * RSEG; ++r) {
-            const int o = swz<DK>(r, ch);
-            const float lr = lam_ws[r * DK + ch];
-            const float e = __expf(lr);
-            const float kk = __bfloat162float(st.k[o]);
-            st.q[o] = __float2bfloat16_rn(__bfloat162float(st.q[o]) * e);
-            st.b[o] = __float2bfloat16_rn(__bfloat162float(st.b[o]) * kk * e);
-            st.la[o] = __float2bfloat16_rn(kk * __expf(lam_end - lr));
+        if (tid < DK) {
+            const float lend = lam_ws[(C - 1) * DK + tid];
+            for (int r = 0; r < C; ++r) {
+                const int o = swz<DK>(r, tid);
+                const float lr = lam_ws[r * DK + tid];
+                const float e = __expf(lr);
+                const float kk = __bfloat162float(st.k[o]);
+                st.q[o] = __float2bfloat16_rn(__bfloat162float(st.q[o]) * e);
+                st.b[o] = __float2bfloat16_rn(__bfloat162float(st.b[o]) * kk * e);
+                st.la[o] = __float2bfloat16_rn(kk * __expf(lend - lr));
+            }
         }
         __syncthreads();
         for (int e = tid; e < C * C; e += NTHR) {
@@ -326,8 +392,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
     }
     __syncthreads();
 
-    // ---- T = (I + A)^{-1}: 16x16 diagonal blocks by substitution, then
-    // off-diagonal blocks level by level: T_RQ = -T_RR sum_J A_RJ T_JQ.
+    // ---- T = (I + A)^{-1}: 16x16 diagonal blocks by substitution in fp32.
     if (tid < 64) {
         const int R = tid >> 4, j = tid & 15;
         float x[16];
@@ -352,52 +417,33 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
         }
     }
     __syncthreads();
+    // Off-diagonal blocks, one warp per block and level, on the tensor cores
+    // in TF32 (T is rounded to bf16 afterwards): X = sum_J A_RJ T_JQ, then
+    // T_RQ = -T_RR X.  Blocks of one level are independent.
 #pragma unroll 1
     for (int lvl = 1; lvl < 4; ++lvl) {
-        const int nb = 4 - lvl;
-        float xv[3];
+        if (warp < 4 - lvl) {
+            const int Q = warp, R = Q + lvl;
+            const int g = lane >> 2, t = lane & 3;
+            float x[2][4] = {};
+            for (int J = Q; J < R; ++J) block16_tf32(x, A32, 16 * R, 16 * J, T32, 16 * Q, lane);
 #pragma unroll
-        for (int s = 0; s < 3; ++s) {
-            const int e = tid + 256 * s;
-            xv[s] = 0.f;
-            if (s < nb) {
-                const int Q = e >> 8, R = Q + lvl, r = (e >> 4) & 15, c = e & 15;
-                float acc = 0.f;
-                for (int J = Q; J < R; ++J)
+            for (int nt = 0; nt < 2; ++nt) {
+                const int c = 16 * Q + 8 * nt + 2 * t;
+                *reinterpret_cast<float2 *>(T32 + (16 * R + g) * C + c) = make_float2(x[nt][0], x[nt][1]);
+                *reinterpret_cast<float2 *>(T32 + (16 * R + g + 8) * C + c) = make_float2(x[nt][2], x[nt][3]);
+            }
+            __syncwarp();
+            float y[2][4] = {};
+            block16_tf32(y, T32, 16 * R, 16 * R, T32, 16 * Q, lane);
+            __syncwarp();
 #pragma unroll
-                    for (int m = 0; m < 16; ++m)
-                        acc += A32[(16 * R + r) * C + 16 * J + m] * T32[(16 * J + m) * C + 16 * Q + c];
-                xv[s] = acc;
+            for (int nt = 0; nt < 2; ++nt) {
+                const int c = 16 * Q + 8 * nt + 2 * t;
+                *reinterpret_cast<float2 *>(T32 + (16 * R + g) * C + c) = make_float2(-y[nt][0], -y[nt][1]);
+                *reinterpret_cast<float2 *>(T32 + (16 * R + g + 8) * C + c) = make_float2(-y[nt][2], -y[nt][3]);
             }
         }
-#pragma unroll
-        for (int s = 0; s < 3; ++s)
-            if (s < nb) {
-                const int e = tid + 256 * s;
-                const int Q = e >> 8, R = Q + lvl, r = (e >> 4) & 15, c = e & 15;
-                T32[(16 * R + r) * C + 16 * Q + c] = xv[s];
-            }
-        __syncthreads();
-#pragma unroll
-        for (int s = 0; s < 3; ++s) {
-            if (s < nb) {
-                const int e = tid + 256 * s;
-                const int Q = e >> 8, R = Q + lvl, r = (e >> 4) & 15, c = e & 15;
-                float acc = 0.f;
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    if (m <= r) acc += T32[(16 * R + r) * C + 16 * R + m] * T32[(16 * R + m) * C + 16 * Q + c];
-                xv[s] = -acc;
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int s = 0; s < 3; ++s)
-            if (s < nb) {
-                const int e = tid + 256 * s;
-                const int Q = e >> 8, R = Q + lvl, r = (e >> 4) & 15, c = e & 15;
-                T32[(16 * R + r) * C + 16 * Q + c] = xv[s];
-            }
         __syncthreads();
     }
     // T32 -> T16, M -> M16 (both bf16, swizzled [64][64])
