@@ -118,7 +118,7 @@ int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return GDN2_ERR_WORKSPACE;
     if (dtype == GDN2_BF16) {
         ChunkFwdArgs a{q, k, v, log_alpha, b, w, S0, o, S_T, static_cast<float *>(ws),
-                       (size_t)64 * dk, nullptr, B, T, H};
+                       (size_t)64 * dk, nullptr, status_ptr(), B, T, H};
         return launch_status(launch_chunk_fwd(a, dk, dv, stream));
     }
     // fp32 precision mode: the recurrence token by token in fp32
@@ -167,7 +167,8 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
         size_t stride = 0, sbytes = 0;
         chunk_bwd_ws_bytes(B, T, H, dk, dv, &stride, &sbytes);
         ChunkBwdArgs a{q, k, v, log_alpha, b, w, S0, dO, dS_T, dq, dk_, dv_, dlog_alpha, db, dw, dS0, ws,
-                       reinterpret_cast<float *>(static_cast<char *>(ws) + sbytes), stride, B, T, H};
+                       reinterpret_cast<float *>(static_cast<char *>(ws) + sbytes), stride, status_ptr(), B, T,
+                       H};
         return launch_status(launch_chunk_bwd(a, dk, dv, stream));
     }
     // fp32 precision mode: reverse-time recurrence token by token in fp32

@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
             const bf16 *src = states + (size_t)n * DK * DV;
             for (int id = tid; id < DK * DV / 8; id += NTHR) {
                 const int r = id / (DV / 8), ch = id % (DV / 8);
-                cp_async16(S16 + swz<DV>(r, ch * 8), src + (size_t)r * DV + ch * 8, true);
+                cp_async16(S16 + swz<DV, DK>(r, ch * 8), src + (size_t)r * DV + ch * 8, true);
             }
         }
         cp_commit();
@@ -173,9 +173,9 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
 #pragma unroll
                 for (int nt = 0; nt < NTS; ++nt) {
                     const int j = j0 + 8 * nt + 2 * (lane & 3);
-                    *reinterpret_cast<uint32_t *>(D16 + swz<DV>(c, j)) =
+                    *reinterpret_cast<uint32_t *>(D16 + swz<DV, DK>(c, j)) =
                         pack_bf16(g0 * dS[mt][nt][0], g0 * dS[mt][nt][1]);
-                    *reinterpret_cast<uint32_t *>(D16 + swz<DV>(c + 8, j)) =
+                    *reinterpret_cast<uint32_t *>(D16 + swz<DV, DK>(c + 8, j)) =
                         pack_bf16(g1 * dS[mt][nt][2], g1 * dS[mt][nt][3]);
                     const __nv_bfloat162 s0 = *reinterpret_cast<const __nv_bfloat162 *>(Snext + (size_t)c * DV + j);
                     const __nv_bfloat162 s1 =
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
         __syncthreads();
         // ---- U = Uv - W S (warps 0..3) into the w slot
         if (warp < 4) {
-            warp_gemm<1, NTV, true, false, DK, DV>(accV, W16, 16 * warp, S16, 0, DK, lane);
+            warp_gemm<1, NTV, true, false, DK, DV, C, DK>(accV, W16, 16 * warp, S16, 0, DK, lane);
             store_tile_bf16<NTV, DV>(accV, U16, 16 * warp, lane, 1.f);
         }
         __syncthreads();
@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
         if (warp < 4) {
             zero(accX);
             warp_gemm<1, NTV, false, false, 64, DV>(accV, M16, 16 * warp, dO16, 0, C, lane);
-            warp_gemm<1, NTV, true, false, DK, DV>(accV, st.la, 16 * warp, D16, 0, DK, lane);
+            warp_gemm<1, NTV, true, false, DK, DV, C, DK>(accV, st.la, 16 * warp, D16, 0, DK, lane);
             store_tile_bf16<NTV, DV>(accV, dU16, 16 * warp, lane, 1.f);
         } else {
             float acc[1][8][4];
@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
             }
         } else {
             zero(accX);
-            warp_gemm<1, NTK, true, true, DV, DV>(accK, U16, 16 * (warp & 3), D16, 0, DV, lane);
+            warp_gemm<1, NTK, true, true, DV, DV, C, DK>(accK, U16, 16 * (warp & 3), D16, 0, DV, lane);
             store_tile_f32<NTK>(accK, DKB, DK, 16 * (warp & 3), lane);
         }
         __syncthreads();
@@ -286,14 +286,14 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
             store_tile_bf16<8, 64>(acc, dA16, 16 * warp, lane, 1.f);
         } else {
             zero(accX);
-            warp_gemm<1, NTK, true, true, DV, DV>(accK, dO16, 16 * (warp & 3), S16, 0, DV, lane);
+            warp_gemm<1, NTK, true, true, DV, DV, C, DK>(accK, dO16, 16 * (warp & 3), S16, 0, DV, lane);
         }
         __syncthreads();
 
         // ---- dGt = nR S^T + dA Kb (warps 0..3) ; dQt += dM Kb, dKb += dA^T Gt + dM^T Qt (warps 4..7)
         if (warp < 4) {
             zero(accX);
-            warp_gemm<1, NTK, true, true, DV, DV>(accK, nR16, 16 * warp, S16, 0, DV, lane);
+            warp_gemm<1, NTK, true, true, DV, DV, C, DK>(accK, nR16, 16 * warp, S16, 0, DV, lane);
             if (!slow) warp_gemm<1, NTK, true, false, 64, DK>(accK, dA16, 16 * warp, st.la, 0, C, lane);
             store_tile_f32<NTK>(accK, DGT, DK, 16 * warp, lane);
         } else {
@@ -462,7 +462,7 @@ template <int DK, int DV>
 cudaError_t launch_t(const ChunkBwdArgs &a, cudaStream_t s) {
     // (1) state pass: the forward with bf16 chunk-boundary states, no output
     ChunkFwdArgs f{a.q, a.k, a.v, a.log_alpha, a.b, a.w, a.S0, nullptr, nullptr, a.scratch, a.scr_stride,
-                   a.states, a.B, a.T, a.H};
+                   a.states, a.status, a.B, a.T, a.H};
     cudaError_t e = launch_chunk_fwd(f, DK, DV, s);
     if (e != cudaSuccess) return e;
     // (2) reverse chunk pass

@@ -26,11 +26,16 @@ constexpr int C = 64;
 constexpr int NTHR = 256;
 constexpr float kSpanGuard = 64.f;  // max in-chunk log-decay span of the fast path
 
-// [rows][D] bf16 tiles: the 16-byte chunk index of a row is XORed with
-// (row & 7) so that ldmatrix row addresses fall in distinct banks.
-template <int D>
+// Shared-memory tiles of R rows x D bf16 columns are stored as D/64 blocks of
+// [R][64] (128-byte rows); within a block the 16-byte chunk index of row r is
+// XORed with (r & 7).  This is the 128-byte-swizzled canonical layout of the
+// tensor-core operand descriptors (8-row x 128-byte atoms, K-major when rows
+// are the M/N index, MN-major when rows are the K index), and it keeps
+// ldmatrix row addresses in distinct banks.  Tiles start on 1 KB boundaries.
+template <int D, int R = 64>
 __device__ __forceinline__ int swz(int r, int c) {
-    return r * D + ((((c >> 3) ^ (r & 7))) << 3) + (c & 7);
+    static_assert(D == 64 || D == 128, "tile width");
+    return (c >> 6) * (R * 64) + r * 64 + ((((c >> 3) & 7) ^ (r & 7)) << 3) + (c & 7);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -67,9 +72,9 @@ template <int N>
 __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
 // acc[MT][NT][4] += A[m0 + 16 mt + .., k] * B[k, n0 + 8 nt + ..], k in [0, K).
-// A_KM: A stored [m][k] in a [.][DA] tile, else stored [k][m].
-// B_KM: B stored [n][k] in a [.][DB] tile, else stored [k][n].
-template <int MT, int NT, bool A_KM, bool B_KM, int DA, int DB>
+// A_KM: A stored [m][k] in a [RA][DA] tile, else stored [k][m].
+// B_KM: B stored [n][k] in a [RB][DB] tile, else stored [k][n].
+template <int MT, int NT, bool A_KM, bool B_KM, int DA, int DB, int RA = C, int RB = C>
 __device__ __forceinline__ void warp_gemm(float (&acc)[MT][NT][4], const bf16 *A, int m0, const bf16 *B,
                                           int n0, int K, int lane) {
     static_assert(NT % 2 == 0, "n tiles come in pairs");
@@ -80,12 +85,12 @@ __device__ __forceinline__ void warp_gemm(float (&acc)[MT][NT][4], const bf16 *A
             if (A_KM) {
                 const int r = m0 + 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
                 const int c = k0 + (lane >> 4) * 8;
-                ldsm4(smem_u32(A + swz<DA>(r, c)), a[mt]);
+                ldsm4(smem_u32(A + swz<DA, RA>(r, c)), a[mt]);
             } else {
                 const int i = lane >> 3;
                 const int kr = k0 + (lane & 7) + (i >> 1) * 8;
                 const int mc = m0 + 16 * mt + (i & 1) * 8;
-                ldsm4t(smem_u32(A + swz<DA>(kr, mc)), a[mt]);
+                ldsm4t(smem_u32(A + swz<DA, RA>(kr, mc)), a[mt]);
             }
         }
 #pragma unroll
@@ -94,11 +99,11 @@ __device__ __forceinline__ void warp_gemm(float (&acc)[MT][NT][4], const bf16 *A
             if (B_KM) {
                 const int r = n0 + 16 * np + (lane & 7) + (lane >> 4) * 8;
                 const int c = k0 + ((lane >> 3) & 1) * 8;
-                ldsm4(smem_u32(B + swz<DB>(r, c)), b);
+                ldsm4(smem_u32(B + swz<DB, RB>(r, c)), b);
             } else {
                 const int kr = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
                 const int nc = n0 + 16 * np + (lane >> 4) * 8;
-                ldsm4t(smem_u32(B + swz<DB>(kr, nc)), b);
+                ldsm4t(smem_u32(B + swz<DB, RB>(kr, nc)), b);
             }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {

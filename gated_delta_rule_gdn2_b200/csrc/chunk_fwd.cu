@@ -123,8 +123,8 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
                 const int j = j0 + 8 * nt + 2 * (lane & 3);
                 const uint32_t lo = pack_bf16(S[mt][nt][0], S[mt][nt][1]);
                 const uint32_t hi = pack_bf16(S[mt][nt][2], S[mt][nt][3]);
-                *reinterpret_cast<uint32_t *>(S16 + swz<DV>(c, j)) = lo;
-                *reinterpret_cast<uint32_t *>(S16 + swz<DV>(c + 8, j)) = hi;
+                *reinterpret_cast<uint32_t *>(S16 + swz<DV, DK>(c, j)) = lo;
+                *reinterpret_cast<uint32_t *>(S16 + swz<DV, DK>(c + 8, j)) = hi;
                 if (gs) {
                     *reinterpret_cast<uint32_t *>(gs + (size_t)c * DV + j) = lo;
                     *reinterpret_cast<uint32_t *>(gs + (size_t)(c + 8) * DV + j) = hi;
@@ -172,10 +172,10 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
 
         // ---- U = Uv - W S (warps 0..3) ; O = Qt S (warps 4..7)
         if (warp < 4) {
-            warp_gemm<1, NTV, true, false, DK, DV>(accV, W16, 16 * warp, S16, 0, DK, lane);
+            warp_gemm<1, NTV, true, false, DK, DV, C, DK>(accV, W16, 16 * warp, S16, 0, DK, lane);
             store_tile_bf16<NTV, DV>(accV, U16, 16 * warp, lane, 1.f);
         } else if (with_o) {
-            warp_gemm<1, NTV, true, false, DK, DV>(accV, st.q, 16 * (warp & 3), S16, 0, DK, lane);
+            warp_gemm<1, NTV, true, false, DK, DV, C, DK>(accV, st.q, 16 * (warp & 3), S16, 0, DK, lane);
         }
         __syncthreads();
 
@@ -253,7 +253,7 @@ cudaError_t launch_t(const ChunkFwdArgs &a, cudaStream_t s) {
 }  // namespace cfwd
 
 cudaError_t launch_chunk_fwd(const ChunkFwdArgs &a, int dk, int dv, cudaStream_t s) {
-    if (dk == 128 && dv == 128) return cfwd::launch_t<128, 128>(a, s);
+    if (dk == 128 && dv == 128) return launch_chunk_fwd_tc(a, s);
     if (dk == 128 && dv == 64) return cfwd::launch_t<128, 64>(a, s);
     if (dk == 64 && dv == 128) return cfwd::launch_t<64, 128>(a, s);
     return cfwd::launch_t<64, 64>(a, s);

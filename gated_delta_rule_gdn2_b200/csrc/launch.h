@@ -39,10 +39,12 @@ struct ChunkFwdArgs {
     float *ws;
     size_t ws_stride;
     void *states;
+    int *status;  // device status word (bounded waits record GDN2_ERR_TIMEOUT here)
     int B, T, H;
 };
 
 cudaError_t launch_chunk_fwd(const ChunkFwdArgs &a, int dk, int dv, cudaStream_t s);
+cudaError_t launch_chunk_fwd_tc(const ChunkFwdArgs &a, cudaStream_t s);  // dk = dv = 128, tcgen05
 size_t chunk_fwd_ws_bytes(int B, int H, int dk);
 
 // Chunk-parallel gate-aware backward (bf16 tokens): a state pass (the
@@ -58,6 +60,7 @@ struct ChunkBwdArgs {
     void *states;
     float *scratch;
     size_t scr_stride;
+    int *status;
     int B, T, H;
 };
 
