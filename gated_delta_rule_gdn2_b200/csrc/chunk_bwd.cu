@@ -17,7 +17,7 @@
 //
 //   dU   = M^T dO + Kb Dh                    dM = strict_lower(dO U^T), diag(dO U^T)
 //   nR   = -T^T dU      (= -dRHS)            dA = strict_lower(nR U^T)
-//   dv   = -nR . w,  dw = -nR . v            dKb = U Dh^T + dA^T Gt + dM^T Qt
+//   dv   = -nR . w,  dw = -nR . v (bf16 nR)  dKb = U Dh^T + dA^T Gt + dM^T Qt
 //   dQt  = dO S^T + dM Kb                    dGt = nR S^T + dA Kb
 //   dS   = Dh + Qt^T dO + Gt^T nR            (-> dSigma of the previous chunk)
 //   dq = dQt e^{L} + dMd k,  dg = dGt e^{L},  dk = dKb e^{-L} + dMd q + dg . b,
@@ -240,29 +240,11 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
         }
         __syncthreads();
 
-        // ---- nR = -T^T dU, dv, dw (warps 0..3) ; dKb(state) = U Dh^T (warps 4..7)
+        // ---- nR = -T^T dU (warps 0..3) ; dKb(state) = U Dh^T (warps 4..7)
         if (warp < 4) {
             zero(accX);
             warp_gemm<1, NTV, false, false, 64, DV>(accV, T16, 16 * warp, dU16, 0, C, lane);
             store_tile_bf16<NTV, DV>(accV, nR16, 16 * warp, lane, -1.f);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int r = 16 * warp + (lane >> 2) + 8 * half;
-                if (r < Cn) {
-                    const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV;
-#pragma unroll
-                    for (int nt = 0; nt < NTV; ++nt) {
-                        const int j = 8 * nt + 2 * (lane & 3);
-                        const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162 *>(gv + o + j);
-                        const __nv_bfloat162 w2 = *reinterpret_cast<const __nv_bfloat162 *>(gw + o + j);
-                        const float d0 = accV[0][nt][2 * half], d1 = accV[0][nt][2 * half + 1];
-                        *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dv) + o + j) =
-                            pack_bf16(d0 * __low2float(w2), d1 * __high2float(w2));
-                        *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dw) + o + j) =
-                            pack_bf16(d0 * __low2float(v2), d1 * __high2float(v2));
-                    }
-                }
-            }
         } else {
             zero(accX);
             warp_gemm<1, NTK, true, true, DV, DV, C, DK>(accK, U16, 16 * (warp & 3), D16, 0, DV, lane);
@@ -375,10 +357,35 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
             const float2 lend = *reinterpret_cast<const float2 *>(LAM + (Cn - 1) * DK + c2);
             const float2 rs0 = *reinterpret_cast<const float2 *>(RS + c2);
             const float2 rs1 = *reinterpret_cast<const float2 *>(RS + DK + c2);
-            float pa = 0.f, pb = 0.f;
-#pragma unroll 4
-            for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r) {
+            // dv = dRHS . w, dw = dRHS . v from the bf16 -dRHS tile, 16-byte coalesced
+            for (int id = tid; id < C * DV / 8; id += NTHR) {
+                const int r = id / (DV / 8), j = (id % (DV / 8)) * 8;
                 if (r < Cn) {
+                    const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV + j;
+                    const uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, j));
+                    const uint4 v8 = *reinterpret_cast<const uint4 *>(gv + o);
+                    const uint4 w8 = *reinterpret_cast<const uint4 *>(gw + o);
+                    const __nv_bfloat162 *n2 = reinterpret_cast<const __nv_bfloat162 *>(&nr);
+                    const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&v8);
+                    const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w8);
+                    uint4 dv8, dw8;
+                    uint32_t *dvp = reinterpret_cast<uint32_t *>(&dv8), *dwp = reinterpret_cast<uint32_t *>(&dw8);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 d = __bfloat1622float2(n2[e]), vv = __bfloat1622float2(v2[e]),
+                                     ww = __bfloat1622float2(w2[e]);
+                        dvp[e] = pack_bf16(-d.x * ww.x, -d.y * ww.y);
+                        dwp[e] = pack_bf16(-d.x * vv.x, -d.y * vv.y);
+                    }
+                    *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dv) + o) = dv8;
+                    *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dw) + o) = dw8;
+                }
+            }
+            float pa = 0.f, pb = 0.f;
+            const int rlo = s2 * RS2, rhi = min(Cn, (s2 + 1) * RS2);
+#pragma unroll 4
+            for (int r = rlo; r < rhi; ++r) {
+                {
                     const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c2;
                     const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(gq + o));
                     const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(gk + o));

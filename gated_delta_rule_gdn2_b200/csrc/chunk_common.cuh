@@ -399,18 +399,17 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
 
     // ---- T = (I + A)^{-1}: 16x16 diagonal blocks by substitution in fp32.
     if (tid < 64) {
+        // column j of the inverse of unit lower-triangular block R, column by
+        // column: once x_r is final, every later row takes its update at once
         const int R = tid >> 4, j = tid & 15;
+        const float *Ablk = A32 + (16 * R) * C + 16 * R;
         float x[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float v = (r == j) ? 1.f : 0.f;
-            if (r > j) {
+        for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-                for (int i = 0; i < r; ++i)
-                    if (i >= j) v -= A32[(16 * R + r) * C + 16 * R + i] * x[i];
-            }
-            x[r] = v;
-        }
+        for (int r = 0; r < 15; ++r)
+#pragma unroll
+            for (int s2 = r + 1; s2 < 16; ++s2) x[s2] -= Ablk[s2 * C + r] * x[r];
 #pragma unroll
         for (int r = 0; r < 16; ++r) T32[(16 * R + r) * C + 16 * R + j] = x[r];
     } else {

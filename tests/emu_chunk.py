@@ -140,8 +140,8 @@ def chunk_bwd_head(q, k, v, la, b, w, S0, dO, dST, bf16=False, opts=()):
         dU = rd(Mb.T @ dOc + Kb @ Dh)
         dRHS = Tm.T @ dU
         nR = rd(-dRHS)
-        g["dv"][n0:n1] = out_rd(dRHS * wc)
-        g["dw"][n0:n1] = out_rd(dRHS * vc)
+        g["dv"][n0:n1] = out_rd(-nR * wc)  # the kernel forms dv, dw from the bf16 -dRHS tile
+        g["dw"][n0:n1] = out_rd(-nR * vc)
         dKb = U @ Dh.T
         dMm = np.tril(dOc @ U.T, 0)
         dAm = np.tril(nR @ U.T, -1)
