@@ -1,11 +1,13 @@
 #!/usr/bin/env python3
 """Benchmark of the GDN-2 mixer hot path on B200.
 
-One step = gdn2_chunk_fwd + gdn2_chunk_bwd over the training batch
-(B=8, T=4096, H=16, dk=dv=128, bf16 tokens, fp32 state, do ~ N(0,1),
-dS_T = 0) -- the 1.3B-layer shape of the pages.  The decode step
-(B=256, H=16, fp32 state of 268 MB updated in place) is timed in the same
-run and reported under "decode".  Inputs are seeded synthetic data of the
+One step = a training forward + backward over the batch (B=8, T=4096, H=16,
+dk=dv=128, bf16 tokens, fp32 state, do ~ N(0,1), dS_T = 0) -- the 1.3B-layer
+shape of the pages: gdn2_chunk_fwd_save (the forward that keeps its
+chunk-boundary states) + gdn2_chunk_bwd_saved (the gate-aware backward using
+them).  The plain forward (prefill, gdn2_chunk_fwd) and the decode step
+(B=256, H=16, fp32 state of 268 MB updated in place) are timed in the same
+run and reported under "prefill" and "decode".  Inputs are seeded synthetic data of the
 pages' distributions (gated_delta_rule_gdn2_b200.inputs); they are larger
 than L2 (about 1 GB per step), so no separate flush is needed.
 
@@ -31,13 +33,14 @@ sys.path.insert(0, ROOT)
 
 B, T, H, D = 8, 4096, 16, 128  # B can be lowered with --batch for profiling captures
 DEC_B, DEC_H = 256, 16
-WORKLOAD = "train fwd+bwd B8 T4096 H16 dk=dv=128 bf16 (prefill shape; decode B256 H16 alongside)"
+WORKLOAD = "train fwd+bwd B8 T4096 H16 dk=dv=128 bf16 (prefill and decode B256 H16 alongside)"
 METRIC = "GDN-2 chunk fwd+bwd tokens/s & TFLOP/s (H16 dk=dv=128); decode state GB/s"
 # algorithmic work per (token, head), d = 128, C = 64: dense-counted products and bytes read + written once
 FLOP_FWD = 6 * D * D + 10 * 64 * D          # 180,224
-FLOP_BWD = 524288                            # state recompute + reverse pass + intra-chunk grads
+FLOP_BWD = 524288 - (4 * D * D + 8 * 64 * D)  # 393,216: backward without the state recompute
 BYTES_FWD = 7 * D * 2                        # q,k,v,log_alpha,b,w in + o out, bf16
 BYTES_BWD = 13 * D * 2                       # 6 inputs + dO in, 6 gradients out, bf16
+BYTES_STATES = D * D * 2 // 64               # bf16 chunk-boundary state per token (written once, read once)
 STATE_BYTES = D * D * 4
 
 
@@ -167,18 +170,24 @@ def run_gpu(args):
     grads = [torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev) for _ in range(6)]
     dS0 = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
     nfw = g.gdn2_chunk_fwd_workspace(B, T, H, D, D, g.GDN2_BF16)
-    nbw = g.gdn2_chunk_bwd_workspace(B, T, H, D, D, g.GDN2_BF16)
+    nbw = g.gdn2_chunk_bwd_saved_workspace(B, T, H, D, D, g.GDN2_BF16)
+    nst = g.gdn2_chunk_states_bytes(B, T, H, D, D, g.GDN2_BF16)
     wsf = torch.empty(max(nfw, 16), dtype=torch.uint8, device=dev)
     wsb = torch.empty(max(nbw, 16), dtype=torch.uint8, device=dev)
+    states = torch.empty(nst, dtype=torch.uint8, device=dev)
     toks = [d[n] for n in ("q", "k", "v", "log_alpha", "b", "w")]
 
     def fwd():
-        st = g.gdn2_chunk_fwd(*toks, d["S0"], o, ST, B, T, H, D, D, g.GDN2_BF16, wsf, nfw, sh)
+        st = g.gdn2_chunk_fwd_save(*toks, d["S0"], o, ST, states, B, T, H, D, D, g.GDN2_BF16, wsf, nfw, sh)
         assert st == 0, st
 
     def bwd():
-        st = g.gdn2_chunk_bwd(*toks, d["S0"], d["dO"], None, *grads, dS0, B, T, H, D, D, g.GDN2_BF16,
-                              wsb, nbw, sh)
+        st = g.gdn2_chunk_bwd_saved(*toks, d["S0"], d["dO"], None, states, *grads, dS0, B, T, H, D, D,
+                                    g.GDN2_BF16, wsb, nbw, sh)
+        assert st == 0, st
+
+    def prefill():
+        st = g.gdn2_chunk_fwd(*toks, d["S0"], o, ST, B, T, H, D, D, g.GDN2_BF16, wsf, nfw, sh)
         assert st == 0, st
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -221,6 +230,18 @@ def run_gpu(args):
         total_ms = float(t.item())
     ms_step = total_ms / args.steps
 
+    # ---- prefill forward (gdn2_chunk_fwd, no states kept)
+    for _ in range(3):
+        prefill()
+    torch.cuda.synchronize()
+    p0, p1 = ev(), ev()
+    p0.record(stream)
+    for _ in range(args.steps):
+        prefill()
+    p1.record(stream)
+    torch.cuda.synchronize()
+    pre_ms = p0.elapsed_time(p1) / args.steps
+
     # ---- decode step, state of B256 H16 d128 resident and updated in place
     from gated_delta_rule_gdn2_b200.inputs import decode_initial_state, decode_step_inputs
     Sdec = torch.from_numpy(decode_initial_state(DEC_B, DEC_H, D, D, seed=1002)).to(dev)
@@ -259,8 +280,9 @@ def run_gpu(args):
     def e2e_step():
         nonlocal outs_host
         dv_ = {n: t.to(dev, non_blocking=True) for n, t in host.items()}
-        oo, SS = g.chunk_fwd(*[dv_[n] for n in ("q", "k", "v", "log_alpha", "b", "w")], S0=dv_["S0"])
-        gg = g.chunk_bwd(*[dv_[n] for n in ("q", "k", "v", "log_alpha", "b", "w")], dv_["S0"], dv_["dO"])
+        tk = [dv_[n] for n in ("q", "k", "v", "log_alpha", "b", "w")]
+        oo, SS, stt = g.chunk_fwd(*tk, S0=dv_["S0"], save_states=True)
+        gg = g.chunk_bwd(*tk, dv_["S0"], dv_["dO"], states=stt)
         res = [oo, SS] + [gg[n] for n in ("dq", "dk", "dv", "dlog_alpha", "db", "dw", "dS0")]
         outs_host = [r.to("cpu", non_blocking=True) for r in res]
         return res
@@ -284,13 +306,13 @@ def run_gpu(args):
     hbm, tf_burst, tf_sus, src = peaks()
     tokens = B * T * world
     th = B * T * H
-    fwd_gbs = (th * BYTES_FWD + 2 * B * H * STATE_BYTES) / (fwd_ms * 1e-3) / 1e9
-    bwd_gbs = (th * BYTES_BWD + 2 * B * H * STATE_BYTES) / (bwd_ms * 1e-3) / 1e9
+    fwd_gbs = (th * (BYTES_FWD + BYTES_STATES) + 2 * B * H * STATE_BYTES) / (fwd_ms * 1e-3) / 1e9
+    bwd_gbs = (th * (BYTES_BWD + BYTES_STATES) + 2 * B * H * STATE_BYTES) / (bwd_ms * 1e-3) / 1e9
+    pre_gbs = (th * BYTES_FWD + 2 * B * H * STATE_BYTES) / (pre_ms * 1e-3) / 1e9
     dom = "bwd" if bwd_ms >= fwd_ms else "fwd"
-    kname = {"fwd": "chunk_fwd_kernel",
-             "bwd": "gdn2_chunk_bwd (state pass chunk_fwd_kernel + chunk_bwd_kernel)"}[dom]
+    kname = {"fwd": "chunk_fwd_tc_kernel (with state output)", "bwd": "chunk_bwd_kernel"}[dom]
     achieved = bwd_gbs if dom == "bwd" else fwd_gbs
-    traffic = kernel_traffic("chunk_fwd_kernel" if dom == "fwd" else "chunk_bwd")
+    traffic = kernel_traffic("chunk_fwd_tc_kernel" if dom == "fwd" else "chunk_bwd_kernel")
     clocks = clk.summary()
     out = {
         "metric": METRIC,
@@ -310,13 +332,16 @@ def run_gpu(args):
                    "l2": "inputs larger than L2 (about 1 GB per step)"},
         "tflops": th * world * (FLOP_FWD + FLOP_BWD) / (ms_step * 1e-3) / 1e12,
         "breakdown": {
-            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
-            "fwd_tokens_per_s": B * T / (fwd_ms * 1e-3),
+            "fwd_save_ms": fwd_ms, "bwd_saved_ms": bwd_ms,
             "fwd_tflops": th * FLOP_FWD / (fwd_ms * 1e-3) / 1e12,
             "fwd_gbs": fwd_gbs, "fwd_hbm_frac": fwd_gbs / hbm,
             "bwd_tflops": th * FLOP_BWD / (bwd_ms * 1e-3) / 1e12,
             "bwd_gbs": bwd_gbs, "bwd_hbm_frac": bwd_gbs / hbm,
         },
+        "prefill": {"workload": "B8 T4096 H16 dk=dv=128 forward (gdn2_chunk_fwd)", "ms": pre_ms,
+                    "tokens_per_s": B * T / (pre_ms * 1e-3), "tflops": th * FLOP_FWD / (pre_ms * 1e-3) / 1e12,
+                    "gbs": pre_gbs, "hbm_frac": pre_gbs / hbm,
+                    "tensor_frac_of_bf16": th * FLOP_FWD / (pre_ms * 1e-3) / 1e12 / tf_burst},
         "decode": {"workload": "B256 H16 dk=dv=128, fp32 state in place", "us_per_step": dec_us,
                    "tokens_per_s": DEC_B / (dec_us * 1e-6), "state_gbs": dec_bytes / (dec_us * 1e-6) / 1e9,
                    "hbm_frac": dec_bytes / (dec_us * 1e-6) / 1e9 / hbm, "peak_gbs": hbm},
@@ -327,7 +352,7 @@ def run_gpu(args):
                                              / ((fwd_ms if dom == "fwd" else bwd_ms) * 1e-3) / 1e12) / tf_sus},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * args.steps,  # chunk_fwd_kernel, then the backward's state pass + reverse kernel
+        "gpu_launches": 2 * args.steps,  # chunk_fwd_tc_kernel (with states) + chunk_bwd_kernel per step
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -33,6 +33,10 @@ SIGNATURES = {
     "gdn2_chunk_bwd_workspace": (_Z, [_I] * 6),
     "gdn2_chunk_bwd": (_I, [_P] * 16 + [_I] * 6 + [_P, _Z, _P]),
     "gdn2_chunk_fwd_noalloc": (_I, [_P] * 9 + [_I] * 6 + [_P]),
+    "gdn2_chunk_states_bytes": (_Z, [_I] * 6),
+    "gdn2_chunk_fwd_save": (_I, [_P] * 10 + [_I] * 6 + [_P, _Z, _P]),
+    "gdn2_chunk_bwd_saved_workspace": (_Z, [_I] * 6),
+    "gdn2_chunk_bwd_saved": (_I, [_P] * 17 + [_I] * 6 + [_P, _Z, _P]),
 }
 
 _lib = None
@@ -118,6 +122,29 @@ def gdn2_chunk_fwd_noalloc(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, dk, dv
                                          _stream(stream))
 
 
+def gdn2_chunk_states_bytes(B, T, H, dk, dv, dtype) -> int:
+    return load().gdn2_chunk_states_bytes(B, T, H, dk, dv, dtype)
+
+
+def gdn2_chunk_bwd_saved_workspace(B, T, H, dk, dv, dtype) -> int:
+    return load().gdn2_chunk_bwd_saved_workspace(B, T, H, dk, dv, dtype)
+
+
+def gdn2_chunk_fwd_save(q, k, v, log_alpha, b, w, S0, o, S_T, states, B, T, H, dk, dv, dtype, ws, ws_bytes,
+                        stream=None) -> int:
+    return load().gdn2_chunk_fwd_save(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                                      _ptr(S0), _ptr(o), _ptr(S_T), _ptr(states), B, T, H, dk, dv, dtype,
+                                      _ptr(ws), ws_bytes, _stream(stream))
+
+
+def gdn2_chunk_bwd_saved(q, k, v, log_alpha, b, w, S0, dO, dS_T, states, dq, dk_, dv_, dlog_alpha, db, dw,
+                         dS0, B, T, H, dk, dv, dtype, ws, ws_bytes, stream=None) -> int:
+    return load().gdn2_chunk_bwd_saved(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                                       _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(states), _ptr(dq), _ptr(dk_),
+                                       _ptr(dv_), _ptr(dlog_alpha), _ptr(db), _ptr(dw), _ptr(dS0), B, T, H,
+                                       dk, dv, dtype, _ptr(ws), ws_bytes, _stream(stream))
+
+
 def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o, B, H, dk, dv, dtype, stream=None) -> int:
     return load().gdn2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
                                    _ptr(S), _ptr(o), B, H, dk, dv, dtype, _stream(stream))
@@ -162,8 +189,11 @@ def _raise(st, what):
         raise Gdn2Error(st, what)
 
 
-def chunk_fwd(q, k, v, log_alpha, b, w, S0=None, output_final_state=True, stream=None):
-    """o, S_T = chunk_fwd(...) for token tensors [B,T,H,D] (bf16 or fp32)."""
+def chunk_fwd(q, k, v, log_alpha, b, w, S0=None, output_final_state=True, save_states=False, stream=None):
+    """o, S_T = chunk_fwd(...) for token tensors [B,T,H,D] (bf16 or fp32).
+
+    With save_states=True returns (o, S_T, states): the chunk-boundary states
+    for chunk_bwd(..., states=states)."""
     import torch
     _check_tokens(q, k, v, log_alpha, b, w, 3)
     B, T, H, dk = q.shape
@@ -173,9 +203,15 @@ def chunk_fwd(q, k, v, log_alpha, b, w, S0=None, output_final_state=True, stream
     S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if output_final_state else None
     nws = gdn2_chunk_fwd_workspace(B, T, H, dk, dv, dt)
     ws = torch.empty(nws, dtype=torch.uint8, device=q.device) if nws else None
-    _raise(gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, dk, dv, dt, ws, nws, stream),
-           "gdn2_chunk_fwd")
-    return o, S_T
+    if not save_states:
+        _raise(gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, dk, dv, dt, ws, nws, stream),
+               "gdn2_chunk_fwd")
+        return o, S_T
+    nst = gdn2_chunk_states_bytes(B, T, H, dk, dv, dt)
+    states = torch.empty(nst, dtype=torch.uint8, device=q.device) if nst else None
+    _raise(gdn2_chunk_fwd_save(q, k, v, log_alpha, b, w, S0, o, S_T, states, B, T, H, dk, dv, dt, ws, nws,
+                               stream), "gdn2_chunk_fwd_save")
+    return o, S_T, states
 
 
 def decode_step(q, k, v, log_alpha, b, w, S, stream=None):
@@ -192,8 +228,10 @@ def decode_step(q, k, v, log_alpha, b, w, S, stream=None):
     return o
 
 
-def chunk_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None, need_dS0=True, stream=None):
-    """Gradients (dq, dk, dv, dlog_alpha, db, dw, dS0) of gdn2_chunk_fwd."""
+def chunk_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None, need_dS0=True, states=None, stream=None):
+    """Gradients (dq, dk, dv, dlog_alpha, db, dw, dS0) of gdn2_chunk_fwd.
+
+    `states` from chunk_fwd(..., save_states=True) skips the state recompute."""
     import torch
     _check_tokens(q, k, v, log_alpha, b, w, 3)
     B, T, H, dk = q.shape
@@ -202,9 +240,16 @@ def chunk_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T=None, need_dS0=True, stream
     g = {n: torch.empty_like(q) for n in ("dq", "dk", "dlog_alpha", "db")}
     g.update({n: torch.empty_like(v) for n in ("dv", "dw")})
     g["dS0"] = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device) if need_dS0 else None
-    nws = gdn2_chunk_bwd_workspace(B, T, H, dk, dv, dt)
+    if states is None:
+        nws = gdn2_chunk_bwd_workspace(B, T, H, dk, dv, dt)
+        ws = torch.empty(nws, dtype=torch.uint8, device=q.device) if nws else None
+        _raise(gdn2_chunk_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T, g["dq"], g["dk"], g["dv"],
+                              g["dlog_alpha"], g["db"], g["dw"], g["dS0"], B, T, H, dk, dv, dt, ws, nws,
+                              stream), "gdn2_chunk_bwd")
+        return g
+    nws = gdn2_chunk_bwd_saved_workspace(B, T, H, dk, dv, dt)
     ws = torch.empty(nws, dtype=torch.uint8, device=q.device) if nws else None
-    _raise(gdn2_chunk_bwd(q, k, v, log_alpha, b, w, S0, dO, dS_T, g["dq"], g["dk"], g["dv"],
-                          g["dlog_alpha"], g["db"], g["dw"], g["dS0"], B, T, H, dk, dv, dt, ws, nws,
-                          stream), "gdn2_chunk_bwd")
+    _raise(gdn2_chunk_bwd_saved(q, k, v, log_alpha, b, w, S0, dO, dS_T, states, g["dq"], g["dk"], g["dv"],
+                                g["dlog_alpha"], g["db"], g["dw"], g["dS0"], B, T, H, dk, dv, dt, ws, nws,
+                                stream), "gdn2_chunk_bwd_saved")
     return g

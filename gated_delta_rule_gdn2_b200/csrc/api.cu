@@ -146,12 +146,16 @@ size_t gdn2_chunk_bwd_workspace(int B, int T, int H, int dk, int dv, int dtype) 
     return recurrent_bwd_ws_bytes(B, T, H, dk, dv);
 }
 
-int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_alpha,
-                   const void *b, const void *w, const float *S0, const void *dO,
-                   const float *dS_T, void *dq, void *dk_, void *dv_, void *dlog_alpha,
-                   void *db, void *dw, float *dS0,
-                   int B, int T, int H, int dk, int dv, int dtype,
-                   void *ws, size_t ws_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of gdn2_chunk_bwd (states == nullptr: recomputed into the
+// workspace) and gdn2_chunk_bwd_saved (states from gdn2_chunk_fwd_save).
+int chunk_bwd_impl(const void *q, const void *k, const void *v, const void *log_alpha, const void *b,
+                   const void *w, const float *S0, const void *dO, const float *dS_T, const void *states,
+                   void *dq, void *dk_, void *dv_, void *dlog_alpha, void *db, void *dw, float *dS0, int B, int T,
+                   int H, int dk, int dv, int dtype, void *ws, size_t ws_bytes, cudaStream_t stream) {
     int st = check_sizes(B, T, H, dk, dv, dtype);
     if (st != GDN2_OK) return st;
     if (!ok_opt(S0) || !ok_opt(dS_T) || !ok_opt(dS0) || !ok_opt(ws)) return GDN2_ERR_INVALID_ARG;
@@ -161,20 +165,84 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
         !ok_ptr(dO) || !ok_ptr(dq) || !ok_ptr(dk_) || !ok_ptr(dv_) || !ok_ptr(dlog_alpha) ||
         !ok_ptr(db) || !ok_ptr(dw))
         return GDN2_ERR_INVALID_ARG;
-    const size_t need = gdn2_chunk_bwd_workspace(B, T, H, dk, dv, dtype);
+    const bool saved = states != nullptr && dtype == GDN2_BF16;
+    if (saved && !aligned16(states)) return GDN2_ERR_INVALID_ARG;
+    const size_t need = saved ? gdn2_chunk_bwd_saved_workspace(B, T, H, dk, dv, dtype)
+                              : gdn2_chunk_bwd_workspace(B, T, H, dk, dv, dtype);
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return GDN2_ERR_WORKSPACE;
     if (dtype == GDN2_BF16) {
         size_t stride = 0, sbytes = 0;
         chunk_bwd_ws_bytes(B, T, H, dk, dv, &stride, &sbytes);
-        ChunkBwdArgs a{q, k, v, log_alpha, b, w, S0, dO, dS_T, dq, dk_, dv_, dlog_alpha, db, dw, dS0, ws,
-                       reinterpret_cast<float *>(static_cast<char *>(ws) + sbytes), stride, status_ptr(), B, T,
-                       H};
+        void *st_buf = saved ? const_cast<void *>(states) : ws;
+        float *scr = reinterpret_cast<float *>(static_cast<char *>(ws) + (saved ? 0 : sbytes));
+        ChunkBwdArgs a{q, k, v, log_alpha, b, w, S0, dO, dS_T, dq, dk_, dv_, dlog_alpha, db, dw, dS0, st_buf,
+                       scr, stride, status_ptr(), saved ? 1 : 0, B, T, H};
         return launch_status(launch_chunk_bwd(a, dk, dv, stream));
     }
     // fp32 precision mode: reverse-time recurrence token by token in fp32
     RecurrentBwdArgs a{q, k, v, log_alpha, b, w, S0, dO, dS_T, dq, dk_, dv_, dlog_alpha, db, dw,
                        dS0, static_cast<float *>(ws), B, T, H};
     return launch_status(launch_recurrent_bwd(a, dk, dv, false, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_alpha,
+                   const void *b, const void *w, const float *S0, const void *dO,
+                   const float *dS_T, void *dq, void *dk_, void *dv_, void *dlog_alpha,
+                   void *db, void *dw, float *dS0,
+                   int B, int T, int H, int dk, int dv, int dtype,
+                   void *ws, size_t ws_bytes, cudaStream_t stream) {
+    return chunk_bwd_impl(q, k, v, log_alpha, b, w, S0, dO, dS_T, nullptr, dq, dk_, dv_, dlog_alpha, db, dw, dS0,
+                          B, T, H, dk, dv, dtype, ws, ws_bytes, stream);
+}
+
+size_t gdn2_chunk_states_bytes(int B, int T, int H, int dk, int dv, int dtype) {
+    if (check_sizes(B, T, H, dk, dv, dtype) != GDN2_OK) return 0;
+    if (B == 0 || H == 0 || T == 0 || dtype != GDN2_BF16) return 0;
+    size_t sbytes = 0;
+    chunk_bwd_ws_bytes(B, T, H, dk, dv, nullptr, &sbytes);
+    return sbytes;
+}
+
+int gdn2_chunk_fwd_save(const void *q, const void *k, const void *v, const void *log_alpha,
+                        const void *b, const void *w, const float *S0, void *o, float *S_T, void *states,
+                        int B, int T, int H, int dk, int dv, int dtype,
+                        void *ws, size_t ws_bytes, cudaStream_t stream) {
+    int st = check_sizes(B, T, H, dk, dv, dtype);
+    if (st != GDN2_OK) return st;
+    if (dtype != GDN2_BF16 || B == 0 || H == 0 || T == 0)
+        return gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0, o, S_T, B, T, H, dk, dv, dtype, ws, ws_bytes, stream);
+    if (!ok_opt(S0) || !ok_opt(S_T) || !ok_opt(ws) || !ok_ptr(states)) return GDN2_ERR_INVALID_ARG;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) ||
+        !ok_ptr(o))
+        return GDN2_ERR_INVALID_ARG;
+    const size_t need = gdn2_chunk_fwd_workspace(B, T, H, dk, dv, dtype);
+    if (ws_bytes < need || (need > 0 && ws == nullptr)) return GDN2_ERR_WORKSPACE;
+    ChunkFwdArgs a{q, k, v, log_alpha, b, w, S0, o, S_T, static_cast<float *>(ws), (size_t)64 * dk, states,
+                   status_ptr(), B, T, H};
+    return launch_status(launch_chunk_fwd(a, dk, dv, stream));
+}
+
+size_t gdn2_chunk_bwd_saved_workspace(int B, int T, int H, int dk, int dv, int dtype) {
+    if (check_sizes(B, T, H, dk, dv, dtype) != GDN2_OK) return 0;
+    if (B == 0 || H == 0 || T == 0) return 0;
+    if (dtype != GDN2_BF16) return gdn2_chunk_bwd_workspace(B, T, H, dk, dv, dtype);
+    size_t sbytes = 0;
+    return chunk_bwd_ws_bytes(B, T, H, dk, dv, nullptr, &sbytes) - sbytes;
+}
+
+int gdn2_chunk_bwd_saved(const void *q, const void *k, const void *v, const void *log_alpha,
+                         const void *b, const void *w, const float *S0, const void *dO,
+                         const float *dS_T, const void *states, void *dq, void *dk_, void *dv_,
+                         void *dlog_alpha, void *db, void *dw, float *dS0,
+                         int B, int T, int H, int dk, int dv, int dtype,
+                         void *ws, size_t ws_bytes, cudaStream_t stream) {
+    if (dtype == GDN2_BF16 && B > 0 && H > 0 && T > 0 && states == nullptr) return GDN2_ERR_INVALID_ARG;
+    return chunk_bwd_impl(q, k, v, log_alpha, b, w, S0, dO, dS_T, states, dq, dk_, dv_, dlog_alpha, db, dw, dS0,
+                          B, T, H, dk, dv, dtype, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

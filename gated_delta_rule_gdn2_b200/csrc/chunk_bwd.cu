@@ -28,8 +28,9 @@
 // A slow chunk (decay beyond e^{-64} inside the chunk) uses Kt = k e^{L_end-L}
 // with Dh = dSigma, and takes the Gram gradients term by term in fp32.
 //
-// Per-CTA fp32 scratch (L, dQt, dGt, dKb, dL and the slow-path partial
-// gradients) lives in the caller's workspace and stays resident in L2.
+// dQt, dGt and dKb are staged in fp32 in shared-memory regions that are dead by
+// then; the per-CTA fp32 scratch of the caller's workspace (L2-resident) holds
+// the slow-path partial gradients and a few row sums.
 #include "chunk_common.cuh"
 #include "launch.h"
 
@@ -47,7 +48,13 @@ struct BSmem {
     static constexpr int OAT = OD + TS;              // A32 | T32 (2 x 16 KB fp32)
     static constexpr bool AM_IN_K = (DK == 128);     // dM16 | dA16 in the k slot
     static constexpr int OAM = OAT + 32768;
-    static constexpr int BYTES = OAM + (AM_IN_K ? 0 : 16384);
+    // fp32 [64][DK] staging of dQt, dGt, dKb for the elementwise phase:
+    // (128,128) reuses the dead S, Dh and WY-solve regions; dk = 64 gets
+    // dedicated regions; (128,64) stages through the global scratch.
+    static constexpr bool STAGE_REUSE = (DK == 128 && DV == 128);
+    static constexpr bool STAGE_DED = (DK == 64);
+    static constexpr int OSTG = OAM + (AM_IN_K ? 0 : 16384);
+    static constexpr int BYTES = OSTG + (STAGE_DED ? 3 * C * DK * 4 : 0);
 };
 
 template <int DK>
@@ -70,6 +77,8 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ IntraShared<DK> sh;
     __shared__ float s_dpart[NTHR / (DK / 2)][DK];
+    __shared__ float s_dmd[C];      // diagonal of dO U^T
+    __shared__ float s_rs[2][DK];   // row sums of dSigma . Sigma (two column halves)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
@@ -97,7 +106,16 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
     float *LAM = scr + SC::LAM * SC::TILE, *DQT = scr + SC::DQT * SC::TILE, *DGT = scr + SC::DGT * SC::TILE;
     float *DKB = scr + SC::DKB * SC::TILE, *DLAM = scr + SC::DLAM * SC::TILE;
     float *PQ = scr + SC::PQ * SC::TILE, *PG = scr + SC::PG * SC::TILE, *PK = scr + SC::PK * SC::TILE;
-    float *PL = scr + SC::PL * SC::TILE, *RS = scr + SC::RS, *DMD = scr + SC::DMD;
+    float *PL = scr + SC::PL * SC::TILE;
+    if (L::STAGE_REUSE) {
+        DQT = reinterpret_cast<float *>(smem + L::OS);
+        DKB = reinterpret_cast<float *>(smem + L::OD);
+        DGT = reinterpret_cast<float *>(smem + L::OAT);
+    } else if (L::STAGE_DED) {
+        DQT = reinterpret_cast<float *>(smem + L::OSTG);
+        DKB = DQT + C * DK;
+        DGT = DKB + C * DK;
+    }
     const bf16 *states = static_cast<const bf16 *>(a.states) + (size_t)bh * (nchunks + 1) * DK * DV;
     const bf16 *gq = static_cast<const bf16 *>(a.q), *gk = static_cast<const bf16 *>(a.k);
     const bf16 *gb = static_cast<const bf16 *>(a.b), *gv = static_cast<const bf16 *>(a.v);
@@ -159,7 +177,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
             }
         }
 
-        const bool slow = intra_chunk<DK, DV>(st, A32, T32, sh, LAM, true);
+        const bool slow = intra_chunk<DK, DV>(st, A32, T32, sh, LAM, false);
 
         // ---- Dh = gam . dSigma (fast) or dSigma (slow) as bf16; row sums of
         // dSigma . Sigma (Sigma = next chunk-boundary state) for dL_end
@@ -188,8 +206,8 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
                 r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
                 r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
                 if ((lane & 3) == 0) {
-                    RS[(warp & 1) * DK + c] = r0;
-                    RS[(warp & 1) * DK + c + 8] = r1;
+                    s_rs[warp & 1][c] = r0;
+                    s_rs[warp & 1][c + 8] = r1;
                 }
             }
         }
@@ -233,22 +251,18 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
                     // its gradient goes straight to dq and dk in fp32 and is kept
                     // out of the Gram products, where it would cancel in dL.
                     const int r = r0 + (e >> 1) * 8, i = 8 * nt + 2 * (lane & 3) + (e & 1);
-                    if (i == r) DMD[r] = acc[0][nt][e];
+                    if (i == r) s_dmd[r] = acc[0][nt][e];
                     if (i >= r) acc[0][nt][e] = 0.f;
                 }
             store_tile_bf16<8, 64>(acc, dM16, 16 * (warp & 3), lane, 1.f);
         }
         __syncthreads();
 
-        // ---- nR = -T^T dU (warps 0..3) ; dKb(state) = U Dh^T (warps 4..7)
+        // ---- nR = -T^T dU (warps 0..3)
         if (warp < 4) {
             zero(accX);
             warp_gemm<1, NTV, false, false, 64, DV>(accV, T16, 16 * warp, dU16, 0, C, lane);
             store_tile_bf16<NTV, DV>(accV, nR16, 16 * warp, lane, -1.f);
-        } else {
-            zero(accX);
-            warp_gemm<1, NTK, true, true, DV, DV, C, DK>(accK, U16, 16 * (warp & 3), D16, 0, DV, lane);
-            store_tile_f32<NTK>(accK, DKB, DK, 16 * (warp & 3), lane);
         }
         __syncthreads();
 
@@ -272,33 +286,29 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
         }
         __syncthreads();
 
-        // ---- dGt = nR S^T + dA Kb (warps 0..3) ; dQt += dM Kb, dKb += dA^T Gt + dM^T Qt (warps 4..7)
+        // ---- dGt = nR S^T + dA Kb (warps 0..3) ; dQt += dM Kb (warps 4..7)
         if (warp < 4) {
             zero(accX);
             warp_gemm<1, NTK, true, true, DV, DV, C, DK>(accK, nR16, 16 * warp, S16, 0, DV, lane);
             if (!slow) warp_gemm<1, NTK, true, false, 64, DK>(accK, dA16, 16 * warp, st.la, 0, C, lane);
-            store_tile_f32<NTK>(accK, DGT, DK, 16 * warp, lane);
-        } else {
+            store_tile_f32<NTK>(accK, DGT, DK, 16 * warp, lane);  // the WY-solve area is dead
+        } else if (!slow) {
+            warp_gemm<1, NTK, true, false, 64, DK>(accK, dM16, 16 * (warp & 3), st.la, 0, C, lane);
+        }
+        __syncthreads();  // S is no longer read: its region takes dQt
+
+        // ---- dKb = U Dh^T + dA^T Gt + dM^T Qt (warps 4..7), then dSigma (all warps)
+        if (warp >= 4) {
             const int m0 = 16 * (warp & 3);
-            if (!slow) warp_gemm<1, NTK, true, false, 64, DK>(accK, dM16, m0, st.la, 0, C, lane);
             store_tile_f32<NTK>(accK, DQT, DK, m0, lane);
+            zero(accX);
+            warp_gemm<1, NTK, true, true, DV, DV, C, DK>(accK, U16, m0, D16, 0, DV, lane);
             if (!slow) {
-                zero(accX);
                 warp_gemm<1, NTK, false, false, 64, DK>(accK, dA16, m0, st.b, 0, C, lane);
                 warp_gemm<1, NTK, false, false, 64, DK>(accK, dM16, m0, st.q, 0, C, lane);
-                const int r = m0 + (lane >> 2);
-#pragma unroll
-                for (int nt = 0; nt < NTK; ++nt) {
-                    const int c = 8 * nt + 2 * (lane & 3);
-                    float2 *p0 = reinterpret_cast<float2 *>(DKB + r * DK + c);
-                    float2 *p1 = reinterpret_cast<float2 *>(DKB + (r + 8) * DK + c);
-                    float2 x0 = *p0, x1 = *p1;
-                    x0.x += accK[0][nt][0]; x0.y += accK[0][nt][1];
-                    x1.x += accK[0][nt][2]; x1.y += accK[0][nt][3];
-                    *p0 = x0;
-                    *p1 = x1;
-                }
             }
+            asm volatile("bar.sync 1, 128;\n" ::: "memory");  // warps 4..7 are done reading Dh
+            store_tile_f32<NTK>(accK, DKB, DK, m0, lane);
         }
 
         // ---- dSigma <- Diag(gam) dSigma + Qt^T dO + Gt^T nR (all warps)
@@ -354,47 +364,93 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
         {
             constexpr int NP = DK / 2, P2 = NTHR / NP, RS2 = C / P2;
             const int cp = tid % NP, s2 = tid / NP, c2 = 2 * cp;
-            const float2 lend = *reinterpret_cast<const float2 *>(LAM + (Cn - 1) * DK + c2);
-            const float2 rs0 = *reinterpret_cast<const float2 *>(RS + c2);
-            const float2 rs1 = *reinterpret_cast<const float2 *>(RS + DK + c2);
-            // dv = dRHS . w, dw = dRHS . v from the bf16 -dRHS tile, 16-byte coalesced
-            for (int id = tid; id < C * DV / 8; id += NTHR) {
-                const int r = id / (DV / 8), j = (id % (DV / 8)) * 8;
-                if (r < Cn) {
-                    const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV + j;
-                    const uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, j));
-                    const uint4 v8 = *reinterpret_cast<const uint4 *>(gv + o);
-                    const uint4 w8 = *reinterpret_cast<const uint4 *>(gw + o);
-                    const __nv_bfloat162 *n2 = reinterpret_cast<const __nv_bfloat162 *>(&nr);
-                    const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&v8);
-                    const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w8);
-                    uint4 dv8, dw8;
-                    uint32_t *dvp = reinterpret_cast<uint32_t *>(&dv8), *dwp = reinterpret_cast<uint32_t *>(&dw8);
+            const float2 lend = slow ? *reinterpret_cast<const float2 *>(LAM + (Cn - 1) * DK + c2)
+                                     : make_float2(0.f, 0.f);
+            const float2 rs0 = make_float2(s_rs[0][c2], s_rs[0][c2 + 1]);
+            const float2 rs1 = make_float2(s_rs[1][c2], s_rs[1][c2 + 1]);
+            // dv = dRHS . w, dw = dRHS . v from the bf16 -dRHS tile, 16-byte coalesced;
+            // every global load of the pass is issued before the first use
+            {
+                constexpr int NV = C * DV / 8 / NTHR;
+                uint4 v8[NV], w8[NV];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 d = __bfloat1622float2(n2[e]), vv = __bfloat1622float2(v2[e]),
-                                     ww = __bfloat1622float2(w2[e]);
-                        dvp[e] = pack_bf16(-d.x * ww.x, -d.y * ww.y);
-                        dwp[e] = pack_bf16(-d.x * vv.x, -d.y * vv.y);
+                for (int it = 0; it < NV; ++it) {
+                    const int id = tid + it * NTHR, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
+                    const size_t o = (((size_t)b * T + n * C + min(r, Cn - 1)) * H + h) * DV + j;
+                    v8[it] = *reinterpret_cast<const uint4 *>(gv + o);
+                    w8[it] = *reinterpret_cast<const uint4 *>(gw + o);
+                }
+#pragma unroll
+                for (int it = 0; it < NV; ++it) {
+                    const int id = tid + it * NTHR, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
+                    if (r < Cn) {
+                        const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV + j;
+                        const uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, j));
+                        const __nv_bfloat162 *n2 = reinterpret_cast<const __nv_bfloat162 *>(&nr);
+                        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&v8[it]);
+                        const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w8[it]);
+                        uint4 dv8, dw8;
+                        uint32_t *dvp = reinterpret_cast<uint32_t *>(&dv8), *dwp = reinterpret_cast<uint32_t *>(&dw8);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 d = __bfloat1622float2(n2[e]), vv = __bfloat1622float2(v2[e]),
+                                         ww = __bfloat1622float2(w2[e]);
+                            dvp[e] = pack_bf16(-d.x * ww.x, -d.y * ww.y);
+                            dwp[e] = pack_bf16(-d.x * vv.x, -d.y * vv.y);
+                        }
+                        *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dv) + o) = dv8;
+                        *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dw) + o) = dw8;
                     }
-                    *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dv) + o) = dv8;
-                    *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dw) + o) = dw8;
                 }
             }
+            // in-chunk decay prefix of this thread's rows (the prep's segment sums,
+            // or the slow chunk's L in the workspace)
+            float la_run = 0.f, lb_run = 0.f;
+#pragma unroll
+            for (int s = 0; s < P2; ++s)
+                if (s < s2) { la_run += sh.part[s][c2]; lb_run += sh.part[s][c2 + 1]; }
+            const bf16 *gla = static_cast<const bf16 *>(a.log_alpha);
+            bf16 *__restrict__ gdq = static_cast<bf16 *>(a.dq);
+            bf16 *__restrict__ gdk = static_cast<bf16 *>(a.dk);
+            bf16 *__restrict__ gdb = static_cast<bf16 *>(a.db);
+            const float *__restrict__ sQT = DQT;
+            const float *__restrict__ sGT = DGT;
+            const float *__restrict__ sKB = DKB;
+            __nv_bfloat162 rq[RS2], rk[RS2], rb[RS2], rl[RS2];
+#pragma unroll
+            for (int i = 0; i < RS2; ++i) {
+                const int r = min(s2 * RS2 + i, Cn - 1);
+                const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c2;
+                rq[i] = *reinterpret_cast<const __nv_bfloat162 *>(gq + o);
+                rk[i] = *reinterpret_cast<const __nv_bfloat162 *>(gk + o);
+                rb[i] = *reinterpret_cast<const __nv_bfloat162 *>(gb + o);
+                rl[i] = *reinterpret_cast<const __nv_bfloat162 *>(gla + o);
+            }
+            float dla_r[RS2], dlb_r[RS2];
             float pa = 0.f, pb = 0.f;
-            const int rlo = s2 * RS2, rhi = min(Cn, (s2 + 1) * RS2);
-#pragma unroll 4
-            for (int r = rlo; r < rhi; ++r) {
-                {
+#pragma unroll
+            for (int i = 0; i < RS2; ++i) {
+                const int r = s2 * RS2 + i;
+                dla_r[i] = 0.f;
+                dlb_r[i] = 0.f;
+                if (r < Cn) {
                     const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c2;
-                    const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(gq + o));
-                    const float2 kk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(gk + o));
-                    const float2 bb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(gb + o));
-                    const float2 lam = *reinterpret_cast<const float2 *>(LAM + r * DK + c2);
-                    const float2 dqt = *reinterpret_cast<const float2 *>(DQT + r * DK + c2);
-                    const float2 dgt = *reinterpret_cast<const float2 *>(DGT + r * DK + c2);
-                    const float2 dkb = *reinterpret_cast<const float2 *>(DKB + r * DK + c2);
-                    const float mdiag = DMD[r];
+                    const float2 q = __bfloat1622float2(rq[i]);
+                    const float2 kk = __bfloat1622float2(rk[i]);
+                    const float2 bb = __bfloat1622float2(rb[i]);
+                    float2 lam;
+                    if (!slow) {
+                        const float2 l = __bfloat1622float2(rl[i]);
+                        la_run += l.x;
+                        lb_run += l.y;
+                        lam = make_float2(la_run, lb_run);
+                    } else {
+                        lam = *reinterpret_cast<const float2 *>(LAM + r * DK + c2);
+                    }
+                    const float2 dqt = *reinterpret_cast<const float2 *>(sQT + r * DK + c2);
+                    const float2 dgt = *reinterpret_cast<const float2 *>(sGT + r * DK + c2);
+                    const float2 dkb = *reinterpret_cast<const float2 *>(sKB + r * DK + c2);
+                    const float mdiag = s_dmd[r];
                     const float ea = __expf(lam.x), eb = __expf(lam.y);
                     float dqa, dqb, dga, dgb, dka, dkb2, dla, dlb;
                     if (!slow) {
@@ -419,11 +475,11 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
                     dqa += mdiag * kk.x; dqb += mdiag * kk.y;
                     dka += mdiag * q.x; dkb2 += mdiag * q.y;
                     if (r == Cn - 1) { dla += rs0.x + rs1.x; dlb += rs0.y + rs1.y; }
-                    *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dq) + o) = pack_bf16(dqa, dqb);
-                    *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dk) + o) =
-                        pack_bf16(dka + dga * bb.x, dkb2 + dgb * bb.y);
-                    *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.db) + o) = pack_bf16(dga * kk.x, dgb * kk.y);
-                    *reinterpret_cast<float2 *>(DLAM + r * DK + c2) = make_float2(dla, dlb);
+                    *reinterpret_cast<uint32_t *>(gdq + o) = pack_bf16(dqa, dqb);
+                    *reinterpret_cast<uint32_t *>(gdk + o) = pack_bf16(dka + dga * bb.x, dkb2 + dgb * bb.y);
+                    *reinterpret_cast<uint32_t *>(gdb + o) = pack_bf16(dga * kk.x, dgb * kk.y);
+                    dla_r[i] = dla;
+                    dlb_r[i] = dlb;
                     pa += dla;
                     pb += dlb;
                 }
@@ -435,12 +491,12 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
 #pragma unroll
             for (int s = 0; s < P2; ++s)
                 if (s > s2) { acca += s_dpart[s][c2]; accb += s_dpart[s][c2 + 1]; }
-#pragma unroll 4
-            for (int r = (s2 + 1) * RS2 - 1; r >= s2 * RS2; --r) {
+#pragma unroll
+            for (int i = RS2 - 1; i >= 0; --i) {
+                const int r = s2 * RS2 + i;
                 if (r < Cn) {
-                    const float2 d = *reinterpret_cast<const float2 *>(DLAM + r * DK + c2);
-                    acca += d.x;
-                    accb += d.y;
+                    acca += dla_r[i];
+                    accb += dlb_r[i];
                     *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dlog_alpha) +
                                                   (((size_t)b * T + n * C + r) * H + h) * DK + c2) =
                         pack_bf16(acca, accb);
@@ -468,10 +524,14 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
 template <int DK, int DV>
 cudaError_t launch_t(const ChunkBwdArgs &a, cudaStream_t s) {
     // (1) state pass: the forward with bf16 chunk-boundary states, no output
-    ChunkFwdArgs f{a.q, a.k, a.v, a.log_alpha, a.b, a.w, a.S0, nullptr, nullptr, a.scratch, a.scr_stride,
-                   a.states, a.status, a.B, a.T, a.H};
-    cudaError_t e = launch_chunk_fwd(f, DK, DV, s);
-    if (e != cudaSuccess) return e;
+    // (skipped when the forward already saved them)
+    cudaError_t e = cudaSuccess;
+    if (!a.states_given) {
+        ChunkFwdArgs f{a.q, a.k, a.v, a.log_alpha, a.b, a.w, a.S0, nullptr, nullptr, a.scratch, a.scr_stride,
+                       a.states, a.status, a.B, a.T, a.H};
+        e = launch_chunk_fwd(f, DK, DV, s);
+        if (e != cudaSuccess) return e;
+    }
     // (2) reverse chunk pass
     constexpr int bytes = BSmem<DK, DV>::BYTES;
     e = cudaFuncSetAttribute(chunk_bwd_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);

@@ -61,6 +61,7 @@ struct ChunkBwdArgs {
     float *scratch;
     size_t scr_stride;
     int *status;
+    int states_given;  // 1: `states` already holds the forward's chunk-boundary states
     int B, T, H;
 };
 

@@ -108,6 +108,32 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
                    void *ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
+ * Saved-state training path.  gdn2_chunk_fwd_save is gdn2_chunk_fwd that
+ * also writes the state at every chunk boundary (bf16, [B][H][ceil(T/64)+1]
+ * [dk][dv], gdn2_chunk_states_bytes(...) bytes, caller-owned, 16-byte
+ * aligned) to `states`; gdn2_chunk_bwd_saved is gdn2_chunk_bwd that reads
+ * those states instead of re-running the forward to recompute them, with the
+ * smaller workspace gdn2_chunk_bwd_saved_workspace(...).  The states must come
+ * from gdn2_chunk_fwd_save on the same inputs; results equal those of
+ * gdn2_chunk_fwd / gdn2_chunk_bwd.  (The backward of the pages' method needs
+ * the chunk-start states; this pair keeps them instead of recomputing them.)
+ * For GDN2_FP32 the state buffer is not used (gdn2_chunk_states_bytes = 0):
+ * the fp32 mode checkpoints inside its own workspace.
+ */
+size_t gdn2_chunk_states_bytes(int B, int T, int H, int dk, int dv, int dtype);
+int gdn2_chunk_fwd_save(const void *q, const void *k, const void *v, const void *log_alpha,
+                        const void *b, const void *w, const float *S0, void *o, float *S_T, void *states,
+                        int B, int T, int H, int dk, int dv, int dtype,
+                        void *ws, size_t ws_bytes, cudaStream_t stream);
+size_t gdn2_chunk_bwd_saved_workspace(int B, int T, int H, int dk, int dv, int dtype);
+int gdn2_chunk_bwd_saved(const void *q, const void *k, const void *v, const void *log_alpha,
+                         const void *b, const void *w, const float *S0, const void *dO,
+                         const float *dS_T, const void *states, void *dq, void *dk_, void *dv_,
+                         void *dlog_alpha, void *db, void *dw, float *dS0,
+                         int B, int T, int H, int dk, int dv, int dtype,
+                         void *ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * gdn2_chunk_fwd without a caller-provided workspace, for callers that cannot
  * allocate device memory (no cudaMalloc available to them, or a code path
  * that must not allocate).  The pages have no counterpart to this call; it is

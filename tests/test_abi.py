@@ -81,3 +81,19 @@ def test_workspace_sizes():
     assert g.gdn2_chunk_fwd_workspace(0, 4096, 16, 128, 128, g.GDN2_BF16) == 0
     assert g.gdn2_chunk_bwd_workspace(8, 4096, 16, 128, 128, g.GDN2_BF16) > 0
     assert g.gdn2_chunk_bwd_workspace(8, 4096, 16, 96, 128, g.GDN2_BF16) == 0
+
+
+def test_saved_state_entry_points_validate():
+    B, T, H = 2, 100, 3
+    n = g.gdn2_chunk_states_bytes(B, T, H, 128, 128, g.GDN2_BF16)
+    assert n == B * H * (2 + 1) * 128 * 128 * 2  # ceil(100/64) + 1 boundaries, bf16
+    assert g.gdn2_chunk_states_bytes(B, T, H, 128, 128, g.GDN2_FP32) == 0
+    assert 0 < g.gdn2_chunk_bwd_saved_workspace(B, T, H, 128, 128, g.GDN2_BF16) < \
+        g.gdn2_chunk_bwd_workspace(B, T, H, 128, 128, g.GDN2_BF16)
+    # missing or misaligned state buffer is refused before any launch
+    args = [16] * 6 + [None, 16, None, None] + [16] * 6 + [None]
+    assert g.gdn2_chunk_bwd_saved(*args, B, T, H, 128, 128, 0, 16, 1 << 40, 0) == -1
+    args[9] = 24
+    assert g.gdn2_chunk_bwd_saved(*args, B, T, H, 128, 128, 0, 16, 1 << 40, 0) == -1
+    assert g.gdn2_chunk_fwd_save(16, 16, 16, 16, 16, 16, None, 16, None, None, B, T, H, 128, 128, 0, 16,
+                                 1 << 40, 0) == -1

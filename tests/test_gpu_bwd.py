@@ -74,3 +74,24 @@ def test_bwd_deterministic():
     g2 = run_bwd(x, "bf16")
     for n in GRADS:
         np.testing.assert_array_equal(g1[n], g2[n])
+
+
+@pytest.mark.parametrize("dk,dv,T", [(128, 128, 200), (64, 64, 130), (128, 64, 64)])
+def test_saved_state_path_equals_recompute(dk, dv, T):
+    """gdn2_chunk_fwd_save + gdn2_chunk_bwd_saved give exactly the results of
+    gdn2_chunk_fwd + gdn2_chunk_bwd (same kernels, states kept instead of
+    recomputed)."""
+    import gated_delta_rule_gdn2_b200 as g
+    x = make_inputs(2, T, 2, dk, dv, seed=91, dtype="bf16", with_do=True)
+    toks = tokens(x, "bf16")
+    S0 = dev_state(x["S0"])
+    o1, S1 = g.chunk_fwd(*toks, S0=S0)
+    o2, S2, states = g.chunk_fwd(*toks, S0=S0, save_states=True)
+    np.testing.assert_array_equal(host(o1), host(o2))
+    np.testing.assert_array_equal(host(S1), host(S2))
+    dO = dev(x["dO"], "bf16")
+    g1 = g.chunk_bwd(*toks, S0, dO)
+    g2 = g.chunk_bwd(*toks, S0, dO, states=states)
+    assert g.gdn2_get_device_status() == 0
+    for n in GRADS:
+        np.testing.assert_array_equal(host(g1[n]), host(g2[n]))
