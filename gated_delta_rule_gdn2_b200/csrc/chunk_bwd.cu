@@ -39,6 +39,10 @@ namespace cbwd {
 
 using namespace chunk;
 
+// k-loop unroll of the backward's warp products: rolled by two so that the
+// kernel's hot path stays inside the instruction cache
+constexpr int KU = 2;
+
 template <int DK, int DV>
 struct BSmem {
     static constexpr int TQ = C * DK * 2, TV = C * DV * 2, TS = DK * DV * 2;
@@ -95,10 +99,9 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
     float *T32 = A32 + C * C;
     bf16 *T16 = reinterpret_cast<bf16 *>(T32);
     bf16 *M16 = T16 + C * C;
-    bf16 *W16 = reinterpret_cast<bf16 *>(A32);   // after the solve
-    bf16 *dU16 = reinterpret_cast<bf16 *>(A32);  // after U
-    bf16 *U16 = st.w;                            // w . v went to the v slot
-    bf16 *nR16 = st.v;                           // after Uv
+    bf16 *dU16 = reinterpret_cast<bf16 *>(A32);
+    bf16 *U16 = st.w;                            // the forward's U
+    bf16 *nR16 = st.v;
     bf16 *dM16 = reinterpret_cast<bf16 *>(L::AM_IN_K ? smem + L::OK : smem + L::OAM);
     bf16 *dA16 = dM16 + C * C;
 
@@ -117,6 +120,8 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
         DGT = DKB + C * DK;
     }
     const bf16 *states = static_cast<const bf16 *>(a.states) + (size_t)bh * (nchunks + 1) * DK * DV;
+    constexpr int TM_BYTES = 2 * C * C * 2, U_BYTES = C * DV * 2, I_BYTES = TM_BYTES + U_BYTES;
+    const unsigned char *intra = static_cast<const unsigned char *>(a.intra) + (size_t)bh * nchunks * I_BYTES;
     const bf16 *gq = static_cast<const bf16 *>(a.q), *gk = static_cast<const bf16 *>(a.k);
     const bf16 *gb = static_cast<const bf16 *>(a.b), *gv = static_cast<const bf16 *>(a.v);
     const bf16 *gw = static_cast<const bf16 *>(a.w);
@@ -137,13 +142,13 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
 
     for (int n = nchunks - 1; n >= 0; --n) {
         const int Cn = min(C, T - n * C);
-        // ---- loads: six token tiles, dO, the chunk-start state
+        // ---- loads: four token tiles, dO, the chunk-start state and the
+        // forward's T, M (into the WY-solve area) and U (into the w slot), which
+        // are stored as their shared-memory images
         load_token_tile<DK>(st.q, gq, b, h, n, T, H);
         load_token_tile<DK>(st.k, gk, b, h, n, T, H);
         load_token_tile<DK>(st.la, static_cast<const bf16 *>(a.log_alpha), b, h, n, T, H);
         load_token_tile<DK>(st.b, gb, b, h, n, T, H);
-        load_token_tile<DV>(st.v, gv, b, h, n, T, H);
-        load_token_tile<DV>(st.w, gw, b, h, n, T, H);
         load_token_tile<DV>(dO16, static_cast<const bf16 *>(a.dO), b, h, n, T, H);
         {
             const bf16 *src = states + (size_t)n * DK * DV;
@@ -151,6 +156,11 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
                 const int r = id / (DV / 8), ch = id % (DV / 8);
                 cp_async16(S16 + swz<DV, DK>(r, ch * 8), src + (size_t)r * DV + ch * 8, true);
             }
+            const unsigned char *it = intra + (size_t)n * I_BYTES;
+            for (int id = tid; id < TM_BYTES / 16; id += NTHR)
+                cp_async16(reinterpret_cast<unsigned char *>(T16) + 16 * id, it + 16 * id, true);
+            for (int id = tid; id < U_BYTES / 16; id += NTHR)
+                cp_async16(reinterpret_cast<unsigned char *>(U16) + 16 * id, it + TM_BYTES + 16 * id, true);
         }
         cp_commit();
         cp_wait<0>();
@@ -173,11 +183,15 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
                     const bf16 *sp = states + (size_t)(n - 1) * DK * DV + (size_t)slot * (DK * DV / 16);
                     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(sp), "r"(DK * DV * 2 / 16)
                                  : "memory");
+                } else if (slot < 32) {
+                    const unsigned char *ip = intra + (size_t)(n - 1) * I_BYTES + (size_t)(slot - 16) * (I_BYTES / 16);
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(ip), "r"(I_BYTES / 16)
+                                 : "memory");
                 }
             }
         }
 
-        const bool slow = intra_chunk<DK, DV>(st, A32, T32, sh, LAM, false);
+        const bool slow = intra_chunk<DK, DV>(st, A32, T32, sh, LAM, false, /*prep_only=*/true);
 
         // ---- Dh = gam . dSigma (fast) or dSigma (slow) as bf16; row sums of
         // dSigma . Sigma (Sigma = next chunk-boundary state) for dL_end
@@ -212,36 +226,22 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
             }
         }
 
-        // ---- W = T Gt (warps 4..7, stored negated), Uv = T WV (warps 0..3)
         constexpr int NTX = NTV > NTK ? NTV : NTK;
         float accX[1][NTX][4];
         auto &accV = reinterpret_cast<float(&)[1][NTV][4]>(accX);
         auto &accK = reinterpret_cast<float(&)[1][NTK][4]>(accX);
-        zero(accX);
-        if (warp < 4) {
-            warp_gemm<1, NTV, true, false, 64, DV>(accV, T16, 16 * warp, st.v, 0, C, lane);
-        } else {
-            warp_gemm<1, NTK, true, false, 64, DK>(accK, T16, 16 * (warp & 3), st.b, 0, C, lane);
-            store_tile_bf16<NTK, DK>(accK, W16, 16 * (warp & 3), lane, -1.f);
-        }
-        __syncthreads();
-        // ---- U = Uv - W S (warps 0..3) into the w slot
-        if (warp < 4) {
-            warp_gemm<1, NTV, true, false, DK, DV, C, DK>(accV, W16, 16 * warp, S16, 0, DK, lane);
-            store_tile_bf16<NTV, DV>(accV, U16, 16 * warp, lane, 1.f);
-        }
-        __syncthreads();
+        __syncthreads();  // D16 and the row sums are complete
 
         // ---- dU = M^T dO + Kh Dh (warps 0..3) ; dM = lower(dO U^T) (warps 4..7)
         if (warp < 4) {
             zero(accX);
-            warp_gemm<1, NTV, false, false, 64, DV>(accV, M16, 16 * warp, dO16, 0, C, lane);
-            warp_gemm<1, NTV, true, false, DK, DV, C, DK>(accV, st.la, 16 * warp, D16, 0, DK, lane);
+            warp_gemm<1, NTV, false, false, 64, DV, C, C, KU>(accV, M16, 16 * warp, dO16, 0, C, lane);
+            warp_gemm<1, NTV, true, false, DK, DV, C, DK, KU>(accV, st.la, 16 * warp, D16, 0, DK, lane);
             store_tile_bf16<NTV, DV>(accV, dU16, 16 * warp, lane, 1.f);
         } else {
             float acc[1][8][4];
             zero(acc);
-            warp_gemm<1, 8, true, true, DV, DV>(acc, dO16, 16 * (warp & 3), U16, 0, DV, lane);
+            warp_gemm<1, 8, true, true, DV, DV, C, C, KU>(acc, dO16, 16 * (warp & 3), U16, 0, DV, lane);
             const int r0 = 16 * (warp & 3) + (lane >> 2);
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
         // ---- nR = -T^T dU (warps 0..3)
         if (warp < 4) {
             zero(accX);
-            warp_gemm<1, NTV, false, false, 64, DV>(accV, T16, 16 * warp, dU16, 0, C, lane);
+            warp_gemm<1, NTV, false, false, 64, DV, C, C, KU>(accV, T16, 16 * warp, dU16, 0, C, lane);
             store_tile_bf16<NTV, DV>(accV, nR16, 16 * warp, lane, -1.f);
         }
         __syncthreads();
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
         if (warp < 4) {
             float acc[1][8][4];
             zero(acc);
-            warp_gemm<1, 8, true, true, DV, DV>(acc, nR16, 16 * warp, U16, 0, DV, lane);
+            warp_gemm<1, 8, true, true, DV, DV, C, C, KU>(acc, nR16, 16 * warp, U16, 0, DV, lane);
             const int r0 = 16 * warp + (lane >> 2);
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
@@ -282,18 +282,18 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
             store_tile_bf16<8, 64>(acc, dA16, 16 * warp, lane, 1.f);
         } else {
             zero(accX);
-            warp_gemm<1, NTK, true, true, DV, DV, C, DK>(accK, dO16, 16 * (warp & 3), S16, 0, DV, lane);
+            warp_gemm<1, NTK, true, true, DV, DV, C, DK, KU>(accK, dO16, 16 * (warp & 3), S16, 0, DV, lane);
         }
         __syncthreads();
 
         // ---- dGt = nR S^T + dA Kb (warps 0..3) ; dQt += dM Kb (warps 4..7)
         if (warp < 4) {
             zero(accX);
-            warp_gemm<1, NTK, true, true, DV, DV, C, DK>(accK, nR16, 16 * warp, S16, 0, DV, lane);
-            if (!slow) warp_gemm<1, NTK, true, false, 64, DK>(accK, dA16, 16 * warp, st.la, 0, C, lane);
+            warp_gemm<1, NTK, true, true, DV, DV, C, DK, KU>(accK, nR16, 16 * warp, S16, 0, DV, lane);
+            if (!slow) warp_gemm<1, NTK, true, false, 64, DK, C, C, KU>(accK, dA16, 16 * warp, st.la, 0, C, lane);
             store_tile_f32<NTK>(accK, DGT, DK, 16 * warp, lane);  // the WY-solve area is dead
         } else if (!slow) {
-            warp_gemm<1, NTK, true, false, 64, DK>(accK, dM16, 16 * (warp & 3), st.la, 0, C, lane);
+            warp_gemm<1, NTK, true, false, 64, DK, C, C, KU>(accK, dM16, 16 * (warp & 3), st.la, 0, C, lane);
         }
         __syncthreads();  // S is no longer read: its region takes dQt
 
@@ -302,10 +302,10 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
             const int m0 = 16 * (warp & 3);
             store_tile_f32<NTK>(accK, DQT, DK, m0, lane);
             zero(accX);
-            warp_gemm<1, NTK, true, true, DV, DV, C, DK>(accK, U16, m0, D16, 0, DV, lane);
+            warp_gemm<1, NTK, true, true, DV, DV, C, DK, KU>(accK, U16, m0, D16, 0, DV, lane);
             if (!slow) {
-                warp_gemm<1, NTK, false, false, 64, DK>(accK, dA16, m0, st.b, 0, C, lane);
-                warp_gemm<1, NTK, false, false, 64, DK>(accK, dM16, m0, st.q, 0, C, lane);
+                warp_gemm<1, NTK, false, false, 64, DK, C, C, KU>(accK, dA16, m0, st.b, 0, C, lane);
+                warp_gemm<1, NTK, false, false, 64, DK, C, C, KU>(accK, dM16, m0, st.q, 0, C, lane);
             }
             asm volatile("bar.sync 1, 128;\n" ::: "memory");  // warps 4..7 are done reading Dh
             store_tile_f32<NTK>(accK, DKB, DK, m0, lane);
@@ -320,8 +320,8 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
                 dS[mt][nt][0] *= g0; dS[mt][nt][1] *= g0; dS[mt][nt][2] *= g1; dS[mt][nt][3] *= g1;
             }
         }
-        warp_gemm<MTS, NTS, false, false, DK, DV>(dS, st.q, c0, dO16, j0, C, lane);
-        warp_gemm<MTS, NTS, false, false, DK, DV>(dS, st.b, c0, nR16, j0, C, lane);
+        warp_gemm<MTS, NTS, false, false, DK, DV, C, C, KU>(dS, st.q, c0, dO16, j0, C, lane);
+        warp_gemm<MTS, NTS, false, false, DK, DV, C, C, KU>(dS, st.b, c0, nR16, j0, C, lane);
         __syncthreads();
 
         // ---- slow chunk: Gram gradients term by term, e^{L_r - L_i} <= 1
@@ -528,7 +528,7 @@ cudaError_t launch_t(const ChunkBwdArgs &a, cudaStream_t s) {
     cudaError_t e = cudaSuccess;
     if (!a.states_given) {
         ChunkFwdArgs f{a.q, a.k, a.v, a.log_alpha, a.b, a.w, a.S0, nullptr, nullptr, a.scratch, a.scr_stride,
-                       a.states, a.status, a.B, a.T, a.H};
+                       a.states, a.intra, a.status, a.B, a.T, a.H};
         e = launch_chunk_fwd(f, DK, DV, s);
         if (e != cudaSuccess) return e;
     }
@@ -542,8 +542,7 @@ cudaError_t launch_t(const ChunkBwdArgs &a, cudaStream_t s) {
 
 template <int DK, int DV>
 size_t ws_t(int B, int T, int H, size_t *scr_stride, size_t *states_bytes) {
-    const size_t nc = (size_t)((T + C - 1) / C);
-    const size_t sb = ((size_t)B * H * (nc + 1) * DK * DV * 2 + 255) / 256 * 256;
+    const size_t sb = states_region_bytes(B, T, H, DK, DV) + intra_region_bytes(B, T, H, DV);
     const size_t stride = (Scratch<DK>::FLOATS + 63) / 64 * 64;
     if (scr_stride) *scr_stride = stride;
     if (states_bytes) *states_bytes = sb;

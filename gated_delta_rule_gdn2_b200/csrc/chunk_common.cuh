@@ -74,43 +74,61 @@ __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0
 // acc[MT][NT][4] += A[m0 + 16 mt + .., k] * B[k, n0 + 8 nt + ..], k in [0, K).
 // A_KM: A stored [m][k] in a [RA][DA] tile, else stored [k][m].
 // B_KM: B stored [n][k] in a [RB][DB] tile, else stored [k][n].
-template <int MT, int NT, bool A_KM, bool B_KM, int DA, int DB, int RA = C, int RB = C>
+// One k-step of 16 of warp_gemm below.
+template <int MT, int NT, bool A_KM, bool B_KM, int DA, int DB, int RA, int RB>
+__device__ __forceinline__ void warp_gemm_kstep(float (&acc)[MT][NT][4], const bf16 *A, int m0, const bf16 *B,
+                                                int n0, int k0, int lane) {
+    uint32_t a[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        if (A_KM) {
+            const int r = m0 + 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int c = k0 + (lane >> 4) * 8;
+            ldsm4(smem_u32(A + swz<DA, RA>(r, c)), a[mt]);
+        } else {
+            const int i = lane >> 3;
+            const int kr = k0 + (lane & 7) + (i >> 1) * 8;
+            const int mc = m0 + 16 * mt + (i & 1) * 8;
+            ldsm4t(smem_u32(A + swz<DA, RA>(kr, mc)), a[mt]);
+        }
+    }
+#pragma unroll
+    for (int np = 0; np < NT / 2; ++np) {
+        uint32_t b[4];
+        if (B_KM) {
+            const int r = n0 + 16 * np + (lane & 7) + (lane >> 4) * 8;
+            const int c = k0 + ((lane >> 3) & 1) * 8;
+            ldsm4(smem_u32(B + swz<DB, RB>(r, c)), b);
+        } else {
+            const int kr = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int nc = n0 + 16 * np + (lane >> 4) * 8;
+            ldsm4t(smem_u32(B + swz<DB, RB>(kr, nc)), b);
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            mma16816(acc[mt][2 * np], a[mt], b[0], b[1]);
+            mma16816(acc[mt][2 * np + 1], a[mt], b[2], b[3]);
+        }
+    }
+}
+
+// acc[MT][NT][4] += A[m0 + 16 mt + .., k] * B[k, n0 + 8 nt + ..], k in [0, K).
+// A_KM: A stored [m][k] in a [RA][DA] tile, else stored [k][m].
+// B_KM: B stored [n][k] in a [RB][DB] tile, else stored [k][n].
+// UNR: unroll factor of the k loop (0 = full); a rolled loop keeps long
+// straight-line kernels inside the instruction cache.
+template <int MT, int NT, bool A_KM, bool B_KM, int DA, int DB, int RA = C, int RB = C, int UNR = 0>
 __device__ __forceinline__ void warp_gemm(float (&acc)[MT][NT][4], const bf16 *A, int m0, const bf16 *B,
                                           int n0, int K, int lane) {
     static_assert(NT % 2 == 0, "n tiles come in pairs");
-    for (int k0 = 0; k0 < K; k0 += 16) {
-        uint32_t a[MT][4];
+    if constexpr (UNR == 0) {
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            if (A_KM) {
-                const int r = m0 + 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int c = k0 + (lane >> 4) * 8;
-                ldsm4(smem_u32(A + swz<DA, RA>(r, c)), a[mt]);
-            } else {
-                const int i = lane >> 3;
-                const int kr = k0 + (lane & 7) + (i >> 1) * 8;
-                const int mc = m0 + 16 * mt + (i & 1) * 8;
-                ldsm4t(smem_u32(A + swz<DA, RA>(kr, mc)), a[mt]);
-            }
-        }
-#pragma unroll
-        for (int np = 0; np < NT / 2; ++np) {
-            uint32_t b[4];
-            if (B_KM) {
-                const int r = n0 + 16 * np + (lane & 7) + (lane >> 4) * 8;
-                const int c = k0 + ((lane >> 3) & 1) * 8;
-                ldsm4(smem_u32(B + swz<DB, RB>(r, c)), b);
-            } else {
-                const int kr = k0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int nc = n0 + 16 * np + (lane >> 4) * 8;
-                ldsm4t(smem_u32(B + swz<DB, RB>(kr, nc)), b);
-            }
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                mma16816(acc[mt][2 * np], a[mt], b[0], b[1]);
-                mma16816(acc[mt][2 * np + 1], a[mt], b[2], b[3]);
-            }
-        }
+        for (int k0 = 0; k0 < K; k0 += 16)
+            warp_gemm_kstep<MT, NT, A_KM, B_KM, DA, DB, RA, RB>(acc, A, m0, B, n0, k0, lane);
+    } else {
+#pragma unroll UNR
+        for (int k0 = 0; k0 < K; k0 += 16)
+            warp_gemm_kstep<MT, NT, A_KM, B_KM, DA, DB, RA, RB>(acc, A, m0, B, n0, k0, lane);
     }
 }
 
@@ -180,6 +198,13 @@ __device__ __forceinline__ void prefetch_token_rows_l2(const bf16 *src, int b, i
     }
 }
 
+// Block-wide 16-byte copy of `bytes` (a multiple of 16) from shared to global memory.
+__device__ __forceinline__ void copy_smem_to_global(void *dst, const void *src, int bytes) {
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+    for (int i = threadIdx.x; i < bytes / 16; i += NTHR) d4[i] = s4[i];
+}
+
 struct ChunkTiles {
     bf16 *q, *k, *la, *b, *v, *w;
 };
@@ -227,8 +252,9 @@ __device__ __forceinline__ void block16_tf32(float (&acc)[2][4], const float *X,
 }
 
 // Intra-chunk stage.  On entry the six raw token tiles of the chunk are in
-// shared memory (and visible to all threads).  On exit (all threads, after a
-// barrier):
+// shared memory (and visible to all threads).  With prep_only only the decay
+// prefix and the operands Qt, Gt, Kb/Kt are formed (v, w untouched; T, M
+// come from elsewhere).  Otherwise, on exit (all threads, after a barrier):
 //   st.q -> Qt, st.b -> Gt, st.la -> Kb (fast) or Kt (slow), st.v -> w . v;
 //   T16 = bf16 (I + A)^{-1} and M16 = bf16 M (swizzled [64][64]);
 //   sh.gamma = e^{L_end}; returns true for a slow chunk.
@@ -237,7 +263,7 @@ __device__ __forceinline__ void block16_tf32(float (&acc)[2][4], const float *X,
 // keep_lam is set and is always used by a slow chunk.
 template <int DK, int DV>
 __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<DK> &sh, float *lam_ws,
-                            bool keep_lam) {
+                            bool keep_lam, bool prep_only = false) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     bf16 *T16 = reinterpret_cast<bf16 *>(T32);
     bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
@@ -256,7 +282,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
         }
         sh.part[s2][c2] = pa;
         sh.part[s2][c2 + 1] = pb;
-        for (int id = tid; id < C * DV / 8; id += NTHR) {
+        for (int id = tid; id < (prep_only ? 0 : C * DV / 8); id += NTHR) {
             uint4 wv = reinterpret_cast<const uint4 *>(st.w)[id];
             uint4 vv = reinterpret_cast<const uint4 *>(st.v)[id];
             const bf16 *w8 = reinterpret_cast<const bf16 *>(&wv);
@@ -307,6 +333,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
             *reinterpret_cast<uint32_t *>(st.la + o) = pack_bf16(k2.x * iea, k2.y * ieb);
         }
         __syncthreads();
+        if (prep_only) return false;
         // ---- Grams: [Gt; Qt] Kb^T, warp w -> rows 16w..16w+15 of the stacked operand
         float acc[1][8][4];
         zero(acc);
@@ -339,7 +366,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
             pa[s] = 0.f;
             pm[s] = 0.f;
             const int p = tid + NTHR * s;
-            if (p < C * (C + 1) / 2) {
+            if (!prep_only && p < C * (C + 1) / 2) {
                 int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
                 while ((r + 1) * (r + 2) / 2 <= p) ++r;
                 while (r * (r + 1) / 2 > p) --r;
@@ -368,6 +395,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
             }
         }
         __syncthreads();
+        if (prep_only) return true;
         for (int e = tid; e < C * C; e += NTHR) {
             A32[e] = 0.f;
             T32[e] = 0.f;

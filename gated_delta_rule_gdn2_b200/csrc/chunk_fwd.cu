@@ -98,6 +98,9 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
     bf16 *S16 = reinterpret_cast<bf16 *>(smem + L::OS16);
     float *lam_ws = a.ws ? a.ws + (size_t)bh * a.ws_stride : nullptr;
     const bool with_o = a.o != nullptr;
+    auto keep_tile = [&](int n) {
+        return static_cast<unsigned char *>(a.intra) + ((size_t)bh * nchunks + n) * intra_tile_bytes(DV);
+    };
 
     // ---- state tile of this warp, fp32 in registers
     const int c0 = (warp >> 1) * WR, j0 = (warp & 1) * WC;
@@ -152,6 +155,8 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
         cp_wait<1>();
         __syncthreads();
         const bool slow = intra_chunk<DK, DV>(st, A32, T32, sh, lam_ws, false);
+        // T and M (then U, below) for the backward, as their shared-memory images
+        if (a.intra) copy_smem_to_global(keep_tile(n), T16, 2 * C * C * 2);
 
         // ---- W = T Gt (warps 4..7, stored negated), Uv = T WV (warps 0..3, kept).
         // One accumulator per warp serves Uv -> U (warps 0..3) and W -> O
@@ -179,6 +184,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
         }
         __syncthreads();
 
+        if (a.intra) copy_smem_to_global(keep_tile(n) + 2 * C * C * 2, U16, C * DV * 2);
         // ---- O += M U, store o
         if (warp >= 4 && with_o) {
             warp_gemm<1, NTV, true, false, 64, DV>(accV, M16, 16 * (warp & 3), U16, 0, C, lane);

@@ -77,6 +77,9 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
     const int nchunks = (a.T + C - 1) / C;
     const bool with_o = a.o != nullptr;
+    auto keep_tile = [&](int n) {
+        return static_cast<unsigned char *>(a.intra) + ((size_t)bh * nchunks + n) * intra_tile_bytes(D);
+    };
     float *lam_ws = a.ws ? a.ws + (size_t)bh * a.ws_stride : nullptr;
     bf16 *S16 = reinterpret_cast<bf16 *>(smem + OS16);
 
@@ -160,6 +163,8 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
         __syncthreads();
         if (sm.abort) break;
         const bool slow = intra_chunk<D, D>(st, A32, T32, sm.intra, lam_ws, false);
+        // T and M (then U, below) for the backward, as their shared-memory images
+        if (a.intra) copy_smem_to_global(keep_tile(n), T16, 2 * C * C * 2);
 
         // ---- Uv = T WV (warps 0..3, registers) ; -W = -T Gt (warps 4..7, shared)
         float acc[1][16][4];
@@ -218,6 +223,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
         __syncthreads();
         if (sm.abort) break;
 
+        if (a.intra) copy_smem_to_global(keep_tile(n) + 2 * C * C * 2, U16, C * D * 2);
         // ---- slow chunk: S <- Diag(gam) S before adding Kt^T U
         if (slow) {
             float v[64];

@@ -39,6 +39,7 @@ struct ChunkFwdArgs {
     float *ws;
     size_t ws_stride;
     void *states;
+    void *intra;  // optional: per chunk the bf16 tiles T, M (64x64 each) and U (64 x dv), as in shared memory
     int *status;  // device status word (bounded waits record GDN2_ERR_TIMEOUT here)
     int B, T, H;
 };
@@ -57,13 +58,26 @@ struct ChunkBwdArgs {
     const float *dS_T;
     void *dq, *dk, *dv, *dlog_alpha, *db, *dw;
     float *dS0;
-    void *states;
+    void *states;      // bf16 chunk-boundary states [B*H][nchunks+1][dk][dv]
+    void *intra;       // per chunk the bf16 tiles T, M, U of the forward (intra_tile_bytes each)
     float *scratch;
     size_t scr_stride;
     int *status;
-    int states_given;  // 1: `states` already holds the forward's chunk-boundary states
+    int states_given;  // 1: `states` already holds what the training forward kept
     int B, T, H;
 };
+
+// Bytes per chunk of the saved intra-chunk tiles (T, M: 64x64 bf16; U: 64 x dv bf16).
+__host__ __device__ inline size_t intra_tile_bytes(int dv) { return (size_t)2 * 64 * 64 * 2 + (size_t)64 * dv * 2; }
+// The saved-state buffer: the chunk-boundary states, then (256-byte aligned) the intra tiles.
+inline size_t states_region_bytes(int B, int T, int H, int dk, int dv) {
+    const size_t nc = (size_t)((T + 63) / 64);
+    return ((size_t)B * H * (nc + 1) * dk * dv * 2 + 255) / 256 * 256;
+}
+inline size_t intra_region_bytes(int B, int T, int H, int dv) {
+    const size_t nc = (size_t)((T + 63) / 64);
+    return ((size_t)B * H * nc * intra_tile_bytes(dv) + 255) / 256 * 256;
+}
 
 cudaError_t launch_chunk_bwd(const ChunkBwdArgs &a, int dk, int dv, cudaStream_t s);
 size_t chunk_bwd_ws_bytes(int B, int T, int H, int dk, int dv, size_t *scr_stride, size_t *states_bytes);

@@ -109,14 +109,18 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
 
 /*
  * Saved-state training path.  gdn2_chunk_fwd_save is gdn2_chunk_fwd that
- * also writes the state at every chunk boundary (bf16, [B][H][ceil(T/64)+1]
- * [dk][dv], gdn2_chunk_states_bytes(...) bytes, caller-owned, 16-byte
- * aligned) to `states`; gdn2_chunk_bwd_saved is gdn2_chunk_bwd that reads
- * those states instead of re-running the forward to recompute them, with the
- * smaller workspace gdn2_chunk_bwd_saved_workspace(...).  The states must come
- * from gdn2_chunk_fwd_save on the same inputs; results equal those of
- * gdn2_chunk_fwd / gdn2_chunk_bwd.  (The backward of the pages' method needs
- * the chunk-start states; this pair keeps them instead of recomputing them.)
+ * also keeps, in `states` (gdn2_chunk_states_bytes(...) bytes, caller-owned,
+ * 16-byte aligned, contents private to this library), what the backward
+ * needs from the forward: the state at every chunk boundary (bf16,
+ * [B][H][ceil(T/64)+1][dk][dv]) and, per chunk, the bf16 WY factor
+ * T = (I + A)^{-1}, the decayed query-key Gram M (64 x 64 each) and the
+ * chunk's WY-form write U (64 x dv).  gdn2_chunk_bwd_saved is gdn2_chunk_bwd
+ * that reads these instead of re-running the forward to recompute them, with
+ * the smaller workspace gdn2_chunk_bwd_saved_workspace(...).  The buffer must
+ * come from gdn2_chunk_fwd_save on the same inputs; results equal those of
+ * gdn2_chunk_fwd / gdn2_chunk_bwd bit for bit.  (The backward of the pages'
+ * method needs the chunk-start states and these per-chunk products; this pair
+ * keeps them instead of recomputing them.)
  * For GDN2_FP32 the state buffer is not used (gdn2_chunk_states_bytes = 0):
  * the fp32 mode checkpoints inside its own workspace.
  */
