@@ -1,0 +1,374 @@
+// Pieces of the backward's reverse chunk pass shared by its two kernels
+// (chunk_bwd.cu: warp-level products for any head size; chunk_bwd_tc.cu:
+// tensor-memory products for dk = dv = 128): the shared-memory plan, the
+// per-chunk loads, the term-by-term Gram gradients of a slow chunk and the
+// token-level gradients (dv, dw, dq, dk, db and the in-chunk reverse
+// cumulative sum that gives dlog_alpha).  The algebra is set out at the top
+// of chunk_bwd.cu.
+#pragma once
+
+#include "chunk_common.cuh"
+#include "launch.h"
+
+namespace gdn2 {
+namespace cbwd {
+
+using namespace chunk;
+
+// k-loop unroll of the backward's warp products: rolled by two so that the
+// kernel's hot path stays inside the instruction cache
+constexpr int KU = 2;
+
+template <int DK, int DV>
+struct BSmem {
+    static constexpr int TQ = C * DK * 2, TV = C * DV * 2, TS = DK * DV * 2;
+    static constexpr int OQ = 0, OK = TQ, OLA = 2 * TQ, OB = 3 * TQ;
+    static constexpr int OV = 4 * TQ, OW = OV + TV, ODO = OW + TV;
+    static constexpr int OS = ODO + TV, OD = OS + TS;
+    static constexpr int OAT = OD + TS;              // A32 | T32 (2 x 16 KB fp32)
+    static constexpr bool AM_IN_K = (DK == 128);     // dM16 | dA16 in the k slot
+    static constexpr int OAM = OAT + 32768;
+    // fp32 [64][DK] staging of dQt, dGt, dKb for the elementwise phase:
+    // (128,128) reuses the dead S, Dh and WY-solve regions; dk = 64 gets
+    // dedicated regions; (128,64) stages through the global scratch.
+    static constexpr bool STAGE_REUSE = (DK == 128 && DV == 128);
+    static constexpr bool STAGE_DED = (DK == 64);
+    static constexpr int OSTG = OAM + (AM_IN_K ? 0 : 16384);
+    static constexpr int BYTES = OSTG + (STAGE_DED ? 3 * C * DK * 4 : 0);
+};
+
+template <int DK>
+struct Scratch {
+    static constexpr int TILE = C * DK;
+    static constexpr int LAM = 0, DQT = 1, DGT = 2, DKB = 3, DLAM = 4, PQ = 5, PG = 6, PK = 7, PL = 8;
+    static constexpr int RS = 9 * TILE;              // 2 x DK row sums
+    static constexpr int DMD = 9 * TILE + 2 * DK;    // diagonal of dM (C floats)
+    static constexpr size_t FLOATS = 9 * TILE + 2 * DK + C;
+};
+
+// fp32 staging tiles [64][DK] of dQt, dGt, dKb: row-major with the 8-column
+// groups of row r permuted by r mod 8, so that the fragment-layout writes
+// (8 rows x 32 bytes per instruction) fill both halves of the banks instead
+// of one; a warp's read of 64 consecutive columns of one row stays a permutation
+// of the same 256 bytes.
+template <int DK>
+__device__ __forceinline__ int stg(int r, int c) { return r * DK + (c ^ ((r & 7) << 3)); }
+
+// Writes a 16-row accumulator fragment (rows m0.., columns n0..) into a staging tile.
+template <int DK, int NT>
+__device__ __forceinline__ void store_stage(const float (&acc)[1][NT][4], float *dst, int m0, int n0, int lane) {
+    const int r = m0 + (lane >> 2);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int c = n0 + 8 * nt + 2 * (lane & 3);
+        *reinterpret_cast<float2 *>(dst + stg<DK>(r, c)) = make_float2(acc[0][nt][0], acc[0][nt][1]);
+        *reinterpret_cast<float2 *>(dst + stg<DK>(r + 8, c)) = make_float2(acc[0][nt][2], acc[0][nt][3]);
+    }
+}
+
+// Per-CTA view of one (batch, head) sequence in the reverse chunk pass: the
+// shared-memory tiles, the caller's per-CTA scratch and the global tensors.
+template <int DK, int DV>
+struct BwdChunk {
+    using L = BSmem<DK, DV>;
+    using SC = Scratch<DK>;
+    static constexpr int TM_BYTES = 2 * C * C * 2, U_BYTES = C * DV * 2, I_BYTES = TM_BYTES + U_BYTES;
+
+    const ChunkBwdArgs &a;
+    IntraShared<DK> &sh;
+    float (*s_dpart)[DK];  // [NTHR / (DK / 2)][DK] segment sums of dL
+    float *s_dmd;          // [C] diagonal of dO U^T
+    float (*s_rs)[DK];     // [2][DK] row sums of dSigma . Sigma (two column halves)
+    int tid, warp, lane, b, h, T, H, nchunks;
+    ChunkTiles st;
+    bf16 *dO16, *S16, *D16, *T16, *M16, *dU16, *U16, *nR16, *dM16, *dA16;
+    float *A32, *T32;
+    float *LAM, *DQT, *DGT, *DKB, *PQ, *PG, *PK, *PL;
+    const bf16 *states, *gq, *gk, *gb, *gv, *gw;
+    const unsigned char *intra;
+
+    __device__ BwdChunk(const ChunkBwdArgs &args, unsigned char *smem, IntraShared<DK> &sh_, float (*dpart)[DK],
+                        float *dmd, float (*rs)[DK])
+        : a(args), sh(sh_), s_dpart(dpart), s_dmd(dmd), s_rs(rs) {
+        tid = threadIdx.x; warp = tid >> 5; lane = tid & 31;
+        const int bh = blockIdx.x;
+        b = bh / a.H; h = bh % a.H; T = a.T; H = a.H;
+        nchunks = (T + C - 1) / C;
+        st = ChunkTiles{reinterpret_cast<bf16 *>(smem + L::OQ), reinterpret_cast<bf16 *>(smem + L::OK),
+                        reinterpret_cast<bf16 *>(smem + L::OLA), reinterpret_cast<bf16 *>(smem + L::OB),
+                        reinterpret_cast<bf16 *>(smem + L::OV), reinterpret_cast<bf16 *>(smem + L::OW)};
+        dO16 = reinterpret_cast<bf16 *>(smem + L::ODO);
+        S16 = reinterpret_cast<bf16 *>(smem + L::OS);
+        D16 = reinterpret_cast<bf16 *>(smem + L::OD);
+        A32 = reinterpret_cast<float *>(smem + L::OAT);
+        T32 = A32 + C * C;
+        T16 = reinterpret_cast<bf16 *>(T32);
+        M16 = T16 + C * C;
+        dU16 = reinterpret_cast<bf16 *>(A32);
+        U16 = st.w;   // the forward's U
+        nR16 = st.v;
+        dM16 = reinterpret_cast<bf16 *>(L::AM_IN_K ? smem + L::OK : smem + L::OAM);
+        dA16 = dM16 + C * C;
+        float *scr = a.scratch + (size_t)bh * a.scr_stride;
+        LAM = scr + SC::LAM * SC::TILE; DQT = scr + SC::DQT * SC::TILE; DGT = scr + SC::DGT * SC::TILE;
+        DKB = scr + SC::DKB * SC::TILE;
+        PQ = scr + SC::PQ * SC::TILE; PG = scr + SC::PG * SC::TILE; PK = scr + SC::PK * SC::TILE;
+        PL = scr + SC::PL * SC::TILE;
+        if (L::STAGE_REUSE) {
+            DQT = reinterpret_cast<float *>(smem + L::OS);
+            DKB = reinterpret_cast<float *>(smem + L::OD);
+            DGT = reinterpret_cast<float *>(smem + L::OAT);
+        } else if (L::STAGE_DED) {
+            DQT = reinterpret_cast<float *>(smem + L::OSTG);
+            DKB = DQT + C * DK;
+            DGT = DKB + C * DK;
+        }
+        states = static_cast<const bf16 *>(a.states) + (size_t)bh * (nchunks + 1) * DK * DV;
+        intra = static_cast<const unsigned char *>(a.intra) + (size_t)bh * nchunks * I_BYTES;
+        gq = static_cast<const bf16 *>(a.q); gk = static_cast<const bf16 *>(a.k);
+        gb = static_cast<const bf16 *>(a.b); gv = static_cast<const bf16 *>(a.v);
+        gw = static_cast<const bf16 *>(a.w);
+    }
+
+    // Chunk n's tiles into shared memory (visible to all threads on return);
+    // the next chunk of the reverse walk is prefetched into L2.
+    __device__ void load(int n) {
+        // ---- loads: four token tiles, dO, the chunk-start state and the
+        // forward's T, M (into the WY-solve area) and U (into the w slot), which
+        // are stored as their shared-memory images
+        load_token_tile<DK>(st.q, gq, b, h, n, T, H);
+        load_token_tile<DK>(st.k, gk, b, h, n, T, H);
+        load_token_tile<DK>(st.la, static_cast<const bf16 *>(a.log_alpha), b, h, n, T, H);
+        load_token_tile<DK>(st.b, gb, b, h, n, T, H);
+        load_token_tile<DV>(dO16, static_cast<const bf16 *>(a.dO), b, h, n, T, H);
+        {
+            const bf16 *src = states + (size_t)n * DK * DV;
+            for (int id = tid; id < DK * DV / 8; id += NTHR) {
+                const int r = id / (DV / 8), ch = id % (DV / 8);
+                cp_async16(S16 + swz<DV, DK>(r, ch * 8), src + (size_t)r * DV + ch * 8, true);
+            }
+            const unsigned char *it = intra + (size_t)n * I_BYTES;
+            for (int id = tid; id < TM_BYTES / 16; id += NTHR)
+                cp_async16(reinterpret_cast<unsigned char *>(T16) + 16 * id, it + 16 * id, true);
+            for (int id = tid; id < U_BYTES / 16; id += NTHR)
+                cp_async16(reinterpret_cast<unsigned char *>(U16) + 16 * id, it + TM_BYTES + 16 * id, true);
+        }
+        cp_commit();
+        cp_wait<0>();
+        __syncthreads();
+        if (n > 0) {
+            // warm L2 with the next chunk of the reverse walk while this one computes
+            const int slot = tid & 63, grp = tid >> 6;
+            if (grp == 0) {
+                prefetch_token_rows_l2<DK>(gq, b, h, n - 1, T, H, slot, 64);
+                prefetch_token_rows_l2<DK>(gk, b, h, n - 1, T, H, slot, 64);
+            } else if (grp == 1) {
+                prefetch_token_rows_l2<DK>(static_cast<const bf16 *>(a.log_alpha), b, h, n - 1, T, H, slot, 64);
+                prefetch_token_rows_l2<DK>(gb, b, h, n - 1, T, H, slot, 64);
+            } else if (grp == 2) {
+                prefetch_token_rows_l2<DV>(gv, b, h, n - 1, T, H, slot, 64);
+                prefetch_token_rows_l2<DV>(gw, b, h, n - 1, T, H, slot, 64);
+            } else {
+                prefetch_token_rows_l2<DV>(static_cast<const bf16 *>(a.dO), b, h, n - 1, T, H, slot, 64);
+                if (slot < 16) {
+                    const bf16 *sp = states + (size_t)(n - 1) * DK * DV + (size_t)slot * (DK * DV / 16);
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(sp), "r"(DK * DV * 2 / 16)
+                                 : "memory");
+                } else if (slot < 32) {
+                    const unsigned char *ip = intra + (size_t)(n - 1) * I_BYTES + (size_t)(slot - 16) * (I_BYTES / 16);
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(ip), "r"(I_BYTES / 16)
+                                 : "memory");
+                }
+            }
+        }
+
+    }
+
+    // Slow chunk: the Gram gradients term by term into the scratch tiles PQ,
+    // PG, PK, PL (dM16 and dA16 hold the masked dO U^T and nR U^T).
+    __device__ void slow_grams(int n, int Cn) {
+        const int ch = tid % DK, seg = tid / DK;
+        if (seg == 0) {
+            for (int r = 0; r < C; ++r) {
+                PQ[r * DK + ch] = 0.f; PG[r * DK + ch] = 0.f; PK[r * DK + ch] = 0.f; PL[r * DK + ch] = 0.f;
+            }
+            for (int r = 0; r < Cn; ++r) {
+                const size_t orr = (((size_t)b * T + n * C + r) * H + h) * DK + ch;
+                const float qr = __bfloat162float(gq[orr]);
+                const float gr = __bfloat162float(gb[orr]) * __bfloat162float(gk[orr]);
+                const float lr = LAM[r * DK + ch];
+                float pq = 0.f, pg = 0.f, pl = 0.f;
+                for (int i = 0; i <= r; ++i) {
+                    const size_t oi = (((size_t)b * T + n * C + i) * H + h) * DK + ch;
+                    const float ki = __bfloat162float(gk[oi]);
+                    const float e = __expf(lr - LAM[i * DK + ch]);
+                    const float wA = i < r ? __bfloat162float(dA16[swz<64>(r, i)]) * e : 0.f;
+                    const float wM = __bfloat162float(dM16[swz<64>(r, i)]) * e;
+                    pg += wA * ki;
+                    pq += wM * ki;
+                    const float tk = wA * gr + wM * qr;
+                    PK[i * DK + ch] += tk;
+                    const float tl = tk * ki;
+                    pl += tl;
+                    PL[i * DK + ch] -= tl;
+                }
+                PQ[r * DK + ch] += pq;
+                PG[r * DK + ch] += pg;
+                PL[r * DK + ch] += pl;
+            }
+        }
+        __syncthreads();
+    }
+
+    // dv, dw from the bf16 -dRHS tile nR16, then dq, dk, db and dlog_alpha from
+    // the fp32 staging tiles DQT, DGT, DKB (and PQ.. for a slow chunk).
+    __device__ void token_grads(int n, int Cn, bool slow) {
+        // ---- elementwise gradients and the in-chunk reverse cumulative sum
+        // (two key channels per thread, rows split into P2 segments)
+        {
+            constexpr int NP = DK / 2, P2 = NTHR / NP, RS2 = C / P2;
+            const int cp = tid % NP, s2 = tid / NP, c2 = 2 * cp;
+            const float2 lend = slow ? *reinterpret_cast<const float2 *>(LAM + (Cn - 1) * DK + c2)
+                                     : make_float2(0.f, 0.f);
+            const float2 rs0 = make_float2(s_rs[0][c2], s_rs[0][c2 + 1]);
+            const float2 rs1 = make_float2(s_rs[1][c2], s_rs[1][c2 + 1]);
+            // dv = dRHS . w, dw = dRHS . v from the bf16 -dRHS tile, 16-byte coalesced;
+            // every global load of the pass is issued before the first use
+            {
+                constexpr int NV = C * DV / 8 / NTHR;
+                uint4 v8[NV], w8[NV];
+#pragma unroll
+                for (int it = 0; it < NV; ++it) {
+                    const int id = tid + it * NTHR, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
+                    const size_t o = (((size_t)b * T + n * C + min(r, Cn - 1)) * H + h) * DV + j;
+                    v8[it] = *reinterpret_cast<const uint4 *>(gv + o);
+                    w8[it] = *reinterpret_cast<const uint4 *>(gw + o);
+                }
+#pragma unroll
+                for (int it = 0; it < NV; ++it) {
+                    const int id = tid + it * NTHR, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
+                    if (r < Cn) {
+                        const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV + j;
+                        const uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, j));
+                        const __nv_bfloat162 *n2 = reinterpret_cast<const __nv_bfloat162 *>(&nr);
+                        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&v8[it]);
+                        const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w8[it]);
+                        uint4 dv8, dw8;
+                        uint32_t *dvp = reinterpret_cast<uint32_t *>(&dv8), *dwp = reinterpret_cast<uint32_t *>(&dw8);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 d = __bfloat1622float2(n2[e]), vv = __bfloat1622float2(v2[e]),
+                                         ww = __bfloat1622float2(w2[e]);
+                            dvp[e] = pack_bf16(-d.x * ww.x, -d.y * ww.y);
+                            dwp[e] = pack_bf16(-d.x * vv.x, -d.y * vv.y);
+                        }
+                        *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dv) + o) = dv8;
+                        *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dw) + o) = dw8;
+                    }
+                }
+            }
+            // in-chunk decay prefix of this thread's rows (the prep's segment sums,
+            // or the slow chunk's L in the workspace)
+            float la_run = 0.f, lb_run = 0.f;
+#pragma unroll
+            for (int s = 0; s < P2; ++s)
+                if (s < s2) { la_run += sh.part[s][c2]; lb_run += sh.part[s][c2 + 1]; }
+            const bf16 *gla = static_cast<const bf16 *>(a.log_alpha);
+            bf16 *__restrict__ gdq = static_cast<bf16 *>(a.dq);
+            bf16 *__restrict__ gdk = static_cast<bf16 *>(a.dk);
+            bf16 *__restrict__ gdb = static_cast<bf16 *>(a.db);
+            const float *__restrict__ sQT = DQT;
+            const float *__restrict__ sGT = DGT;
+            const float *__restrict__ sKB = DKB;
+            __nv_bfloat162 rq[RS2], rk[RS2], rb[RS2], rl[RS2];
+#pragma unroll
+            for (int i = 0; i < RS2; ++i) {
+                const int r = min(s2 * RS2 + i, Cn - 1);
+                const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c2;
+                rq[i] = *reinterpret_cast<const __nv_bfloat162 *>(gq + o);
+                rk[i] = *reinterpret_cast<const __nv_bfloat162 *>(gk + o);
+                rb[i] = *reinterpret_cast<const __nv_bfloat162 *>(gb + o);
+                rl[i] = *reinterpret_cast<const __nv_bfloat162 *>(gla + o);
+            }
+            float dla_r[RS2], dlb_r[RS2];
+            float pa = 0.f, pb = 0.f;
+#pragma unroll
+            for (int i = 0; i < RS2; ++i) {
+                const int r = s2 * RS2 + i;
+                dla_r[i] = 0.f;
+                dlb_r[i] = 0.f;
+                if (r < Cn) {
+                    const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c2;
+                    const float2 q = __bfloat1622float2(rq[i]);
+                    const float2 kk = __bfloat1622float2(rk[i]);
+                    const float2 bb = __bfloat1622float2(rb[i]);
+                    float2 lam;
+                    if (!slow) {
+                        const float2 l = __bfloat1622float2(rl[i]);
+                        la_run += l.x;
+                        lb_run += l.y;
+                        lam = make_float2(la_run, lb_run);
+                    } else {
+                        lam = *reinterpret_cast<const float2 *>(LAM + r * DK + c2);
+                    }
+                    const float2 dqt = *reinterpret_cast<const float2 *>(sQT + stg<DK>(r, c2));
+                    const float2 dgt = *reinterpret_cast<const float2 *>(sGT + stg<DK>(r, c2));
+                    const float2 dkb = *reinterpret_cast<const float2 *>(sKB + stg<DK>(r, c2));
+                    const float mdiag = s_dmd[r];
+                    const float ea = __expf(lam.x), eb = __expf(lam.y);
+                    float dqa, dqb, dga, dgb, dka, dkb2, dla, dlb;
+                    if (!slow) {
+                        const float iea = __expf(-lam.x), ieb = __expf(-lam.y);
+                        dqa = dqt.x * ea; dqb = dqt.y * eb;
+                        dga = dgt.x * ea; dgb = dgt.y * eb;
+                        dka = dkb.x * iea; dkb2 = dkb.y * ieb;
+                        dla = dqt.x * q.x * ea + dgt.x * bb.x * kk.x * ea - dkb.x * kk.x * iea;
+                        dlb = dqt.y * q.y * eb + dgt.y * bb.y * kk.y * eb - dkb.y * kk.y * ieb;
+                    } else {
+                        const float kea = __expf(lend.x - lam.x), keb = __expf(lend.y - lam.y);
+                        const float2 pq = *reinterpret_cast<const float2 *>(PQ + r * DK + c2);
+                        const float2 pg = *reinterpret_cast<const float2 *>(PG + r * DK + c2);
+                        const float2 pk = *reinterpret_cast<const float2 *>(PK + r * DK + c2);
+                        const float2 pl = *reinterpret_cast<const float2 *>(PL + r * DK + c2);
+                        dqa = dqt.x * ea + pq.x; dqb = dqt.y * eb + pq.y;
+                        dga = dgt.x * ea + pg.x; dgb = dgt.y * eb + pg.y;
+                        dka = dkb.x * kea + pk.x; dkb2 = dkb.y * keb + pk.y;
+                        dla = dqt.x * q.x * ea + dgt.x * bb.x * kk.x * ea - dkb.x * kk.x * kea + pl.x;
+                        dlb = dqt.y * q.y * eb + dgt.y * bb.y * kk.y * eb - dkb.y * kk.y * keb + pl.y;
+                    }
+                    dqa += mdiag * kk.x; dqb += mdiag * kk.y;
+                    dka += mdiag * q.x; dkb2 += mdiag * q.y;
+                    if (r == Cn - 1) { dla += rs0.x + rs1.x; dlb += rs0.y + rs1.y; }
+                    *reinterpret_cast<uint32_t *>(gdq + o) = pack_bf16(dqa, dqb);
+                    *reinterpret_cast<uint32_t *>(gdk + o) = pack_bf16(dka + dga * bb.x, dkb2 + dgb * bb.y);
+                    *reinterpret_cast<uint32_t *>(gdb + o) = pack_bf16(dga * kk.x, dgb * kk.y);
+                    dla_r[i] = dla;
+                    dlb_r[i] = dlb;
+                    pa += dla;
+                    pb += dlb;
+                }
+            }
+            s_dpart[s2][c2] = pa;
+            s_dpart[s2][c2 + 1] = pb;
+            __syncthreads();
+            float acca = 0.f, accb = 0.f;
+#pragma unroll
+            for (int s = 0; s < P2; ++s)
+                if (s > s2) { acca += s_dpart[s][c2]; accb += s_dpart[s][c2 + 1]; }
+#pragma unroll
+            for (int i = RS2 - 1; i >= 0; --i) {
+                const int r = s2 * RS2 + i;
+                if (r < Cn) {
+                    acca += dla_r[i];
+                    accb += dlb_r[i];
+                    *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dlog_alpha) +
+                                                  (((size_t)b * T + n * C + r) * H + h) * DK + c2) =
+                        pack_bf16(acca, accb);
+                }
+            }
+        }
+    }
+};
+
+}  // namespace cbwd
+}  // namespace gdn2

@@ -1,0 +1,336 @@
+// Reverse chunk pass of the backward for dk = dv = 128 with every chunk
+// product on the fifth-generation tensor cores (tcgen05, accumulators in
+// tensor memory).
+//
+// Same algebra as chunk_bwd.cu ("Why NVIDIA Gated DeltaNet-2 separates erase
+// and write gates", section "Gated Delta Rule-2: per-channel erase/write
+// split"; the gradients of the WY form follow from the laonpeople Gated
+// DeltaNet page's chunk equations).  Tensor memory (512 columns x 128 lanes)
+// holds, per CTA:
+//   cols   0..127  R_A: dO U^T (0..63), nR U^T (64..127), then dQt
+//   cols 128..255  R_B: -nR = T^T dU, then dGt
+//   cols 256..383  R_C: dU, then dKb
+//   cols 384..511  R_S: dSigma (128 key rows x 128 value columns, fp32)
+// One thread issues four groups of MMAs per chunk; after each group the warps
+// read the results back (16x256b shape for the 64-row products, which lands
+// in the register layout of a warp-level m16n8 fragment; 32x32b rows for
+// dSigma), form the next bf16 operands in shared memory, and hand over:
+//   M1  dU = M^T dO + Kx D ;  dO U^T ;  dSigma += Qt^T dO      (D = g . dSigma)
+//   M2  T^T dU
+//   M3  nR U^T ;  dGt = nR S^T ;  dKb = U D^T ;  dSigma += Gt^T nR
+//   M4  dQt = dO S^T (+ dM Kb) ;  dGt += dA Kb ;  dKb += dA^T Gt + dM^T Qt
+// (the Gram terms in M4 only on a fast chunk; a slow chunk takes them term by
+// term in fp32, as in chunk_bwd.cu).  dQt, dGt and dKb then go to the fp32
+// staging tiles and the token-level gradients follow (chunk_bwd_common.cuh).
+// Every wait on the MMA completion barrier is bounded: on expiry the kernel
+// records GDN2_ERR_TIMEOUT in the device status word, frees its tensor memory
+// and returns.
+#include "chunk_bwd_common.cuh"
+#include "gdn2.h"
+#include "tc.cuh"
+
+namespace gdn2 {
+namespace cbwd_tc {
+
+using namespace chunk;
+using cbwd::BSmem;
+using cbwd::BwdChunk;
+
+constexpr int D = 128;
+using L = BSmem<D, D>;
+constexpr int BYTES = L::BYTES + 1024;  // + room to align the tiles to 1 KB
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t COL_A = 0, COL_B = 128, COL_C = 256, COL_S = 384;
+// instruction descriptors: shape, then the majorness of A and B (MN = the
+// operand is stored with its M (or N) index along the rows' contiguous axis)
+constexpr uint32_t ID64x128_MN_MN = tc::idesc_bf16(64, 128, true, true);
+constexpr uint32_t ID64x128_K_MN = tc::idesc_bf16(64, 128, false, true);
+constexpr uint32_t ID64x128_K_K = tc::idesc_bf16(64, 128, false, false);
+constexpr uint32_t ID64x64_K_K = tc::idesc_bf16(64, 64, false, false);
+constexpr uint32_t ID128x128_MN_MN = tc::idesc_bf16(128, 128, true, true);
+
+// Operand descriptors of a swizzled [R][64 k] tile (chunk_common.cuh's swz):
+// k-step s (16 elements) of a K-major operand (rows = M or N, columns = K) ...
+__device__ __forceinline__ uint64_t kmaj(const void *tile, int R, int s) {
+    return tc::sdesc(tc::smem_addr(tile) + (uint32_t)((s >> 2) * (R * 128) + (s & 3) * 32), 16, 1024);
+}
+// ... and of an MN-major operand (rows = K, columns = M or N).
+__device__ __forceinline__ uint64_t mnmaj(const void *tile, int R, int s) {
+    return tc::sdesc(tc::smem_addr(tile) + (uint32_t)(s * 2048), (uint32_t)(R * 128), 1024);
+}
+
+// D (+)= A B over K = 16 ks, issued by one thread.  A_K / B_K: K-major operand.
+template <bool A_K, bool B_K>
+__device__ __forceinline__ void mma_tiles(uint32_t d, const void *A, int RA, const void *B, int RB, int ks,
+                                          uint32_t idesc, bool accumulate) {
+    for (int s = 0; s < ks; ++s) {
+        const uint64_t da = A_K ? kmaj(A, RA, s) : mnmaj(A, RA, s);
+        const uint64_t db = B_K ? kmaj(B, RB, s) : mnmaj(B, RB, s);
+        tc::mma_bf16(d, da, db, idesc, accumulate || s > 0);
+    }
+}
+
+// A 64-column fragment read with ld_16x256b_x8, as a warp-level [1][8][4] tile.
+using Frag = float[1][8][4];
+__device__ __forceinline__ void ld_frag(uint32_t taddr, Frag &f) {
+    tc::ld_16x256b_x8(taddr, reinterpret_cast<float(&)[32]>(f));
+}
+
+// bf16 store of a fragment (rows m0.., columns n0..) into a swizzled [.][DC] tile.
+template <int DC>
+__device__ __forceinline__ void store_frag_bf16(const Frag &f, bf16 *dst, int m0, int n0, int lane, float scale) {
+    const int r = m0 + (lane >> 2);
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+        const int c = n0 + 8 * nt + 2 * (lane & 3);
+        *reinterpret_cast<uint32_t *>(dst + swz<DC>(r, c)) = pack_bf16(scale * f[0][nt][0], scale * f[0][nt][1]);
+        *reinterpret_cast<uint32_t *>(dst + swz<DC>(r + 8, c)) = pack_bf16(scale * f[0][nt][2], scale * f[0][nt][3]);
+    }
+}
+
+__global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u);
+    __shared__ IntraShared<D> sh;
+    __shared__ float s_dpart[NTHR / (D / 2)][D];
+    __shared__ float s_dmd[C];
+    __shared__ float s_rs[2][D];
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
+
+    BwdChunk<D, D> x(a, smem, sh, s_dpart, s_dmd, s_rs);
+    const int tid = x.tid, warp = x.warp, lane = x.lane, bh = blockIdx.x;
+    const ChunkTiles st = x.st;
+
+    if (warp == 0) tc::tmem_alloc(&tmem_slot, kTmemCols);
+    if (tid == 0) {
+        tc::mbar_init(&mbar, 1);
+        tc::fence_mbar_init();
+        abort_flag = 0;
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = tmem_slot;
+
+    // Thread <-> dSigma row c = 32 p + lane of sub-partition p; warps p and
+    // p + 4 take the column halves hc = 0, 1.  For the 64-row products the
+    // same warp reads rows 16 p .. 16 p + 15, columns 64 hc .. 64 hc + 63.
+    const int p = warp & 3, hc = warp >> 2, c = 32 * p + lane;
+    const uint32_t lane_base = (uint32_t)(32 * p) << 16;
+    const uint32_t t_srow = tmem + lane_base + COL_S + 64 * hc;
+
+    {  // dSigma of the last chunk end = dS_T (or zero)
+        float v[64];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float4 y = a.dS_T ? reinterpret_cast<const float4 *>(a.dS_T + (size_t)bh * D * D + (size_t)c * D +
+                                                                       64 * hc)[i]
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * i] = y.x; v[4 * i + 1] = y.y; v[4 * i + 2] = y.z; v[4 * i + 3] = y.w;
+        }
+        tc::st_32x32b_x32(t_srow, *reinterpret_cast<const float(*)[32]>(&v[0]));
+        tc::st_32x32b_x32(t_srow + 32, *reinterpret_cast<const float(*)[32]>(&v[32]));
+        tc::wait_st();
+    }
+
+    uint32_t phase = 0;
+    // Commit the MMAs issued so far and wait for them (all threads); false on timeout.
+    auto mma_done = [&]() {
+        if (tid == 0) tc::commit(&mbar);
+        if (!tc::mbar_wait(&mbar, phase)) {
+            abort_flag = 1;
+            record_status(a.status, GDN2_ERR_TIMEOUT);
+        }
+        phase ^= 1;
+        tc::fence_after();
+    };
+    // Shared-memory operands written by the threads -> visible to the tensor
+    // cores, and everybody's tensor-memory accesses ordered before the next MMA.
+    auto handoff = [&]() {
+        tc::fence_async_smem();
+        tc::fence_before();
+        __syncthreads();
+        tc::fence_after();
+    };
+
+    for (int n = x.nchunks - 1; n >= 0; --n) {
+        const int Cn = min(C, a.T - n * C);
+        x.load(n);
+        const bool slow = intra_chunk<D, D>(st, x.A32, x.T32, sh, x.LAM, false, /*prep_only=*/true);
+
+        // ---- E0: D = g . dSigma (g = gam on a fast chunk, else 1) as bf16;
+        // row sums of dSigma . Sigma for dL_end; dSigma <- gam . dSigma
+        {
+            float v[64];
+            tc::ld_32x32b_x32(t_srow, *reinterpret_cast<float(*)[32]>(&v[0]));
+            tc::ld_32x32b_x32(t_srow + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+            tc::wait_ld();
+            const float gm = sh.gamma[c], g = slow ? 1.f : gm;
+            bf16 *row = x.D16 + hc * (D * 64) + c * 64;
+            const uint4 *sig = reinterpret_cast<const uint4 *>(x.states + (size_t)(n + 1) * D * D + (size_t)c * D +
+                                                               64 * hc);
+            float rs = 0.f;
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8) {
+                uint4 u;
+                u.x = pack_bf16(g * v[8 * q8 + 0], g * v[8 * q8 + 1]);
+                u.y = pack_bf16(g * v[8 * q8 + 2], g * v[8 * q8 + 3]);
+                u.z = pack_bf16(g * v[8 * q8 + 4], g * v[8 * q8 + 5]);
+                u.w = pack_bf16(g * v[8 * q8 + 6], g * v[8 * q8 + 7]);
+                *reinterpret_cast<uint4 *>(row + ((q8 ^ (c & 7)) << 3)) = u;
+                const uint4 sv = sig[q8];
+                const __nv_bfloat162 *s2 = reinterpret_cast<const __nv_bfloat162 *>(&sv);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(s2[e]);
+                    rs += v[8 * q8 + 2 * e] * f.x + v[8 * q8 + 2 * e + 1] * f.y;
+                }
+            }
+            s_rs[hc][c] = rs;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] *= gm;
+            tc::st_32x32b_x32(t_srow, *reinterpret_cast<const float(*)[32]>(&v[0]));
+            tc::st_32x32b_x32(t_srow + 32, *reinterpret_cast<const float(*)[32]>(&v[32]));
+            tc::wait_st();
+        }
+        handoff();
+
+        // ---- M1: dU = M^T dO + Kx D ; dO U^T ; dSigma += Qt^T dO
+        if (tid == 0) {
+            mma_tiles<false, false>(tmem + COL_C, x.M16, 64, x.dO16, 64, 4, ID64x128_MN_MN, false);
+            mma_tiles<true, false>(tmem + COL_C, st.la, 64, x.D16, D, 8, ID64x128_K_MN, true);
+            mma_tiles<true, true>(tmem + COL_A, x.dO16, 64, x.U16, 64, 8, ID64x64_K_K, false);
+            mma_tiles<false, false>(tmem + COL_S, st.q, 64, x.dO16, 64, 4, ID128x128_MN_MN, true);
+        }
+        mma_done();
+        // ---- E1: dU -> bf16 (all warps, column halves) ; dM = strict_lower(dO U^T) with
+        // its diagonal kept aside in fp32 (warps 0..3)
+        {
+            Frag f;
+            ld_frag(tmem + lane_base + COL_C + 64 * hc, f);
+            tc::wait_ld();
+            store_frag_bf16<D>(f, x.dU16, 16 * p, 64 * hc, lane, 1.f);
+            if (hc == 0) {
+                ld_frag(tmem + lane_base + COL_A, f);
+                tc::wait_ld();
+                const int r0 = 16 * p + (lane >> 2);
+#pragma unroll
+                for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        // The diagonal of M carries no decay factor: its gradient goes
+                        // straight to dq and dk in fp32 and stays out of the Gram products.
+                        const int r = r0 + (e >> 1) * 8, i = 8 * nt + 2 * (lane & 3) + (e & 1);
+                        if (i == r) s_dmd[r] = f[0][nt][e];
+                        if (i >= r) f[0][nt][e] = 0.f;
+                    }
+                store_frag_bf16<64>(f, x.dM16, 16 * p, 0, lane, 1.f);
+            }
+        }
+        handoff();
+        if (abort_flag) break;
+
+        // ---- M2: T^T dU
+        if (tid == 0) mma_tiles<false, false>(tmem + COL_B, x.T16, 64, x.dU16, 64, 4, ID64x128_MN_MN, false);
+        mma_done();
+        // ---- E2: nR = -T^T dU -> bf16
+        {
+            Frag f;
+            ld_frag(tmem + lane_base + COL_B + 64 * hc, f);
+            tc::wait_ld();
+            store_frag_bf16<D>(f, x.nR16, 16 * p, 64 * hc, lane, -1.f);
+        }
+        handoff();
+        if (abort_flag) break;
+
+        // ---- M3: nR U^T ; dGt = nR S^T ; dKb = U D^T ; dSigma += Gt^T nR
+        if (tid == 0) {
+            mma_tiles<true, true>(tmem + COL_A + 64, x.nR16, 64, x.U16, 64, 8, ID64x64_K_K, false);
+            mma_tiles<true, true>(tmem + COL_B, x.nR16, 64, x.S16, D, 8, ID64x128_K_K, false);
+            mma_tiles<true, true>(tmem + COL_C, x.U16, 64, x.D16, D, 8, ID64x128_K_K, false);
+            mma_tiles<false, false>(tmem + COL_S, st.b, 64, x.nR16, 64, 4, ID128x128_MN_MN, true);
+        }
+        mma_done();
+        // ---- E3: dA = strict_lower(nR U^T) -> bf16 (warps 0..3)
+        if (hc == 0) {
+            Frag f;
+            ld_frag(tmem + lane_base + COL_A + 64, f);
+            tc::wait_ld();
+            const int r0 = 16 * p + (lane >> 2);
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = r0 + (e >> 1) * 8, i = 8 * nt + 2 * (lane & 3) + (e & 1);
+                    if (i >= r) f[0][nt][e] = 0.f;
+                }
+            store_frag_bf16<64>(f, x.dA16, 16 * p, 0, lane, 1.f);
+        }
+        handoff();
+        if (abort_flag) break;
+
+        // ---- M4: dQt = dO S^T (+ dM Kb) ; dGt += dA Kb ; dKb += dA^T Gt + dM^T Qt
+        if (tid == 0) {
+            mma_tiles<true, true>(tmem + COL_A, x.dO16, 64, x.S16, D, 8, ID64x128_K_K, false);
+            if (!slow) {
+                mma_tiles<true, false>(tmem + COL_A, x.dM16, 64, st.la, 64, 4, ID64x128_K_MN, true);
+                mma_tiles<true, false>(tmem + COL_B, x.dA16, 64, st.la, 64, 4, ID64x128_K_MN, true);
+                mma_tiles<false, false>(tmem + COL_C, x.dA16, 64, st.b, 64, 4, ID64x128_MN_MN, true);
+                mma_tiles<false, false>(tmem + COL_C, x.dM16, 64, st.q, 64, 4, ID64x128_MN_MN, true);
+            }
+        }
+        mma_done();
+        // ---- E4: dQt, dGt, dKb -> fp32 staging (the S, D and T/M/dU regions are dead)
+        {
+            Frag f;
+            ld_frag(tmem + lane_base + COL_A + 64 * hc, f);
+            tc::wait_ld();
+            cbwd::store_stage<D, 8>(f, x.DQT, 16 * p, 64 * hc, lane);
+            ld_frag(tmem + lane_base + COL_B + 64 * hc, f);
+            tc::wait_ld();
+            cbwd::store_stage<D, 8>(f, x.DGT, 16 * p, 64 * hc, lane);
+            ld_frag(tmem + lane_base + COL_C + 64 * hc, f);
+            tc::wait_ld();
+            cbwd::store_stage<D, 8>(f, x.DKB, 16 * p, 64 * hc, lane);
+        }
+        tc::fence_before();
+        __syncthreads();
+        if (abort_flag) break;
+
+        if (slow) x.slow_grams(n, Cn);
+        x.token_grads(n, Cn, slow);
+        __syncthreads();
+    }
+
+    if (a.dS0 && !abort_flag) {
+        tc::fence_after();
+        float v[64];
+        tc::ld_32x32b_x32(t_srow, *reinterpret_cast<float(*)[32]>(&v[0]));
+        tc::ld_32x32b_x32(t_srow + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+        tc::wait_ld();
+        float4 *dst = reinterpret_cast<float4 *>(a.dS0 + (size_t)bh * D * D + (size_t)c * D + 64 * hc);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace cbwd_tc
+
+cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs &a, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(cbwd_tc::chunk_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         cbwd_tc::BYTES);
+    if (e != cudaSuccess) return e;
+    cbwd_tc::chunk_bwd_tc_kernel<<<(unsigned)(a.B * a.H), chunk::NTHR, cbwd_tc::BYTES, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn2

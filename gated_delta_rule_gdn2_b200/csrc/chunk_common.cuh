@@ -157,19 +157,6 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[1][NT][4], bf
     }
 }
 
-// Writes a 16-row accumulator tile as fp32 into a plain row-major [.][ld] array.
-template <int NT>
-__device__ __forceinline__ void store_tile_f32(const float (&acc)[1][NT][4], float *dst, int ld, int m0,
-                                               int lane) {
-    const int r = m0 + (lane >> 2);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int c = 8 * nt + 2 * (lane & 3);
-        *reinterpret_cast<float2 *>(dst + r * ld + c) = make_float2(acc[0][nt][0], acc[0][nt][1]);
-        *reinterpret_cast<float2 *>(dst + (r + 8) * ld + c) = make_float2(acc[0][nt][2], acc[0][nt][3]);
-    }
-}
-
 // cp.async of rows [n*C, n*C + C) of a token tensor [B,T,H,D] (head h of
 // batch b) into a swizzled [C][D] tile; rows past T are zero-filled.
 template <int D>

@@ -79,6 +79,7 @@ inline size_t intra_region_bytes(int B, int T, int H, int dv) {
     return ((size_t)B * H * nc * intra_tile_bytes(dv) + 255) / 256 * 256;
 }
 
+cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs &a, cudaStream_t s);  // reverse pass, dk = dv = 128, tcgen05
 cudaError_t launch_chunk_bwd(const ChunkBwdArgs &a, int dk, int dv, cudaStream_t s);
 size_t chunk_bwd_ws_bytes(int B, int T, int H, int dk, int dv, size_t *scr_stride, size_t *states_bytes);
 
