@@ -130,58 +130,75 @@ struct BwdChunk {
         gw = static_cast<const bf16 *>(a.w);
     }
 
-    // Chunk n's tiles into shared memory (visible to all threads on return);
-    // the next chunk of the reverse walk is prefetched into L2.
-    __device__ void load(int n) {
-        // ---- loads: four token tiles, dO, the chunk-start state and the
-        // forward's T, M (into the WY-solve area) and U (into the w slot), which
-        // are stored as their shared-memory images
+    // Chunk n's tiles are loaded in two cp.async groups, each committed:
+    // group A = the four token tiles, dO and the forward's U (into the w slot);
+    // group B = the chunk-start state and the forward's T, M (into the WY-solve
+    // area).  The forward's tiles are stored as their shared-memory images.
+    __device__ void issue_a(int n) {
         load_token_tile<DK>(st.q, gq, b, h, n, T, H);
         load_token_tile<DK>(st.k, gk, b, h, n, T, H);
         load_token_tile<DK>(st.la, static_cast<const bf16 *>(a.log_alpha), b, h, n, T, H);
         load_token_tile<DK>(st.b, gb, b, h, n, T, H);
         load_token_tile<DV>(dO16, static_cast<const bf16 *>(a.dO), b, h, n, T, H);
-        {
-            const bf16 *src = states + (size_t)n * DK * DV;
-            for (int id = tid; id < DK * DV / 8; id += NTHR) {
-                const int r = id / (DV / 8), ch = id % (DV / 8);
-                cp_async16(S16 + swz<DV, DK>(r, ch * 8), src + (size_t)r * DV + ch * 8, true);
-            }
-            const unsigned char *it = intra + (size_t)n * I_BYTES;
-            for (int id = tid; id < TM_BYTES / 16; id += NTHR)
-                cp_async16(reinterpret_cast<unsigned char *>(T16) + 16 * id, it + 16 * id, true);
-            for (int id = tid; id < U_BYTES / 16; id += NTHR)
-                cp_async16(reinterpret_cast<unsigned char *>(U16) + 16 * id, it + TM_BYTES + 16 * id, true);
-        }
+        const unsigned char *it = intra + (size_t)n * I_BYTES + TM_BYTES;
+        for (int id = tid; id < U_BYTES / 16; id += NTHR)
+            cp_async16(reinterpret_cast<unsigned char *>(U16) + 16 * id, it + 16 * id, true);
         cp_commit();
+    }
+    __device__ void issue_b(int n) {
+        const bf16 *src = states + (size_t)n * DK * DV;
+        for (int id = tid; id < DK * DV / 8; id += NTHR) {
+            const int r = id / (DV / 8), ch = id % (DV / 8);
+            cp_async16(S16 + swz<DV, DK>(r, ch * 8), src + (size_t)r * DV + ch * 8, true);
+        }
+        const unsigned char *it = intra + (size_t)n * I_BYTES;
+        for (int id = tid; id < TM_BYTES / 16; id += NTHR)
+            cp_async16(reinterpret_cast<unsigned char *>(T16) + 16 * id, it + 16 * id, true);
+        cp_commit();
+    }
+    // Warm L2 with chunk n of the reverse walk.
+    __device__ void prefetch_l2(int n) {
+        const int slot = tid & 63, grp = tid >> 6;
+        if (grp == 0) {
+            prefetch_token_rows_l2<DK>(gq, b, h, n, T, H, slot, 64);
+            prefetch_token_rows_l2<DK>(gk, b, h, n, T, H, slot, 64);
+        } else if (grp == 1) {
+            prefetch_token_rows_l2<DK>(static_cast<const bf16 *>(a.log_alpha), b, h, n, T, H, slot, 64);
+            prefetch_token_rows_l2<DK>(gb, b, h, n, T, H, slot, 64);
+        } else if (grp == 2) {
+            prefetch_token_rows_l2<DV>(gv, b, h, n, T, H, slot, 64);
+            prefetch_token_rows_l2<DV>(gw, b, h, n, T, H, slot, 64);
+        } else {
+            prefetch_token_rows_l2<DV>(static_cast<const bf16 *>(a.dO), b, h, n, T, H, slot, 64);
+            if (slot < 16) {
+                const bf16 *sp = states + (size_t)n * DK * DV + (size_t)slot * (DK * DV / 16);
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(sp), "r"(DK * DV * 2 / 16)
+                             : "memory");
+            } else if (slot < 32) {
+                const unsigned char *ip = intra + (size_t)n * I_BYTES + (size_t)(slot - 16) * (I_BYTES / 16);
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(ip), "r"(I_BYTES / 16)
+                             : "memory");
+            }
+        }
+    }
+    // Warm L2 with the rows of v and w of chunk n, which the dv/dw pass reads
+    // straight from global memory (one 128-byte line per thread).
+    __device__ void prefetch_vw_l2(int n) {
+        const int t = n * C + ((tid >> 1) & (C - 1));
+        if (t >= T) return;
+        const bf16 *src = (tid < 2 * C) ? gv : gw;
+        const bf16 *row = src + (((size_t)b * T + t) * H + h) * DV;
+        if ((tid & 1) * 64 < DV)
+            asm volatile("prefetch.global.L2 [%0];\n" ::"l"(row + (tid & 1) * 64) : "memory");
+    }
+    // All of chunk n's tiles, visible to all threads on return; the next chunk
+    // of the reverse walk is prefetched into L2.
+    __device__ void load(int n) {
+        issue_a(n);
+        issue_b(n);
         cp_wait<0>();
         __syncthreads();
-        if (n > 0) {
-            // warm L2 with the next chunk of the reverse walk while this one computes
-            const int slot = tid & 63, grp = tid >> 6;
-            if (grp == 0) {
-                prefetch_token_rows_l2<DK>(gq, b, h, n - 1, T, H, slot, 64);
-                prefetch_token_rows_l2<DK>(gk, b, h, n - 1, T, H, slot, 64);
-            } else if (grp == 1) {
-                prefetch_token_rows_l2<DK>(static_cast<const bf16 *>(a.log_alpha), b, h, n - 1, T, H, slot, 64);
-                prefetch_token_rows_l2<DK>(gb, b, h, n - 1, T, H, slot, 64);
-            } else if (grp == 2) {
-                prefetch_token_rows_l2<DV>(gv, b, h, n - 1, T, H, slot, 64);
-                prefetch_token_rows_l2<DV>(gw, b, h, n - 1, T, H, slot, 64);
-            } else {
-                prefetch_token_rows_l2<DV>(static_cast<const bf16 *>(a.dO), b, h, n - 1, T, H, slot, 64);
-                if (slot < 16) {
-                    const bf16 *sp = states + (size_t)(n - 1) * DK * DV + (size_t)slot * (DK * DV / 16);
-                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(sp), "r"(DK * DV * 2 / 16)
-                                 : "memory");
-                } else if (slot < 32) {
-                    const unsigned char *ip = intra + (size_t)(n - 1) * I_BYTES + (size_t)(slot - 16) * (I_BYTES / 16);
-                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(ip), "r"(I_BYTES / 16)
-                                 : "memory");
-                }
-            }
-        }
-
+        if (n > 0) prefetch_l2(n - 1);
     }
 
     // Slow chunk: the Gram gradients term by term into the scratch tiles PQ,

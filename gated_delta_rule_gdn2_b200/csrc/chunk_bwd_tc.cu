@@ -71,6 +71,18 @@ __device__ __forceinline__ void mma_tiles(uint32_t d, const void *A, int RA, con
     }
 }
 
+// sum_e v[e] * y[e] over 8 fp32 values and 8 packed bf16 values
+__device__ __forceinline__ float dot8(const float *v, uint4 y) {
+    const __nv_bfloat162 *y2 = reinterpret_cast<const __nv_bfloat162 *>(&y);
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(y2[e]);
+        acc += v[2 * e] * f.x + v[2 * e + 1] * f.y;
+    }
+    return acc;
+}
+
 // A 64-column fragment read with ld_16x256b_x8, as a warp-level [1][8][4] tile.
 using Frag = float[1][8][4];
 __device__ __forceinline__ void ld_frag(uint32_t taddr, Frag &f) {
@@ -95,12 +107,12 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
     __shared__ IntraShared<D> sh;
     __shared__ float s_dpart[NTHR / (D / 2)][D];
     __shared__ float s_dmd[C];
-    __shared__ float s_rs[2][D];
+    __shared__ float s_rs[2][2][D];  // by chunk parity: row sums of dSigma . Sigma (two column halves)
     __shared__ uint64_t mbar;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
-    BwdChunk<D, D> x(a, smem, sh, s_dpart, s_dmd, s_rs);
+    BwdChunk<D, D> x(a, smem, sh, s_dpart, s_dmd, s_rs[0]);
     const int tid = x.tid, warp = x.warp, lane = x.lane, bh = blockIdx.x;
     const ChunkTiles st = x.st;
 
@@ -156,13 +168,21 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
         tc::fence_after();
     };
 
+    // Loads run one chunk ahead: group A of chunk n - 1 (token tiles, dO, U)
+    // lands while chunk n's token-level gradients are formed, group B (S, T, M)
+    // while chunk n - 1's decay prep and E0 run.
+    x.issue_a(x.nchunks - 1);
+    x.issue_b(x.nchunks - 1);
     for (int n = x.nchunks - 1; n >= 0; --n) {
         const int Cn = min(C, a.T - n * C);
-        x.load(n);
+        cp_wait<1>();
+        __syncthreads();
+        if (n > 0) x.prefetch_vw_l2(n - 1);
         const bool slow = intra_chunk<D, D>(st, x.A32, x.T32, sh, x.LAM, false, /*prep_only=*/true);
 
-        // ---- E0: D = g . dSigma (g = gam on a fast chunk, else 1) as bf16;
-        // row sums of dSigma . Sigma for dL_end; dSigma <- gam . dSigma
+        // ---- E0: D = g . dSigma (g = gam on a fast chunk, else 1) as bf16 and
+        // dSigma <- gam . dSigma; on the last chunk also the row sums of
+        // dSigma . Sigma (Sigma = the final state) for dL_end
         {
             float v[64];
             tc::ld_32x32b_x32(t_srow, *reinterpret_cast<float(*)[32]>(&v[0]));
@@ -170,9 +190,6 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
             tc::wait_ld();
             const float gm = sh.gamma[c], g = slow ? 1.f : gm;
             bf16 *row = x.D16 + hc * (D * 64) + c * 64;
-            const uint4 *sig = reinterpret_cast<const uint4 *>(x.states + (size_t)(n + 1) * D * D + (size_t)c * D +
-                                                               64 * hc);
-            float rs = 0.f;
 #pragma unroll
             for (int q8 = 0; q8 < 8; ++q8) {
                 uint4 u;
@@ -181,21 +198,22 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
                 u.z = pack_bf16(g * v[8 * q8 + 4], g * v[8 * q8 + 5]);
                 u.w = pack_bf16(g * v[8 * q8 + 6], g * v[8 * q8 + 7]);
                 *reinterpret_cast<uint4 *>(row + ((q8 ^ (c & 7)) << 3)) = u;
-                const uint4 sv = sig[q8];
-                const __nv_bfloat162 *s2 = reinterpret_cast<const __nv_bfloat162 *>(&sv);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(s2[e]);
-                    rs += v[8 * q8 + 2 * e] * f.x + v[8 * q8 + 2 * e + 1] * f.y;
-                }
             }
-            s_rs[hc][c] = rs;
+            if (n == x.nchunks - 1) {
+                const uint4 *sig = reinterpret_cast<const uint4 *>(x.states + (size_t)(n + 1) * D * D +
+                                                                   (size_t)c * D + 64 * hc);
+                float rs = 0.f;
+#pragma unroll
+                for (int q8 = 0; q8 < 8; ++q8) rs += dot8(v + 8 * q8, sig[q8]);
+                s_rs[n & 1][hc][c] = rs;
+            }
 #pragma unroll
             for (int i = 0; i < 64; ++i) v[i] *= gm;
             tc::st_32x32b_x32(t_srow, *reinterpret_cast<const float(*)[32]>(&v[0]));
             tc::st_32x32b_x32(t_srow + 32, *reinterpret_cast<const float(*)[32]>(&v[32]));
             tc::wait_st();
         }
+        cp_wait<0>();  // group B: S, T, M
         handoff();
 
         // ---- M1: dU = M^T dO + Kx D ; dO U^T ; dSigma += Qt^T dO
@@ -254,6 +272,20 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
             mma_tiles<false, false>(tmem + COL_S, st.b, 64, x.nR16, 64, 4, ID128x128_MN_MN, true);
         }
         mma_done();
+        // ---- row sums of dSigma . Sigma for chunk n - 1: dSigma is now its
+        // chunk-end gradient and Sigma = this chunk's start state S
+        if (n > 0) {
+            float v[64];
+            tc::ld_32x32b_x32(t_srow, *reinterpret_cast<float(*)[32]>(&v[0]));
+            tc::ld_32x32b_x32(t_srow + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+            tc::wait_ld();
+            const bf16 *srow = x.S16 + hc * (D * 64) + c * 64;
+            float rs = 0.f;
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8)
+                rs += dot8(v + 8 * q8, *reinterpret_cast<const uint4 *>(srow + ((q8 ^ (c & 7)) << 3)));
+            s_rs[(n - 1) & 1][hc][c] = rs;
+        }
         // ---- E3: dA = strict_lower(nR U^T) -> bf16 (warps 0..3)
         if (hc == 0) {
             Frag f;
@@ -301,9 +333,13 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
         if (abort_flag) break;
 
         if (slow) x.slow_grams(n, Cn);
+        if (n > 0) x.issue_a(n - 1);  // the token, dO and U slots are free now
+        x.s_rs = s_rs[n & 1];
         x.token_grads(n, Cn, slow);
         __syncthreads();
+        if (n > 0) x.issue_b(n - 1);  // the staging tiles in the S and T/M regions are consumed
     }
+    cp_wait<0>();
 
     if (a.dS0 && !abort_flag) {
         tc::fence_after();
