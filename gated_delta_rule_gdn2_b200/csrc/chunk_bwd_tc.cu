@@ -28,6 +28,7 @@
 #include "chunk_bwd_common.cuh"
 #include "gdn2.h"
 #include "tc.cuh"
+#include "tma_host.h"
 
 namespace gdn2 {
 namespace cbwd_tc {
@@ -38,6 +39,13 @@ using cbwd::BwdChunk;
 
 constexpr int D = 128;
 using L = BSmem<D, D>;
+constexpr int TILE_BYTES = C * D * 2;
+constexpr int TM_BYTES = 2 * C * C * 2;
+
+// TMA tensor maps of the token tensors and of the saved chunk-boundary states.
+struct BwdMaps {
+    CUtensorMap q, k, la, b, dO, S;
+};
 constexpr int BYTES = L::BYTES + 1024;  // + room to align the tiles to 1 KB
 
 constexpr uint32_t kTmemCols = 512;
@@ -101,7 +109,7 @@ __device__ __forceinline__ void store_frag_bf16(const Frag &f, bf16 *dst, int m0
     }
 }
 
-__global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
+__global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, const __grid_constant__ BwdMaps maps) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u);
     __shared__ IntraShared<D> sh;
@@ -109,6 +117,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
     __shared__ float s_dmd[C];
     __shared__ float s_rs[2][2][D];  // by chunk parity: row sums of dSigma . Sigma (two column halves)
     __shared__ uint64_t mbar;
+    __shared__ uint64_t mbar_ld[2];  // load groups A and B
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -119,6 +128,8 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
     if (warp == 0) tc::tmem_alloc(&tmem_slot, kTmemCols);
     if (tid == 0) {
         tc::mbar_init(&mbar, 1);
+        tc::mbar_init(&mbar_ld[0], 1);
+        tc::mbar_init(&mbar_ld[1], 1);
         tc::fence_mbar_init();
         abort_flag = 0;
     }
@@ -168,15 +179,52 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
         tc::fence_after();
     };
 
-    // Loads run one chunk ahead: group A of chunk n - 1 (token tiles, dO, U)
-    // lands while chunk n's token-level gradients are formed, group B (S, T, M)
-    // while chunk n - 1's decay prep and E0 run.
-    x.issue_a(x.nchunks - 1);
-    x.issue_b(x.nchunks - 1);
+    // Tile loads, issued by one thread through the TMA and counted in bytes on
+    // mbar_ld: group A = the four token tiles and dO (64 x 64 boxes of the
+    // tensor maps, two per tile) and the forward's U (a bulk copy of its
+    // shared-memory image); group B = the chunk-start state (two 64-column
+    // boxes) and the forward's T, M (bulk).  They run one chunk ahead: group A
+    // of chunk n - 1 lands while chunk n's token-level gradients are formed,
+    // group B while chunk n - 1's decay prep and E0 run.
+    uint32_t ph_ld[2] = {0, 0};
+    auto issue_a = [&](int m) {
+        tc::mbar_expect_tx(&mbar_ld[0], 6 * TILE_BYTES);
+        const unsigned char *img = x.intra + (size_t)m * x.I_BYTES + TM_BYTES;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int cx = 64 * half, off = half * C * 64;
+            tc::tma_load_4d(st.q + off, &maps.q, cx, x.h, m * C, x.b, &mbar_ld[0]);
+            tc::tma_load_4d(st.k + off, &maps.k, cx, x.h, m * C, x.b, &mbar_ld[0]);
+            tc::tma_load_4d(st.la + off, &maps.la, cx, x.h, m * C, x.b, &mbar_ld[0]);
+            tc::tma_load_4d(st.b + off, &maps.b, cx, x.h, m * C, x.b, &mbar_ld[0]);
+            tc::tma_load_4d(x.dO16 + off, &maps.dO, cx, x.h, m * C, x.b, &mbar_ld[0]);
+        }
+        tc::bulk_load(x.U16, img, TILE_BYTES, &mbar_ld[0]);
+    };
+    auto issue_b = [&](int m) {
+        tc::mbar_expect_tx(&mbar_ld[1], D * D * 2 + TM_BYTES);
+        const int row = (bh * (x.nchunks + 1) + m) * D;
+        tc::tma_load_2d(x.S16, &maps.S, 0, row, &mbar_ld[1]);
+        tc::tma_load_2d(x.S16 + D * 64, &maps.S, 64, row, &mbar_ld[1]);
+        tc::bulk_load(x.T16, x.intra + (size_t)m * x.I_BYTES, TM_BYTES, &mbar_ld[1]);
+    };
+    auto wait_loads = [&](int g) {
+        if (!tc::mbar_wait(&mbar_ld[g], ph_ld[g])) {
+            abort_flag = 1;
+            record_status(a.status, GDN2_ERR_TIMEOUT);
+        }
+        ph_ld[g] ^= 1;
+    };
+
+    if (tid == 0) {
+        issue_a(x.nchunks - 1);
+        issue_b(x.nchunks - 1);
+    }
     for (int n = x.nchunks - 1; n >= 0; --n) {
         const int Cn = min(C, a.T - n * C);
-        cp_wait<1>();
+        wait_loads(0);
         __syncthreads();
+        if (abort_flag) break;
         if (n > 0) x.prefetch_vw_l2(n - 1);
         const bool slow = intra_chunk<D, D>(st, x.A32, x.T32, sh, x.LAM, false, /*prep_only=*/true);
 
@@ -213,8 +261,9 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
             tc::st_32x32b_x32(t_srow + 32, *reinterpret_cast<const float(*)[32]>(&v[32]));
             tc::wait_st();
         }
-        cp_wait<0>();  // group B: S, T, M
+        wait_loads(1);  // group B: S, T, M
         handoff();
+        if (abort_flag) break;
 
         // ---- M1: dU = M^T dO + Kx D ; dO U^T ; dSigma += Qt^T dO
         if (tid == 0) {
@@ -328,18 +377,24 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
             tc::wait_ld();
             cbwd::store_stage<D, 8>(f, x.DKB, 16 * p, 64 * hc, lane);
         }
+        // (every generic access of a tile is fenced against the TMA before it is refilled)
+        tc::fence_async_smem();
         tc::fence_before();
         __syncthreads();
         if (abort_flag) break;
 
-        if (slow) x.slow_grams(n, Cn);
-        if (n > 0) x.issue_a(n - 1);  // the token, dO and U slots are free now
+        if (slow) {
+            x.slow_grams(n, Cn);
+            tc::fence_async_smem();
+            __syncthreads();
+        }
+        if (n > 0 && tid == 0) issue_a(n - 1);  // the token, dO and U slots are free now
         x.s_rs = s_rs[n & 1];
         x.token_grads(n, Cn, slow);
+        tc::fence_async_smem();
         __syncthreads();
-        if (n > 0) x.issue_b(n - 1);  // the staging tiles in the S and T/M regions are consumed
+        if (n > 0 && tid == 0) issue_b(n - 1);  // the staging tiles in the S and T/M regions are consumed
     }
-    cp_wait<0>();
 
     if (a.dS0 && !abort_flag) {
         tc::fence_after();
@@ -362,10 +417,19 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a) {
 }  // namespace cbwd_tc
 
 cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs &a, cudaStream_t s) {
+    cbwd_tc::BwdMaps m;
+    const uint64_t state_rows = (uint64_t)a.B * a.H * ((a.T + chunk::C - 1) / chunk::C + 1) * cbwd_tc::D;
+    if (!token_tensor_map(&m.q, a.q, a.B, a.T, a.H, cbwd_tc::D) ||
+        !token_tensor_map(&m.k, a.k, a.B, a.T, a.H, cbwd_tc::D) ||
+        !token_tensor_map(&m.la, a.log_alpha, a.B, a.T, a.H, cbwd_tc::D) ||
+        !token_tensor_map(&m.b, a.b, a.B, a.T, a.H, cbwd_tc::D) ||
+        !token_tensor_map(&m.dO, a.dO, a.B, a.T, a.H, cbwd_tc::D) ||
+        !matrix_tensor_map(&m.S, a.states, state_rows, cbwd_tc::D, cbwd_tc::D))
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(cbwd_tc::chunk_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          cbwd_tc::BYTES);
     if (e != cudaSuccess) return e;
-    cbwd_tc::chunk_bwd_tc_kernel<<<(unsigned)(a.B * a.H), chunk::NTHR, cbwd_tc::BYTES, s>>>(a);
+    cbwd_tc::chunk_bwd_tc_kernel<<<(unsigned)(a.B * a.H), chunk::NTHR, cbwd_tc::BYTES, s>>>(a, m);
     return cudaGetLastError();
 }
 
