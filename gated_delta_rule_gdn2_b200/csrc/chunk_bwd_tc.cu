@@ -42,9 +42,9 @@ using L = BSmem<D, D>;
 constexpr int TILE_BYTES = C * D * 2;
 constexpr int TM_BYTES = 2 * C * C * 2;
 
-// TMA tensor maps of the token tensors and of the saved chunk-boundary states.
+// TMA tensor maps of the token tensors.
 struct BwdMaps {
-    CUtensorMap q, k, la, b, dO, S;
+    CUtensorMap q, k, la, b, dO;
 };
 constexpr int BYTES = L::BYTES + 1024;  // + room to align the tiles to 1 KB
 
@@ -181,9 +181,9 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, c
 
     // Tile loads, issued by one thread through the TMA and counted in bytes on
     // mbar_ld: group A = the four token tiles and dO (64 x 64 boxes of the
-    // tensor maps, two per tile) and the forward's U (a bulk copy of its
-    // shared-memory image); group B = the chunk-start state (two 64-column
-    // boxes) and the forward's T, M (bulk).  They run one chunk ahead: group A
+    // tensor maps, two per tile) and the forward's U; group B = the chunk-start
+    // state and the forward's T, M.  The forward stores U, T, M and the states
+    // as images of their shared-memory tiles, which come back as bulk copies.  They run one chunk ahead: group A
     // of chunk n - 1 lands while chunk n's token-level gradients are formed,
     // group B while chunk n - 1's decay prep and E0 run.
     uint32_t ph_ld[2] = {0, 0};
@@ -203,9 +203,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, c
     };
     auto issue_b = [&](int m) {
         tc::mbar_expect_tx(&mbar_ld[1], D * D * 2 + TM_BYTES);
-        const int row = (bh * (x.nchunks + 1) + m) * D;
-        tc::tma_load_2d(x.S16, &maps.S, 0, row, &mbar_ld[1]);
-        tc::tma_load_2d(x.S16 + D * 64, &maps.S, 64, row, &mbar_ld[1]);
+        tc::bulk_load(x.S16, x.states + (size_t)m * D * D, D * D * 2, &mbar_ld[1]);
         tc::bulk_load(x.T16, x.intra + (size_t)m * x.I_BYTES, TM_BYTES, &mbar_ld[1]);
     };
     auto wait_loads = [&](int g) {
@@ -248,11 +246,11 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, c
                 *reinterpret_cast<uint4 *>(row + ((q8 ^ (c & 7)) << 3)) = u;
             }
             if (n == x.nchunks - 1) {
-                const uint4 *sig = reinterpret_cast<const uint4 *>(x.states + (size_t)(n + 1) * D * D +
-                                                                   (size_t)c * D + 64 * hc);
+                const bf16 *sig = x.states + (size_t)(n + 1) * D * D + hc * (D * 64) + c * 64;
                 float rs = 0.f;
 #pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8) rs += dot8(v + 8 * q8, sig[q8]);
+                for (int q8 = 0; q8 < 8; ++q8)
+                    rs += dot8(v + 8 * q8, *reinterpret_cast<const uint4 *>(sig + ((q8 ^ (c & 7)) << 3)));
                 s_rs[n & 1][hc][c] = rs;
             }
 #pragma unroll
@@ -418,13 +416,11 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, c
 
 cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs &a, cudaStream_t s) {
     cbwd_tc::BwdMaps m;
-    const uint64_t state_rows = (uint64_t)a.B * a.H * ((a.T + chunk::C - 1) / chunk::C + 1) * cbwd_tc::D;
     if (!token_tensor_map(&m.q, a.q, a.B, a.T, a.H, cbwd_tc::D) ||
         !token_tensor_map(&m.k, a.k, a.B, a.T, a.H, cbwd_tc::D) ||
         !token_tensor_map(&m.la, a.log_alpha, a.B, a.T, a.H, cbwd_tc::D) ||
         !token_tensor_map(&m.b, a.b, a.B, a.T, a.H, cbwd_tc::D) ||
-        !token_tensor_map(&m.dO, a.dO, a.B, a.T, a.H, cbwd_tc::D) ||
-        !matrix_tensor_map(&m.S, a.states, state_rows, cbwd_tc::D, cbwd_tc::D))
+        !token_tensor_map(&m.dO, a.dO, a.B, a.T, a.H, cbwd_tc::D))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(cbwd_tc::chunk_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          cbwd_tc::BYTES);

@@ -23,6 +23,7 @@
 #include "gdn2.h"
 #include "launch.h"
 #include "tc.cuh"
+#include "tma_host.h"
 
 namespace gdn2 {
 namespace cfwd_tc {
@@ -38,6 +39,7 @@ constexpr int OSMALL = OS16 + D * D * 2;
 struct Small {
     IntraShared<D> intra;
     uint64_t mbar[2];
+    uint64_t mbar_ld[2];  // tile loads of stage 0 and 1
     uint32_t tmem;
     int abort;
 };
@@ -56,17 +58,28 @@ __device__ __forceinline__ ChunkTiles stage_tiles(unsigned char *smem, int s) {
             reinterpret_cast<bf16 *>(p + 5 * TILE)};
 }
 
-__device__ __forceinline__ void issue_chunk(const ChunkFwdArgs &a, ChunkTiles st, int b, int h, int n) {
-    load_token_tile<D>(st.q, static_cast<const bf16 *>(a.q), b, h, n, a.T, a.H);
-    load_token_tile<D>(st.k, static_cast<const bf16 *>(a.k), b, h, n, a.T, a.H);
-    load_token_tile<D>(st.la, static_cast<const bf16 *>(a.log_alpha), b, h, n, a.T, a.H);
-    load_token_tile<D>(st.b, static_cast<const bf16 *>(a.b), b, h, n, a.T, a.H);
-    load_token_tile<D>(st.v, static_cast<const bf16 *>(a.v), b, h, n, a.T, a.H);
-    load_token_tile<D>(st.w, static_cast<const bf16 *>(a.w), b, h, n, a.T, a.H);
-    cp_commit();
+// TMA tensor maps of the six token tensors.
+struct FwdMaps {
+    CUtensorMap q, k, la, b, v, w;
+};
+
+// Chunk n's six token tiles into a stage (one thread; 64 x 64 boxes, two per
+// tile), completion counted in bytes on the stage's mbarrier.
+__device__ __forceinline__ void issue_chunk(const FwdMaps &m, ChunkTiles st, int b, int h, int n, uint64_t *mbar) {
+    tc::mbar_expect_tx(mbar, 6 * TILE);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int cx = 64 * half, off = half * C * 64;
+        tc::tma_load_4d(st.q + off, &m.q, cx, h, n * C, b, mbar);
+        tc::tma_load_4d(st.k + off, &m.k, cx, h, n * C, b, mbar);
+        tc::tma_load_4d(st.la + off, &m.la, cx, h, n * C, b, mbar);
+        tc::tma_load_4d(st.b + off, &m.b, cx, h, n * C, b, mbar);
+        tc::tma_load_4d(st.v + off, &m.v, cx, h, n * C, b, mbar);
+        tc::tma_load_4d(st.w + off, &m.w, cx, h, n * C, b, mbar);
+    }
 }
 
-__global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
+__global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, const __grid_constant__ FwdMaps maps) {
     extern __shared__ __align__(1024) unsigned char smem[];
     Small &sm = *reinterpret_cast<Small *>(smem + OSMALL);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -87,6 +100,8 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
     if (tid == 0) {
         tc::mbar_init(&sm.mbar[0], 1);
         tc::mbar_init(&sm.mbar[1], 1);
+        tc::mbar_init(&sm.mbar_ld[0], 1);
+        tc::mbar_init(&sm.mbar_ld[1], 1);
         tc::fence_mbar_init();
         sm.abort = 0;
     }
@@ -100,13 +115,9 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
     const int p = warp & 3, hc = warp >> 2, c = 32 * p + lane;
     const uint32_t t_row = tmem + ((uint32_t)(32 * p) << 16) + COL_S + 64 * hc;
 
-    // bf16 copy of this thread's 64 state values into S16 (and the chunk-boundary
-    // state output when requested)
-    auto put_state = [&](const float (&v)[64], int n) {
+    // bf16 copy of this thread's 64 state values into S16
+    auto put_state = [&](const float (&v)[64]) {
         bf16 *row = S16 + hc * (D * 64) + c * 64;
-        bf16 *g = a.states ? static_cast<bf16 *>(a.states) + ((size_t)bh * (nchunks + 1) + n) * D * D +
-                                 (size_t)c * D + 64 * hc
-                           : nullptr;
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) {
             uint4 u;
@@ -115,7 +126,14 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
             u.z = pack_bf16(v[8 * q8 + 4], v[8 * q8 + 5]);
             u.w = pack_bf16(v[8 * q8 + 6], v[8 * q8 + 7]);
             *reinterpret_cast<uint4 *>(row + ((q8 ^ (c & 7)) << 3)) = u;
-            if (g) *reinterpret_cast<uint4 *>(g + 8 * q8) = u;
+        }
+    };
+    // The chunk-boundary state n (when requested) as the image of S16, by one
+    // thread after the writers' proxy fence and a barrier.
+    auto keep_state = [&](int n) {
+        if (a.states) {
+            tc::bulk_store(static_cast<bf16 *>(a.states) + ((size_t)bh * (nchunks + 1) + n) * D * D, S16, D * D * 2);
+            tc::bulk_commit();
         }
     };
     auto load_state = [&](float (&v)[64]) {
@@ -140,16 +158,18 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
             v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
         }
         store_state(v);
-        put_state(v, 0);
+        put_state(v);
     }
     tc::fence_async_smem();
     tc::fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        keep_state(0);
+        issue_chunk(maps, stage_tiles(smem, 0), b, h, 0, &sm.mbar_ld[0]);
+        if (nchunks > 1) issue_chunk(maps, stage_tiles(smem, 1), b, h, 1, &sm.mbar_ld[1]);
+    }
 
-    issue_chunk(a, stage_tiles(smem, 0), b, h, 0);
-    if (nchunks > 1) issue_chunk(a, stage_tiles(smem, 1), b, h, 1);
-    else cp_commit();
-
-    uint32_t ph0 = 0, ph1 = 0;
+    uint32_t ph0 = 0, ph1 = 0, ph_ld[2] = {0, 0};
     for (int n = 0; n < nchunks; ++n) {
         ChunkTiles st = stage_tiles(smem, n & 1);
         float *A32 = reinterpret_cast<float *>(st.k);  // k and w slots are free after the prep
@@ -159,12 +179,14 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
         bf16 *M16 = T16 + C * C;
         bf16 *U16 = st.v;                              // after Uv
 
-        cp_wait<1>();
+        if (!tc::mbar_wait(&sm.mbar_ld[n & 1], ph_ld[n & 1])) {
+            sm.abort = 1;
+            record_status(a.status, GDN2_ERR_TIMEOUT);
+        }
+        ph_ld[n & 1] ^= 1;
         __syncthreads();
         if (sm.abort) break;
         const bool slow = intra_chunk<D, D>(st, A32, T32, sm.intra, lam_ws, false);
-        // T and M (then U, below) for the backward, as their shared-memory images
-        if (a.intra) copy_smem_to_global(keep_tile(n), T16, 2 * C * C * 2);
 
         // ---- Uv = T WV (warps 0..3, registers) ; -W = -T Gt (warps 4..7, shared)
         float acc[1][16][4];
@@ -178,8 +200,13 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
         tc::fence_async_smem();
         __syncthreads();
 
-        // ---- D_W = -W S, D_Q = Qt S on the tensor cores
+        // ---- D_W = -W S, D_Q = Qt S on the tensor cores; T and M (and U,
+        // below) go out for the backward as their shared-memory images
         if (tid == 0) {
+            if (a.intra) {
+                tc::bulk_store(keep_tile(n), T16, 2 * C * C * 2);
+                tc::bulk_commit();
+            }
             tc::fence_after();
             const uint32_t sS = tc::smem_addr(S16), sW = tc::smem_addr(W16), sQ = tc::smem_addr(st.q);
 #pragma unroll
@@ -218,12 +245,16 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
                     for (int e = 0; e < 4; ++e) acc[0][nt][e] = d[4 * nt + e];
             }
         }
+        if (tid == 0) tc::bulk_wait_read();  // the previous state image is out: S16 may be rewritten below
         tc::fence_async_smem();
         tc::fence_before();
         __syncthreads();
         if (sm.abort) break;
 
-        if (a.intra) copy_smem_to_global(keep_tile(n) + 2 * C * C * 2, U16, C * D * 2);
+        if (tid == 0 && a.intra) {
+            tc::bulk_store(keep_tile(n) + 2 * C * C * 2, U16, C * D * 2);
+            tc::bulk_commit();
+        }
         // ---- slow chunk: S <- Diag(gam) S before adding Kt^T U
         if (slow) {
             float v[64];
@@ -279,15 +310,19 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
                 for (int i = 0; i < 64; ++i) v[i] *= gm;
                 store_state(v);
             }
-            put_state(v, n + 1);
+            put_state(v);
         }
         tc::fence_async_smem();
         tc::fence_before();
         __syncthreads();
-        if (n + 2 < nchunks) issue_chunk(a, st, b, h, n + 2);
-        else cp_commit();
+        if (tid == 0) {
+            // this stage's T, M and U images are out before the stage is refilled
+            tc::bulk_wait_read();
+            if (n + 2 < nchunks) issue_chunk(maps, st, b, h, n + 2, &sm.mbar_ld[n & 1]);
+            keep_state(n + 1);
+        }
     }
-    cp_wait<0>();
+    if (tid == 0) tc::bulk_wait();
     __syncthreads();
 
     if (a.S_T && !sm.abort) {
@@ -309,10 +344,16 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a) {
 }  // namespace cfwd_tc
 
 cudaError_t launch_chunk_fwd_tc(const ChunkFwdArgs &a, cudaStream_t s) {
+    cfwd_tc::FwdMaps m;
+    const int D = cfwd_tc::D;
+    if (!token_tensor_map(&m.q, a.q, a.B, a.T, a.H, D) || !token_tensor_map(&m.k, a.k, a.B, a.T, a.H, D) ||
+        !token_tensor_map(&m.la, a.log_alpha, a.B, a.T, a.H, D) || !token_tensor_map(&m.b, a.b, a.B, a.T, a.H, D) ||
+        !token_tensor_map(&m.v, a.v, a.B, a.T, a.H, D) || !token_tensor_map(&m.w, a.w, a.B, a.T, a.H, D))
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(cfwd_tc::chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          cfwd_tc::BYTES);
     if (e != cudaSuccess) return e;
-    cfwd_tc::chunk_fwd_tc_kernel<<<(unsigned)(a.B * a.H), chunk::NTHR, cfwd_tc::BYTES, s>>>(a);
+    cfwd_tc::chunk_fwd_tc_kernel<<<(unsigned)(a.B * a.H), chunk::NTHR, cfwd_tc::BYTES, s>>>(a, m);
     return cudaGetLastError();
 }
 

@@ -101,14 +101,6 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *map, int x, i
         "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(mbar))
         : "memory");
 }
-// Tiled box of a 2-D tensor map at coordinates (x, y), x innermost.
-__device__ __forceinline__ void tma_load_2d(void *dst, const void *map, int x, int y, uint64_t *mbar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];\n" ::"r"(smem_addr(dst)),
-        "l"(map), "r"(x), "r"(y), "r"(smem_addr(mbar))
-        : "memory");
-}
 // Contiguous copy (addresses 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *mbar) {
     asm volatile(
@@ -117,6 +109,21 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         "l"(src), "r"(bytes), "r"(smem_addr(mbar))
         : "memory");
 }
+
+// Contiguous store from shared to global memory in the current bulk group
+// (addresses 16-byte aligned, bytes a multiple of 16); the source must have
+// been written before a proxy fence and a barrier.
+__device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(gdst), "r"(smem_addr(ssrc)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+// Until the sources of every committed bulk store have been read (the shared
+// memory may then be overwritten) ...
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+// ... or until the stores are complete.
+__device__ __forceinline__ void bulk_wait() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 
 // Generic-proxy shared-memory writes -> visible to the tensor cores.
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
