@@ -68,17 +68,19 @@ __device__ __forceinline__ void store_stage(const float (&acc)[1][NT][4], float 
 
 // Per-CTA view of one (batch, head) sequence in the reverse chunk pass: the
 // shared-memory tiles, the caller's per-CTA scratch and the global tensors.
-template <int DK, int DV>
+// NT: threads of the CTA (256 or 512).
+template <int DK, int DV, int NT = NTHR>
 struct BwdChunk {
     using L = BSmem<DK, DV>;
     using SC = Scratch<DK>;
     static constexpr int TM_BYTES = 2 * C * C * 2, U_BYTES = C * DV * 2, I_BYTES = TM_BYTES + U_BYTES;
+    static constexpr int NRS = NT / 128;  // partial row sums of dSigma . Sigma (column parts)
 
     const ChunkBwdArgs &a;
-    IntraShared<DK> &sh;
-    float (*s_dpart)[DK];  // [NTHR / (DK / 2)][DK] segment sums of dL
+    IntraShared<DK, NT> &sh;
+    float (*s_dpart)[DK];  // [NT / (DK / 2)][DK] segment sums of dL
     float *s_dmd;          // [C] diagonal of dO U^T
-    float (*s_rs)[DK];     // [2][DK] row sums of dSigma . Sigma (two column halves)
+    float (*s_rs)[DK];     // [NRS][DK] row sums of dSigma . Sigma over NRS column parts
     int tid, warp, lane, b, h, T, H, nchunks;
     ChunkTiles st;
     bf16 *dO16, *S16, *D16, *T16, *M16, *dU16, *U16, *nR16, *dM16, *dA16;
@@ -87,7 +89,7 @@ struct BwdChunk {
     const bf16 *states, *gq, *gk, *gb, *gv, *gw;
     const unsigned char *intra;
 
-    __device__ BwdChunk(const ChunkBwdArgs &args, unsigned char *smem, IntraShared<DK> &sh_, float (*dpart)[DK],
+    __device__ BwdChunk(const ChunkBwdArgs &args, unsigned char *smem, IntraShared<DK, NT> &sh_, float (*dpart)[DK],
                         float *dmd, float (*rs)[DK])
         : a(args), sh(sh_), s_dpart(dpart), s_dmd(dmd), s_rs(rs) {
         tid = threadIdx.x; warp = tid >> 5; lane = tid & 31;
@@ -135,29 +137,30 @@ struct BwdChunk {
     // group B = the chunk-start state and the forward's T, M (into the WY-solve
     // area).  The forward's tiles are stored as their shared-memory images.
     __device__ void issue_a(int n) {
-        load_token_tile<DK>(st.q, gq, b, h, n, T, H);
-        load_token_tile<DK>(st.k, gk, b, h, n, T, H);
-        load_token_tile<DK>(st.la, static_cast<const bf16 *>(a.log_alpha), b, h, n, T, H);
-        load_token_tile<DK>(st.b, gb, b, h, n, T, H);
-        load_token_tile<DV>(dO16, static_cast<const bf16 *>(a.dO), b, h, n, T, H);
+        load_token_tile<DK, NT>(st.q, gq, b, h, n, T, H);
+        load_token_tile<DK, NT>(st.k, gk, b, h, n, T, H);
+        load_token_tile<DK, NT>(st.la, static_cast<const bf16 *>(a.log_alpha), b, h, n, T, H);
+        load_token_tile<DK, NT>(st.b, gb, b, h, n, T, H);
+        load_token_tile<DV, NT>(dO16, static_cast<const bf16 *>(a.dO), b, h, n, T, H);
         const unsigned char *it = intra + (size_t)n * I_BYTES + TM_BYTES;
-        for (int id = tid; id < U_BYTES / 16; id += NTHR)
+        for (int id = tid; id < U_BYTES / 16; id += NT)
             cp_async16(reinterpret_cast<unsigned char *>(U16) + 16 * id, it + 16 * id, true);
         cp_commit();
     }
     __device__ void issue_b(int n) {
         const bf16 *src = states + (size_t)n * DK * DV;
-        for (int id = tid; id < DK * DV / 8; id += NTHR) {
+        for (int id = tid; id < DK * DV / 8; id += NT) {
             const int r = id / (DV / 8), ch = id % (DV / 8);
             cp_async16(S16 + swz<DV, DK>(r, ch * 8), src + (size_t)r * DV + ch * 8, true);
         }
         const unsigned char *it = intra + (size_t)n * I_BYTES;
-        for (int id = tid; id < TM_BYTES / 16; id += NTHR)
+        for (int id = tid; id < TM_BYTES / 16; id += NT)
             cp_async16(reinterpret_cast<unsigned char *>(T16) + 16 * id, it + 16 * id, true);
         cp_commit();
     }
     // Warm L2 with chunk n of the reverse walk.
     __device__ void prefetch_l2(int n) {
+        if (tid >= 256) return;
         const int slot = tid & 63, grp = tid >> 6;
         if (grp == 0) {
             prefetch_token_rows_l2<DK>(gq, b, h, n, T, H, slot, 64);
@@ -185,7 +188,7 @@ struct BwdChunk {
     // straight from global memory (one 128-byte line per thread).
     __device__ void prefetch_vw_l2(int n) {
         const int t = n * C + ((tid >> 1) & (C - 1));
-        if (t >= T) return;
+        if (tid >= 4 * C || t >= T) return;
         const bf16 *src = (tid < 2 * C) ? gv : gw;
         const bf16 *row = src + (((size_t)b * T + t) * H + h) * DV;
         if ((tid & 1) * 64 < DV)
@@ -243,27 +246,31 @@ struct BwdChunk {
         // ---- elementwise gradients and the in-chunk reverse cumulative sum
         // (two key channels per thread, rows split into P2 segments)
         {
-            constexpr int NP = DK / 2, P2 = NTHR / NP, RS2 = C / P2;
+            constexpr int NP = DK / 2, P2 = NT / NP, RS2 = C / P2;
             const int cp = tid % NP, s2 = tid / NP, c2 = 2 * cp;
             const float2 lend = slow ? *reinterpret_cast<const float2 *>(LAM + (Cn - 1) * DK + c2)
                                      : make_float2(0.f, 0.f);
-            const float2 rs0 = make_float2(s_rs[0][c2], s_rs[0][c2 + 1]);
-            const float2 rs1 = make_float2(s_rs[1][c2], s_rs[1][c2 + 1]);
+            float2 rsum = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < NRS; ++i) {
+                rsum.x += s_rs[i][c2];
+                rsum.y += s_rs[i][c2 + 1];
+            }
             // dv = dRHS . w, dw = dRHS . v from the bf16 -dRHS tile, 16-byte coalesced;
             // every global load of the pass is issued before the first use
             {
-                constexpr int NV = C * DV / 8 / NTHR;
+                constexpr int NV = C * DV / 8 / NT;
                 uint4 v8[NV], w8[NV];
 #pragma unroll
                 for (int it = 0; it < NV; ++it) {
-                    const int id = tid + it * NTHR, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
+                    const int id = tid + it * NT, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
                     const size_t o = (((size_t)b * T + n * C + min(r, Cn - 1)) * H + h) * DV + j;
                     v8[it] = *reinterpret_cast<const uint4 *>(gv + o);
                     w8[it] = *reinterpret_cast<const uint4 *>(gw + o);
                 }
 #pragma unroll
                 for (int it = 0; it < NV; ++it) {
-                    const int id = tid + it * NTHR, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
+                    const int id = tid + it * NT, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
                     if (r < Cn) {
                         const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV + j;
                         const uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, j));
@@ -355,7 +362,7 @@ struct BwdChunk {
                     }
                     dqa += mdiag * kk.x; dqb += mdiag * kk.y;
                     dka += mdiag * q.x; dkb2 += mdiag * q.y;
-                    if (r == Cn - 1) { dla += rs0.x + rs1.x; dlb += rs0.y + rs1.y; }
+                    if (r == Cn - 1) { dla += rsum.x; dlb += rsum.y; }
                     *reinterpret_cast<uint32_t *>(gdq + o) = pack_bf16(dqa, dqb);
                     *reinterpret_cast<uint32_t *>(gdk + o) = pack_bf16(dka + dga * bb.x, dkb2 + dgb * bb.y);
                     *reinterpret_cast<uint32_t *>(gdb + o) = pack_bf16(dga * kk.x, dgb * kk.y);

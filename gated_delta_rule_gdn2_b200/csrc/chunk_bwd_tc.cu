@@ -38,7 +38,9 @@ using cbwd::BSmem;
 using cbwd::BwdChunk;
 
 constexpr int D = 128;
+constexpr int NT = 512;  // 16 warps: four per tensor-memory sub-partition
 using L = BSmem<D, D>;
+using Chunk = BwdChunk<D, D, NT>;
 constexpr int TILE_BYTES = C * D * 2;
 constexpr int TM_BYTES = 2 * C * C * 2;
 
@@ -91,10 +93,10 @@ __device__ __forceinline__ float dot8(const float *v, uint4 y) {
     return acc;
 }
 
-// A 64-column fragment read with ld_16x256b_x8, as a warp-level [1][8][4] tile.
-using Frag = float[1][8][4];
+// A 32-column fragment read with ld_16x256b_x4, as a warp-level [1][4][4] tile.
+using Frag = float[1][4][4];
 __device__ __forceinline__ void ld_frag(uint32_t taddr, Frag &f) {
-    tc::ld_16x256b_x8(taddr, reinterpret_cast<float(&)[32]>(f));
+    tc::ld_16x256b_x4(taddr, reinterpret_cast<float(&)[16]>(f));
 }
 
 // bf16 store of a fragment (rows m0.., columns n0..) into a swizzled [.][DC] tile.
@@ -102,26 +104,26 @@ template <int DC>
 __device__ __forceinline__ void store_frag_bf16(const Frag &f, bf16 *dst, int m0, int n0, int lane, float scale) {
     const int r = m0 + (lane >> 2);
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
+    for (int nt = 0; nt < 4; ++nt) {
         const int c = n0 + 8 * nt + 2 * (lane & 3);
         *reinterpret_cast<uint32_t *>(dst + swz<DC>(r, c)) = pack_bf16(scale * f[0][nt][0], scale * f[0][nt][1]);
         *reinterpret_cast<uint32_t *>(dst + swz<DC>(r + 8, c)) = pack_bf16(scale * f[0][nt][2], scale * f[0][nt][3]);
     }
 }
 
-__global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, const __grid_constant__ BwdMaps maps) {
+__global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, const __grid_constant__ BwdMaps maps) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u);
-    __shared__ IntraShared<D> sh;
-    __shared__ float s_dpart[NTHR / (D / 2)][D];
+    __shared__ IntraShared<D, NT> sh;
+    __shared__ float s_dpart[NT / (D / 2)][D];
     __shared__ float s_dmd[C];
-    __shared__ float s_rs[2][2][D];  // by chunk parity: row sums of dSigma . Sigma (two column halves)
+    __shared__ float s_rs[2][Chunk::NRS][D];  // by chunk parity: row sums of dSigma . Sigma (column quarters)
     __shared__ uint64_t mbar;
     __shared__ uint64_t mbar_ld[2];  // load groups A and B
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
-    BwdChunk<D, D> x(a, smem, sh, s_dpart, s_dmd, s_rs[0]);
+    Chunk x(a, smem, sh, s_dpart, s_dmd, s_rs[0]);
     const int tid = x.tid, warp = x.warp, lane = x.lane, bh = blockIdx.x;
     const ChunkTiles st = x.st;
 
@@ -138,24 +140,27 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, c
     tc::fence_after();
     const uint32_t tmem = tmem_slot;
 
-    // Thread <-> dSigma row c = 32 p + lane of sub-partition p; warps p and
-    // p + 4 take the column halves hc = 0, 1.  For the 64-row products the
-    // same warp reads rows 16 p .. 16 p + 15, columns 64 hc .. 64 hc + 63.
-    const int p = warp & 3, hc = warp >> 2, c = 32 * p + lane;
+    // Thread <-> dSigma row c = 32 p + lane of sub-partition p; warps p,
+    // p + 4, p + 8, p + 12 take the column quarters qc = 0..3.  For the 64-row
+    // products the same warp reads rows 16 p .. 16 p + 15, columns 32 qc ...
+    const int p = warp & 3, qc = warp >> 2, c = 32 * p + lane;
     const uint32_t lane_base = (uint32_t)(32 * p) << 16;
-    const uint32_t t_srow = tmem + lane_base + COL_S + 64 * hc;
+    const uint32_t t_srow = tmem + lane_base + COL_S + 32 * qc;
+    // this thread's 32 columns of a swizzled [128][128] bf16 tile row c, as 4 x 8
+    auto tile_row = [&](const bf16 *tile, int i) {
+        return tile + (qc >> 1) * (D * 64) + c * 64 + (((4 * (qc & 1) + i) ^ (c & 7)) << 3);
+    };
 
     {  // dSigma of the last chunk end = dS_T (or zero)
-        float v[64];
+        float v[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 8; ++i) {
             const float4 y = a.dS_T ? reinterpret_cast<const float4 *>(a.dS_T + (size_t)bh * D * D + (size_t)c * D +
-                                                                       64 * hc)[i]
+                                                                       32 * qc)[i]
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
             v[4 * i] = y.x; v[4 * i + 1] = y.y; v[4 * i + 2] = y.z; v[4 * i + 3] = y.w;
         }
-        tc::st_32x32b_x32(t_srow, *reinterpret_cast<const float(*)[32]>(&v[0]));
-        tc::st_32x32b_x32(t_srow + 32, *reinterpret_cast<const float(*)[32]>(&v[32]));
+        tc::st_32x32b_x32(t_srow, v);
         tc::wait_st();
     }
 
@@ -224,39 +229,35 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, c
         __syncthreads();
         if (abort_flag) break;
         if (n > 0) x.prefetch_vw_l2(n - 1);
-        const bool slow = intra_chunk<D, D>(st, x.A32, x.T32, sh, x.LAM, false, /*prep_only=*/true);
+        const bool slow = intra_chunk<D, D, NT>(st, x.A32, x.T32, sh, x.LAM, false, /*prep_only=*/true);
 
         // ---- E0: D = g . dSigma (g = gam on a fast chunk, else 1) as bf16 and
         // dSigma <- gam . dSigma; on the last chunk also the row sums of
         // dSigma . Sigma (Sigma = the final state) for dL_end
         {
-            float v[64];
-            tc::ld_32x32b_x32(t_srow, *reinterpret_cast<float(*)[32]>(&v[0]));
-            tc::ld_32x32b_x32(t_srow + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+            float v[32];
+            tc::ld_32x32b_x32(t_srow, v);
             tc::wait_ld();
             const float gm = sh.gamma[c], g = slow ? 1.f : gm;
-            bf16 *row = x.D16 + hc * (D * 64) + c * 64;
 #pragma unroll
-            for (int q8 = 0; q8 < 8; ++q8) {
+            for (int i = 0; i < 4; ++i) {
                 uint4 u;
-                u.x = pack_bf16(g * v[8 * q8 + 0], g * v[8 * q8 + 1]);
-                u.y = pack_bf16(g * v[8 * q8 + 2], g * v[8 * q8 + 3]);
-                u.z = pack_bf16(g * v[8 * q8 + 4], g * v[8 * q8 + 5]);
-                u.w = pack_bf16(g * v[8 * q8 + 6], g * v[8 * q8 + 7]);
-                *reinterpret_cast<uint4 *>(row + ((q8 ^ (c & 7)) << 3)) = u;
+                u.x = pack_bf16(g * v[8 * i + 0], g * v[8 * i + 1]);
+                u.y = pack_bf16(g * v[8 * i + 2], g * v[8 * i + 3]);
+                u.z = pack_bf16(g * v[8 * i + 4], g * v[8 * i + 5]);
+                u.w = pack_bf16(g * v[8 * i + 6], g * v[8 * i + 7]);
+                *reinterpret_cast<uint4 *>(const_cast<bf16 *>(tile_row(x.D16, i))) = u;
             }
             if (n == x.nchunks - 1) {
-                const bf16 *sig = x.states + (size_t)(n + 1) * D * D + hc * (D * 64) + c * 64;
+                const bf16 *sig = x.states + (size_t)(n + 1) * D * D;
                 float rs = 0.f;
 #pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8)
-                    rs += dot8(v + 8 * q8, *reinterpret_cast<const uint4 *>(sig + ((q8 ^ (c & 7)) << 3)));
-                s_rs[n & 1][hc][c] = rs;
+                for (int i = 0; i < 4; ++i) rs += dot8(v + 8 * i, *reinterpret_cast<const uint4 *>(tile_row(sig, i)));
+                s_rs[n & 1][qc][c] = rs;
             }
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] *= gm;
-            tc::st_32x32b_x32(t_srow, *reinterpret_cast<const float(*)[32]>(&v[0]));
-            tc::st_32x32b_x32(t_srow + 32, *reinterpret_cast<const float(*)[32]>(&v[32]));
+            for (int i = 0; i < 32; ++i) v[i] *= gm;
+            tc::st_32x32b_x32(t_srow, v);
             tc::wait_st();
         }
         wait_loads(1);  // group B: S, T, M
@@ -271,28 +272,28 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, c
             mma_tiles<false, false>(tmem + COL_S, st.q, 64, x.dO16, 64, 4, ID128x128_MN_MN, true);
         }
         mma_done();
-        // ---- E1: dU -> bf16 (all warps, column halves) ; dM = strict_lower(dO U^T) with
-        // its diagonal kept aside in fp32 (warps 0..3)
+        // ---- E1: dU -> bf16 (all warps, column quarters) ; dM = strict_lower(dO U^T)
+        // with its diagonal kept aside in fp32 (warps with qc < 2)
         {
             Frag f;
-            ld_frag(tmem + lane_base + COL_C + 64 * hc, f);
+            ld_frag(tmem + lane_base + COL_C + 32 * qc, f);
             tc::wait_ld();
-            store_frag_bf16<D>(f, x.dU16, 16 * p, 64 * hc, lane, 1.f);
-            if (hc == 0) {
-                ld_frag(tmem + lane_base + COL_A, f);
+            store_frag_bf16<D>(f, x.dU16, 16 * p, 32 * qc, lane, 1.f);
+            if (qc < 2) {
+                ld_frag(tmem + lane_base + COL_A + 32 * qc, f);
                 tc::wait_ld();
                 const int r0 = 16 * p + (lane >> 2);
 #pragma unroll
-                for (int nt = 0; nt < 8; ++nt)
+                for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         // The diagonal of M carries no decay factor: its gradient goes
                         // straight to dq and dk in fp32 and stays out of the Gram products.
-                        const int r = r0 + (e >> 1) * 8, i = 8 * nt + 2 * (lane & 3) + (e & 1);
+                        const int r = r0 + (e >> 1) * 8, i = 32 * qc + 8 * nt + 2 * (lane & 3) + (e & 1);
                         if (i == r) s_dmd[r] = f[0][nt][e];
                         if (i >= r) f[0][nt][e] = 0.f;
                     }
-                store_frag_bf16<64>(f, x.dM16, 16 * p, 0, lane, 1.f);
+                store_frag_bf16<64>(f, x.dM16, 16 * p, 32 * qc, lane, 1.f);
             }
         }
         handoff();
@@ -304,9 +305,9 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, c
         // ---- E2: nR = -T^T dU -> bf16
         {
             Frag f;
-            ld_frag(tmem + lane_base + COL_B + 64 * hc, f);
+            ld_frag(tmem + lane_base + COL_B + 32 * qc, f);
             tc::wait_ld();
-            store_frag_bf16<D>(f, x.nR16, 16 * p, 64 * hc, lane, -1.f);
+            store_frag_bf16<D>(f, x.nR16, 16 * p, 32 * qc, lane, -1.f);
         }
         handoff();
         if (abort_flag) break;
@@ -322,31 +323,28 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, c
         // ---- row sums of dSigma . Sigma for chunk n - 1: dSigma is now its
         // chunk-end gradient and Sigma = this chunk's start state S
         if (n > 0) {
-            float v[64];
-            tc::ld_32x32b_x32(t_srow, *reinterpret_cast<float(*)[32]>(&v[0]));
-            tc::ld_32x32b_x32(t_srow + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+            float v[32];
+            tc::ld_32x32b_x32(t_srow, v);
             tc::wait_ld();
-            const bf16 *srow = x.S16 + hc * (D * 64) + c * 64;
             float rs = 0.f;
 #pragma unroll
-            for (int q8 = 0; q8 < 8; ++q8)
-                rs += dot8(v + 8 * q8, *reinterpret_cast<const uint4 *>(srow + ((q8 ^ (c & 7)) << 3)));
-            s_rs[(n - 1) & 1][hc][c] = rs;
+            for (int i = 0; i < 4; ++i) rs += dot8(v + 8 * i, *reinterpret_cast<const uint4 *>(tile_row(x.S16, i)));
+            s_rs[(n - 1) & 1][qc][c] = rs;
         }
-        // ---- E3: dA = strict_lower(nR U^T) -> bf16 (warps 0..3)
-        if (hc == 0) {
+        // ---- E3: dA = strict_lower(nR U^T) -> bf16 (warps with qc < 2)
+        if (qc < 2) {
             Frag f;
-            ld_frag(tmem + lane_base + COL_A + 64, f);
+            ld_frag(tmem + lane_base + COL_A + 64 + 32 * qc, f);
             tc::wait_ld();
             const int r0 = 16 * p + (lane >> 2);
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
+            for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int r = r0 + (e >> 1) * 8, i = 8 * nt + 2 * (lane & 3) + (e & 1);
+                    const int r = r0 + (e >> 1) * 8, i = 32 * qc + 8 * nt + 2 * (lane & 3) + (e & 1);
                     if (i >= r) f[0][nt][e] = 0.f;
                 }
-            store_frag_bf16<64>(f, x.dA16, 16 * p, 0, lane, 1.f);
+            store_frag_bf16<64>(f, x.dA16, 16 * p, 32 * qc, lane, 1.f);
         }
         handoff();
         if (abort_flag) break;
@@ -365,15 +363,15 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, c
         // ---- E4: dQt, dGt, dKb -> fp32 staging (the S, D and T/M/dU regions are dead)
         {
             Frag f;
-            ld_frag(tmem + lane_base + COL_A + 64 * hc, f);
+            ld_frag(tmem + lane_base + COL_A + 32 * qc, f);
             tc::wait_ld();
-            cbwd::store_stage<D, 8>(f, x.DQT, 16 * p, 64 * hc, lane);
-            ld_frag(tmem + lane_base + COL_B + 64 * hc, f);
+            cbwd::store_stage<D, 4>(f, x.DQT, 16 * p, 32 * qc, lane);
+            ld_frag(tmem + lane_base + COL_B + 32 * qc, f);
             tc::wait_ld();
-            cbwd::store_stage<D, 8>(f, x.DGT, 16 * p, 64 * hc, lane);
-            ld_frag(tmem + lane_base + COL_C + 64 * hc, f);
+            cbwd::store_stage<D, 4>(f, x.DGT, 16 * p, 32 * qc, lane);
+            ld_frag(tmem + lane_base + COL_C + 32 * qc, f);
             tc::wait_ld();
-            cbwd::store_stage<D, 8>(f, x.DKB, 16 * p, 64 * hc, lane);
+            cbwd::store_stage<D, 4>(f, x.DKB, 16 * p, 32 * qc, lane);
         }
         // (every generic access of a tile is fenced against the TMA before it is refilled)
         tc::fence_async_smem();
@@ -396,13 +394,12 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, c
 
     if (a.dS0 && !abort_flag) {
         tc::fence_after();
-        float v[64];
-        tc::ld_32x32b_x32(t_srow, *reinterpret_cast<float(*)[32]>(&v[0]));
-        tc::ld_32x32b_x32(t_srow + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+        float v[32];
+        tc::ld_32x32b_x32(t_srow, v);
         tc::wait_ld();
-        float4 *dst = reinterpret_cast<float4 *>(a.dS0 + (size_t)bh * D * D + (size_t)c * D + 64 * hc);
+        float4 *dst = reinterpret_cast<float4 *>(a.dS0 + (size_t)bh * D * D + (size_t)c * D + 32 * qc);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
     tc::fence_before();
     __syncthreads();
@@ -425,7 +422,7 @@ cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(cbwd_tc::chunk_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          cbwd_tc::BYTES);
     if (e != cudaSuccess) return e;
-    cbwd_tc::chunk_bwd_tc_kernel<<<(unsigned)(a.B * a.H), chunk::NTHR, cbwd_tc::BYTES, s>>>(a, m);
+    cbwd_tc::chunk_bwd_tc_kernel<<<(unsigned)(a.B * a.H), cbwd_tc::NT, cbwd_tc::BYTES, s>>>(a, m);
     return cudaGetLastError();
 }
 

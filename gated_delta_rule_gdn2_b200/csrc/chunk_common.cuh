@@ -159,10 +159,10 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[1][NT][4], bf
 
 // cp.async of rows [n*C, n*C + C) of a token tensor [B,T,H,D] (head h of
 // batch b) into a swizzled [C][D] tile; rows past T are zero-filled.
-template <int D>
+template <int D, int NT = NTHR>
 __device__ __forceinline__ void load_token_tile(bf16 *dst, const bf16 *src, int b, int h, int n, int T, int H) {
     constexpr int CPR = D / 8;  // 16-byte chunks per row
-    for (int id = threadIdx.x; id < C * CPR; id += NTHR) {
+    for (int id = threadIdx.x; id < C * CPR; id += NT) {
         const int r = id / CPR, ch = id % CPR;
         const int t = n * C + r;
         const bool ok = t < T;
@@ -196,10 +196,10 @@ struct ChunkTiles {
     bf16 *q, *k, *la, *b, *v, *w;
 };
 
-// Shared-memory scratch of the intra-chunk stage (static, per CTA).
-template <int DK>
+// Shared-memory scratch of the intra-chunk stage (static, per CTA of NT threads).
+template <int DK, int NT = NTHR>
 struct IntraShared {
-    float part[NTHR / (DK / 2)][DK];  // segment sums of log_alpha (channel-pair layout)
+    float part[NT / (DK / 2)][DK];  // segment sums of log_alpha (channel-pair layout)
     float gamma[DK];
     int slow;
 };
@@ -248,16 +248,18 @@ __device__ __forceinline__ void block16_tf32(float (&acc)[2][4], const float *X,
 // A32 and T32 are 64x64 fp32 work areas; A32 is free on return, T32 holds
 // T16 and M16.  lam_ws (per-CTA [64][DK] fp32, global) receives L when
 // keep_lam is set and is always used by a slow chunk.
-template <int DK, int DV>
-__device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<DK> &sh, float *lam_ws,
+// NT: threads of the CTA (a multiple of 64, at least 256).
+template <int DK, int DV, int NT = NTHR>
+__device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<DK, NT> &sh, float *lam_ws,
                             bool keep_lam, bool prep_only = false) {
+    static_assert(NT % 64 == 0 && NT >= 256, "thread count");
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     bf16 *T16 = reinterpret_cast<bf16 *>(T32);
     bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
 
     if (tid == 0) sh.slow = 0;
     // ---- pass 1: segment sums of log_alpha per channel pair, and w . v in place of v
-    constexpr int NP = DK / 2, P2 = NTHR / NP, RS2 = C / P2;
+    constexpr int NP = DK / 2, P2 = NT / NP, RS2 = C / P2;
     const int cp = tid % NP, s2 = tid / NP, c2 = 2 * cp;
     {
         float pa = 0.f, pb = 0.f;
@@ -269,7 +271,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
         }
         sh.part[s2][c2] = pa;
         sh.part[s2][c2 + 1] = pb;
-        for (int id = tid; id < (prep_only ? 0 : C * DV / 8); id += NTHR) {
+        for (int id = tid; id < (prep_only ? 0 : C * DV / 8); id += NT) {
             uint4 wv = reinterpret_cast<const uint4 *>(st.w)[id];
             uint4 vv = reinterpret_cast<const uint4 *>(st.v)[id];
             const bf16 *w8 = reinterpret_cast<const bf16 *>(&wv);
@@ -321,20 +323,22 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
         }
         __syncthreads();
         if (prep_only) return false;
-        // ---- Grams: [Gt; Qt] Kb^T, warp w -> rows 16w..16w+15 of the stacked operand
-        float acc[1][8][4];
-        zero(acc);
-        const bf16 *Aop = warp < 4 ? st.b : st.q;
-        warp_gemm<1, 8, true, true, DK, DK>(acc, Aop, 16 * (warp & 3), st.la, 0, DK, lane);
-        const int r0 = 16 * (warp & 3) + (lane >> 2);
+        // ---- Grams: [Gt; Qt] Kb^T, warp w < 8 -> rows 16w..16w+15 of the stacked operand
+        if (warp < 8) {
+            float acc[1][8][4];
+            zero(acc);
+            const bf16 *Aop = warp < 4 ? st.b : st.q;
+            warp_gemm<1, 8, true, true, DK, DK>(acc, Aop, 16 * (warp & 3), st.la, 0, DK, lane);
+            const int r0 = 16 * (warp & 3) + (lane >> 2);
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
+            for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = r0 + (e >> 1) * 8, i = 8 * nt + 2 * (lane & 3) + (e & 1);
-                if (warp < 4) A32[r * C + i] = i < r ? acc[0][nt][e] : 0.f;
-                else accM[0][nt][e] = i <= r ? acc[0][nt][e] : 0.f;
-            }
+                for (int e = 0; e < 4; ++e) {
+                    const int r = r0 + (e >> 1) * 8, i = 8 * nt + 2 * (lane & 3) + (e & 1);
+                    if (warp < 4) A32[r * C + i] = i < r ? acc[0][nt][e] : 0.f;
+                    else accM[0][nt][e] = i <= r ? acc[0][nt][e] : 0.f;
+                }
+        }
     } else {
         // ---- slow chunk: exact per-term decays.  L goes to the per-CTA
         // workspace (one thread per key channel); raw q, k, b stay in shared
@@ -347,12 +351,13 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
             }
         }
         __syncthreads();
-        float pa[9], pm[9];
+        constexpr int NPAIR = C * (C + 1) / 2, NS = (NPAIR + NT - 1) / NT;
+        float pa[NS], pm[NS];
 #pragma unroll
-        for (int s = 0; s < 9; ++s) {
+        for (int s = 0; s < NS; ++s) {
             pa[s] = 0.f;
             pm[s] = 0.f;
-            const int p = tid + NTHR * s;
+            const int p = tid + NT * s;
             if (!prep_only && p < C * (C + 1) / 2) {
                 int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
                 while ((r + 1) * (r + 2) / 2 <= p) ++r;
@@ -383,14 +388,14 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
         }
         __syncthreads();
         if (prep_only) return true;
-        for (int e = tid; e < C * C; e += NTHR) {
+        for (int e = tid; e < C * C; e += NT) {
             A32[e] = 0.f;
             T32[e] = 0.f;
         }
         __syncthreads();
 #pragma unroll
-        for (int s = 0; s < 9; ++s) {
-            const int p = tid + NTHR * s;
+        for (int s = 0; s < NS; ++s) {
+            const int p = tid + NT * s;
             if (p < C * (C + 1) / 2) {
                 int r = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
                 while ((r + 1) * (r + 2) / 2 <= p) ++r;
@@ -401,7 +406,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
             }
         }
         __syncthreads();
-        if (warp >= 4) {
+        if (warp >= 4 && warp < 8) {
             const int r0 = 16 * (warp & 3) + (lane >> 2);
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt)
@@ -428,7 +433,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
 #pragma unroll
         for (int r = 0; r < 16; ++r) T32[(16 * R + r) * C + 16 * R + j] = x[r];
     } else {
-        for (int e = tid - 64; e < 6 * 256; e += NTHR - 64) {
+        for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
             const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
             const int R = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
             const int Q = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
@@ -467,15 +472,16 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
     }
     // T32 -> T16, M -> M16 (both bf16, swizzled [64][64])
     {
-        float tv[16];
+        constexpr int EPT = C * C / NT;  // elements per thread
+        float tv[EPT];
 #pragma unroll
-        for (int s = 0; s < 16; ++s) tv[s] = T32[tid * 16 + s];
+        for (int s = 0; s < EPT; ++s) tv[s] = T32[tid * EPT + s];
         __syncthreads();
-        const int r = tid >> 2, cb = (tid & 3) * 16;
+        const int r = tid / (C / EPT), cb = (tid % (C / EPT)) * EPT;
 #pragma unroll
-        for (int s = 0; s < 16; s += 2)
+        for (int s = 0; s < EPT; s += 2)
             *reinterpret_cast<uint32_t *>(T16 + swz<64>(r, cb + s)) = pack_bf16(tv[s], tv[s + 1]);
-        if (warp >= 4) store_tile_bf16<8, 64>(accM, M16, 16 * (warp & 3), lane, 1.f);
+        if (warp >= 4 && warp < 8) store_tile_bf16<8, 64>(accM, M16, 16 * (warp & 3), lane, 1.f);
     }
     __syncthreads();
     return slow;

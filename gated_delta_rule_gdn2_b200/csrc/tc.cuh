@@ -155,6 +155,18 @@ __device__ __forceinline__ void ld_16x256b_x16(uint32_t taddr, float (&v)[64]) {
         : "r"(taddr));
 }
 
+// The same shape over 32 columns (4 repetitions, 16 registers).
+__device__ __forceinline__ void ld_16x256b_x4(uint32_t taddr, float (&v)[16]) {
+    uint32_t *r = reinterpret_cast<uint32_t *>(v);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15])
+        : "r"(taddr));
+}
+
 // The same shape over 64 columns (8 repetitions, 32 registers).
 __device__ __forceinline__ void ld_16x256b_x8(uint32_t taddr, float (&v)[32]) {
     uint32_t *r = reinterpret_cast<uint32_t *>(v);
