@@ -246,12 +246,13 @@ cudaError_t launch_t(const ChunkBwdArgs &a, cudaStream_t s) {
     // (2) reverse chunk pass (tensor-memory products for dk = dv = 128)
     if constexpr (DK == 128 && DV == 128) {
         return launch_chunk_bwd_tc(a, s);
+    } else {
+        constexpr int bytes = BSmem<DK, DV>::BYTES;
+        e = cudaFuncSetAttribute(chunk_bwd_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return e;
+        chunk_bwd_kernel<DK, DV><<<(unsigned)(a.B * a.H), NTHR, bytes, s>>>(a);
+        return cudaGetLastError();
     }
-    constexpr int bytes = BSmem<DK, DV>::BYTES;
-    e = cudaFuncSetAttribute(chunk_bwd_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    chunk_bwd_kernel<DK, DV><<<(unsigned)(a.B * a.H), NTHR, bytes, s>>>(a);
-    return cudaGetLastError();
 }
 
 template <int DK, int DV>

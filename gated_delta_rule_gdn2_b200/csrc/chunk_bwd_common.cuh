@@ -240,13 +240,74 @@ struct BwdChunk {
         __syncthreads();
     }
 
-    // dv, dw from the bf16 -dRHS tile nR16, then dq, dk, db and dlog_alpha from
-    // the fp32 staging tiles DQT, DGT, DKB (and PQ.. for a slow chunk).
-    __device__ void token_grads(int n, int Cn, bool slow) {
+    // dv = dRHS . w, dw = dRHS . v from the bf16 -dRHS tile nR16 (16-byte
+    // coalesced; every global load is issued before the first use).
+    __device__ void dvdw(int n, int Cn) {
+        constexpr int NV = C * DV / 8 / NT;
+        uint4 v8[NV], w8[NV];
+#pragma unroll
+        for (int it = 0; it < NV; ++it) {
+            const int id = tid + it * NT, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
+            const size_t o = (((size_t)b * T + n * C + min(r, Cn - 1)) * H + h) * DV + j;
+            v8[it] = *reinterpret_cast<const uint4 *>(gv + o);
+            w8[it] = *reinterpret_cast<const uint4 *>(gw + o);
+        }
+#pragma unroll
+        for (int it = 0; it < NV; ++it) {
+            const int id = tid + it * NT, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
+            if (r < Cn) {
+                const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV + j;
+                const uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, j));
+                const __nv_bfloat162 *n2 = reinterpret_cast<const __nv_bfloat162 *>(&nr);
+                const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&v8[it]);
+                const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w8[it]);
+                uint4 dv8, dw8;
+                uint32_t *dvp = reinterpret_cast<uint32_t *>(&dv8), *dwp = reinterpret_cast<uint32_t *>(&dw8);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 d = __bfloat1622float2(n2[e]), vv = __bfloat1622float2(v2[e]),
+                                 ww = __bfloat1622float2(w2[e]);
+                    dvp[e] = pack_bf16(-d.x * ww.x, -d.y * ww.y);
+                    dwp[e] = pack_bf16(-d.x * vv.x, -d.y * vv.y);
+                }
+                *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dv) + o) = dv8;
+                *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dw) + o) = dw8;
+            }
+        }
+    }
+
+    // The raw q, k, b, log_alpha of this thread's rows and channel pair in the
+    // token-gradient layout (two key channels per thread, rows in P2 segments).
+    static constexpr int NP = DK / 2, P2 = NT / NP, RS2 = C / P2;
+    struct RawRows {
+        __nv_bfloat162 q[RS2], k[RS2], b[RS2], la[RS2];
+    };
+    __device__ void load_rows(RawRows &raw, int n, int Cn) const {
+        const int c2 = 2 * (tid % NP), s2 = tid / NP;
+        const bf16 *gla = static_cast<const bf16 *>(a.log_alpha);
+#pragma unroll
+        for (int i = 0; i < RS2; ++i) {
+            const int r = min(s2 * RS2 + i, Cn - 1);
+            const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c2;
+            raw.q[i] = *reinterpret_cast<const __nv_bfloat162 *>(gq + o);
+            raw.k[i] = *reinterpret_cast<const __nv_bfloat162 *>(gk + o);
+            raw.b[i] = *reinterpret_cast<const __nv_bfloat162 *>(gb + o);
+            raw.la[i] = *reinterpret_cast<const __nv_bfloat162 *>(gla + o);
+        }
+    }
+
+    // dv, dw (unless done already), then dq, dk, db and dlog_alpha from the fp32
+    // staging tiles DQT, DGT, DKB (and PQ.. for a slow chunk).
+    __device__ void token_grads(int n, int Cn, bool slow, bool with_dvdw = true) {
+        RawRows raw;
+        load_rows(raw, n, Cn);
+        token_grads(n, Cn, slow, raw, with_dvdw);
+    }
+    // ... with the raw rows loaded already (load_rows, issued early to hide its latency)
+    __device__ void token_grads(int n, int Cn, bool slow, const RawRows &raw, bool with_dvdw) {
         // ---- elementwise gradients and the in-chunk reverse cumulative sum
         // (two key channels per thread, rows split into P2 segments)
         {
-            constexpr int NP = DK / 2, P2 = NT / NP, RS2 = C / P2;
             const int cp = tid % NP, s2 = tid / NP, c2 = 2 * cp;
             const float2 lend = slow ? *reinterpret_cast<const float2 *>(LAM + (Cn - 1) * DK + c2)
                                      : make_float2(0.f, 0.f);
@@ -256,64 +317,19 @@ struct BwdChunk {
                 rsum.x += s_rs[i][c2];
                 rsum.y += s_rs[i][c2 + 1];
             }
-            // dv = dRHS . w, dw = dRHS . v from the bf16 -dRHS tile, 16-byte coalesced;
-            // every global load of the pass is issued before the first use
-            {
-                constexpr int NV = C * DV / 8 / NT;
-                uint4 v8[NV], w8[NV];
-#pragma unroll
-                for (int it = 0; it < NV; ++it) {
-                    const int id = tid + it * NT, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
-                    const size_t o = (((size_t)b * T + n * C + min(r, Cn - 1)) * H + h) * DV + j;
-                    v8[it] = *reinterpret_cast<const uint4 *>(gv + o);
-                    w8[it] = *reinterpret_cast<const uint4 *>(gw + o);
-                }
-#pragma unroll
-                for (int it = 0; it < NV; ++it) {
-                    const int id = tid + it * NT, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
-                    if (r < Cn) {
-                        const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV + j;
-                        const uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, j));
-                        const __nv_bfloat162 *n2 = reinterpret_cast<const __nv_bfloat162 *>(&nr);
-                        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&v8[it]);
-                        const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w8[it]);
-                        uint4 dv8, dw8;
-                        uint32_t *dvp = reinterpret_cast<uint32_t *>(&dv8), *dwp = reinterpret_cast<uint32_t *>(&dw8);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 d = __bfloat1622float2(n2[e]), vv = __bfloat1622float2(v2[e]),
-                                         ww = __bfloat1622float2(w2[e]);
-                            dvp[e] = pack_bf16(-d.x * ww.x, -d.y * ww.y);
-                            dwp[e] = pack_bf16(-d.x * vv.x, -d.y * vv.y);
-                        }
-                        *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dv) + o) = dv8;
-                        *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dw) + o) = dw8;
-                    }
-                }
-            }
+            if (with_dvdw) dvdw(n, Cn);
             // in-chunk decay prefix of this thread's rows (the prep's segment sums,
             // or the slow chunk's L in the workspace)
             float la_run = 0.f, lb_run = 0.f;
 #pragma unroll
             for (int s = 0; s < P2; ++s)
                 if (s < s2) { la_run += sh.part[s][c2]; lb_run += sh.part[s][c2 + 1]; }
-            const bf16 *gla = static_cast<const bf16 *>(a.log_alpha);
             bf16 *__restrict__ gdq = static_cast<bf16 *>(a.dq);
             bf16 *__restrict__ gdk = static_cast<bf16 *>(a.dk);
             bf16 *__restrict__ gdb = static_cast<bf16 *>(a.db);
             const float *__restrict__ sQT = DQT;
             const float *__restrict__ sGT = DGT;
             const float *__restrict__ sKB = DKB;
-            __nv_bfloat162 rq[RS2], rk[RS2], rb[RS2], rl[RS2];
-#pragma unroll
-            for (int i = 0; i < RS2; ++i) {
-                const int r = min(s2 * RS2 + i, Cn - 1);
-                const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c2;
-                rq[i] = *reinterpret_cast<const __nv_bfloat162 *>(gq + o);
-                rk[i] = *reinterpret_cast<const __nv_bfloat162 *>(gk + o);
-                rb[i] = *reinterpret_cast<const __nv_bfloat162 *>(gb + o);
-                rl[i] = *reinterpret_cast<const __nv_bfloat162 *>(gla + o);
-            }
             float dla_r[RS2], dlb_r[RS2];
             float pa = 0.f, pb = 0.f;
 #pragma unroll
@@ -323,12 +339,12 @@ struct BwdChunk {
                 dlb_r[i] = 0.f;
                 if (r < Cn) {
                     const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c2;
-                    const float2 q = __bfloat1622float2(rq[i]);
-                    const float2 kk = __bfloat1622float2(rk[i]);
-                    const float2 bb = __bfloat1622float2(rb[i]);
+                    const float2 q = __bfloat1622float2(raw.q[i]);
+                    const float2 kk = __bfloat1622float2(raw.k[i]);
+                    const float2 bb = __bfloat1622float2(raw.b[i]);
                     float2 lam;
                     if (!slow) {
-                        const float2 l = __bfloat1622float2(rl[i]);
+                        const float2 l = __bfloat1622float2(raw.la[i]);
                         la_run += l.x;
                         lb_run += l.y;
                         lam = make_float2(la_run, lb_run);

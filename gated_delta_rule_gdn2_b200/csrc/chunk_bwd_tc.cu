@@ -165,15 +165,19 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
     }
 
     uint32_t phase = 0;
-    // Commit the MMAs issued so far and wait for them (all threads); false on timeout.
-    auto mma_done = [&]() {
-        if (tid == 0) tc::commit(&mbar);
+    // Wait for the MMAs committed last (all threads) ...
+    auto mma_wait = [&]() {
         if (!tc::mbar_wait(&mbar, phase)) {
             abort_flag = 1;
             record_status(a.status, GDN2_ERR_TIMEOUT);
         }
         phase ^= 1;
         tc::fence_after();
+    };
+    // ... or commit the MMAs issued so far and wait for them.
+    auto mma_done = [&]() {
+        if (tid == 0) tc::commit(&mbar);
+        mma_wait();
     };
     // Shared-memory operands written by the threads -> visible to the tensor
     // cores, and everybody's tensor-memory accesses ordered before the next MMA.
@@ -318,8 +322,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
             mma_tiles<true, true>(tmem + COL_B, x.nR16, 64, x.S16, D, 8, ID64x128_K_K, false);
             mma_tiles<true, true>(tmem + COL_C, x.U16, 64, x.D16, D, 8, ID64x128_K_K, false);
             mma_tiles<false, false>(tmem + COL_S, st.b, 64, x.nR16, 64, 4, ID128x128_MN_MN, true);
+            tc::commit(&mbar);
         }
-        mma_done();
+        x.dvdw(n, Cn);  // while the tensor cores run: dv, dw from nR and the global v, w
+        mma_wait();
         // ---- row sums of dSigma . Sigma for chunk n - 1: dSigma is now its
         // chunk-end gradient and Sigma = this chunk's start state S
         if (n > 0) {
@@ -358,8 +364,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
                 mma_tiles<false, false>(tmem + COL_C, x.dA16, 64, st.b, 64, 4, ID64x128_MN_MN, true);
                 mma_tiles<false, false>(tmem + COL_C, x.dM16, 64, st.q, 64, 4, ID64x128_MN_MN, true);
             }
+            tc::commit(&mbar);
         }
-        mma_done();
+        Chunk::RawRows raw;
+        x.load_rows(raw, n, Cn);  // while the tensor cores run
+        mma_wait();
         // ---- E4: dQt, dGt, dKb -> fp32 staging (the S, D and T/M/dU regions are dead)
         {
             Frag f;
@@ -386,7 +395,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         }
         if (n > 0 && tid == 0) issue_a(n - 1);  // the token, dO and U slots are free now
         x.s_rs = s_rs[n & 1];
-        x.token_grads(n, Cn, slow);
+        x.token_grads(n, Cn, slow, raw, /*with_dvdw=*/false);
         tc::fence_async_smem();
         __syncthreads();
         if (n > 0 && tid == 0) issue_b(n - 1);  // the staging tiles in the S and T/M regions are consumed
