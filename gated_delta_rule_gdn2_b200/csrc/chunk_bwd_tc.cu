@@ -27,7 +27,7 @@
 // and returns.
 #include "chunk_bwd_common.cuh"
 #include "gdn2.h"
-#include "tc.cuh"
+#include "tc_tiles.cuh"
 #include "tma_host.h"
 
 namespace gdn2 {
@@ -60,56 +60,11 @@ constexpr uint32_t ID64x128_K_K = tc::idesc_bf16(64, 128, false, false);
 constexpr uint32_t ID64x64_K_K = tc::idesc_bf16(64, 64, false, false);
 constexpr uint32_t ID128x128_MN_MN = tc::idesc_bf16(128, 128, true, true);
 
-// Operand descriptors of a swizzled [R][64 k] tile (chunk_common.cuh's swz):
-// k-step s (16 elements) of a K-major operand (rows = M or N, columns = K) ...
-__device__ __forceinline__ uint64_t kmaj(const void *tile, int R, int s) {
-    return tc::sdesc(tc::smem_addr(tile) + (uint32_t)((s >> 2) * (R * 128) + (s & 3) * 32), 16, 1024);
-}
-// ... and of an MN-major operand (rows = K, columns = M or N).
-__device__ __forceinline__ uint64_t mnmaj(const void *tile, int R, int s) {
-    return tc::sdesc(tc::smem_addr(tile) + (uint32_t)(s * 2048), (uint32_t)(R * 128), 1024);
-}
-
-// D (+)= A B over K = 16 ks, issued by one thread.  A_K / B_K: K-major operand.
-template <bool A_K, bool B_K>
-__device__ __forceinline__ void mma_tiles(uint32_t d, const void *A, int RA, const void *B, int RB, int ks,
-                                          uint32_t idesc, bool accumulate) {
-    for (int s = 0; s < ks; ++s) {
-        const uint64_t da = A_K ? kmaj(A, RA, s) : mnmaj(A, RA, s);
-        const uint64_t db = B_K ? kmaj(B, RB, s) : mnmaj(B, RB, s);
-        tc::mma_bf16(d, da, db, idesc, accumulate || s > 0);
-    }
-}
-
-// sum_e v[e] * y[e] over 8 fp32 values and 8 packed bf16 values
-__device__ __forceinline__ float dot8(const float *v, uint4 y) {
-    const __nv_bfloat162 *y2 = reinterpret_cast<const __nv_bfloat162 *>(&y);
-    float acc = 0.f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(y2[e]);
-        acc += v[2 * e] * f.x + v[2 * e + 1] * f.y;
-    }
-    return acc;
-}
-
-// A 32-column fragment read with ld_16x256b_x4, as a warp-level [1][4][4] tile.
-using Frag = float[1][4][4];
-__device__ __forceinline__ void ld_frag(uint32_t taddr, Frag &f) {
-    tc::ld_16x256b_x4(taddr, reinterpret_cast<float(&)[16]>(f));
-}
-
-// bf16 store of a fragment (rows m0.., columns n0..) into a swizzled [.][DC] tile.
-template <int DC>
-__device__ __forceinline__ void store_frag_bf16(const Frag &f, bf16 *dst, int m0, int n0, int lane, float scale) {
-    const int r = m0 + (lane >> 2);
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-        const int c = n0 + 8 * nt + 2 * (lane & 3);
-        *reinterpret_cast<uint32_t *>(dst + swz<DC>(r, c)) = pack_bf16(scale * f[0][nt][0], scale * f[0][nt][1]);
-        *reinterpret_cast<uint32_t *>(dst + swz<DC>(r + 8, c)) = pack_bf16(scale * f[0][nt][2], scale * f[0][nt][3]);
-    }
-}
+using tct::Frag;
+using tct::dot8;
+using tct::ld_frag;
+using tct::mma_tiles;
+using tct::store_frag_bf16;
 
 __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, const __grid_constant__ BwdMaps maps) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -279,10 +234,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         // ---- E1: dU -> bf16 (all warps, column quarters) ; dM = strict_lower(dO U^T)
         // with its diagonal kept aside in fp32 (warps with qc < 2)
         {
-            Frag f;
+            Frag<4> f;
             ld_frag(tmem + lane_base + COL_C + 32 * qc, f);
             tc::wait_ld();
-            store_frag_bf16<D>(f, x.dU16, 16 * p, 32 * qc, lane, 1.f);
+            store_frag_bf16<D, 4>(f, x.dU16, 16 * p, 32 * qc, lane, 1.f);
             if (qc < 2) {
                 ld_frag(tmem + lane_base + COL_A + 32 * qc, f);
                 tc::wait_ld();
@@ -297,7 +252,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
                         if (i == r) s_dmd[r] = f[0][nt][e];
                         if (i >= r) f[0][nt][e] = 0.f;
                     }
-                store_frag_bf16<64>(f, x.dM16, 16 * p, 32 * qc, lane, 1.f);
+                store_frag_bf16<64, 4>(f, x.dM16, 16 * p, 32 * qc, lane, 1.f);
             }
         }
         handoff();
@@ -308,10 +263,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         mma_done();
         // ---- E2: nR = -T^T dU -> bf16
         {
-            Frag f;
+            Frag<4> f;
             ld_frag(tmem + lane_base + COL_B + 32 * qc, f);
             tc::wait_ld();
-            store_frag_bf16<D>(f, x.nR16, 16 * p, 32 * qc, lane, -1.f);
+            store_frag_bf16<D, 4>(f, x.nR16, 16 * p, 32 * qc, lane, -1.f);
         }
         handoff();
         if (abort_flag) break;
@@ -339,7 +294,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         }
         // ---- E3: dA = strict_lower(nR U^T) -> bf16 (warps with qc < 2)
         if (qc < 2) {
-            Frag f;
+            Frag<4> f;
             ld_frag(tmem + lane_base + COL_A + 64 + 32 * qc, f);
             tc::wait_ld();
             const int r0 = 16 * p + (lane >> 2);
@@ -350,7 +305,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
                     const int r = r0 + (e >> 1) * 8, i = 32 * qc + 8 * nt + 2 * (lane & 3) + (e & 1);
                     if (i >= r) f[0][nt][e] = 0.f;
                 }
-            store_frag_bf16<64>(f, x.dA16, 16 * p, 32 * qc, lane, 1.f);
+            store_frag_bf16<64, 4>(f, x.dA16, 16 * p, 32 * qc, lane, 1.f);
         }
         handoff();
         if (abort_flag) break;
@@ -371,7 +326,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         mma_wait();
         // ---- E4: dQt, dGt, dKb -> fp32 staging (the S, D and T/M/dU regions are dead)
         {
-            Frag f;
+            Frag<4> f;
             ld_frag(tmem + lane_base + COL_A + 32 * qc, f);
             tc::wait_ld();
             cbwd::store_stage<D, 4>(f, x.DQT, 16 * p, 32 * qc, lane);

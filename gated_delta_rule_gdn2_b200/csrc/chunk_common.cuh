@@ -238,6 +238,81 @@ __device__ __forceinline__ void block16_tf32(float (&acc)[2][4], const float *X,
     }
 }
 
+// WY solve: T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 area
+// A32, into T32 (fp32) and then T16 = bf16 T (swizzled [64][64], first half of
+// the T32 area).  All NT threads; on return the area past T16 may be written,
+// and T16 is complete after the caller's next barrier.
+template <int NT>
+__device__ void wy_solve(const float *A32, float *T32) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    bf16 *T16 = reinterpret_cast<bf16 *>(T32);
+    // 16x16 diagonal blocks by substitution in fp32.
+    if (tid < 64) {
+        // column j of the inverse of unit lower-triangular block R, column by
+        // column: once x_r is final, every later row takes its update at once
+        const int R = tid >> 4, j = tid & 15;
+        const float *Ablk = A32 + (16 * R) * C + 16 * R;
+        float x[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int r = 0; r < 15; ++r)
+#pragma unroll
+            for (int s2 = r + 1; s2 < 16; ++s2) x[s2] -= Ablk[s2 * C + r] * x[r];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) T32[(16 * R + r) * C + 16 * R + j] = x[r];
+    } else {
+        for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
+            const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            const int R = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+            const int Q = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            T32[(16 * R + r) * C + 16 * Q + c] = 0.f;
+        }
+    }
+    __syncthreads();
+    // Off-diagonal blocks, one warp per block and level, on the tensor cores
+    // in TF32 (T is rounded to bf16 afterwards): X = sum_J A_RJ T_JQ, then
+    // T_RQ = -T_RR X.  Blocks of one level are independent.
+#pragma unroll 1
+    for (int lvl = 1; lvl < 4; ++lvl) {
+        if (warp < 4 - lvl) {
+            const int Q = warp, R = Q + lvl;
+            const int g = lane >> 2, t = lane & 3;
+            float x[2][4] = {};
+            for (int J = Q; J < R; ++J) block16_tf32(x, A32, 16 * R, 16 * J, T32, 16 * Q, lane);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int c = 16 * Q + 8 * nt + 2 * t;
+                *reinterpret_cast<float2 *>(T32 + (16 * R + g) * C + c) = make_float2(x[nt][0], x[nt][1]);
+                *reinterpret_cast<float2 *>(T32 + (16 * R + g + 8) * C + c) = make_float2(x[nt][2], x[nt][3]);
+            }
+            __syncwarp();
+            float y[2][4] = {};
+            block16_tf32(y, T32, 16 * R, 16 * R, T32, 16 * Q, lane);
+            __syncwarp();
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const int c = 16 * Q + 8 * nt + 2 * t;
+                *reinterpret_cast<float2 *>(T32 + (16 * R + g) * C + c) = make_float2(-y[nt][0], -y[nt][1]);
+                *reinterpret_cast<float2 *>(T32 + (16 * R + g + 8) * C + c) = make_float2(-y[nt][2], -y[nt][3]);
+            }
+        }
+        __syncthreads();
+    }
+    // T32 -> T16 (bf16, swizzled [64][64], the first half of the T32 area)
+    {
+        constexpr int EPT = C * C / NT;  // elements per thread
+        float tv[EPT];
+#pragma unroll
+        for (int s = 0; s < EPT; ++s) tv[s] = T32[tid * EPT + s];
+        __syncthreads();
+        const int r = tid / (C / EPT), cb = (tid % (C / EPT)) * EPT;
+#pragma unroll
+        for (int s = 0; s < EPT; s += 2)
+            *reinterpret_cast<uint32_t *>(T16 + swz<64>(r, cb + s)) = pack_bf16(tv[s], tv[s + 1]);
+    }
+}
+
 // Intra-chunk stage.  On entry the six raw token tiles of the chunk are in
 // shared memory (and visible to all threads).  With prep_only only the decay
 // prefix and the operands Qt, Gt, Kb/Kt are formed (v, w untouched; T, M
@@ -251,7 +326,7 @@ __device__ __forceinline__ void block16_tf32(float (&acc)[2][4], const float *X,
 // NT: threads of the CTA (a multiple of 64, at least 256).
 template <int DK, int DV, int NT = NTHR>
 __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<DK, NT> &sh, float *lam_ws,
-                            bool keep_lam, bool prep_only = false) {
+                            bool keep_lam, bool prep_only = false, bool grams_ext = false) {
     static_assert(NT % 64 == 0 && NT >= 256, "thread count");
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     bf16 *T16 = reinterpret_cast<bf16 *>(T32);
@@ -322,7 +397,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
             *reinterpret_cast<uint32_t *>(st.la + o) = pack_bf16(k2.x * iea, k2.y * ieb);
         }
         __syncthreads();
-        if (prep_only) return false;
+        if (prep_only || grams_ext) return false;
         // ---- Grams: [Gt; Qt] Kb^T, warp w < 8 -> rows 16w..16w+15 of the stacked operand
         if (warp < 8) {
             float acc[1][8][4];
@@ -417,72 +492,9 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
     }
     __syncthreads();
 
-    // ---- T = (I + A)^{-1}: 16x16 diagonal blocks by substitution in fp32.
-    if (tid < 64) {
-        // column j of the inverse of unit lower-triangular block R, column by
-        // column: once x_r is final, every later row takes its update at once
-        const int R = tid >> 4, j = tid & 15;
-        const float *Ablk = A32 + (16 * R) * C + 16 * R;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
-#pragma unroll
-        for (int r = 0; r < 15; ++r)
-#pragma unroll
-            for (int s2 = r + 1; s2 < 16; ++s2) x[s2] -= Ablk[s2 * C + r] * x[r];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) T32[(16 * R + r) * C + 16 * R + j] = x[r];
-    } else {
-        for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
-            const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
-            const int R = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-            const int Q = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            T32[(16 * R + r) * C + 16 * Q + c] = 0.f;
-        }
-    }
-    __syncthreads();
-    // Off-diagonal blocks, one warp per block and level, on the tensor cores
-    // in TF32 (T is rounded to bf16 afterwards): X = sum_J A_RJ T_JQ, then
-    // T_RQ = -T_RR X.  Blocks of one level are independent.
-#pragma unroll 1
-    for (int lvl = 1; lvl < 4; ++lvl) {
-        if (warp < 4 - lvl) {
-            const int Q = warp, R = Q + lvl;
-            const int g = lane >> 2, t = lane & 3;
-            float x[2][4] = {};
-            for (int J = Q; J < R; ++J) block16_tf32(x, A32, 16 * R, 16 * J, T32, 16 * Q, lane);
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int c = 16 * Q + 8 * nt + 2 * t;
-                *reinterpret_cast<float2 *>(T32 + (16 * R + g) * C + c) = make_float2(x[nt][0], x[nt][1]);
-                *reinterpret_cast<float2 *>(T32 + (16 * R + g + 8) * C + c) = make_float2(x[nt][2], x[nt][3]);
-            }
-            __syncwarp();
-            float y[2][4] = {};
-            block16_tf32(y, T32, 16 * R, 16 * R, T32, 16 * Q, lane);
-            __syncwarp();
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int c = 16 * Q + 8 * nt + 2 * t;
-                *reinterpret_cast<float2 *>(T32 + (16 * R + g) * C + c) = make_float2(-y[nt][0], -y[nt][1]);
-                *reinterpret_cast<float2 *>(T32 + (16 * R + g + 8) * C + c) = make_float2(-y[nt][2], -y[nt][3]);
-            }
-        }
-        __syncthreads();
-    }
-    // T32 -> T16, M -> M16 (both bf16, swizzled [64][64])
-    {
-        constexpr int EPT = C * C / NT;  // elements per thread
-        float tv[EPT];
-#pragma unroll
-        for (int s = 0; s < EPT; ++s) tv[s] = T32[tid * EPT + s];
-        __syncthreads();
-        const int r = tid / (C / EPT), cb = (tid % (C / EPT)) * EPT;
-#pragma unroll
-        for (int s = 0; s < EPT; s += 2)
-            *reinterpret_cast<uint32_t *>(T16 + swz<64>(r, cb + s)) = pack_bf16(tv[s], tv[s + 1]);
-        if (warp >= 4 && warp < 8) store_tile_bf16<8, 64>(accM, M16, 16 * (warp & 3), lane, 1.f);
-    }
+    wy_solve<NT>(A32, T32);
+    // M -> M16 (bf16, swizzled [64][64]; the second half of the T32 area)
+    if (warp >= 4 && warp < 8) store_tile_bf16<8, 64>(accM, M16, 16 * (warp & 3), lane, 1.f);
     __syncthreads();
     return slow;
 }

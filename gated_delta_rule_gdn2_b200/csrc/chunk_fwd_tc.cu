@@ -1,28 +1,31 @@
-// Chunk-parallel forward for dk = dv = 128 with the inter-chunk state
-// propagation on the fifth-generation tensor cores (tcgen05, accumulators in
-// tensor memory).
+// Chunk-parallel forward for dk = dv = 128 with every chunk product on the
+// fifth-generation tensor cores (tcgen05, accumulators in tensor memory).
 //
 // Same algebra as chunk_fwd.cu ("Why NVIDIA Gated DeltaNet-2 separates erase
 // and write gates", section "Gated Delta Rule-2: per-channel erase/write
 // split"; WY form from the laonpeople Gated DeltaNet page): per chunk
-//   U = Uv - W S,   O = Qt S + M U,   S <- Diag(gam) (S + Kb^T U).
+//   A = Gt Kb^T, M = Qt Kb^T,  T = (I + A)^{-1},
+//   U = T (w . v) - (T Gt) S,   O = Qt S + M U,   S <- Diag(gam) (S + Kb^T U).
 // The fp32 state S lives in TMEM (128 lanes = key channels x 128 columns)
-// for the whole sequence.  Per chunk one thread issues
-//   D_W = (-W) S   and   D_Q = Qt S     (two M=64, N=128, K=128 MMAs, bf16 S
-//                                        copy in shared memory as operand B)
-//   S  += Kb^T U                        (M=128, N=128, K=64, accumulating in TMEM)
-// and the warps read D_W / D_Q back with the 16x256b TMEM load shape, which
-// lands in the register layout of the warp-level m16n8 products that form Uv
-// and M U.  S is scaled by gam in TMEM (32x32b load/store) and copied to bf16
-// for the next chunk.  The intra-chunk stage (decay prefix, operands, Grams,
-// WY solve, W and Uv) is shared with the other kernels (chunk_common.cuh).
-// Every wait on the MMA completion barrier is bounded: on expiry the kernel
-// records GDN2_ERR_TIMEOUT in the device status word, frees its tensor memory
-// and returns.
+// for the whole sequence.  Per chunk one thread issues four MMA groups:
+//   the two Grams (M = N = 64, K = 128);
+//   T (w . v) into U's columns and T Gt (M = 64, N = 128, K = 64);
+//   U += (-W) S and O = Qt S (K = 128, bf16 S copy in shared memory as B);
+//   S += Kb^T U (M = 128) and O += M U,
+// and between them the warps read the results back with the 16x256b TMEM
+// load shape (the register layout of a warp-level m16n8 fragment) to form
+// the next bf16 operands: A in fp32 for the WY solve (TF32 tensor-core levels
+// on fp32 16x16 diagonal blocks, chunk_common.cuh), M, -W and U in bf16.  S is
+// scaled by gam in TMEM (32x32b load/store) and copied to bf16 for the next
+// chunk.  A chunk whose decay spans more than e^{-64} takes its Grams term by
+// term in fp32 inside the shared intra-chunk stage.  Tiles arrive by TMA and
+// the tiles kept for the backward leave as bulk stores.  Every wait on an
+// mbarrier is bounded: on expiry the kernel records GDN2_ERR_TIMEOUT in the
+// device status word, frees its tensor memory and returns.
 #include "chunk_common.cuh"
 #include "gdn2.h"
 #include "launch.h"
-#include "tc.cuh"
+#include "tc_tiles.cuh"
 #include "tma_host.h"
 
 namespace gdn2 {
@@ -38,7 +41,7 @@ constexpr int OSMALL = OS16 + D * D * 2;
 
 struct Small {
     IntraShared<D> intra;
-    uint64_t mbar[2];
+    uint64_t mbar[1];     // MMA completion
     uint64_t mbar_ld[2];  // tile loads of stage 0 and 1
     uint32_t tmem;
     int abort;
@@ -46,10 +49,19 @@ struct Small {
 constexpr int BYTES = OSMALL + (int)sizeof(Small);
 static_assert(BYTES <= 232448, "shared memory per block");
 
+// Tensor memory: U (Uv, then + (-W) S), O (Qt S, then + M U), the state S
+// (fp32, 128 key rows x 128 value columns) and a work region for the Grams
+// (A | M, 64 columns each) and then T Gt.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t COL_W = 0, COL_Q = 128, COL_S = 256;
-constexpr uint32_t IDESC_WQ = tc::idesc_bf16(64, 128, false, true);  // A K-major, B MN-major
-constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, true, true);   // A, B MN-major
+constexpr uint32_t COL_U = 0, COL_O = 128, COL_S = 256, COL_G = 384;
+constexpr uint32_t ID64x64_K_K = tc::idesc_bf16(64, 64, false, false);
+constexpr uint32_t ID64x128_K_MN = tc::idesc_bf16(64, 128, false, true);
+constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, true, true);  // A, B MN-major
+
+using tct::Frag;
+using tct::ld_frag;
+using tct::mma_tiles;
+using tct::store_frag_bf16;
 
 __device__ __forceinline__ ChunkTiles stage_tiles(unsigned char *smem, int s) {
     unsigned char *p = smem + s * STAGE;
@@ -99,7 +111,6 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, c
     if (warp == 0) tc::tmem_alloc(&sm.tmem, kTmemCols);
     if (tid == 0) {
         tc::mbar_init(&sm.mbar[0], 1);
-        tc::mbar_init(&sm.mbar[1], 1);
         tc::mbar_init(&sm.mbar_ld[0], 1);
         tc::mbar_init(&sm.mbar_ld[1], 1);
         tc::fence_mbar_init();
@@ -169,7 +180,26 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, c
         if (nchunks > 1) issue_chunk(maps, stage_tiles(smem, 1), b, h, 1, &sm.mbar_ld[1]);
     }
 
-    uint32_t ph0 = 0, ph1 = 0, ph_ld[2] = {0, 0};
+    uint32_t ph_mma = 0, ph_ld[2] = {0, 0};
+    // Commit the MMAs issued so far (thread 0) and wait for them (all threads).
+    auto mma_done = [&]() {
+        if (tid == 0) tc::commit(&sm.mbar[0]);
+        if (!tc::mbar_wait(&sm.mbar[0], ph_mma)) {
+            sm.abort = 1;
+            record_status(a.status, GDN2_ERR_TIMEOUT);
+        }
+        ph_mma ^= 1;
+        tc::fence_after();
+    };
+    // Shared-memory operands written by the threads -> visible to the tensor cores.
+    auto handoff = [&]() {
+        tc::fence_async_smem();
+        tc::fence_before();
+        __syncthreads();
+        tc::fence_after();
+    };
+    const uint32_t lane_base = (uint32_t)(32 * p) << 16;  // this warp's 16 rows of a 64-row product
+
     for (int n = 0; n < nchunks; ++n) {
         ChunkTiles st = stage_tiles(smem, n & 1);
         float *A32 = reinterpret_cast<float *>(st.k);  // k and w slots are free after the prep
@@ -186,69 +216,84 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, c
         ph_ld[n & 1] ^= 1;
         __syncthreads();
         if (sm.abort) break;
-        const bool slow = intra_chunk<D, D>(st, A32, T32, sm.intra, lam_ws, false);
-
-        // ---- Uv = T WV (warps 0..3, registers) ; -W = -T Gt (warps 4..7, shared)
-        float acc[1][16][4];
-        zero(acc);
-        if (warp < 4) {
-            warp_gemm<1, 16, true, false, 64, D>(acc, T16, 16 * warp, st.v, 0, C, lane);
-        } else {
-            warp_gemm<1, 16, true, false, 64, D>(acc, T16, 16 * p, st.b, 0, C, lane);
-            store_tile_bf16<16, D>(acc, W16, 16 * p, lane, -1.f);
+        // decay prep and w . v; a slow chunk also takes its Grams term by term and
+        // its WY solve here, a fast chunk continues below
+        const bool slow = intra_chunk<D, D>(st, A32, T32, sm.intra, lam_ws, false, false, /*grams_ext=*/true);
+        if (!slow) {
+            // ---- Grams on the tensor cores: A = Gt Kb^T, M = Qt Kb^T (M = N = 64, K = 128)
+            handoff();
+            if (tid == 0) {
+                mma_tiles<true, true>(tmem + COL_G, st.b, 64, st.la, 64, 8, ID64x64_K_K, false);
+                mma_tiles<true, true>(tmem + COL_G + 64, st.q, 64, st.la, 64, 8, ID64x64_K_K, false);
+            }
+            mma_done();
+            {  // A (strictly lower) -> fp32 for the solve
+                Frag<4> f;
+                ld_frag(tmem + lane_base + COL_G + 32 * hc, f);
+                tc::wait_ld();
+                const int r0 = 16 * p + (lane >> 2);
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int r = r0 + 8 * h2, i = 32 * hc + 8 * nt + 2 * (lane & 3);
+                        *reinterpret_cast<float2 *>(A32 + r * C + i) =
+                            make_float2(i < r ? f[0][nt][2 * h2] : 0.f, i + 1 < r ? f[0][nt][2 * h2 + 1] : 0.f);
+                    }
+            }
+            __syncthreads();
+            wy_solve<NTHR>(A32, T32);
+            {  // M (lower with the diagonal) -> bf16, past T16
+                Frag<4> f;
+                ld_frag(tmem + lane_base + COL_G + 64 + 32 * hc, f);
+                tc::wait_ld();
+                const int r0 = 16 * p + (lane >> 2);
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int r = r0 + (e >> 1) * 8, i = 32 * hc + 8 * nt + 2 * (lane & 3) + (e & 1);
+                        if (i > r) f[0][nt][e] = 0.f;
+                    }
+                store_frag_bf16<64, 4>(f, M16, 16 * p, 32 * hc, lane, 1.f);
+            }
         }
-        tc::fence_async_smem();
-        __syncthreads();
+        handoff();
+        if (sm.abort) break;
 
-        // ---- D_W = -W S, D_Q = Qt S on the tensor cores; T and M (and U,
+        // ---- Uv = T (w . v) and T Gt on the tensor cores (M = 64, N = 128, K = 64)
+        if (tid == 0) {
+            mma_tiles<true, false>(tmem + COL_U, T16, 64, st.v, 64, 4, ID64x128_K_MN, false);
+            mma_tiles<true, false>(tmem + COL_G, T16, 64, st.b, 64, 4, ID64x128_K_MN, false);
+        }
+        mma_done();
+        {  // -W = -(T Gt) -> bf16 in the k slot
+            Frag<8> f;
+            ld_frag(tmem + lane_base + COL_G + 64 * hc, f);
+            tc::wait_ld();
+            store_frag_bf16<D, 8>(f, W16, 16 * p, 64 * hc, lane, -1.f);
+        }
+        handoff();
+
+        // ---- U = Uv + (-W) S and O = Qt S on the tensor cores; T and M (and U,
         // below) go out for the backward as their shared-memory images
         if (tid == 0) {
             if (a.intra) {
                 tc::bulk_store(keep_tile(n), T16, 2 * C * C * 2);
                 tc::bulk_commit();
             }
-            tc::fence_after();
-            const uint32_t sS = tc::smem_addr(S16), sW = tc::smem_addr(W16), sQ = tc::smem_addr(st.q);
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const uint32_t koff = (s >> 2) * 8192 + (s & 3) * 32;
-                const uint64_t bd = tc::sdesc(sS + s * 2048, D * 128, 1024);
-                tc::mma_bf16(tmem + COL_W, tc::sdesc(sW + koff, 16, 1024), bd, IDESC_WQ, s > 0);
-                if (with_o) tc::mma_bf16(tmem + COL_Q, tc::sdesc(sQ + koff, 16, 1024), bd, IDESC_WQ, s > 0);
-            }
-            tc::commit(&sm.mbar[0]);
+            mma_tiles<true, false>(tmem + COL_U, W16, 64, S16, D, 8, ID64x128_K_MN, true);
+            if (with_o) mma_tiles<true, false>(tmem + COL_O, st.q, 64, S16, D, 8, ID64x128_K_MN, false);
         }
-        if (!tc::mbar_wait(&sm.mbar[0], ph0)) {
-            sm.abort = 1;
-            record_status(a.status, GDN2_ERR_TIMEOUT);
-        }
-        ph0 ^= 1;
-        tc::fence_after();
-
-        // ---- U = Uv + D_W (warps 0..3) -> bf16 ; O starts as D_Q (warps 4..7)
-        {
-            float d[64];
-            if (warp < 4) {
-                tc::ld_16x256b_x16(tmem + ((uint32_t)(32 * warp) << 16) + COL_W, d);
-                tc::wait_ld();
-#pragma unroll
-                for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[0][nt][e] += d[4 * nt + e];
-                store_tile_bf16<16, D>(acc, U16, 16 * warp, lane, 1.f);
-            } else if (with_o) {
-                tc::ld_16x256b_x16(tmem + ((uint32_t)(32 * p) << 16) + COL_Q, d);
-                tc::wait_ld();
-#pragma unroll
-                for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[0][nt][e] = d[4 * nt + e];
-            }
+        mma_done();
+        {  // U -> bf16 in the v slot (w . v is consumed)
+            Frag<8> f;
+            ld_frag(tmem + lane_base + COL_U + 64 * hc, f);
+            tc::wait_ld();
+            store_frag_bf16<D, 8>(f, U16, 16 * p, 64 * hc, lane, 1.f);
         }
         if (tid == 0) tc::bulk_wait_read();  // the previous state image is out: S16 may be rewritten below
-        tc::fence_async_smem();
-        tc::fence_before();
-        __syncthreads();
+        handoff();
         if (sm.abort) break;
 
         if (tid == 0 && a.intra) {
@@ -265,40 +310,32 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, c
             store_state(v);
             tc::fence_before();
             __syncthreads();
-        }
-        // ---- S += Kh^T U in TMEM
-        if (tid == 0) {
             tc::fence_after();
-            const uint32_t sK = tc::smem_addr(st.la), sU = tc::smem_addr(U16);
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                tc::mma_bf16(tmem + COL_S, tc::sdesc(sK + s * 2048, 8192, 1024), tc::sdesc(sU + s * 2048, 8192, 1024),
-                             IDESC_S, true);
-            tc::commit(&sm.mbar[1]);
         }
-        // ---- O += M U (warps 4..7), store o
-        if (warp >= 4 && with_o) {
-            warp_gemm<1, 16, true, false, 64, D>(acc, M16, 16 * p, U16, 0, C, lane);
+        // ---- S += Kx^T U ; O += M U
+        if (tid == 0) {
+            mma_tiles<false, false>(tmem + COL_S, st.la, 64, U16, 64, 4, IDESC_S, true);
+            if (with_o) mma_tiles<true, false>(tmem + COL_O, M16, 64, U16, 64, 4, ID64x128_K_MN, true);
+        }
+        mma_done();
+        if (with_o) {  // O -> o (bf16), straight from the fragment layout
+            Frag<8> f;
+            ld_frag(tmem + lane_base + COL_O + 64 * hc, f);
+            tc::wait_ld();
             const int rl = 16 * p + (lane >> 2);
             bf16 *o = static_cast<bf16 *>(a.o);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const int t = n * C + rl + 8 * half;
                 if (t < a.T) {
-                    bf16 *orow = o + (((size_t)b * a.T + t) * a.H + h) * D;
+                    bf16 *orow = o + (((size_t)b * a.T + t) * a.H + h) * D + 64 * hc;
 #pragma unroll
-                    for (int nt = 0; nt < 16; ++nt)
+                    for (int nt = 0; nt < 8; ++nt)
                         *reinterpret_cast<uint32_t *>(orow + 8 * nt + 2 * (lane & 3)) =
-                            pack_bf16(acc[0][nt][2 * half], acc[0][nt][2 * half + 1]);
+                            pack_bf16(f[0][nt][2 * half], f[0][nt][2 * half + 1]);
                 }
             }
         }
-        if (!tc::mbar_wait(&sm.mbar[1], ph1)) {
-            sm.abort = 1;
-            record_status(a.status, GDN2_ERR_TIMEOUT);
-        }
-        ph1 ^= 1;
-        tc::fence_after();
 
         // ---- S <- Diag(gam) S (fast chunk), bf16 copy for the next chunk
         {

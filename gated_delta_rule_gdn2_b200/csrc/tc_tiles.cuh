@@ -1,0 +1,74 @@
+// tcgen05 operands and results on the swizzled shared-memory tiles of
+// chunk_common.cuh (64-column blocks of 128-byte rows, 16-byte chunks permuted
+// by row mod 8 — the 128-byte-swizzle canonical layout): operand descriptors,
+// an MMA group over K, and the 16x256b tensor-memory fragments that land in
+// the register layout of a warp-level m16n8 product.
+#pragma once
+
+#include "chunk_common.cuh"
+#include "tc.cuh"
+
+namespace gdn2 {
+namespace tct {
+
+using namespace chunk;
+
+// k-step s (16 elements) of a K-major operand in an [R][.] tile (rows = M or N,
+// columns = K) ...
+__device__ __forceinline__ uint64_t kmaj(const void *tile, int R, int s) {
+    return tc::sdesc(tc::smem_addr(tile) + (uint32_t)((s >> 2) * (R * 128) + (s & 3) * 32), 16, 1024);
+}
+// ... and of an MN-major operand (rows = K, columns = M or N).
+__device__ __forceinline__ uint64_t mnmaj(const void *tile, int R, int s) {
+    return tc::sdesc(tc::smem_addr(tile) + (uint32_t)(s * 2048), (uint32_t)(R * 128), 1024);
+}
+
+// D (+)= A B over K = 16 ks, issued by one thread.  A_K / B_K: K-major operand.
+template <bool A_K, bool B_K>
+__device__ __forceinline__ void mma_tiles(uint32_t d, const void *A, int RA, const void *B, int RB, int ks,
+                                          uint32_t idesc, bool accumulate) {
+    for (int s = 0; s < ks; ++s) {
+        const uint64_t da = A_K ? kmaj(A, RA, s) : mnmaj(A, RA, s);
+        const uint64_t db = B_K ? kmaj(B, RB, s) : mnmaj(B, RB, s);
+        tc::mma_bf16(d, da, db, idesc, accumulate || s > 0);
+    }
+}
+
+// A fragment of 8 NTL columns of a 64-row accumulator (16 rows per warp),
+// read with the 16x256b shape, as a warp-level [1][NTL][4] tile.
+template <int NTL>
+using Frag = float[1][NTL][4];
+__device__ __forceinline__ void ld_frag(uint32_t taddr, Frag<4> &f) {
+    tc::ld_16x256b_x4(taddr, reinterpret_cast<float(&)[16]>(f));
+}
+__device__ __forceinline__ void ld_frag(uint32_t taddr, Frag<8> &f) {
+    tc::ld_16x256b_x8(taddr, reinterpret_cast<float(&)[32]>(f));
+}
+
+// bf16 store of a fragment (rows m0.., columns n0..) into a swizzled [.][DC] tile.
+template <int DC, int NTL>
+__device__ __forceinline__ void store_frag_bf16(const Frag<NTL> &f, bf16 *dst, int m0, int n0, int lane,
+                                                float scale) {
+    const int r = m0 + (lane >> 2);
+#pragma unroll
+    for (int nt = 0; nt < NTL; ++nt) {
+        const int c = n0 + 8 * nt + 2 * (lane & 3);
+        *reinterpret_cast<uint32_t *>(dst + swz<DC>(r, c)) = pack_bf16(scale * f[0][nt][0], scale * f[0][nt][1]);
+        *reinterpret_cast<uint32_t *>(dst + swz<DC>(r + 8, c)) = pack_bf16(scale * f[0][nt][2], scale * f[0][nt][3]);
+    }
+}
+
+// sum_e v[e] * y[e] over 8 fp32 values and 8 packed bf16 values
+__device__ __forceinline__ float dot8(const float *v, uint4 y) {
+    const __nv_bfloat162 *y2 = reinterpret_cast<const __nv_bfloat162 *>(&y);
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(y2[e]);
+        acc += v[2 * e] * f.x + v[2 * e + 1] * f.y;
+    }
+    return acc;
+}
+
+}  // namespace tct
+}  // namespace gdn2
