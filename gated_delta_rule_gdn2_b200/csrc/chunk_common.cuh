@@ -329,7 +329,6 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
                             bool keep_lam, bool prep_only = false, bool grams_ext = false) {
     static_assert(NT % 64 == 0 && NT >= 256, "thread count");
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    bf16 *T16 = reinterpret_cast<bf16 *>(T32);
     bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
 
     if (tid == 0) sh.slow = 0;

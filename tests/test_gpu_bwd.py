@@ -19,7 +19,7 @@ def run_bwd(x, dtype, dST=None):
 
 
 @pytest.mark.parametrize("dtype,tol", [("bf16", TOL_BF16_GRAD), ("fp32", TOL_FP32)])
-@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128)])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64), (64, 128)])
 @pytest.mark.parametrize("T", [1, 64, 150])
 def test_bwd_matches_oracle(dtype, tol, dk, dv, T):
     x = make_inputs(2, T, 2, dk, dv, seed=300 + T, dtype=dtype, with_do=True)
