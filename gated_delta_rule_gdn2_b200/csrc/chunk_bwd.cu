@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
         const int Cn = min(C, T - n * C);
         x.load(n);
 
-        const bool slow = intra_chunk<DK, DV>(st, A32, T32, sh, LAM, false, /*prep_only=*/true);
+        const bool slow = intra_chunk<DK, DV>(st, A32, T32, view(sh), LAM, false, /*prep_only=*/true);
 
         // ---- Dh = gam . dSigma (fast) or dSigma (slow) as bf16; row sums of
         // dSigma . Sigma (Sigma = next chunk-boundary state) for dL_end

@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         __syncthreads();
         if (abort_flag) break;
         if (n > 0) x.prefetch_vw_l2(n - 1);
-        const bool slow = intra_chunk<D, D, NT>(st, x.A32, x.T32, sh, x.LAM, false, /*prep_only=*/true);
+        const bool slow = intra_chunk<D, D, NT>(st, x.A32, x.T32, view(sh), x.LAM, false, /*prep_only=*/true);
 
         // ---- E0: D = g . dSigma (g = gam on a fast chunk, else 1) as bf16 and
         // dSigma <- gam . dSigma; on the last chunk also the row sums of

@@ -203,6 +203,28 @@ struct IntraShared {
     float gamma[DK];
     int slow;
 };
+// Where the intra-chunk stage keeps that scratch (which may be split).
+template <int DK>
+struct IntraView {
+    float (*part)[DK];
+    float *gamma;
+    int *slow;
+};
+template <int DK, int NT>
+__device__ __forceinline__ IntraView<DK> view(IntraShared<DK, NT> &s) {
+    return {s.part, s.gamma, &s.slow};
+}
+
+// The threads that run a stage: the whole CTA (BAR = 0, __syncthreads), or
+// the NT threads from thread BASE on, which meet at the named barrier BAR.
+template <int BAR, int NT, int BASE>
+struct Grp {
+    static __device__ __forceinline__ void sync() {
+        if constexpr (BAR == 0) __syncthreads();
+        else asm volatile("bar.sync %0, %1;\n" ::"n"(BAR), "n"(NT) : "memory");
+    }
+    static __device__ __forceinline__ int tid() { return (int)threadIdx.x - BASE; }
+};
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
@@ -242,9 +264,9 @@ __device__ __forceinline__ void block16_tf32(float (&acc)[2][4], const float *X,
 // A32, into T32 (fp32) and then T16 = bf16 T (swizzled [64][64], first half of
 // the T32 area).  All NT threads; on return the area past T16 may be written,
 // and T16 is complete after the caller's next barrier.
-template <int NT>
+template <int NT, class G = Grp<0, NT, 0>>
 __device__ void wy_solve(const float *A32, float *T32) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = G::tid(), warp = tid >> 5, lane = tid & 31;
     bf16 *T16 = reinterpret_cast<bf16 *>(T32);
     // 16x16 diagonal blocks by substitution in fp32.
     if (tid < 64) {
@@ -269,7 +291,7 @@ __device__ void wy_solve(const float *A32, float *T32) {
             T32[(16 * R + r) * C + 16 * Q + c] = 0.f;
         }
     }
-    __syncthreads();
+    G::sync();
     // Off-diagonal blocks, one warp per block and level, on the tensor cores
     // in TF32 (T is rounded to bf16 afterwards): X = sum_J A_RJ T_JQ, then
     // T_RQ = -T_RR X.  Blocks of one level are independent.
@@ -297,7 +319,7 @@ __device__ void wy_solve(const float *A32, float *T32) {
                 *reinterpret_cast<float2 *>(T32 + (16 * R + g + 8) * C + c) = make_float2(-y[nt][2], -y[nt][3]);
             }
         }
-        __syncthreads();
+        G::sync();
     }
     // T32 -> T16 (bf16, swizzled [64][64], the first half of the T32 area)
     {
@@ -305,7 +327,7 @@ __device__ void wy_solve(const float *A32, float *T32) {
         float tv[EPT];
 #pragma unroll
         for (int s = 0; s < EPT; ++s) tv[s] = T32[tid * EPT + s];
-        __syncthreads();
+        G::sync();
         const int r = tid / (C / EPT), cb = (tid % (C / EPT)) * EPT;
 #pragma unroll
         for (int s = 0; s < EPT; s += 2)
@@ -324,28 +346,21 @@ __device__ void wy_solve(const float *A32, float *T32) {
 // T16 and M16.  lam_ws (per-CTA [64][DK] fp32, global) receives L when
 // keep_lam is set and is always used by a slow chunk.
 // NT: threads of the CTA (a multiple of 64, at least 256).
-template <int DK, int DV, int NT = NTHR>
-__device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<DK, NT> &sh, float *lam_ws,
+// G: the threads that run it (the whole CTA by default).
+template <int DK, int DV, int NT = NTHR, class G = Grp<0, NT, 0>>
+__device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK> sh, float *lam_ws,
                             bool keep_lam, bool prep_only = false, bool grams_ext = false) {
     static_assert(NT % 64 == 0 && NT >= 256, "thread count");
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = G::tid(), warp = tid >> 5, lane = tid & 31;
     bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
 
-    if (tid == 0) sh.slow = 0;
-    // ---- pass 1: segment sums of log_alpha per channel pair, and w . v in place of v
+    if (tid == 0) *sh.slow = 0;
+    // ---- pass 1: w . v in place of v (then w is dead: the segment sums may
+    // live in its tile), and the segment sums of log_alpha per channel pair
     constexpr int NP = DK / 2, P2 = NT / NP, RS2 = C / P2;
     const int cp = tid % NP, s2 = tid / NP, c2 = 2 * cp;
-    {
-        float pa = 0.f, pb = 0.f;
-#pragma unroll 4
-        for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r) {
-            const float2 l = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.la + swz<DK>(r, c2)));
-            pa += l.x;
-            pb += l.y;
-        }
-        sh.part[s2][c2] = pa;
-        sh.part[s2][c2 + 1] = pb;
-        for (int id = tid; id < (prep_only ? 0 : C * DV / 8); id += NT) {
+    if (!prep_only) {
+        for (int id = tid; id < C * DV / 8; id += NT) {
             uint4 wv = reinterpret_cast<const uint4 *>(st.w)[id];
             uint4 vv = reinterpret_cast<const uint4 *>(st.v)[id];
             const bf16 *w8 = reinterpret_cast<const bf16 *>(&wv);
@@ -358,8 +373,20 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
                                   __bfloat162float(w8[2 * e + 1]) * __bfloat162float(v8[2 * e + 1]));
             reinterpret_cast<uint4 *>(st.v)[id] = o;
         }
+        G::sync();
     }
-    __syncthreads();
+    {
+        float pa = 0.f, pb = 0.f;
+#pragma unroll 4
+        for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r) {
+            const float2 l = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.la + swz<DK>(r, c2)));
+            pa += l.x;
+            pb += l.y;
+        }
+        sh.part[s2][c2] = pa;
+        sh.part[s2][c2 + 1] = pb;
+    }
+    G::sync();
     float la0 = 0.f, lb0 = 0.f, la_end = 0.f, lb_end = 0.f;
 #pragma unroll
     for (int s = 0; s < P2; ++s) {
@@ -371,10 +398,10 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
     if (s2 == 0) {
         sh.gamma[c2] = __expf(la_end);
         sh.gamma[c2 + 1] = __expf(lb_end);
-        if (-la_end > kSpanGuard || -lb_end > kSpanGuard) sh.slow = 1;
+        if (-la_end > kSpanGuard || -lb_end > kSpanGuard) *sh.slow = 1;
     }
-    __syncthreads();
-    const bool slow = sh.slow != 0;
+    G::sync();
+    const bool slow = *sh.slow != 0;
 
     float accM[1][8][4];  // M rows of warps 4..7 (lower incl. diagonal)
     if (!slow) {
@@ -395,7 +422,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
             *reinterpret_cast<uint32_t *>(st.b + o) = pack_bf16(b2.x * k2.x * ea, b2.y * k2.y * eb);
             *reinterpret_cast<uint32_t *>(st.la + o) = pack_bf16(k2.x * iea, k2.y * ieb);
         }
-        __syncthreads();
+        G::sync();
         if (prep_only || grams_ext) return false;
         // ---- Grams: [Gt; Qt] Kb^T, warp w < 8 -> rows 16w..16w+15 of the stacked operand
         if (warp < 8) {
@@ -424,7 +451,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
                 lam_ws[r * DK + tid] = lam;
             }
         }
-        __syncthreads();
+        G::sync();
         constexpr int NPAIR = C * (C + 1) / 2, NS = (NPAIR + NT - 1) / NT;
         float pa[NS], pm[NS];
 #pragma unroll
@@ -446,7 +473,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
                 }
             }
         }
-        __syncthreads();
+        G::sync();
         // Qt, Gt and Kt = k e^{L_end - L} in place of q, b, log_alpha
         if (tid < DK) {
             const float lend = lam_ws[(C - 1) * DK + tid];
@@ -460,13 +487,13 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
                 st.la[o] = __float2bfloat16_rn(kk * __expf(lend - lr));
             }
         }
-        __syncthreads();
+        G::sync();
         if (prep_only) return true;
         for (int e = tid; e < C * C; e += NT) {
             A32[e] = 0.f;
             T32[e] = 0.f;
         }
-        __syncthreads();
+        G::sync();
 #pragma unroll
         for (int s = 0; s < NS; ++s) {
             const int p = tid + NT * s;
@@ -479,7 +506,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
                 T32[r * C + i] = pm[s];  // M parked in the T region
             }
         }
-        __syncthreads();
+        G::sync();
         if (warp >= 4 && warp < 8) {
             const int r0 = 16 * (warp & 3) + (lane >> 2);
 #pragma unroll
@@ -489,12 +516,12 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraShared<D
                     accM[0][nt][e] = T32[(r0 + (e >> 1) * 8) * C + 8 * nt + 2 * (lane & 3) + (e & 1)];
         }
     }
-    __syncthreads();
+    G::sync();
 
-    wy_solve<NT>(A32, T32);
+    wy_solve<NT, G>(A32, T32);
     // M -> M16 (bf16, swizzled [64][64]; the second half of the T32 area)
     if (warp >= 4 && warp < 8) store_tile_bf16<8, 64>(accM, M16, 16 * (warp & 3), lane, 1.f);
-    __syncthreads();
+    G::sync();
     return slow;
 }
 

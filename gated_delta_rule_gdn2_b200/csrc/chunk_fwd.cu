@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
 
         cp_wait<1>();
         __syncthreads();
-        const bool slow = intra_chunk<DK, DV>(st, A32, T32, sh, lam_ws, false);
+        const bool slow = intra_chunk<DK, DV>(st, A32, T32, view(sh), lam_ws, false);
         // T and M (then U, below) for the backward, as their shared-memory images
         if (a.intra) copy_smem_to_global(keep_tile(n), T16, 2 * C * C * 2);
 

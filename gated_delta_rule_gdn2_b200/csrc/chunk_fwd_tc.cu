@@ -39,19 +39,29 @@ constexpr int STAGE = 6 * TILE;          // q k log_alpha b v w
 constexpr int OS16 = 2 * STAGE;          // bf16 copy of S: [2 col blocks][128 rows][64]
 constexpr int OSMALL = OS16 + D * D * 2;
 
+// Two warp groups of 256 threads: A (warps 0..7) runs the intra-chunk stage
+// of chunk m while B (warps 8..15) runs the state chain of chunk m - 1; the
+// two stages of input tiles are the pipeline's buffers.
+constexpr int NT = 512, NG = 256;
+using GA = Grp<1, NG, 0>;
+using GB = Grp<2, NG, NG>;
+
 struct Small {
-    IntraShared<D> intra;
-    uint64_t mbar[1];     // MMA completion
+    float gamma[2][D];    // per stage: gam = e^{L_end} of its chunk
+    int slow[2];          // per stage: the chunk took the exact path
+    uint64_t mbar_a;      // MMA completion, group A
+    uint64_t mbar_b;      // MMA completion, group B
     uint64_t mbar_ld[2];  // tile loads of stage 0 and 1
+    uint64_t ready[2];    // stage s: its intra-chunk stage is done
     uint32_t tmem;
     int abort;
 };
 constexpr int BYTES = OSMALL + (int)sizeof(Small);
 static_assert(BYTES <= 232448, "shared memory per block");
 
-// Tensor memory: U (Uv, then + (-W) S), O (Qt S, then + M U), the state S
-// (fp32, 128 key rows x 128 value columns) and a work region for the Grams
-// (A | M, 64 columns each) and then T Gt.
+// Tensor memory: group B's U (T Gt, then T (w . v) + (-W) S), O (Qt S, then
+// + M U) and the state S (fp32, 128 key rows x 128 value columns); group A's
+// Grams (A | M, 64 columns each).
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t COL_U = 0, COL_O = 128, COL_S = 256, COL_G = 384;
 constexpr uint32_t ID64x64_K_K = tc::idesc_bf16(64, 64, false, false);
@@ -91,7 +101,7 @@ __device__ __forceinline__ void issue_chunk(const FwdMaps &m, ChunkTiles st, int
     }
 }
 
-__global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, const __grid_constant__ FwdMaps maps) {
+__global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, const __grid_constant__ FwdMaps maps) {
     extern __shared__ __align__(1024) unsigned char smem[];
     Small &sm = *reinterpret_cast<Small *>(smem + OSMALL);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -101,18 +111,15 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, c
     }
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
     const int nchunks = (a.T + C - 1) / C;
-    const bool with_o = a.o != nullptr;
-    auto keep_tile = [&](int n) {
-        return static_cast<unsigned char *>(a.intra) + ((size_t)bh * nchunks + n) * intra_tile_bytes(D);
-    };
-    float *lam_ws = a.ws ? a.ws + (size_t)bh * a.ws_stride : nullptr;
-    bf16 *S16 = reinterpret_cast<bf16 *>(smem + OS16);
 
     if (warp == 0) tc::tmem_alloc(&sm.tmem, kTmemCols);
     if (tid == 0) {
-        tc::mbar_init(&sm.mbar[0], 1);
-        tc::mbar_init(&sm.mbar_ld[0], 1);
-        tc::mbar_init(&sm.mbar_ld[1], 1);
+        tc::mbar_init(&sm.mbar_a, 1);
+        tc::mbar_init(&sm.mbar_b, 1);
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&sm.mbar_ld[i], 1);
+            tc::mbar_init(&sm.ready[i], 1);
+        }
         tc::fence_mbar_init();
         sm.abort = 0;
     }
@@ -120,255 +127,293 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, c
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = sm.tmem;
-
-    // Thread <-> state row c = 32 p + lane of sub-partition p; warps p and
-    // p + 4 share the rows and take column halves hc = 0, 1.
-    const int p = warp & 3, hc = warp >> 2, c = 32 * p + lane;
-    const uint32_t t_row = tmem + ((uint32_t)(32 * p) << 16) + COL_S + 64 * hc;
-
-    // bf16 copy of this thread's 64 state values into S16
-    auto put_state = [&](const float (&v)[64]) {
-        bf16 *row = S16 + hc * (D * 64) + c * 64;
-#pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) {
-            uint4 u;
-            u.x = pack_bf16(v[8 * q8 + 0], v[8 * q8 + 1]);
-            u.y = pack_bf16(v[8 * q8 + 2], v[8 * q8 + 3]);
-            u.z = pack_bf16(v[8 * q8 + 4], v[8 * q8 + 5]);
-            u.w = pack_bf16(v[8 * q8 + 6], v[8 * q8 + 7]);
-            *reinterpret_cast<uint4 *>(row + ((q8 ^ (c & 7)) << 3)) = u;
-        }
-    };
-    // The chunk-boundary state n (when requested) as the image of S16, by one
-    // thread after the writers' proxy fence and a barrier.
-    auto keep_state = [&](int n) {
-        if (a.states) {
-            tc::bulk_store(static_cast<bf16 *>(a.states) + ((size_t)bh * (nchunks + 1) + n) * D * D, S16, D * D * 2);
-            tc::bulk_commit();
-        }
-    };
-    auto load_state = [&](float (&v)[64]) {
-        tc::ld_32x32b_x32(t_row, *reinterpret_cast<float(*)[32]>(&v[0]));
-        tc::ld_32x32b_x32(t_row + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
-        tc::wait_ld();
-    };
-    auto store_state = [&](const float (&v)[64]) {
-        tc::st_32x32b_x32(t_row, *reinterpret_cast<const float(*)[32]>(&v[0]));
-        tc::st_32x32b_x32(t_row + 32, *reinterpret_cast<const float(*)[32]>(&v[32]));
-        tc::wait_st();
-    };
-
-    // ---- initial state into TMEM and S16
-    {
-        float v[64];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float4 x = a.S0 ? reinterpret_cast<const float4 *>(a.S0 + (size_t)bh * D * D + (size_t)c * D +
-                                                                     64 * hc)[i]
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-            v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
-        }
-        store_state(v);
-        put_state(v);
-    }
-    tc::fence_async_smem();
-    tc::fence_before();
-    __syncthreads();
-    if (tid == 0) {
-        keep_state(0);
-        issue_chunk(maps, stage_tiles(smem, 0), b, h, 0, &sm.mbar_ld[0]);
-        if (nchunks > 1) issue_chunk(maps, stage_tiles(smem, 1), b, h, 1, &sm.mbar_ld[1]);
-    }
-
-    uint32_t ph_mma = 0, ph_ld[2] = {0, 0};
-    // Commit the MMAs issued so far (thread 0) and wait for them (all threads).
-    auto mma_done = [&]() {
-        if (tid == 0) tc::commit(&sm.mbar[0]);
-        if (!tc::mbar_wait(&sm.mbar[0], ph_mma)) {
+    // TMEM sub-partition of this warp: its 32 lanes (state rows 32 p ..) and
+    // the rows 16 p .. 16 p + 15 of a 64-row product; two warps of each group
+    // share a sub-partition and take the column halves hc = 0, 1.
+    const int p = warp & 3, hc = (warp >> 2) & 1;
+    const uint32_t lane_base = (uint32_t)(32 * p) << 16;
+    // Bounded wait on an mbarrier phase; a timeout is recorded and ends the pass.
+    auto wait_on = [&](uint64_t *mbar, uint32_t &phase) {
+        if (!tc::mbar_wait(mbar, phase)) {
             sm.abort = 1;
             record_status(a.status, GDN2_ERR_TIMEOUT);
         }
-        ph_mma ^= 1;
+        phase ^= 1;
         tc::fence_after();
     };
-    // Shared-memory operands written by the threads -> visible to the tensor cores.
-    auto handoff = [&]() {
-        tc::fence_async_smem();
-        tc::fence_before();
-        __syncthreads();
-        tc::fence_after();
-    };
-    const uint32_t lane_base = (uint32_t)(32 * p) << 16;  // this warp's 16 rows of a 64-row product
 
-    for (int n = 0; n < nchunks; ++n) {
-        ChunkTiles st = stage_tiles(smem, n & 1);
-        float *A32 = reinterpret_cast<float *>(st.k);  // k and w slots are free after the prep
-        float *T32 = reinterpret_cast<float *>(st.w);
-        bf16 *W16 = reinterpret_cast<bf16 *>(A32);     // -W, after the solve
-        bf16 *T16 = reinterpret_cast<bf16 *>(T32);
-        bf16 *M16 = T16 + C * C;
-        bf16 *U16 = st.v;                              // after Uv
+    if (warp < 8) {
+        // ================= group A: decay prep, Grams, WY solve, M =================
+        float *lam_ws = a.ws ? a.ws + (size_t)bh * a.ws_stride : nullptr;
+        uint32_t ph_a = 0, ph_ld[2] = {0, 0};
+        for (int m = 0; m < nchunks; ++m) {
+            const int s = m & 1;
+            ChunkTiles st = stage_tiles(smem, s);
+            float *A32 = reinterpret_cast<float *>(st.k);  // k and w slots are free after the prep
+            float *T32 = reinterpret_cast<float *>(st.w);
+            bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
 
-        if (!tc::mbar_wait(&sm.mbar_ld[n & 1], ph_ld[n & 1])) {
-            sm.abort = 1;
-            record_status(a.status, GDN2_ERR_TIMEOUT);
-        }
-        ph_ld[n & 1] ^= 1;
-        __syncthreads();
-        if (sm.abort) break;
-        // decay prep and w . v; a slow chunk also takes its Grams term by term and
-        // its WY solve here, a fast chunk continues below
-        const bool slow = intra_chunk<D, D>(st, A32, T32, sm.intra, lam_ws, false, false, /*grams_ext=*/true);
-        if (!slow) {
-            // ---- Grams on the tensor cores: A = Gt Kb^T, M = Qt Kb^T (M = N = 64, K = 128)
-            handoff();
-            if (tid == 0) {
-                mma_tiles<true, true>(tmem + COL_G, st.b, 64, st.la, 64, 8, ID64x64_K_K, false);
-                mma_tiles<true, true>(tmem + COL_G + 64, st.q, 64, st.la, 64, 8, ID64x64_K_K, false);
-            }
-            mma_done();
-            {  // A (strictly lower) -> fp32 for the solve
-                Frag<4> f;
-                ld_frag(tmem + lane_base + COL_G + 32 * hc, f);
-                tc::wait_ld();
-                const int r0 = 16 * p + (lane >> 2);
+            wait_on(&sm.mbar_ld[s], ph_ld[s]);
+            GA::sync();
+            if (sm.abort) break;
+            // the segment sums live in the w tile once w . v is formed
+            const IntraView<D> iv{reinterpret_cast<float(*)[D]>(st.w), sm.gamma[s], &sm.slow[s]};
+            // a slow chunk takes its Grams term by term and its WY solve in here
+            const bool slow = intra_chunk<D, D, NG, GA>(st, A32, T32, iv, lam_ws, false, false, /*grams_ext=*/true);
+            if (!slow) {
+                // ---- Grams on the tensor cores: A = Gt Kb^T, M = Qt Kb^T (M = N = 64, K = 128)
+                tc::fence_async_smem();
+                tc::fence_before();
+                GA::sync();
+                tc::fence_after();
+                if (tid == 0) {
+                    mma_tiles<true, true>(tmem + COL_G, st.b, 64, st.la, 64, 8, ID64x64_K_K, false);
+                    mma_tiles<true, true>(tmem + COL_G + 64, st.q, 64, st.la, 64, 8, ID64x64_K_K, false);
+                    tc::commit(&sm.mbar_a);
+                }
+                wait_on(&sm.mbar_a, ph_a);
+                {  // A (strictly lower) -> fp32 for the solve
+                    Frag<4> f;
+                    ld_frag(tmem + lane_base + COL_G + 32 * hc, f);
+                    tc::wait_ld();
+                    const int r0 = 16 * p + (lane >> 2);
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
+                    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        const int r = r0 + 8 * h2, i = 32 * hc + 8 * nt + 2 * (lane & 3);
-                        *reinterpret_cast<float2 *>(A32 + r * C + i) =
-                            make_float2(i < r ? f[0][nt][2 * h2] : 0.f, i + 1 < r ? f[0][nt][2 * h2 + 1] : 0.f);
-                    }
-            }
-            __syncthreads();
-            wy_solve<NTHR>(A32, T32);
-            {  // M (lower with the diagonal) -> bf16, past T16
-                Frag<4> f;
-                ld_frag(tmem + lane_base + COL_G + 64 + 32 * hc, f);
-                tc::wait_ld();
-                const int r0 = 16 * p + (lane >> 2);
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            const int r = r0 + 8 * h2, i = 32 * hc + 8 * nt + 2 * (lane & 3);
+                            *reinterpret_cast<float2 *>(A32 + r * C + i) = make_float2(
+                                i < r ? f[0][nt][2 * h2] : 0.f, i + 1 < r ? f[0][nt][2 * h2 + 1] : 0.f);
+                        }
+                }
+                GA::sync();
+                wy_solve<NG, GA>(A32, T32);
+                {  // M (lower with the diagonal) -> bf16, past T16
+                    Frag<4> f;
+                    ld_frag(tmem + lane_base + COL_G + 64 + 32 * hc, f);
+                    tc::wait_ld();
+                    const int r0 = 16 * p + (lane >> 2);
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
+                    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int r = r0 + (e >> 1) * 8, i = 32 * hc + 8 * nt + 2 * (lane & 3) + (e & 1);
-                        if (i > r) f[0][nt][e] = 0.f;
-                    }
-                store_frag_bf16<64, 4>(f, M16, 16 * p, 32 * hc, lane, 1.f);
-            }
-        }
-        handoff();
-        if (sm.abort) break;
-
-        // ---- Uv = T (w . v) and T Gt on the tensor cores (M = 64, N = 128, K = 64)
-        if (tid == 0) {
-            mma_tiles<true, false>(tmem + COL_U, T16, 64, st.v, 64, 4, ID64x128_K_MN, false);
-            mma_tiles<true, false>(tmem + COL_G, T16, 64, st.b, 64, 4, ID64x128_K_MN, false);
-        }
-        mma_done();
-        {  // -W = -(T Gt) -> bf16 in the k slot
-            Frag<8> f;
-            ld_frag(tmem + lane_base + COL_G + 64 * hc, f);
-            tc::wait_ld();
-            store_frag_bf16<D, 8>(f, W16, 16 * p, 64 * hc, lane, -1.f);
-        }
-        handoff();
-
-        // ---- U = Uv + (-W) S and O = Qt S on the tensor cores; T and M (and U,
-        // below) go out for the backward as their shared-memory images
-        if (tid == 0) {
-            if (a.intra) {
-                tc::bulk_store(keep_tile(n), T16, 2 * C * C * 2);
-                tc::bulk_commit();
-            }
-            mma_tiles<true, false>(tmem + COL_U, W16, 64, S16, D, 8, ID64x128_K_MN, true);
-            if (with_o) mma_tiles<true, false>(tmem + COL_O, st.q, 64, S16, D, 8, ID64x128_K_MN, false);
-        }
-        mma_done();
-        {  // U -> bf16 in the v slot (w . v is consumed)
-            Frag<8> f;
-            ld_frag(tmem + lane_base + COL_U + 64 * hc, f);
-            tc::wait_ld();
-            store_frag_bf16<D, 8>(f, U16, 16 * p, 64 * hc, lane, 1.f);
-        }
-        if (tid == 0) tc::bulk_wait_read();  // the previous state image is out: S16 may be rewritten below
-        handoff();
-        if (sm.abort) break;
-
-        if (tid == 0 && a.intra) {
-            tc::bulk_store(keep_tile(n) + 2 * C * C * 2, U16, C * D * 2);
-            tc::bulk_commit();
-        }
-        // ---- slow chunk: S <- Diag(gam) S before adding Kt^T U
-        if (slow) {
-            float v[64];
-            load_state(v);
-            const float gm = sm.intra.gamma[c];
-#pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] *= gm;
-            store_state(v);
-            tc::fence_before();
-            __syncthreads();
-            tc::fence_after();
-        }
-        // ---- S += Kx^T U ; O += M U
-        if (tid == 0) {
-            mma_tiles<false, false>(tmem + COL_S, st.la, 64, U16, 64, 4, IDESC_S, true);
-            if (with_o) mma_tiles<true, false>(tmem + COL_O, M16, 64, U16, 64, 4, ID64x128_K_MN, true);
-        }
-        mma_done();
-        if (with_o) {  // O -> o (bf16), straight from the fragment layout
-            Frag<8> f;
-            ld_frag(tmem + lane_base + COL_O + 64 * hc, f);
-            tc::wait_ld();
-            const int rl = 16 * p + (lane >> 2);
-            bf16 *o = static_cast<bf16 *>(a.o);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int t = n * C + rl + 8 * half;
-                if (t < a.T) {
-                    bf16 *orow = o + (((size_t)b * a.T + t) * a.H + h) * D + 64 * hc;
-#pragma unroll
-                    for (int nt = 0; nt < 8; ++nt)
-                        *reinterpret_cast<uint32_t *>(orow + 8 * nt + 2 * (lane & 3)) =
-                            pack_bf16(f[0][nt][2 * half], f[0][nt][2 * half + 1]);
+                        for (int e = 0; e < 4; ++e) {
+                            const int r = r0 + (e >> 1) * 8, i = 32 * hc + 8 * nt + 2 * (lane & 3) + (e & 1);
+                            if (i > r) f[0][nt][e] = 0.f;
+                        }
+                    store_frag_bf16<64, 4>(f, M16, 16 * p, 32 * hc, lane, 1.f);
                 }
             }
+            // hand the stage to group B: every write of it fenced against the
+            // tensor cores and the TMA, then one arrival
+            tc::fence_async_smem();
+            tc::fence_before();
+            GA::sync();
+            if (tid == 0) tc::mbar_arrive(&sm.ready[s]);
         }
-
-        // ---- S <- Diag(gam) S (fast chunk), bf16 copy for the next chunk
-        {
-            float v[64];
-            load_state(v);
-            if (!slow) {
-                const float gm = sm.intra.gamma[c];
-#pragma unroll
-                for (int i = 0; i < 64; ++i) v[i] *= gm;
-                store_state(v);
+    } else {
+        // ================= group B: the state chain =================
+        const int tb = tid - NG;
+        const bool with_o = a.o != nullptr;
+        bf16 *S16 = reinterpret_cast<bf16 *>(smem + OS16);
+        const int c = 32 * p + lane;  // this thread's state row; columns 64 hc .. 64 hc + 63
+        const uint32_t t_row = tmem + lane_base + COL_S + 64 * hc;
+        auto keep_tile = [&](int n) {
+            return static_cast<unsigned char *>(a.intra) + ((size_t)bh * nchunks + n) * intra_tile_bytes(D);
+        };
+        // the chunk-boundary state n (when requested) as the image of S16 (thread tb = 0)
+        auto keep_state = [&](int n) {
+            if (a.states) {
+                tc::bulk_store(static_cast<bf16 *>(a.states) + ((size_t)bh * (nchunks + 1) + n) * D * D, S16,
+                               D * D * 2);
+                tc::bulk_commit();
             }
-            put_state(v);
-        }
-        tc::fence_async_smem();
-        tc::fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            // this stage's T, M and U images are out before the stage is refilled
-            tc::bulk_wait_read();
-            if (n + 2 < nchunks) issue_chunk(maps, st, b, h, n + 2, &sm.mbar_ld[n & 1]);
-            keep_state(n + 1);
-        }
-    }
-    if (tid == 0) tc::bulk_wait();
-    __syncthreads();
-
-    if (a.S_T && !sm.abort) {
-        tc::fence_after();
-        float v[64];
-        load_state(v);
-        float4 *dst = reinterpret_cast<float4 *>(a.S_T + (size_t)bh * D * D + (size_t)c * D + 64 * hc);
+        };
+        // 32 state values of this thread (half i of its 64 columns) <-> TMEM, and
+        // their bf16 copy into S16
+        auto load_half = [&](int i, float (&v)[32]) {
+            tc::ld_32x32b_x32(t_row + 32 * i, v);
+            tc::wait_ld();
+        };
+        auto store_half = [&](int i, const float (&v)[32]) {
+            tc::st_32x32b_x32(t_row + 32 * i, v);
+            tc::wait_st();
+        };
+        auto put_half = [&](int i, const float (&v)[32]) {
+            bf16 *row = S16 + hc * (D * 64) + c * 64;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            for (int j = 0; j < 4; ++j) {
+                uint4 u;
+                u.x = pack_bf16(v[8 * j + 0], v[8 * j + 1]);
+                u.y = pack_bf16(v[8 * j + 2], v[8 * j + 3]);
+                u.z = pack_bf16(v[8 * j + 4], v[8 * j + 5]);
+                u.w = pack_bf16(v[8 * j + 6], v[8 * j + 7]);
+                *reinterpret_cast<uint4 *>(row + (((4 * i + j) ^ (c & 7)) << 3)) = u;
+            }
+        };
+        auto handoff = [&]() {
+            tc::fence_async_smem();
+            tc::fence_before();
+            GB::sync();
+            tc::fence_after();
+        };
+
+        // initial state into TMEM (its bf16 copy is formed in the first chunk)
+        for (int i = 0; i < 2; ++i) {
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float4 x = a.S0 ? reinterpret_cast<const float4 *>(a.S0 + (size_t)bh * D * D + (size_t)c * D +
+                                                                         64 * hc + 32 * i)[j]
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+            }
+            store_half(i, v);
+        }
+        if (tb == 0) {
+            issue_chunk(maps, stage_tiles(smem, 0), b, h, 0, &sm.mbar_ld[0]);
+            if (nchunks > 1) issue_chunk(maps, stage_tiles(smem, 1), b, h, 1, &sm.mbar_ld[1]);
+        }
+
+        // gam of the previous chunk for this thread's row, when that chunk's
+        // state update still owes the Diag(gam) (a fast chunk)
+        float gm_owed = 1.f;
+        uint32_t ph_b = 0, ph_rdy[2] = {0, 0};
+        for (int n = 0; n < nchunks; ++n) {
+            const int s = n & 1;
+            ChunkTiles st = stage_tiles(smem, s);
+            bf16 *W16 = st.k;  // -W, in the k slot
+            bf16 *T16 = reinterpret_cast<bf16 *>(st.w);
+            bf16 *M16 = T16 + C * C;
+            bf16 *U16 = st.v;  // after T (w . v)
+
+            wait_on(&sm.ready[s], ph_rdy[s]);
+            GB::sync();
+            if (sm.abort) break;
+            const bool slow = sm.slow[s] != 0;
+            const float gm = sm.gamma[s][c];
+
+            // ---- T Gt (M = 64, N = 128, K = 64) -> -W in bf16
+            if (tb == 0) {
+                mma_tiles<true, false>(tmem + COL_U, T16, 64, st.b, 64, 4, ID64x128_K_MN, false);
+                tc::commit(&sm.mbar_b);
+            }
+            wait_on(&sm.mbar_b, ph_b);
+            {
+                Frag<8> f;
+                ld_frag(tmem + lane_base + COL_U + 64 * hc, f);
+                tc::wait_ld();
+                store_frag_bf16<D, 8>(f, W16, 16 * p, 64 * hc, lane, -1.f);
+            }
+            // ---- the chunk-start state: the owed Diag(gam) of the previous chunk, and its bf16 copy
+            for (int i = 0; i < 2; ++i) {
+                float v[32];
+                load_half(i, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] *= gm_owed;
+                store_half(i, v);  // (warp-collective: never behind a per-thread condition)
+                put_half(i, v);
+            }
+            handoff();
+
+            // ---- U = T (w . v) + (-W) S and O = Qt S; the state, T and M (and U,
+            // below) go out for the backward as their shared-memory images
+            if (tb == 0) {
+                keep_state(n);
+                if (a.intra) {
+                    tc::bulk_store(keep_tile(n), T16, 2 * C * C * 2);
+                    tc::bulk_commit();
+                }
+                mma_tiles<true, false>(tmem + COL_U, T16, 64, st.v, 64, 4, ID64x128_K_MN, false);
+                mma_tiles<true, false>(tmem + COL_U, W16, 64, S16, D, 8, ID64x128_K_MN, true);
+                if (with_o) mma_tiles<true, false>(tmem + COL_O, st.q, 64, S16, D, 8, ID64x128_K_MN, false);
+                tc::commit(&sm.mbar_b);
+            }
+            wait_on(&sm.mbar_b, ph_b);
+            {  // U -> bf16 in the v slot (w . v is consumed)
+                Frag<8> f;
+                ld_frag(tmem + lane_base + COL_U + 64 * hc, f);
+                tc::wait_ld();
+                store_frag_bf16<D, 8>(f, U16, 16 * p, 64 * hc, lane, 1.f);
+            }
+            handoff();
+            if (sm.abort) break;
+            if (tb == 0 && a.intra) {
+                tc::bulk_store(keep_tile(n) + 2 * C * C * 2, U16, C * D * 2);
+                tc::bulk_commit();
+            }
+            // ---- slow chunk: S <- Diag(gam) S before adding Kt^T U
+            if (slow) {
+                for (int i = 0; i < 2; ++i) {
+                    float v[32];
+                    load_half(i, v);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] *= gm;
+                    store_half(i, v);
+                }
+                tc::fence_before();
+                GB::sync();
+                tc::fence_after();
+            }
+            // ---- S += Kx^T U ; O += M U
+            if (tb == 0) {
+                mma_tiles<false, false>(tmem + COL_S, st.la, 64, U16, 64, 4, IDESC_S, true);
+                if (with_o) mma_tiles<true, false>(tmem + COL_O, M16, 64, U16, 64, 4, ID64x128_K_MN, true);
+                tc::commit(&sm.mbar_b);
+            }
+            wait_on(&sm.mbar_b, ph_b);
+            gm_owed = slow ? 1.f : gm;  // a fast chunk's Diag(gam) is applied with the next bf16 copy
+            if (with_o) {  // O -> o (bf16), straight from the fragment layout
+                Frag<8> f;
+                ld_frag(tmem + lane_base + COL_O + 64 * hc, f);
+                tc::wait_ld();
+                const int rl = 16 * p + (lane >> 2);
+                bf16 *o = static_cast<bf16 *>(a.o);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int t = n * C + rl + 8 * half;
+                    if (t < a.T) {
+                        bf16 *orow = o + (((size_t)b * a.T + t) * a.H + h) * D + 64 * hc;
+#pragma unroll
+                        for (int nt = 0; nt < 8; ++nt)
+                            *reinterpret_cast<uint32_t *>(orow + 8 * nt + 2 * (lane & 3)) =
+                                pack_bf16(f[0][nt][2 * half], f[0][nt][2 * half + 1]);
+                    }
+                }
+            }
+            tc::fence_before();
+            GB::sync();
+            if (tb == 0) {
+                // the stage's T, M, U images and the state image are out before the
+                // stage is refilled (and before S16 is rewritten, which follows this
+                // thread's next MMA issue)
+                tc::bulk_wait_read();
+                if (n + 2 < nchunks) issue_chunk(maps, st, b, h, n + 2, &sm.mbar_ld[s]);
+            }
+        }
+        GB::sync();
+        if (!sm.abort) {  // the final state: S_T and (when requested) its bf16 image
+            tc::fence_after();
+            for (int i = 0; i < 2; ++i) {
+                float v[32];
+                load_half(i, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] *= gm_owed;
+                if (a.S_T) {
+                    float4 *dst = reinterpret_cast<float4 *>(a.S_T + (size_t)bh * D * D + (size_t)c * D + 64 * hc +
+                                                             32 * i);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                }
+                put_half(i, v);
+            }
+            if (a.states) {
+                tc::fence_async_smem();
+                GB::sync();
+                if (tb == 0) keep_state(nchunks);
+            }
+        }
+        if (tb == 0) tc::bulk_wait();
     }
     tc::fence_before();
     __syncthreads();
@@ -390,7 +435,7 @@ cudaError_t launch_chunk_fwd_tc(const ChunkFwdArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(cfwd_tc::chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          cfwd_tc::BYTES);
     if (e != cudaSuccess) return e;
-    cfwd_tc::chunk_fwd_tc_kernel<<<(unsigned)(a.B * a.H), chunk::NTHR, cfwd_tc::BYTES, s>>>(a, m);
+    cfwd_tc::chunk_fwd_tc_kernel<<<(unsigned)(a.B * a.H), cfwd_tc::NT, cfwd_tc::BYTES, s>>>(a, m);
     return cudaGetLastError();
 }
 

@@ -71,6 +71,11 @@ __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::);
 }
 
+// One arrival (release) on `mbar`.
+__device__ __forceinline__ void mbar_arrive(uint64_t *mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(mbar)) : "memory");
+}
+
 // Bounded wait for the phase `parity` of `mbar`; false when it ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint32_t max_iter = 1u << 22) {
     const uint32_t a = smem_addr(mbar);
