@@ -335,10 +335,32 @@ __device__ void wy_solve(const float *A32, float *T32) {
     }
 }
 
+// w . v in place of v (the NT threads of G; no barrier).
+template <int DV, int NT, class G = Grp<0, NT, 0>>
+__device__ __forceinline__ void form_wv(ChunkTiles st) {
+    for (int id = G::tid(); id < C * DV / 8; id += NT) {
+        uint4 wv = reinterpret_cast<const uint4 *>(st.w)[id];
+        uint4 vv = reinterpret_cast<const uint4 *>(st.v)[id];
+        const bf16 *w8 = reinterpret_cast<const bf16 *>(&wv);
+        const bf16 *v8 = reinterpret_cast<const bf16 *>(&vv);
+        uint4 o;
+        uint32_t *o4 = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            o4[e] = pack_bf16(__bfloat162float(w8[2 * e]) * __bfloat162float(v8[2 * e]),
+                              __bfloat162float(w8[2 * e + 1]) * __bfloat162float(v8[2 * e + 1]));
+        reinterpret_cast<uint4 *>(st.v)[id] = o;
+    }
+}
+
 // Intra-chunk stage.  On entry the six raw token tiles of the chunk are in
 // shared memory (and visible to all threads).  With prep_only only the decay
 // prefix and the operands Qt, Gt, Kb/Kt are formed (v, w untouched; T, M
-// come from elsewhere).  Otherwise, on exit (all threads, after a barrier):
+// come from elsewhere).  With grams_ext a fast chunk stops there too (the
+// caller forms A, M and T); without wv_here the caller forms w . v (form_wv)
+// for a fast chunk, and the slow path forms it before reusing the w tile.
+// The scratch's part array needs NT / (DK / 2) - 1 rows.  Otherwise, on exit
+// (all threads, after a barrier):
 //   st.q -> Qt, st.b -> Gt, st.la -> Kb (fast) or Kt (slow), st.v -> w . v;
 //   T16 = bf16 (I + A)^{-1} and M16 = bf16 M (swizzled [64][64]);
 //   sh.gamma = e^{L_end}; returns true for a slow chunk.
@@ -349,53 +371,36 @@ __device__ void wy_solve(const float *A32, float *T32) {
 // G: the threads that run it (the whole CTA by default).
 template <int DK, int DV, int NT = NTHR, class G = Grp<0, NT, 0>>
 __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK> sh, float *lam_ws,
-                            bool keep_lam, bool prep_only = false, bool grams_ext = false) {
+                            bool keep_lam, bool prep_only = false, bool grams_ext = false, bool wv_here = true) {
     static_assert(NT % 64 == 0 && NT >= 256, "thread count");
     const int tid = G::tid(), warp = tid >> 5, lane = tid & 31;
     bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
 
     if (tid == 0) *sh.slow = 0;
-    // ---- pass 1: w . v in place of v (then w is dead: the segment sums may
-    // live in its tile), and the segment sums of log_alpha per channel pair
+    // ---- pass 1: w . v in place of v (unless the caller forms it later), and the
+    // segment sums of log_alpha per channel pair; only the first P2 - 1 are
+    // stored (the last segment's threads form the chunk total themselves)
     constexpr int NP = DK / 2, P2 = NT / NP, RS2 = C / P2;
     const int cp = tid % NP, s2 = tid / NP, c2 = 2 * cp;
-    if (!prep_only) {
-        for (int id = tid; id < C * DV / 8; id += NT) {
-            uint4 wv = reinterpret_cast<const uint4 *>(st.w)[id];
-            uint4 vv = reinterpret_cast<const uint4 *>(st.v)[id];
-            const bf16 *w8 = reinterpret_cast<const bf16 *>(&wv);
-            const bf16 *v8 = reinterpret_cast<const bf16 *>(&vv);
-            uint4 o;
-            uint32_t *o4 = reinterpret_cast<uint32_t *>(&o);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                o4[e] = pack_bf16(__bfloat162float(w8[2 * e]) * __bfloat162float(v8[2 * e]),
-                                  __bfloat162float(w8[2 * e + 1]) * __bfloat162float(v8[2 * e + 1]));
-            reinterpret_cast<uint4 *>(st.v)[id] = o;
-        }
-        G::sync();
-    }
-    {
-        float pa = 0.f, pb = 0.f;
+    if (!prep_only && wv_here) form_wv<DV, NT, G>(st);
+    float pa = 0.f, pb = 0.f;
 #pragma unroll 4
-        for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r) {
-            const float2 l = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.la + swz<DK>(r, c2)));
-            pa += l.x;
-            pb += l.y;
-        }
+    for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r) {
+        const float2 l = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.la + swz<DK>(r, c2)));
+        pa += l.x;
+        pb += l.y;
+    }
+    if (s2 < P2 - 1) {
         sh.part[s2][c2] = pa;
         sh.part[s2][c2 + 1] = pb;
     }
     G::sync();
-    float la0 = 0.f, lb0 = 0.f, la_end = 0.f, lb_end = 0.f;
+    float la0 = 0.f, lb0 = 0.f;
 #pragma unroll
-    for (int s = 0; s < P2; ++s) {
-        const float pa = sh.part[s][c2], pb = sh.part[s][c2 + 1];
-        if (s < s2) { la0 += pa; lb0 += pb; }
-        la_end += pa;
-        lb_end += pb;
-    }
-    if (s2 == 0) {
+    for (int s = 0; s < P2 - 1; ++s)
+        if (s < s2) { la0 += sh.part[s][c2]; lb0 += sh.part[s][c2 + 1]; }
+    if (s2 == P2 - 1) {
+        const float la_end = la0 + pa, lb_end = lb0 + pb;
         sh.gamma[c2] = __expf(la_end);
         sh.gamma[c2 + 1] = __expf(lb_end);
         if (-la_end > kSpanGuard || -lb_end > kSpanGuard) *sh.slow = 1;
@@ -443,7 +448,9 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK>
     } else {
         // ---- slow chunk: exact per-term decays.  L goes to the per-CTA
         // workspace (one thread per key channel); raw q, k, b stay in shared
-        // memory until A and M exist.
+        // memory until A and M exist.  w . v is formed first when the caller
+        // deferred it: the w tile becomes the T32 work area below.
+        if (!prep_only && !wv_here) form_wv<DV, NT, G>(st);
         if (tid < DK) {
             float lam = 0.f;
             for (int r = 0; r < C; ++r) {

@@ -47,6 +47,7 @@ using GA = Grp<1, NG, 0>;
 using GB = Grp<2, NG, NG>;
 
 struct Small {
+    float part[NG / (D / 2) - 1][D];  // group A: segment sums of log_alpha
     float gamma[2][D];    // per stage: gam = e^{L_end} of its chunk
     int slow[2];          // per stage: the chunk took the exact path
     uint64_t mbar_a;      // MMA completion, group A
@@ -156,10 +157,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             wait_on(&sm.mbar_ld[s], ph_ld[s]);
             GA::sync();
             if (sm.abort) break;
-            // the segment sums live in the w tile once w . v is formed
-            const IntraView<D> iv{reinterpret_cast<float(*)[D]>(st.w), sm.gamma[s], &sm.slow[s]};
-            // a slow chunk takes its Grams term by term and its WY solve in here
-            const bool slow = intra_chunk<D, D, NG, GA>(st, A32, T32, iv, lam_ws, false, false, /*grams_ext=*/true);
+            const IntraView<D> iv{sm.part, sm.gamma[s], &sm.slow[s]};
+            // a slow chunk takes its Grams term by term, its WY solve and w . v in
+            // here; a fast chunk forms w . v below, while its Grams run
+            const bool slow = intra_chunk<D, D, NG, GA>(st, A32, T32, iv, lam_ws, false, false, /*grams_ext=*/true,
+                                                        /*wv_here=*/false);
             if (!slow) {
                 // ---- Grams on the tensor cores: A = Gt Kb^T, M = Qt Kb^T (M = N = 64, K = 128)
                 tc::fence_async_smem();
@@ -171,6 +173,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                     mma_tiles<true, true>(tmem + COL_G + 64, st.q, 64, st.la, 64, 8, ID64x64_K_K, false);
                     tc::commit(&sm.mbar_a);
                 }
+                form_wv<D, NG, GA>(st);  // while the tensor cores run
                 wait_on(&sm.mbar_a, ph_a);
                 {  // A (strictly lower) -> fp32 for the solve
                     Frag<4> f;
