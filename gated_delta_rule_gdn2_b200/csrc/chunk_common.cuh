@@ -292,35 +292,52 @@ __device__ void wy_solve(const float *A32, float *T32) {
         }
     }
     G::sync();
-    // Off-diagonal blocks, one warp per block and level, on the tensor cores
-    // in TF32 (T is rounded to bf16 afterwards): X = sum_J A_RJ T_JQ, then
-    // T_RQ = -T_RR X.  Blocks of one level are independent.
-#pragma unroll 1
-    for (int lvl = 1; lvl < 4; ++lvl) {
-        if (warp < 4 - lvl) {
-            const int Q = warp, R = Q + lvl;
-            const int g = lane >> 2, t = lane & 3;
-            float x[2][4] = {};
-            for (int J = Q; J < R; ++J) block16_tf32(x, A32, 16 * R, 16 * J, T32, 16 * Q, lane);
+    // Off-diagonal blocks on the tensor cores in TF32 (T is rounded to bf16
+    // afterwards), two levels of 32 x 32 blocks, one warp per 16 x 16 block:
+    //   T10 = -T11 A10 T00,  T32 = -T33 A32 T22;
+    //   [T20 T21; T30 T31] = -[T22 0; T32 T33] X,  X = A[2:4, 0:2] [T00 0; T10 T11],
+    // where X's terms that need no T10 start beside T10 and T32.
+    const int g = lane >> 2, t = lane & 3;
+    auto put = [&](const float (&x)[2][4], int R, int Q, float sc) {
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int c = 16 * Q + 8 * nt + 2 * t;
-                *reinterpret_cast<float2 *>(T32 + (16 * R + g) * C + c) = make_float2(x[nt][0], x[nt][1]);
-                *reinterpret_cast<float2 *>(T32 + (16 * R + g + 8) * C + c) = make_float2(x[nt][2], x[nt][3]);
-            }
-            __syncwarp();
-            float y[2][4] = {};
-            block16_tf32(y, T32, 16 * R, 16 * R, T32, 16 * Q, lane);
-            __syncwarp();
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int c = 16 * Q + 8 * nt + 2 * t;
-                *reinterpret_cast<float2 *>(T32 + (16 * R + g) * C + c) = make_float2(-y[nt][0], -y[nt][1]);
-                *reinterpret_cast<float2 *>(T32 + (16 * R + g + 8) * C + c) = make_float2(-y[nt][2], -y[nt][3]);
-            }
+        for (int nt = 0; nt < 2; ++nt) {
+            const int c = 16 * Q + 8 * nt + 2 * t;
+            *reinterpret_cast<float2 *>(T32 + (16 * R + g) * C + c) = make_float2(sc * x[nt][0], sc * x[nt][1]);
+            *reinterpret_cast<float2 *>(T32 + (16 * R + g + 8) * C + c) = make_float2(sc * x[nt][2], sc * x[nt][3]);
         }
+    };
+    float x[2][4] = {};
+    if (warp < 2) {  // T10 (warp 0) and T32 (warp 1): Z = A_RQ T_QQ, then -T_RR Z
+        const int Q = 2 * warp, R = Q + 1;
+        block16_tf32(x, A32, 16 * R, 16 * Q, T32, 16 * Q, lane);
+        put(x, R, Q, 1.f);
+        __syncwarp();
+        float y[2][4] = {};
+        block16_tf32(y, T32, 16 * R, 16 * R, T32, 16 * Q, lane);
+        __syncwarp();
+        put(y, R, Q, -1.f);
+    } else if (warp < 6) {  // X20, X30 (first terms), X21, X31
+        const int R = 2 + (warp & 1), Q = (warp - 2) >> 1;
+        block16_tf32(x, A32, 16 * R, 16 * Q, T32, 16 * Q, lane);  // A_R0 T00 or A_R1 T11
+    }
+    G::sync();
+    if (warp >= 2 && warp < 6) {
+        const int R = 2 + (warp & 1), Q = (warp - 2) >> 1;
+        if (Q == 0) block16_tf32(x, A32, 16 * R, 16, T32, 0, lane);  // + A_R1 T10
+        put(x, R, Q, 1.f);                                           // X_RQ in the T_RQ slot
+    }
+    G::sync();
+    if (warp < 4) {  // Y = [T22 0; T32 T33] X into registers, then -Y
+        const int R = 2 + (warp >> 1), Q = warp & 1;
+        float y[2][4] = {};
+        block16_tf32(y, T32, 16 * R, 32, T32, 16 * Q, lane);                 // T_R2 X_2Q
+        if (R == 3) block16_tf32(y, T32, 48, 48, T32, 16 * Q, lane);         // + T33 X_3Q
+        G::sync();
+        put(y, R, Q, -1.f);
+    } else {
         G::sync();
     }
+    G::sync();
     // T32 -> T16 (bf16, swizzled [64][64], the first half of the T32 area)
     {
         constexpr int EPT = C * C / NT;  // elements per thread
