@@ -118,7 +118,7 @@ int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return GDN2_ERR_WORKSPACE;
     if (dtype == GDN2_BF16) {
         ChunkFwdArgs a{q, k, v, log_alpha, b, w, S0, o, S_T, static_cast<float *>(ws),
-                       (size_t)64 * dk, nullptr, nullptr, status_ptr(), B, T, H};
+                       (size_t)64 * dk, nullptr, nullptr, nullptr, status_ptr(), B, T, H};
         return launch_status(launch_chunk_fwd(a, dk, dv, stream));
     }
     // fp32 precision mode: the recurrence token by token in fp32
@@ -176,7 +176,9 @@ int chunk_bwd_impl(const void *q, const void *k, const void *v, const void *log_
         char *st_buf = saved ? static_cast<char *>(const_cast<void *>(states)) : static_cast<char *>(ws);
         float *scr = reinterpret_cast<float *>(static_cast<char *>(ws) + (saved ? 0 : sbytes));
         ChunkBwdArgs a{q, k, v, log_alpha, b, w, S0, dO, dS_T, dq, dk_, dv_, dlog_alpha, db, dw, dS0, st_buf,
-                       st_buf + states_region_bytes(B, T, H, dk, dv), scr, stride, status_ptr(), saved ? 1 : 0,
+                       st_buf + states_region_bytes(B, T, H, dk, dv),
+                       st_buf + states_region_bytes(B, T, H, dk, dv) + intra_region_bytes(B, T, H, dv), scr, stride,
+                       status_ptr(), saved ? 1 : 0,
                        B, T, H};
         return launch_status(launch_chunk_bwd(a, dk, dv, stream));
     }
@@ -223,7 +225,9 @@ int gdn2_chunk_fwd_save(const void *q, const void *k, const void *v, const void 
     const size_t need = gdn2_chunk_fwd_workspace(B, T, H, dk, dv, dtype);
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return GDN2_ERR_WORKSPACE;
     ChunkFwdArgs a{q, k, v, log_alpha, b, w, S0, o, S_T, static_cast<float *>(ws), (size_t)64 * dk, states,
-                   static_cast<char *>(states) + states_region_bytes(B, T, H, dk, dv), status_ptr(), B, T, H};
+                   static_cast<char *>(states) + states_region_bytes(B, T, H, dk, dv),
+                   static_cast<char *>(states) + states_region_bytes(B, T, H, dk, dv) + intra_region_bytes(B, T, H, dv),
+                   status_ptr(), B, T, H};
     return launch_status(launch_chunk_fwd(a, dk, dv, stream));
 }
 

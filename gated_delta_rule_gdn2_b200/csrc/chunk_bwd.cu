@@ -239,7 +239,7 @@ cudaError_t launch_t(const ChunkBwdArgs &a, cudaStream_t s) {
     cudaError_t e = cudaSuccess;
     if (!a.states_given) {
         ChunkFwdArgs f{a.q, a.k, a.v, a.log_alpha, a.b, a.w, a.S0, nullptr, nullptr, a.scratch, a.scr_stride,
-                       a.states, a.intra, a.status, a.B, a.T, a.H};
+                       a.states, a.intra, a.ops, a.status, a.B, a.T, a.H};
         e = launch_chunk_fwd(f, DK, DV, s);
         if (e != cudaSuccess) return e;
     }
@@ -257,7 +257,8 @@ cudaError_t launch_t(const ChunkBwdArgs &a, cudaStream_t s) {
 
 template <int DK, int DV>
 size_t ws_t(int B, int T, int H, size_t *scr_stride, size_t *states_bytes) {
-    const size_t sb = states_region_bytes(B, T, H, DK, DV) + intra_region_bytes(B, T, H, DV);
+    const size_t sb = states_region_bytes(B, T, H, DK, DV) + intra_region_bytes(B, T, H, DV) +
+                      ops_region_bytes(B, T, H, DK, DV);
     const size_t stride = (Scratch<DK>::FLOATS + 63) / 64 * 64;
     if (scr_stride) *scr_stride = stride;
     if (states_bytes) *states_bytes = sb;

@@ -44,9 +44,9 @@ using Chunk = BwdChunk<D, D, NT>;
 constexpr int TILE_BYTES = C * D * 2;
 constexpr int TM_BYTES = 2 * C * C * 2;
 
-// TMA tensor maps of the token tensors.
+// TMA tensor maps of the token tensors read as tiles.
 struct BwdMaps {
-    CUtensorMap q, k, la, b, dO;
+    CUtensorMap la, dO;
 };
 constexpr int BYTES = L::BYTES + 1024;  // + room to align the tiles to 1 KB
 
@@ -144,25 +144,27 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
     };
 
     // Tile loads, issued by one thread through the TMA and counted in bytes on
-    // mbar_ld: group A = the four token tiles and dO (64 x 64 boxes of the
-    // tensor maps, two per tile) and the forward's U; group B = the chunk-start
-    // state and the forward's T, M.  The forward stores U, T, M and the states
-    // as images of their shared-memory tiles, which come back as bulk copies.  They run one chunk ahead: group A
-    // of chunk n - 1 lands while chunk n's token-level gradients are formed,
-    // group B while chunk n - 1's decay prep and E0 run.
+    // mbar_ld: group A = the forward's Qt, Gt, Kb (or Kt) and U, with the raw
+    // log_alpha (into the k slot, for the decay sums) and dO as 64 x 64 boxes
+    // of the tensor maps; group B = the chunk-start state and the forward's T,
+    // M.  The forward stores its tiles as images of shared memory, which come
+    // back as bulk copies.  They run one chunk ahead: group A of chunk n - 1
+    // lands while chunk n's token-level gradients are formed, group B while
+    // chunk n - 1's decay sums and E0 run.
     uint32_t ph_ld[2] = {0, 0};
     auto issue_a = [&](int m) {
         tc::mbar_expect_tx(&mbar_ld[0], 6 * TILE_BYTES);
         const unsigned char *img = x.intra + (size_t)m * x.I_BYTES + TM_BYTES;
+        const unsigned char *op = static_cast<const unsigned char *>(a.ops) + ((size_t)bh * x.nchunks + m) * kOpsTileBytes;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             const int cx = 64 * half, off = half * C * 64;
-            tc::tma_load_4d(st.q + off, &maps.q, cx, x.h, m * C, x.b, &mbar_ld[0]);
-            tc::tma_load_4d(st.k + off, &maps.k, cx, x.h, m * C, x.b, &mbar_ld[0]);
-            tc::tma_load_4d(st.la + off, &maps.la, cx, x.h, m * C, x.b, &mbar_ld[0]);
-            tc::tma_load_4d(st.b + off, &maps.b, cx, x.h, m * C, x.b, &mbar_ld[0]);
+            tc::tma_load_4d(st.k + off, &maps.la, cx, x.h, m * C, x.b, &mbar_ld[0]);
             tc::tma_load_4d(x.dO16 + off, &maps.dO, cx, x.h, m * C, x.b, &mbar_ld[0]);
         }
+        tc::bulk_load(st.q, op, TILE_BYTES, &mbar_ld[0]);
+        tc::bulk_load(st.b, op + TILE_BYTES, TILE_BYTES, &mbar_ld[0]);
+        tc::bulk_load(st.la, op + 2 * TILE_BYTES, TILE_BYTES, &mbar_ld[0]);
         tc::bulk_load(x.U16, img, TILE_BYTES, &mbar_ld[0]);
     };
     auto issue_b = [&](int m) {
@@ -188,7 +190,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         __syncthreads();
         if (abort_flag) break;
         if (n > 0) x.prefetch_vw_l2(n - 1);
-        const bool slow = intra_chunk<D, D, NT>(st, x.A32, x.T32, view(sh), x.LAM, false, /*prep_only=*/true);
+        // gam, the decay segment sums and (slow chunk) L from the raw log_alpha in the k slot
+        ChunkTiles rawla = st;
+        rawla.la = st.k;
+        const bool slow = intra_chunk<D, D, NT>(rawla, x.A32, x.T32, view(sh), x.LAM, false, /*prep_only=*/true,
+                                                false, true, /*pass1_only=*/true);
 
         // ---- E0: D = g . dSigma (g = gam on a fast chunk, else 1) as bf16 and
         // dSigma <- gam . dSigma; on the last chunk also the row sums of
@@ -377,10 +383,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
 
 cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs &a, cudaStream_t s) {
     cbwd_tc::BwdMaps m;
-    if (!token_tensor_map(&m.q, a.q, a.B, a.T, a.H, cbwd_tc::D) ||
-        !token_tensor_map(&m.k, a.k, a.B, a.T, a.H, cbwd_tc::D) ||
-        !token_tensor_map(&m.la, a.log_alpha, a.B, a.T, a.H, cbwd_tc::D) ||
-        !token_tensor_map(&m.b, a.b, a.B, a.T, a.H, cbwd_tc::D) ||
+    if (!token_tensor_map(&m.la, a.log_alpha, a.B, a.T, a.H, cbwd_tc::D) ||
         !token_tensor_map(&m.dO, a.dO, a.B, a.T, a.H, cbwd_tc::D))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(cbwd_tc::chunk_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

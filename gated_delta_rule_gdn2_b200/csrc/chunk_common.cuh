@@ -374,7 +374,9 @@ __device__ __forceinline__ void form_wv(ChunkTiles st) {
 // shared memory (and visible to all threads).  With prep_only only the decay
 // prefix and the operands Qt, Gt, Kb/Kt are formed (v, w untouched; T, M
 // come from elsewhere).  With grams_ext a fast chunk stops there too (the
-// caller forms A, M and T); without wv_here the caller forms w . v (form_wv)
+// caller forms A, M and T); with pass1_only (which implies prep_only) only the
+// segment sums, gam and a slow chunk's L are formed (the operands come from
+// elsewhere); without wv_here the caller forms w . v (form_wv)
 // for a fast chunk, and the slow path forms it before reusing the w tile.
 // The scratch's part array needs NT / (DK / 2) - 1 rows.  Otherwise, on exit
 // (all threads, after a barrier):
@@ -388,7 +390,8 @@ __device__ __forceinline__ void form_wv(ChunkTiles st) {
 // G: the threads that run it (the whole CTA by default).
 template <int DK, int DV, int NT = NTHR, class G = Grp<0, NT, 0>>
 __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK> sh, float *lam_ws,
-                            bool keep_lam, bool prep_only = false, bool grams_ext = false, bool wv_here = true) {
+                            bool keep_lam, bool prep_only = false, bool grams_ext = false, bool wv_here = true,
+                            bool pass1_only = false) {
     static_assert(NT % 64 == 0 && NT >= 256, "thread count");
     const int tid = G::tid(), warp = tid >> 5, lane = tid & 31;
     bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
@@ -424,6 +427,19 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK>
     }
     G::sync();
     const bool slow = *sh.slow != 0;
+    if (pass1_only) {  // the operands come from elsewhere: gam, the segment sums and a slow chunk's L
+        if (slow) {
+            if (tid < DK) {
+                float lam = 0.f;
+                for (int r = 0; r < C; ++r) {
+                    lam += __bfloat162float(st.la[swz<DK>(r, tid)]);
+                    lam_ws[r * DK + tid] = lam;
+                }
+            }
+            G::sync();
+        }
+        return slow;
+    }
 
     float accM[1][8][4];  // M rows of warps 4..7 (lower incl. diagonal)
     if (!slow) {

@@ -295,8 +295,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             const bool slow = sm.slow[s] != 0;
             const float gm = sm.gamma[s][c];
 
-            // ---- T Gt (M = 64, N = 128, K = 64) -> -W in bf16
+            // ---- T Gt (M = 64, N = 128, K = 64) -> -W in bf16; the decayed
+            // operands Qt, Gt, Kb (or Kt) go out for the backward
             if (tb == 0) {
+                if (a.ops) {
+                    unsigned char *op = static_cast<unsigned char *>(a.ops) + ((size_t)bh * nchunks + n) * kOpsTileBytes;
+                    tc::bulk_store(op, st.q, TILE);
+                    tc::bulk_store(op + TILE, st.b, TILE);
+                    tc::bulk_store(op + 2 * TILE, st.la, TILE);
+                    tc::bulk_commit();
+                }
                 mma_tiles<true, false>(tmem + COL_U, T16, 64, st.b, 64, 4, ID64x128_K_MN, false);
                 tc::commit(&sm.mbar_b);
             }
@@ -326,6 +334,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                     tc::bulk_store(keep_tile(n), T16, 2 * C * C * 2);
                     tc::bulk_commit();
                 }
+
                 mma_tiles<true, false>(tmem + COL_U, T16, 64, st.v, 64, 4, ID64x128_K_MN, false);
                 mma_tiles<true, false>(tmem + COL_U, W16, 64, S16, D, 8, ID64x128_K_MN, true);
                 if (with_o) mma_tiles<true, false>(tmem + COL_O, st.q, 64, S16, D, 8, ID64x128_K_MN, false);

@@ -40,6 +40,7 @@ struct ChunkFwdArgs {
     size_t ws_stride;
     void *states;
     void *intra;  // optional: per chunk the bf16 tiles T, M (64x64 each) and U (64 x dv), as in shared memory
+    void *ops;    // optional (dk = dv = 128): per chunk the bf16 operands Qt, Gt, Kb/Kt, as in shared memory
     int *status;  // device status word (bounded waits record GDN2_ERR_TIMEOUT here)
     int B, T, H;
 };
@@ -60,6 +61,7 @@ struct ChunkBwdArgs {
     float *dS0;
     void *states;      // bf16 chunk-boundary states [B*H][nchunks+1][dk][dv]
     void *intra;       // per chunk the bf16 tiles T, M, U of the forward (intra_tile_bytes each)
+    void *ops;         // dk = dv = 128: per chunk the forward's Qt, Gt, Kb/Kt (ops_tile_bytes each)
     float *scratch;
     size_t scr_stride;
     int *status;
@@ -77,6 +79,14 @@ inline size_t states_region_bytes(int B, int T, int H, int dk, int dv) {
 inline size_t intra_region_bytes(int B, int T, int H, int dv) {
     const size_t nc = (size_t)((T + 63) / 64);
     return ((size_t)B * H * nc * intra_tile_bytes(dv) + 255) / 256 * 256;
+}
+// Then, for dk = dv = 128 (the tensor-memory kernels), the decayed operands
+// Qt, Gt and Kb (or Kt) of every chunk, 3 x 64 x 128 bf16 each.
+constexpr size_t kOpsTileBytes = (size_t)3 * 64 * 128 * 2;
+inline size_t ops_region_bytes(int B, int T, int H, int dk, int dv) {
+    if (dk != 128 || dv != 128) return 0;
+    const size_t nc = (size_t)((T + 63) / 64);
+    return (size_t)B * H * nc * kOpsTileBytes;
 }
 
 cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs &a, cudaStream_t s);  // reverse pass, dk = dv = 128, tcgen05

@@ -114,7 +114,8 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
  * needs from the forward: the state at every chunk boundary (bf16,
  * [B][H][ceil(T/64)+1][dk][dv]) and, per chunk, the bf16 WY factor
  * T = (I + A)^{-1}, the decayed query-key Gram M (64 x 64 each) and the
- * chunk's WY-form write U (64 x dv).  gdn2_chunk_bwd_saved is gdn2_chunk_bwd
+ * chunk's WY-form write U (64 x dv), and for dk = dv = 128 also the decayed
+ * operands Qt, Gt, Kb (64 x 128 each).  gdn2_chunk_bwd_saved is gdn2_chunk_bwd
  * that reads these instead of re-running the forward to recompute them, with
  * the smaller workspace gdn2_chunk_bwd_saved_workspace(...).  The buffer must
  * come from gdn2_chunk_fwd_save on the same inputs; results equal those of

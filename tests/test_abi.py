@@ -87,8 +87,13 @@ def test_saved_state_entry_points_validate():
     B, T, H = 2, 100, 3
     n = g.gdn2_chunk_states_bytes(B, T, H, 128, 128, g.GDN2_BF16)
     # ceil(100/64) + 1 bf16 chunk-boundary states, then per chunk the bf16
-    # tiles T, M (64 x 64) and U (64 x dv); both regions are multiples of 256 bytes here
-    assert n == B * H * (2 + 1) * 128 * 128 * 2 + B * H * 2 * (2 * 64 * 64 + 64 * 128) * 2
+    # tiles T, M (64 x 64) and U (64 x dv), then (dk = dv = 128 only) per chunk
+    # the decayed operands Qt, Gt, Kb (64 x 128 each); every region is a
+    # multiple of 256 bytes here
+    assert n == B * H * (2 + 1) * 128 * 128 * 2 + B * H * 2 * (2 * 64 * 64 + 64 * 128) * 2 + \
+        B * H * 2 * 3 * 64 * 128 * 2
+    assert g.gdn2_chunk_states_bytes(B, T, H, 64, 64, g.GDN2_BF16) == \
+        B * H * (2 + 1) * 64 * 64 * 2 + B * H * 2 * (2 * 64 * 64 + 64 * 64) * 2
     assert g.gdn2_chunk_states_bytes(B, T, H, 128, 128, g.GDN2_FP32) == 0
     assert 0 < g.gdn2_chunk_bwd_saved_workspace(B, T, H, 128, 128, g.GDN2_BF16) < \
         g.gdn2_chunk_bwd_workspace(B, T, H, 128, 128, g.GDN2_BF16)
