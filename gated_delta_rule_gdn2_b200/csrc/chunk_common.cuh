@@ -261,13 +261,13 @@ __device__ __forceinline__ void block16_tf32(float (&acc)[2][4], const float *X,
 }
 
 // WY solve: T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 area
-// A32, into T32 (fp32) and then T16 = bf16 T (swizzled [64][64], first half of
-// the T32 area).  All NT threads; on return the area past T16 may be written,
-// and T16 is complete after the caller's next barrier.
+// A32, in the fp32 work area T32 and then as T16 = bf16 T (swizzled [64][64];
+// T16 may be the first half of the T32 area).  All NT threads of G; on return
+// the T32 area past T16 may be written, and T16 is complete after the
+// caller's next barrier.
 template <int NT, class G = Grp<0, NT, 0>>
-__device__ void wy_solve(const float *A32, float *T32) {
+__device__ void wy_solve(const float *A32, float *T32, bf16 *T16) {
     const int tid = G::tid(), warp = tid >> 5, lane = tid & 31;
-    bf16 *T16 = reinterpret_cast<bf16 *>(T32);
     // 16x16 diagonal blocks by substitution in fp32.
     if (tid < 64) {
         // column j of the inverse of unit lower-triangular block R, column by
@@ -558,7 +558,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK>
     }
     G::sync();
 
-    wy_solve<NT, G>(A32, T32);
+    wy_solve<NT, G>(A32, T32, reinterpret_cast<bf16 *>(T32));
     // M -> M16 (bf16, swizzled [64][64]; the second half of the T32 area)
     if (warp >= 4 && warp < 8) store_tile_bf16<8, 64>(accM, M16, 16 * (warp & 3), lane, 1.f);
     G::sync();

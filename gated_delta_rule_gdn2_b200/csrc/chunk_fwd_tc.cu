@@ -144,7 +144,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
     };
 
     if (warp < 8) {
-        // ================= group A: decay prep, Grams, WY solve, M =================
+        // ================= group A: decay prep, Grams, A and M =================
+        // (a fast chunk's WY solve runs in group B; a slow chunk takes its Grams
+        // term by term and its solve in the intra-chunk stage here)
         float *lam_ws = a.ws ? a.ws + (size_t)bh * a.ws_stride : nullptr;
         uint32_t ph_a = 0, ph_ld[2] = {0, 0};
         for (int m = 0; m < nchunks; ++m) {
@@ -189,9 +191,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                                 i < r ? f[0][nt][2 * h2] : 0.f, i + 1 < r ? f[0][nt][2 * h2 + 1] : 0.f);
                         }
                 }
-                GA::sync();
-                wy_solve<NG, GA>(A32, T32);
-                {  // M (lower with the diagonal) -> bf16, past T16
+                GA::sync();  // every thread is done reading w for w . v
+                {  // M (lower with the diagonal) -> bf16 in the second half of the w tile
                     Frag<4> f;
                     ld_frag(tmem + lane_base + COL_G + 64 + 32 * hc, f);
                     tc::wait_ld();
@@ -294,6 +295,14 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             if (sm.abort) break;
             const bool slow = sm.slow[s] != 0;
             const float gm = sm.gamma[s][c];
+            if (!slow) {
+                // ---- WY solve of a fast chunk: A (k slot) -> T16 (first half of the
+                // w tile), with the fp32 work area in the S16 area, free until the
+                // state's bf16 copy below (the previous state image is out)
+                wy_solve<NG, GB>(reinterpret_cast<const float *>(st.k), reinterpret_cast<float *>(S16), T16);
+                tc::fence_async_smem();
+                GB::sync();
+            }
 
             // ---- T Gt (M = 64, N = 128, K = 64) -> -W in bf16; the decayed
             // operands Qt, Gt, Kb (or Kt) go out for the backward
