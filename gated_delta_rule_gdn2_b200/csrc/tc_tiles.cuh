@@ -23,15 +23,25 @@ __device__ __forceinline__ uint64_t mnmaj(const void *tile, int R, int s) {
     return tc::sdesc(tc::smem_addr(tile) + (uint32_t)(s * 2048), (uint32_t)(R * 128), 1024);
 }
 
+// Byte offset of k-step s from k-step 0 of an operand in an [R][.] tile.
+template <bool K_MAJOR>
+__device__ __forceinline__ uint32_t kstep_bytes(int R, int s) {
+    return K_MAJOR ? (uint32_t)((s >> 2) * (R * 128) + (s & 3) * 32) : (uint32_t)(s * 2048);
+}
+
 // D (+)= A B over K = 16 ks, issued by one thread.  A_K / B_K: K-major operand.
+// The descriptors of k-step 0 are built once; a later k-step adds its byte
+// offset / 16 to the start-address field, which cannot carry out of it
+// (shared memory addresses stay below 2^18).
 template <bool A_K, bool B_K>
 __device__ __forceinline__ void mma_tiles(uint32_t d, const void *A, int RA, const void *B, int RB, int ks,
                                           uint32_t idesc, bool accumulate) {
-    for (int s = 0; s < ks; ++s) {
-        const uint64_t da = A_K ? kmaj(A, RA, s) : mnmaj(A, RA, s);
-        const uint64_t db = B_K ? kmaj(B, RB, s) : mnmaj(B, RB, s);
-        tc::mma_bf16(d, da, db, idesc, accumulate || s > 0);
-    }
+    const uint64_t da0 = A_K ? kmaj(A, RA, 0) : mnmaj(A, RA, 0);
+    const uint64_t db0 = B_K ? kmaj(B, RB, 0) : mnmaj(B, RB, 0);
+#pragma unroll
+    for (int s = 0; s < ks; ++s)
+        tc::mma_bf16(d, da0 + (kstep_bytes<A_K>(RA, s) >> 4), db0 + (kstep_bytes<B_K>(RB, s) >> 4), idesc,
+                     accumulate || s > 0);
 }
 
 // A fragment of 8 NTL columns of a 64-row accumulator (16 rows per warp),
