@@ -52,6 +52,7 @@ struct Small {
     int slow[2];          // per stage: the chunk took the exact path
     uint64_t mbar_a;      // MMA completion, group A
     uint64_t mbar_b;      // MMA completion, group B
+    uint64_t mbar_o;      // MMA completion, group B's O = Qt S (a second barrier: each keeps one phase in flight)
     uint64_t mbar_ld[2];  // tile loads of stage 0 and 1
     uint64_t ready[2];    // stage s: its intra-chunk stage is done
     uint32_t tmem;
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
     if (tid == 0) {
         tc::mbar_init(&sm.mbar_a, 1);
         tc::mbar_init(&sm.mbar_b, 1);
+        tc::mbar_init(&sm.mbar_o, 1);
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&sm.mbar_ld[i], 1);
             tc::mbar_init(&sm.ready[i], 1);
@@ -281,7 +283,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         // gam of the previous chunk for this thread's row, when that chunk's
         // state update still owes the Diag(gam) (a fast chunk)
         float gm_owed = 1.f;
-        uint32_t ph_b = 0, ph_rdy[2] = {0, 0};
+        uint32_t ph_b = 0, ph_o = 0, ph_rdy[2] = {0, 0};
         for (int n = 0; n < nchunks; ++n) {
             const int s = n & 1;
             ChunkTiles st = stage_tiles(smem, s);
@@ -304,7 +306,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 GB::sync();
             }
 
-            // ---- T Gt (M = 64, N = 128, K = 64) -> -W in bf16; the decayed
+            // ---- T Gt (M = 64, N = 128, K = 64) on the tensor cores; the decayed
             // operands Qt, Gt, Kb (or Kt) go out for the backward
             if (tb == 0) {
                 if (a.ops) {
@@ -317,14 +319,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 mma_tiles<true, false>(tmem + COL_U, T16, 64, st.b, 64, 4, ID64x128_K_MN, false);
                 tc::commit(&sm.mbar_b);
             }
-            wait_on(&sm.mbar_b, ph_b);
-            {
-                Frag<8> f;
-                ld_frag(tmem + lane_base + COL_U + 64 * hc, f);
-                tc::wait_ld();
-                store_frag_bf16<D, 8>(f, W16, 16 * p, 64 * hc, lane, -1.f);
-            }
-            // ---- the chunk-start state: the owed Diag(gam) of the previous chunk, and its bf16 copy
+            // ---- meanwhile the chunk-start state: the owed Diag(gam) of the
+            // previous chunk, and its bf16 copy (the S16 area is free again)
             for (int i = 0; i < 2; ++i) {
                 float v[32];
                 load_half(i, v);
@@ -334,22 +330,33 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 put_half(i, v);
             }
             handoff();
-
-            // ---- U = T (w . v) + (-W) S and O = Qt S; the state, T and M (and U,
-            // below) go out for the backward as their shared-memory images
+            // ---- O = Qt S; the state, T and M (and U, below) go out for the
+            // backward as their shared-memory images
             if (tb == 0) {
                 keep_state(n);
                 if (a.intra) {
                     tc::bulk_store(keep_tile(n), T16, 2 * C * C * 2);
                     tc::bulk_commit();
                 }
-
+                if (with_o) mma_tiles<true, false>(tmem + COL_O, st.q, 64, S16, D, 8, ID64x128_K_MN, false);
+                tc::commit(&sm.mbar_o);
+            }
+            wait_on(&sm.mbar_b, ph_b);  // T Gt
+            {  // -W = -(T Gt) -> bf16 in the k slot
+                Frag<8> f;
+                ld_frag(tmem + lane_base + COL_U + 64 * hc, f);
+                tc::wait_ld();
+                store_frag_bf16<D, 8>(f, W16, 16 * p, 64 * hc, lane, -1.f);
+            }
+            handoff();
+            // ---- U = T (w . v) + (-W) S
+            if (tb == 0) {
                 mma_tiles<true, false>(tmem + COL_U, T16, 64, st.v, 64, 4, ID64x128_K_MN, false);
                 mma_tiles<true, false>(tmem + COL_U, W16, 64, S16, D, 8, ID64x128_K_MN, true);
-                if (with_o) mma_tiles<true, false>(tmem + COL_O, st.q, 64, S16, D, 8, ID64x128_K_MN, false);
                 tc::commit(&sm.mbar_b);
             }
-            wait_on(&sm.mbar_b, ph_b);
+            wait_on(&sm.mbar_o, ph_o);  // O
+            wait_on(&sm.mbar_b, ph_b);  // U
             {  // U -> bf16 in the v slot (w . v is consumed)
                 Frag<8> f;
                 ld_frag(tmem + lane_base + COL_U + 64 * hc, f);
