@@ -320,10 +320,10 @@ struct BwdChunk {
             if (with_dvdw) dvdw(n, Cn);
             // in-chunk decay prefix of this thread's rows (the prep's segment sums,
             // or the slow chunk's L in the workspace)
-            float la_run = 0.f, lb_run = 0.f;
+            float2 run = make_float2(0.f, 0.f);
 #pragma unroll
             for (int s = 0; s < P2; ++s)
-                if (s < s2) { la_run += sh.part[s][c2]; lb_run += sh.part[s][c2 + 1]; }
+                if (s < s2) { run.x += sh.part[s][c2]; run.y += sh.part[s][c2 + 1]; }
             bf16 *__restrict__ gdq = static_cast<bf16 *>(a.dq);
             bf16 *__restrict__ gdk = static_cast<bf16 *>(a.dk);
             bf16 *__restrict__ gdb = static_cast<bf16 *>(a.db);
@@ -331,7 +331,7 @@ struct BwdChunk {
             const float *__restrict__ sGT = DGT;
             const float *__restrict__ sKB = DKB;
             float dla_r[RS2], dlb_r[RS2];
-            float pa = 0.f, pb = 0.f;
+            float2 psum = make_float2(0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < RS2; ++i) {
                 const int r = s2 * RS2 + i;
@@ -342,54 +342,50 @@ struct BwdChunk {
                     const float2 q = __bfloat1622float2(raw.q[i]);
                     const float2 kk = __bfloat1622float2(raw.k[i]);
                     const float2 bb = __bfloat1622float2(raw.b[i]);
-                    float2 lam;
-                    if (!slow) {
-                        const float2 l = __bfloat1622float2(raw.la[i]);
-                        la_run += l.x;
-                        lb_run += l.y;
-                        lam = make_float2(la_run, lb_run);
-                    } else {
-                        lam = *reinterpret_cast<const float2 *>(LAM + r * DK + c2);
-                    }
                     const float2 dqt = *reinterpret_cast<const float2 *>(sQT + stg<DK>(r, c2));
                     const float2 dgt = *reinterpret_cast<const float2 *>(sGT + stg<DK>(r, c2));
                     const float2 dkb = *reinterpret_cast<const float2 *>(sKB + stg<DK>(r, c2));
-                    const float mdiag = s_dmd[r];
-                    const float ea = __expf(lam.x), eb = __expf(lam.y);
-                    float dqa, dqb, dga, dgb, dka, dkb2, dla, dlb;
+                    const float2 md = make_float2(s_dmd[r], s_dmd[r]);
+                    float2 dq, dg, dk, dl;
                     if (!slow) {
-                        const float iea = __expf(-lam.x), ieb = __expf(-lam.y);
-                        dqa = dqt.x * ea; dqb = dqt.y * eb;
-                        dga = dgt.x * ea; dgb = dgt.y * eb;
-                        dka = dkb.x * iea; dkb2 = dkb.y * ieb;
-                        dla = dqt.x * q.x * ea + dgt.x * bb.x * kk.x * ea - dkb.x * kk.x * iea;
-                        dlb = dqt.y * q.y * eb + dgt.y * bb.y * kk.y * eb - dkb.y * kk.y * ieb;
+                        // both channels at once on the packed fp32x2 pipe
+                        run = __fadd2_rn(run, __bfloat1622float2(raw.la[i]));
+                        const float2 e = make_float2(__expf(run.x), __expf(run.y));
+                        const float2 ie = make_float2(__expf(-run.x), __expf(-run.y));
+                        dq = __fmul2_rn(dqt, e);
+                        dg = __fmul2_rn(dgt, e);
+                        dk = __fmul2_rn(dkb, ie);
+                        dl = __fmul2_rn(dk, make_float2(-kk.x, -kk.y));
+                        dl = __ffma2_rn(dg, __fmul2_rn(bb, kk), dl);
+                        dl = __ffma2_rn(dq, q, dl);
                     } else {
+                        const float2 lam = *reinterpret_cast<const float2 *>(LAM + r * DK + c2);
+                        const float ea = __expf(lam.x), eb = __expf(lam.y);
                         const float kea = __expf(lend.x - lam.x), keb = __expf(lend.y - lam.y);
                         const float2 pq = *reinterpret_cast<const float2 *>(PQ + r * DK + c2);
                         const float2 pg = *reinterpret_cast<const float2 *>(PG + r * DK + c2);
                         const float2 pk = *reinterpret_cast<const float2 *>(PK + r * DK + c2);
                         const float2 pl = *reinterpret_cast<const float2 *>(PL + r * DK + c2);
-                        dqa = dqt.x * ea + pq.x; dqb = dqt.y * eb + pq.y;
-                        dga = dgt.x * ea + pg.x; dgb = dgt.y * eb + pg.y;
-                        dka = dkb.x * kea + pk.x; dkb2 = dkb.y * keb + pk.y;
-                        dla = dqt.x * q.x * ea + dgt.x * bb.x * kk.x * ea - dkb.x * kk.x * kea + pl.x;
-                        dlb = dqt.y * q.y * eb + dgt.y * bb.y * kk.y * eb - dkb.y * kk.y * keb + pl.y;
+                        dq = make_float2(dqt.x * ea + pq.x, dqt.y * eb + pq.y);
+                        dg = make_float2(dgt.x * ea + pg.x, dgt.y * eb + pg.y);
+                        dk = make_float2(dkb.x * kea + pk.x, dkb.y * keb + pk.y);
+                        dl = make_float2(dqt.x * q.x * ea + dgt.x * bb.x * kk.x * ea - dkb.x * kk.x * kea + pl.x,
+                                         dqt.y * q.y * eb + dgt.y * bb.y * kk.y * eb - dkb.y * kk.y * keb + pl.y);
                     }
-                    dqa += mdiag * kk.x; dqb += mdiag * kk.y;
-                    dka += mdiag * q.x; dkb2 += mdiag * q.y;
-                    if (r == Cn - 1) { dla += rsum.x; dlb += rsum.y; }
-                    *reinterpret_cast<uint32_t *>(gdq + o) = pack_bf16(dqa, dqb);
-                    *reinterpret_cast<uint32_t *>(gdk + o) = pack_bf16(dka + dga * bb.x, dkb2 + dgb * bb.y);
-                    *reinterpret_cast<uint32_t *>(gdb + o) = pack_bf16(dga * kk.x, dgb * kk.y);
-                    dla_r[i] = dla;
-                    dlb_r[i] = dlb;
-                    pa += dla;
-                    pb += dlb;
+                    dq = __ffma2_rn(md, kk, dq);
+                    dk = __ffma2_rn(md, q, dk);
+                    if (r == Cn - 1) dl = __fadd2_rn(dl, rsum);
+                    *reinterpret_cast<uint32_t *>(gdq + o) = pack_bf16(dq.x, dq.y);
+                    const float2 dkt = __ffma2_rn(dg, bb, dk), dbt = __fmul2_rn(dg, kk);
+                    *reinterpret_cast<uint32_t *>(gdk + o) = pack_bf16(dkt.x, dkt.y);
+                    *reinterpret_cast<uint32_t *>(gdb + o) = pack_bf16(dbt.x, dbt.y);
+                    dla_r[i] = dl.x;
+                    dlb_r[i] = dl.y;
+                    psum = __fadd2_rn(psum, dl);
                 }
             }
-            s_dpart[s2][c2] = pa;
-            s_dpart[s2][c2 + 1] = pb;
+            s_dpart[s2][c2] = psum.x;
+            s_dpart[s2][c2 + 1] = psum.y;
             __syncthreads();
             float acca = 0.f, accb = 0.f;
 #pragma unroll
