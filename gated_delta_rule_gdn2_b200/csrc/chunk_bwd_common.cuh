@@ -257,18 +257,18 @@ struct BwdChunk {
             const int id = tid + it * NT, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
             if (r < Cn) {
                 const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV + j;
-                const uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, j));
+                uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, j));
+                nr.x ^= 0x80008000u; nr.y ^= 0x80008000u; nr.z ^= 0x80008000u; nr.w ^= 0x80008000u;  // dRHS = -nR
                 const __nv_bfloat162 *n2 = reinterpret_cast<const __nv_bfloat162 *>(&nr);
                 const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&v8[it]);
                 const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&w8[it]);
+                // bf16 x bf16 products: one rounding, as of the exact fp32 product
                 uint4 dv8, dw8;
-                uint32_t *dvp = reinterpret_cast<uint32_t *>(&dv8), *dwp = reinterpret_cast<uint32_t *>(&dw8);
+                __nv_bfloat162 *dvp = reinterpret_cast<__nv_bfloat162 *>(&dv8), *dwp = reinterpret_cast<__nv_bfloat162 *>(&dw8);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float2 d = __bfloat1622float2(n2[e]), vv = __bfloat1622float2(v2[e]),
-                                 ww = __bfloat1622float2(w2[e]);
-                    dvp[e] = pack_bf16(-d.x * ww.x, -d.y * ww.y);
-                    dwp[e] = pack_bf16(-d.x * vv.x, -d.y * vv.y);
+                    dvp[e] = __hmul2(n2[e], w2[e]);
+                    dwp[e] = __hmul2(n2[e], v2[e]);
                 }
                 *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dv) + o) = dv8;
                 *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dw) + o) = dw8;

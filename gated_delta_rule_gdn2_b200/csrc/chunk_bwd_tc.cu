@@ -204,14 +204,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
             tc::ld_32x32b_x32(t_srow, v);
             tc::wait_ld();
             const float gm = sh.gamma[c], g = slow ? 1.f : gm;
+            const float2 g2 = make_float2(g, g), gm2 = make_float2(gm, gm);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                uint4 u;
-                u.x = pack_bf16(g * v[8 * i + 0], g * v[8 * i + 1]);
-                u.y = pack_bf16(g * v[8 * i + 2], g * v[8 * i + 3]);
-                u.z = pack_bf16(g * v[8 * i + 4], g * v[8 * i + 5]);
-                u.w = pack_bf16(g * v[8 * i + 6], g * v[8 * i + 7]);
-                *reinterpret_cast<uint4 *>(const_cast<bf16 *>(tile_row(x.D16, i))) = u;
+                uint32_t u[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 t = __fmul2_rn(make_float2(v[8 * i + 2 * e], v[8 * i + 2 * e + 1]), g2);
+                    u[e] = pack_bf16(t.x, t.y);
+                }
+                *reinterpret_cast<uint4 *>(const_cast<bf16 *>(tile_row(x.D16, i))) = make_uint4(u[0], u[1], u[2], u[3]);
             }
             if (n == x.nchunks - 1) {
                 const bf16 *sig = x.states + (size_t)(n + 1) * D * D;
@@ -221,7 +223,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
                 s_rs[n & 1][qc][c] = rs;
             }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= gm;
+            for (int i = 0; i < 32; i += 2) {
+                const float2 t = __fmul2_rn(make_float2(v[i], v[i + 1]), gm2);
+                v[i] = t.x;
+                v[i + 1] = t.y;
+            }
             tc::st_32x32b_x32(t_srow, v);
             tc::wait_st();
         }

@@ -356,16 +356,16 @@ __device__ void wy_solve(const float *A32, float *T32, bf16 *T16) {
 template <int DV, int NT, class G = Grp<0, NT, 0>>
 __device__ __forceinline__ void form_wv(ChunkTiles st) {
     for (int id = G::tid(); id < C * DV / 8; id += NT) {
+        // the product of two bf16 values is exact in fp32, so the bf16x2 multiply
+        // (one rounding) gives the same bits as an fp32 product rounded to bf16
         uint4 wv = reinterpret_cast<const uint4 *>(st.w)[id];
         uint4 vv = reinterpret_cast<const uint4 *>(st.v)[id];
-        const bf16 *w8 = reinterpret_cast<const bf16 *>(&wv);
-        const bf16 *v8 = reinterpret_cast<const bf16 *>(&vv);
+        const __nv_bfloat162 *w2 = reinterpret_cast<const __nv_bfloat162 *>(&wv);
+        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vv);
         uint4 o;
-        uint32_t *o4 = reinterpret_cast<uint32_t *>(&o);
+        __nv_bfloat162 *o2 = reinterpret_cast<__nv_bfloat162 *>(&o);
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            o4[e] = pack_bf16(__bfloat162float(w8[2 * e]) * __bfloat162float(v8[2 * e]),
-                              __bfloat162float(w8[2 * e + 1]) * __bfloat162float(v8[2 * e + 1]));
+        for (int e = 0; e < 4; ++e) o2[e] = __hmul2(w2[e], v2[e]);
         reinterpret_cast<uint4 *>(st.v)[id] = o;
     }
 }
@@ -403,13 +403,11 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK>
     constexpr int NP = DK / 2, P2 = NT / NP, RS2 = C / P2;
     const int cp = tid % NP, s2 = tid / NP, c2 = 2 * cp;
     if (!prep_only && wv_here) form_wv<DV, NT, G>(st);
-    float pa = 0.f, pb = 0.f;
+    float2 psum = make_float2(0.f, 0.f);
 #pragma unroll 4
-    for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r) {
-        const float2 l = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.la + swz<DK>(r, c2)));
-        pa += l.x;
-        pb += l.y;
-    }
+    for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r)
+        psum = __fadd2_rn(psum, __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.la + swz<DK>(r, c2))));
+    const float pa = psum.x, pb = psum.y;
     if (s2 < P2 - 1) {
         sh.part[s2][c2] = pa;
         sh.part[s2][c2 + 1] = pb;
@@ -444,7 +442,8 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK>
     float accM[1][8][4];  // M rows of warps 4..7 (lower incl. diagonal)
     if (!slow) {
         // ---- pass 2 (fast): Qt, Gt, Kb in place of q, b, log_alpha (two channels per thread)
-        float la = la0, lb = lb0;
+        // (both channels of a thread on the packed fp32x2 pipe)
+        float2 lam = make_float2(la0, lb0);
 #pragma unroll 4
         for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r) {
             const int o = swz<DK>(r, c2);
@@ -452,13 +451,14 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK>
             const float2 q2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.q + o));
             const float2 k2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.k + o));
             const float2 b2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.b + o));
-            la += l.x;
-            lb += l.y;
-            if (keep_lam) *reinterpret_cast<float2 *>(lam_ws + r * DK + c2) = make_float2(la, lb);
-            const float ea = __expf(la), eb = __expf(lb), iea = __expf(-la), ieb = __expf(-lb);
-            *reinterpret_cast<uint32_t *>(st.q + o) = pack_bf16(q2.x * ea, q2.y * eb);
-            *reinterpret_cast<uint32_t *>(st.b + o) = pack_bf16(b2.x * k2.x * ea, b2.y * k2.y * eb);
-            *reinterpret_cast<uint32_t *>(st.la + o) = pack_bf16(k2.x * iea, k2.y * ieb);
+            lam = __fadd2_rn(lam, l);
+            if (keep_lam) *reinterpret_cast<float2 *>(lam_ws + r * DK + c2) = lam;
+            const float2 e = make_float2(__expf(lam.x), __expf(lam.y));
+            const float2 ie = make_float2(__expf(-lam.x), __expf(-lam.y));
+            const float2 qt = __fmul2_rn(q2, e), gt = __fmul2_rn(__fmul2_rn(b2, k2), e), kb = __fmul2_rn(k2, ie);
+            *reinterpret_cast<uint32_t *>(st.q + o) = pack_bf16(qt.x, qt.y);
+            *reinterpret_cast<uint32_t *>(st.b + o) = pack_bf16(gt.x, gt.y);
+            *reinterpret_cast<uint32_t *>(st.la + o) = pack_bf16(kb.x, kb.y);
         }
         G::sync();
         if (prep_only || grams_ext) return false;

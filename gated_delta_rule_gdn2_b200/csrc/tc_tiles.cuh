@@ -69,15 +69,13 @@ __device__ __forceinline__ void store_frag_bf16(const Frag<NTL> &f, bf16 *dst, i
 }
 
 // sum_e v[e] * y[e] over 8 fp32 values and 8 packed bf16 values
+// (pairs on the packed fp32x2 pipe)
 __device__ __forceinline__ float dot8(const float *v, uint4 y) {
     const __nv_bfloat162 *y2 = reinterpret_cast<const __nv_bfloat162 *>(&y);
-    float acc = 0.f;
+    float2 acc = __fmul2_rn(make_float2(v[0], v[1]), __bfloat1622float2(y2[0]));
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(y2[e]);
-        acc += v[2 * e] * f.x + v[2 * e + 1] * f.y;
-    }
-    return acc;
+    for (int e = 1; e < 4; ++e) acc = __ffma2_rn(make_float2(v[2 * e], v[2 * e + 1]), __bfloat1622float2(y2[e]), acc);
+    return acc.x + acc.y;
 }
 
 }  // namespace tct
