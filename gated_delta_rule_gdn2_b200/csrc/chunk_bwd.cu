@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
     __shared__ float s_dpart[NTHR / (DK / 2)][DK];
     __shared__ float s_dmd[C];
     __shared__ float s_rs[2][DK];
-    BwdChunk<DK, DV> x(a, smem, sh, s_dpart, s_dmd, s_rs);
+    BwdChunk<DK, DV> x(a, smem, &sh, s_dpart, s_dmd, s_rs);
     const int warp = x.warp, lane = x.lane, bh = blockIdx.x;
     const int T = a.T, nchunks = x.nchunks;
     const ChunkTiles st = x.st;

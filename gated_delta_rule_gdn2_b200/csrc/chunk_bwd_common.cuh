@@ -77,8 +77,8 @@ struct BwdChunk {
     static constexpr int NRS = NT / 128;  // partial row sums of dSigma . Sigma (column parts)
 
     const ChunkBwdArgs &a;
-    IntraShared<DK, NT> &sh;
-    float (*s_dpart)[DK];  // [NT / (DK / 2)][DK] segment sums of dL
+    IntraShared<DK, NT> *sh;  // decay sums of the two-channel token pass (token_grads)
+    float (*s_dpart)[DK];     // [NT / (DK / 2)][DK] segment sums of dL (token_grads)
     float *s_dmd;          // [C] diagonal of dO U^T
     float (*s_rs)[DK];     // [NRS][DK] row sums of dSigma . Sigma over NRS column parts
     int tid, warp, lane, b, h, T, H, nchunks;
@@ -89,7 +89,7 @@ struct BwdChunk {
     const bf16 *states, *gq, *gk, *gb, *gv, *gw;
     const unsigned char *intra;
 
-    __device__ BwdChunk(const ChunkBwdArgs &args, unsigned char *smem, IntraShared<DK, NT> &sh_, float (*dpart)[DK],
+    __device__ BwdChunk(const ChunkBwdArgs &args, unsigned char *smem, IntraShared<DK, NT> *sh_, float (*dpart)[DK],
                         float *dmd, float (*rs)[DK])
         : a(args), sh(sh_), s_dpart(dpart), s_dmd(dmd), s_rs(rs) {
         tid = threadIdx.x; warp = tid >> 5; lane = tid & 31;
@@ -323,7 +323,7 @@ struct BwdChunk {
             float2 run = make_float2(0.f, 0.f);
 #pragma unroll
             for (int s = 0; s < P2; ++s)
-                if (s < s2) { run.x += sh.part[s][c2]; run.y += sh.part[s][c2 + 1]; }
+                if (s < s2) { run.x += sh->part[s][c2]; run.y += sh->part[s][c2 + 1]; }
             bf16 *__restrict__ gdq = static_cast<bf16 *>(a.dq);
             bf16 *__restrict__ gdk = static_cast<bf16 *>(a.dk);
             bf16 *__restrict__ gdb = static_cast<bf16 *>(a.db);
@@ -401,6 +401,167 @@ struct BwdChunk {
                                                   (((size_t)b * T + n * C + r) * H + h) * DK + c2) =
                         pack_bf16(acca, accb);
                 }
+            }
+        }
+    }
+
+    // ---- Token-level gradients with four key channels per thread: lane =
+    // channel quad, warp = 4-row segment of the chunk (DK = 128, NT = 512), so
+    // that every raw-row load and gradient store moves 8 bytes and a warp's
+    // store covers 256 contiguous bytes of one token row.
+    static constexpr int NQ = DK / 4, P4 = NT / NQ, R4 = C / P4;
+    struct RawRows4 {
+        uint2 q[R4], k[R4], b[R4], la[R4];
+    };
+    __device__ void load_rows4(RawRows4 &raw, int n, int Cn) const {
+        const int c4 = 4 * (tid % NQ), s4 = tid / NQ;
+        const bf16 *gla = static_cast<const bf16 *>(a.log_alpha);
+#pragma unroll
+        for (int i = 0; i < R4; ++i) {
+            const int r = min(s4 * R4 + i, Cn - 1);
+            const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c4;
+            raw.q[i] = *reinterpret_cast<const uint2 *>(gq + o);
+            raw.k[i] = *reinterpret_cast<const uint2 *>(gk + o);
+            raw.b[i] = *reinterpret_cast<const uint2 *>(gb + o);
+            raw.la[i] = *reinterpret_cast<const uint2 *>(gla + o);
+        }
+    }
+    // One channel pair of a fast chunk: dq, dk, db before the diagonal-of-M
+    // terms, and the dlog_alpha term (run = the in-chunk decay prefix L).
+    struct Pair {
+        float2 dq, dg, dk, dl;
+    };
+    static __device__ __forceinline__ Pair fast_pair(float2 dqt, float2 dgt, float2 dkb, float2 q, float2 k, float2 bb,
+                                                     float2 run) {
+        const float2 e = make_float2(__expf(run.x), __expf(run.y));
+        const float2 ie = make_float2(__expf(-run.x), __expf(-run.y));
+        Pair p;
+        p.dq = __fmul2_rn(dqt, e);
+        p.dg = __fmul2_rn(dgt, e);
+        p.dk = __fmul2_rn(dkb, ie);
+        p.dl = __fmul2_rn(p.dk, make_float2(-k.x, -k.y));
+        p.dl = __ffma2_rn(p.dg, __fmul2_rn(bb, k), p.dl);
+        p.dl = __ffma2_rn(p.dq, q, p.dl);
+        return p;
+    }
+    // ... and of a slow chunk, from its exact L and the term-by-term Gram
+    // gradients PQ, PG, PK, PL (lend = L at the chunk's last token).
+    static __device__ __forceinline__ Pair slow_pair(float2 dqt, float2 dgt, float2 dkb, float2 q, float2 k, float2 bb,
+                                                     float2 lam, float2 lend, float2 pq, float2 pg, float2 pk,
+                                                     float2 pl) {
+        const float ea = __expf(lam.x), eb = __expf(lam.y);
+        const float kea = __expf(lend.x - lam.x), keb = __expf(lend.y - lam.y);
+        Pair p;
+        p.dq = make_float2(dqt.x * ea + pq.x, dqt.y * eb + pq.y);
+        p.dg = make_float2(dgt.x * ea + pg.x, dgt.y * eb + pg.y);
+        p.dk = make_float2(dkb.x * kea + pk.x, dkb.y * keb + pk.y);
+        p.dl = make_float2(dqt.x * q.x * ea + dgt.x * bb.x * k.x * ea - dkb.x * k.x * kea + pl.x,
+                           dqt.y * q.y * eb + dgt.y * bb.y * k.y * eb - dkb.y * k.y * keb + pl.y);
+        return p;
+    }
+    // dq, dk, db and dlog_alpha from the fp32 staging tiles DQT, DGT, DKB (and
+    // PQ.. for a slow chunk).  seg: [P4][DK] sums of log_alpha over each 4-row
+    // segment (a fast chunk's decay prefix); dseg: a free [P4][DK] fp32 area
+    // for the segment sums of dL.  All of seg, dseg and s_rs 16-byte aligned.
+    __device__ void token_grads4(int n, int Cn, bool slow, const RawRows4 &raw, const float (*seg)[DK],
+                                 float (*dseg)[DK]) {
+        const int c4 = 4 * (tid % NQ), s4 = tid / NQ;
+        const float4 lend4 = slow ? *reinterpret_cast<const float4 *>(LAM + (Cn - 1) * DK + c4)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 rsum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < NRS; ++i) {
+            const float4 t = *reinterpret_cast<const float4 *>(&s_rs[i][c4]);
+            rsum.x += t.x; rsum.y += t.y; rsum.z += t.z; rsum.w += t.w;
+        }
+        // in-chunk decay prefix at the start of this thread's segment
+        float2 run0 = make_float2(0.f, 0.f), run1 = make_float2(0.f, 0.f);
+        for (int s = 0; s < s4; ++s) {
+            const float4 t = *reinterpret_cast<const float4 *>(&seg[s][c4]);
+            run0 = __fadd2_rn(run0, make_float2(t.x, t.y));
+            run1 = __fadd2_rn(run1, make_float2(t.z, t.w));
+        }
+        bf16 *__restrict__ gdq = static_cast<bf16 *>(a.dq);
+        bf16 *__restrict__ gdk = static_cast<bf16 *>(a.dk);
+        bf16 *__restrict__ gdb = static_cast<bf16 *>(a.db);
+        float2 dl0[R4], dl1[R4];
+        float2 ps0 = make_float2(0.f, 0.f), ps1 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < R4; ++i) {
+            const int r = s4 * R4 + i;
+            dl0[i] = make_float2(0.f, 0.f);
+            dl1[i] = make_float2(0.f, 0.f);
+            if (r < Cn) {
+                const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c4;
+                const float2 q0 = unpack_bf16(raw.q[i].x), q1 = unpack_bf16(raw.q[i].y);
+                const float2 k0 = unpack_bf16(raw.k[i].x), k1 = unpack_bf16(raw.k[i].y);
+                const float2 b0 = unpack_bf16(raw.b[i].x), b1 = unpack_bf16(raw.b[i].y);
+                const float4 dqt = *reinterpret_cast<const float4 *>(DQT + stg<DK>(r, c4));
+                const float4 dgt = *reinterpret_cast<const float4 *>(DGT + stg<DK>(r, c4));
+                const float4 dkb = *reinterpret_cast<const float4 *>(DKB + stg<DK>(r, c4));
+                Pair p0, p1;
+                if (!slow) {
+                    run0 = __fadd2_rn(run0, unpack_bf16(raw.la[i].x));
+                    run1 = __fadd2_rn(run1, unpack_bf16(raw.la[i].y));
+                    p0 = fast_pair(make_float2(dqt.x, dqt.y), make_float2(dgt.x, dgt.y), make_float2(dkb.x, dkb.y),
+                                   q0, k0, b0, run0);
+                    p1 = fast_pair(make_float2(dqt.z, dqt.w), make_float2(dgt.z, dgt.w), make_float2(dkb.z, dkb.w),
+                                   q1, k1, b1, run1);
+                } else {
+                    const float4 lam = *reinterpret_cast<const float4 *>(LAM + r * DK + c4);
+                    const float4 pq = *reinterpret_cast<const float4 *>(PQ + r * DK + c4);
+                    const float4 pg = *reinterpret_cast<const float4 *>(PG + r * DK + c4);
+                    const float4 pk = *reinterpret_cast<const float4 *>(PK + r * DK + c4);
+                    const float4 pl = *reinterpret_cast<const float4 *>(PL + r * DK + c4);
+                    p0 = slow_pair(make_float2(dqt.x, dqt.y), make_float2(dgt.x, dgt.y), make_float2(dkb.x, dkb.y),
+                                   q0, k0, b0, make_float2(lam.x, lam.y), make_float2(lend4.x, lend4.y),
+                                   make_float2(pq.x, pq.y), make_float2(pg.x, pg.y), make_float2(pk.x, pk.y),
+                                   make_float2(pl.x, pl.y));
+                    p1 = slow_pair(make_float2(dqt.z, dqt.w), make_float2(dgt.z, dgt.w), make_float2(dkb.z, dkb.w),
+                                   q1, k1, b1, make_float2(lam.z, lam.w), make_float2(lend4.z, lend4.w),
+                                   make_float2(pq.z, pq.w), make_float2(pg.z, pg.w), make_float2(pk.z, pk.w),
+                                   make_float2(pl.z, pl.w));
+                }
+                // the diagonal of M carries no decay: its gradient s_dmd goes to dq and dk directly
+                const float2 md = make_float2(s_dmd[r], s_dmd[r]);
+                p0.dq = __ffma2_rn(md, k0, p0.dq);
+                p1.dq = __ffma2_rn(md, k1, p1.dq);
+                p0.dk = __ffma2_rn(md, q0, p0.dk);
+                p1.dk = __ffma2_rn(md, q1, p1.dk);
+                if (r == Cn - 1) {
+                    p0.dl = __fadd2_rn(p0.dl, make_float2(rsum.x, rsum.y));
+                    p1.dl = __fadd2_rn(p1.dl, make_float2(rsum.z, rsum.w));
+                }
+                const float2 dk0 = __ffma2_rn(p0.dg, b0, p0.dk), dk1 = __ffma2_rn(p1.dg, b1, p1.dk);
+                const float2 db0 = __fmul2_rn(p0.dg, k0), db1 = __fmul2_rn(p1.dg, k1);
+                *reinterpret_cast<uint2 *>(gdq + o) = make_uint2(pack_bf16(p0.dq.x, p0.dq.y), pack_bf16(p1.dq.x, p1.dq.y));
+                *reinterpret_cast<uint2 *>(gdk + o) = make_uint2(pack_bf16(dk0.x, dk0.y), pack_bf16(dk1.x, dk1.y));
+                *reinterpret_cast<uint2 *>(gdb + o) = make_uint2(pack_bf16(db0.x, db0.y), pack_bf16(db1.x, db1.y));
+                dl0[i] = p0.dl;
+                dl1[i] = p1.dl;
+                ps0 = __fadd2_rn(ps0, p0.dl);
+                ps1 = __fadd2_rn(ps1, p1.dl);
+            }
+        }
+        // in-chunk reverse cumulative sum of dL: the later segments, then this
+        // thread's rows from the last up
+        *reinterpret_cast<float4 *>(&dseg[s4][c4]) = make_float4(ps0.x, ps0.y, ps1.x, ps1.y);
+        __syncthreads();
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        for (int s = s4 + 1; s < P4; ++s) {
+            const float4 t = *reinterpret_cast<const float4 *>(&dseg[s][c4]);
+            acc0 = __fadd2_rn(acc0, make_float2(t.x, t.y));
+            acc1 = __fadd2_rn(acc1, make_float2(t.z, t.w));
+        }
+        bf16 *__restrict__ gdl = static_cast<bf16 *>(a.dlog_alpha);
+#pragma unroll
+        for (int i = R4 - 1; i >= 0; --i) {
+            const int r = s4 * R4 + i;
+            if (r < Cn) {
+                acc0 = __fadd2_rn(acc0, dl0[i]);
+                acc1 = __fadd2_rn(acc1, dl1[i]);
+                *reinterpret_cast<uint2 *>(gdl + (((size_t)b * T + n * C + r) * H + h) * DK + c4) =
+                    make_uint2(pack_bf16(acc0.x, acc0.y), pack_bf16(acc1.x, acc1.y));
             }
         }
     }

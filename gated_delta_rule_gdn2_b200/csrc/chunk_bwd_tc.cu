@@ -66,19 +66,64 @@ using tct::ld_frag;
 using tct::mma_tiles;
 using tct::store_frag_bf16;
 
+// Decay of chunk n from its raw log_alpha tile (bf16, swizzled [64][D]):
+// seg[s][c] = sum of log_alpha[., c] over rows 4 s .. 4 s + 3 (lane = channel
+// quad, warp = segment, as in the token-level gradients), gamma[c] = e^{L_end};
+// true (and L in lam_ws, [64][D] fp32) when the chunk decays by more than
+// e^{-kSpanGuard} in some channel.  Tokens past T read as zeros.
+__device__ bool decay_sums(const bf16 *la, float (*seg)[D], float *gamma, int *slow_flag, float *lam_ws, int tid) {
+    constexpr int P4 = Chunk::P4, R4 = Chunk::R4;
+    const int c4 = 4 * (tid % Chunk::NQ), s4 = tid / Chunk::NQ;
+    if (tid == 0) *slow_flag = 0;
+    float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < R4; ++i) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(la + swz<D>(s4 * R4 + i, c4));
+        s0 = __fadd2_rn(s0, unpack_bf16(v.x));
+        s1 = __fadd2_rn(s1, unpack_bf16(v.y));
+    }
+    *reinterpret_cast<float4 *>(&seg[s4][c4]) = make_float4(s0.x, s0.y, s1.x, s1.y);
+    __syncthreads();
+    if (s4 == P4 - 1) {  // the last segment's warp: the chunk totals L_end
+        float2 t0 = make_float2(0.f, 0.f), t1 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int s = 0; s < P4; ++s) {
+            const float4 t = *reinterpret_cast<const float4 *>(&seg[s][c4]);
+            t0 = __fadd2_rn(t0, make_float2(t.x, t.y));
+            t1 = __fadd2_rn(t1, make_float2(t.z, t.w));
+        }
+        *reinterpret_cast<float4 *>(gamma + c4) = make_float4(__expf(t0.x), __expf(t0.y), __expf(t1.x), __expf(t1.y));
+        if (fminf(fminf(t0.x, t0.y), fminf(t1.x, t1.y)) < -kSpanGuard) *slow_flag = 1;
+    }
+    __syncthreads();
+    const bool slow = *slow_flag != 0;
+    if (slow) {  // the exact path needs L at every token
+        if (tid < D) {
+            float lam = 0.f;
+            for (int r = 0; r < C; ++r) {
+                lam += __bfloat162float(la[swz<D>(r, tid)]);
+                lam_ws[r * D + tid] = lam;
+            }
+        }
+        __syncthreads();
+    }
+    return slow;
+}
+
 __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, const __grid_constant__ BwdMaps maps) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u);
-    __shared__ IntraShared<D, NT> sh;
-    __shared__ float s_dpart[NT / (D / 2)][D];
+    __shared__ __align__(16) float s_seg[Chunk::P4][D];  // log_alpha sums over the 4-row segments of a chunk
+    __shared__ __align__(16) float s_gamma[D];            // e^{L_end} of the chunk
+    __shared__ int s_slow;
     __shared__ float s_dmd[C];
-    __shared__ float s_rs[2][Chunk::NRS][D];  // by chunk parity: row sums of dSigma . Sigma (column quarters)
+    __shared__ __align__(16) float s_rs[2][Chunk::NRS][D];  // by chunk parity: row sums of dSigma . Sigma (column quarters)
     __shared__ uint64_t mbar;
     __shared__ uint64_t mbar_ld[2];  // load groups A and B
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
-    Chunk x(a, smem, sh, s_dpart, s_dmd, s_rs[0]);
+    Chunk x(a, smem, nullptr, nullptr, s_dmd, s_rs[0]);
     const int tid = x.tid, warp = x.warp, lane = x.lane, bh = blockIdx.x;
     const ChunkTiles st = x.st;
 
@@ -191,10 +236,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         if (abort_flag) break;
         if (n > 0) x.prefetch_vw_l2(n - 1);
         // gam, the decay segment sums and (slow chunk) L from the raw log_alpha in the k slot
-        ChunkTiles rawla = st;
-        rawla.la = st.k;
-        const bool slow = intra_chunk<D, D, NT>(rawla, x.A32, x.T32, view(sh), x.LAM, false, /*prep_only=*/true,
-                                                false, true, /*pass1_only=*/true);
+        const bool slow = decay_sums(st.k, s_seg, s_gamma, &s_slow, x.LAM, tid);
 
         // ---- E0: D = g . dSigma (g = gam on a fast chunk, else 1) as bf16 and
         // dSigma <- gam . dSigma; on the last chunk also the row sums of
@@ -203,7 +245,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
             float v[32];
             tc::ld_32x32b_x32(t_srow, v);
             tc::wait_ld();
-            const float gm = sh.gamma[c], g = slow ? 1.f : gm;
+            const float gm = s_gamma[c], g = slow ? 1.f : gm;
             const float2 g2 = make_float2(g, g), gm2 = make_float2(gm, gm);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -333,8 +375,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
             }
             tc::commit(&mbar);
         }
-        Chunk::RawRows raw;
-        x.load_rows(raw, n, Cn);  // while the tensor cores run
+        Chunk::RawRows4 raw;
+        x.load_rows4(raw, n, Cn);  // while the tensor cores run
         mma_wait();
         // ---- E4: dQt, dGt, dKb -> fp32 staging (the S, D and T/M/dU regions are dead)
         {
@@ -362,7 +404,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         }
         if (n > 0 && tid == 0) issue_a(n - 1);  // the token, dO and U slots are free now
         x.s_rs = s_rs[n & 1];
-        x.token_grads(n, Cn, slow, raw, /*with_dvdw=*/false);
+        // (the v slot's nR is consumed: its first 8 KB take the segment sums of dL)
+        x.token_grads4(n, Cn, slow, raw, s_seg, reinterpret_cast<float (*)[D]>(st.v));
         tc::fence_async_smem();
         __syncthreads();
         if (n > 0 && tid == 0) issue_b(n - 1);  // the staging tiles in the S and T/M regions are consumed
