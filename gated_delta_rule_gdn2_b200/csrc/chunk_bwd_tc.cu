@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
     __shared__ float s_dmd[C];
     __shared__ __align__(16) float s_rs[2][Chunk::NRS][D];  // by chunk parity: row sums of dSigma . Sigma (column quarters)
     __shared__ uint64_t mbar;
-    __shared__ uint64_t mbar_ld[2];  // load groups A and B
+    __shared__ uint64_t mbar_ld[3];  // load groups A, B and the state image
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -132,6 +132,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         tc::mbar_init(&mbar, 1);
         tc::mbar_init(&mbar_ld[0], 1);
         tc::mbar_init(&mbar_ld[1], 1);
+        tc::mbar_init(&mbar_ld[2], 1);
         tc::fence_mbar_init();
         abort_flag = 0;
     }
@@ -191,12 +192,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
     // Tile loads, issued by one thread through the TMA and counted in bytes on
     // mbar_ld: group A = the forward's Qt, Gt, Kb (or Kt) and U, with the raw
     // log_alpha (into the k slot, for the decay sums) and dO as 64 x 64 boxes
-    // of the tensor maps; group B = the chunk-start state and the forward's T,
-    // M.  The forward stores its tiles as images of shared memory, which come
-    // back as bulk copies.  They run one chunk ahead: group A of chunk n - 1
-    // lands while chunk n's token-level gradients are formed, group B while
-    // chunk n - 1's decay sums and E0 run.
-    uint32_t ph_ld[2] = {0, 0};
+    // of the tensor maps; group B = the forward's T, M; then the chunk-start
+    // state on a barrier of its own (first needed by M3).  The forward stores
+    // its tiles as images of shared memory, which come back as bulk copies.
+    // They run one chunk ahead: group A of chunk n - 1 lands while chunk n's
+    // token-level gradients are formed, group B and the state while chunk
+    // n - 1's decay sums, E0 and first products run.
+    uint32_t ph_ld[3] = {0, 0, 0};
     auto issue_a = [&](int m) {
         tc::mbar_expect_tx(&mbar_ld[0], 6 * TILE_BYTES);
         const unsigned char *img = x.intra + (size_t)m * x.I_BYTES + TM_BYTES;
@@ -213,9 +215,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         tc::bulk_load(x.U16, img, TILE_BYTES, &mbar_ld[0]);
     };
     auto issue_b = [&](int m) {
-        tc::mbar_expect_tx(&mbar_ld[1], D * D * 2 + TM_BYTES);
-        tc::bulk_load(x.S16, x.states + (size_t)m * D * D, D * D * 2, &mbar_ld[1]);
+        tc::mbar_expect_tx(&mbar_ld[1], TM_BYTES);
         tc::bulk_load(x.T16, x.intra + (size_t)m * x.I_BYTES, TM_BYTES, &mbar_ld[1]);
+        tc::mbar_expect_tx(&mbar_ld[2], D * D * 2);
+        tc::bulk_load(x.S16, x.states + (size_t)m * D * D, D * D * 2, &mbar_ld[2]);
     };
     auto wait_loads = [&](int g) {
         if (!tc::mbar_wait(&mbar_ld[g], ph_ld[g])) {
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
             tc::st_32x32b_x32(t_srow, v);
             tc::wait_st();
         }
-        wait_loads(1);  // group B: S, T, M
+        wait_loads(1);  // group B: T, M
         handoff();
         if (abort_flag) break;
 
@@ -322,6 +325,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
             tc::wait_ld();
             store_frag_bf16<D, 4>(f, x.nR16, 16 * p, 32 * qc, lane, -1.f);
         }
+        wait_loads(2);  // the chunk-start state S
         handoff();
         if (abort_flag) break;
 
