@@ -463,8 +463,11 @@ struct BwdChunk {
     // PQ.. for a slow chunk).  seg: [P4][DK] sums of log_alpha over each 4-row
     // segment (a fast chunk's decay prefix); dseg: a free [P4][DK] fp32 area
     // for the segment sums of dL.  All of seg, dseg and s_rs 16-byte aligned.
+    // rows_done() runs on every thread once all threads have read the staging
+    // tiles and s_rs (after a barrier).
+    template <class F>
     __device__ void token_grads4(int n, int Cn, bool slow, const RawRows4 &raw, const float (*seg)[DK],
-                                 float (*dseg)[DK]) {
+                                 float (*dseg)[DK], F &&rows_done) {
         const int c4 = 4 * (tid % NQ), s4 = tid / NQ;
         const float4 lend4 = slow ? *reinterpret_cast<const float4 *>(LAM + (Cn - 1) * DK + c4)
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -547,6 +550,7 @@ struct BwdChunk {
         // thread's rows from the last up
         *reinterpret_cast<float4 *>(&dseg[s4][c4]) = make_float4(ps0.x, ps0.y, ps1.x, ps1.y);
         __syncthreads();
+        rows_done();
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         for (int s = s4 + 1; s < P4; ++s) {
             const float4 t = *reinterpret_cast<const float4 *>(&dseg[s][c4]);

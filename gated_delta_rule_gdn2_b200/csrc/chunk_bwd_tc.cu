@@ -408,11 +408,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         }
         if (n > 0 && tid == 0) issue_a(n - 1);  // the token, dO and U slots are free now
         x.s_rs = s_rs[n & 1];
-        // (the v slot's nR is consumed: its first 8 KB take the segment sums of dL)
-        x.token_grads4(n, Cn, slow, raw, s_seg, reinterpret_cast<float (*)[D]>(st.v));
-        tc::fence_async_smem();
-        __syncthreads();
-        if (n > 0 && tid == 0) issue_b(n - 1);  // the staging tiles in the S and T/M regions are consumed
+        // (the v slot's nR is consumed: its first 8 KB take the segment sums of
+        // dL).  Group B and the state of chunk n - 1 load once the staging tiles
+        // in the S and T/M regions are read, during the reverse cumulative sum.
+        x.token_grads4(n, Cn, slow, raw, s_seg, reinterpret_cast<float (*)[D]>(st.v), [&] {
+            if (n > 0 && tid == 0) issue_b(n - 1);
+        });
     }
 
     if (a.dS0 && !abort_flag) {
