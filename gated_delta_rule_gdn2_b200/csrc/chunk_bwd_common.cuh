@@ -241,21 +241,26 @@ struct BwdChunk {
     }
 
     // dv = dRHS . w, dw = dRHS . v from the bf16 -dRHS tile nR16 (16-byte
-    // coalesced; every global load is issued before the first use).
+    // coalesced; every global load is issued before the first use).  Threads
+    // below T0 take no part (the thread that issues the tensor-core products
+    // meanwhile sits in that range).
+    template <int T0 = 0>
     __device__ void dvdw(int n, int Cn) {
-        constexpr int NV = C * DV / 8 / NT;
+        constexpr int ITEMS = C * DV / 8, NV = (ITEMS + NT - T0 - 1) / (NT - T0);
+        const int t = tid - T0;
+        if (t < 0) return;
         uint4 v8[NV], w8[NV];
 #pragma unroll
         for (int it = 0; it < NV; ++it) {
-            const int id = tid + it * NT, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
+            const int id = min(t + it * (NT - T0), ITEMS - 1), r = id / (DV / 8), j = (id % (DV / 8)) * 8;
             const size_t o = (((size_t)b * T + n * C + min(r, Cn - 1)) * H + h) * DV + j;
             v8[it] = *reinterpret_cast<const uint4 *>(gv + o);
             w8[it] = *reinterpret_cast<const uint4 *>(gw + o);
         }
 #pragma unroll
         for (int it = 0; it < NV; ++it) {
-            const int id = tid + it * NT, r = id / (DV / 8), j = (id % (DV / 8)) * 8;
-            if (r < Cn) {
+            const int id = t + it * (NT - T0), r = id / (DV / 8), j = (id % (DV / 8)) * 8;
+            if (id < ITEMS && r < Cn) {
                 const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV + j;
                 uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, j));
                 nr.x ^= 0x80008000u; nr.y ^= 0x80008000u; nr.z ^= 0x80008000u; nr.w ^= 0x80008000u;  // dRHS = -nR

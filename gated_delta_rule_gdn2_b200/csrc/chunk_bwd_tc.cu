@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
             mma_tiles<false, false>(tmem + COL_S, st.b, 64, x.nR16, 64, 4, ID128x128_MN_MN, true);
             tc::commit(&mbar);
         }
-        x.dvdw(n, Cn);  // while the tensor cores run: dv, dw from nR and the global v, w
+        x.dvdw<32>(n, Cn);  // while the tensor cores run (warps 1..15): dv, dw from nR and the global v, w
         mma_wait();
         // ---- row sums of dSigma . Sigma for chunk n - 1: dSigma is now its
         // chunk-end gradient and Sigma = this chunk's start state S
