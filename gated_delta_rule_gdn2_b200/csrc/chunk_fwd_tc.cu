@@ -82,9 +82,9 @@ __device__ __forceinline__ ChunkTiles stage_tiles(unsigned char *smem, int s) {
             reinterpret_cast<bf16 *>(p + 5 * TILE)};
 }
 
-// TMA tensor maps of the six token tensors.
+// TMA tensor maps of the six token tensors and of the output o.
 struct FwdMaps {
-    CUtensorMap q, k, la, b, v, w;
+    CUtensorMap q, k, la, b, v, w, o;
 };
 
 // Chunk n's six token tiles into a stage (one thread; 64 x 64 boxes, two per
@@ -390,30 +390,24 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             }
             wait_on(&sm.mbar_b, ph_b);
             gm_owed = slow ? 1.f : gm;  // a fast chunk's Diag(gam) is applied with the next bf16 copy
-            if (with_o) {  // O -> o (bf16), straight from the fragment layout
+            if (with_o) {  // O -> its bf16 image in the k slot (free since U), stored by the TMA
                 Frag<8> f;
                 ld_frag(tmem + lane_base + COL_O + 64 * hc, f);
                 tc::wait_ld();
-                const int rl = 16 * p + (lane >> 2);
-                bf16 *o = static_cast<bf16 *>(a.o);
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int t = n * C + rl + 8 * half;
-                    if (t < a.T) {
-                        bf16 *orow = o + (((size_t)b * a.T + t) * a.H + h) * D + 64 * hc;
-#pragma unroll
-                        for (int nt = 0; nt < 8; ++nt)
-                            *reinterpret_cast<uint32_t *>(orow + 8 * nt + 2 * (lane & 3)) =
-                                pack_bf16(f[0][nt][2 * half], f[0][nt][2 * half + 1]);
-                    }
-                }
+                store_frag_bf16<D, 8>(f, st.k, 16 * p, 64 * hc, lane, 1.f);
+                tc::fence_async_smem();
             }
             tc::fence_before();
             GB::sync();
             if (tb == 0) {
-                // the stage's T, M, U images and the state image are out before the
-                // stage is refilled (and before S16 is rewritten, which follows this
-                // thread's next MMA issue)
+                if (with_o) {  // (tokens past T are clipped)
+                    tc::tma_store_4d(&maps.o, st.k, 0, h, n * C, b);
+                    tc::tma_store_4d(&maps.o, st.k + C * 64, 64, h, n * C, b);
+                    tc::bulk_commit();
+                }
+                // the stage's T, M, U and O images and the state image are out
+                // before the stage is refilled (and before S16 is rewritten, which
+                // follows this thread's next MMA issue)
                 tc::bulk_wait_read();
                 if (n + 2 < nchunks) issue_chunk(maps, st, b, h, n + 2, &sm.mbar_ld[s]);
             }
@@ -454,11 +448,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
 }  // namespace cfwd_tc
 
 cudaError_t launch_chunk_fwd_tc(const ChunkFwdArgs &a, cudaStream_t s) {
-    cfwd_tc::FwdMaps m;
+    cfwd_tc::FwdMaps m{};
     const int D = cfwd_tc::D;
     if (!token_tensor_map(&m.q, a.q, a.B, a.T, a.H, D) || !token_tensor_map(&m.k, a.k, a.B, a.T, a.H, D) ||
         !token_tensor_map(&m.la, a.log_alpha, a.B, a.T, a.H, D) || !token_tensor_map(&m.b, a.b, a.B, a.T, a.H, D) ||
-        !token_tensor_map(&m.v, a.v, a.B, a.T, a.H, D) || !token_tensor_map(&m.w, a.w, a.B, a.T, a.H, D))
+        !token_tensor_map(&m.v, a.v, a.B, a.T, a.H, D) || !token_tensor_map(&m.w, a.w, a.B, a.T, a.H, D) ||
+        (a.o && !token_tensor_map(&m.o, a.o, a.B, a.T, a.H, D)))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(cfwd_tc::chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          cfwd_tc::BYTES);

@@ -123,6 +123,14 @@ __device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_
                  "r"(bytes)
                  : "memory");
 }
+// Tiled box of this CTA's shared memory to a 4-D tensor map at (x, y, z, w)
+// (never at a negative coordinate; the box is clipped at the tensor's end),
+// completion in this thread's bulk group.
+__device__ __forceinline__ void tma_store_4d(const void *map, const void *src, int x, int y, int z, int w) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];\n" ::"l"(map),
+                 "r"(smem_addr(src)), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
 // Until the sources of every committed bulk store have been read (the shared
 // memory may then be overwritten) ...
