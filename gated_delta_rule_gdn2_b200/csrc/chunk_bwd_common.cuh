@@ -465,8 +465,8 @@ struct BwdChunk {
         return p;
     }
     // dq, dk, db and dlog_alpha from the fp32 staging tiles DQT, DGT, DKB (and
-    // PQ.. for a slow chunk).  seg: [P4][DK] sums of log_alpha over each 4-row
-    // segment (a fast chunk's decay prefix); dseg: a free [P4][DK] fp32 area
+    // PQ.. for a slow chunk).  seg: [P4][DK] sums of log_alpha over the rows
+    // before each 4-row segment (a fast chunk's decay prefix); dseg: a free [P4][DK] fp32 area
     // for the segment sums of dL.  All of seg, dseg and s_rs 16-byte aligned.
     // rows_done() runs on every thread once all threads have read the staging
     // tiles and s_rs (after a barrier).
@@ -483,12 +483,8 @@ struct BwdChunk {
             rsum.x += t.x; rsum.y += t.y; rsum.z += t.z; rsum.w += t.w;
         }
         // in-chunk decay prefix at the start of this thread's segment
-        float2 run0 = make_float2(0.f, 0.f), run1 = make_float2(0.f, 0.f);
-        for (int s = 0; s < s4; ++s) {
-            const float4 t = *reinterpret_cast<const float4 *>(&seg[s][c4]);
-            run0 = __fadd2_rn(run0, make_float2(t.x, t.y));
-            run1 = __fadd2_rn(run1, make_float2(t.z, t.w));
-        }
+        const float4 pre = *reinterpret_cast<const float4 *>(&seg[s4][c4]);
+        float2 run0 = make_float2(pre.x, pre.y), run1 = make_float2(pre.z, pre.w);
         bf16 *__restrict__ gdq = static_cast<bf16 *>(a.dq);
         bf16 *__restrict__ gdk = static_cast<bf16 *>(a.dk);
         bf16 *__restrict__ gdb = static_cast<bf16 *>(a.db);

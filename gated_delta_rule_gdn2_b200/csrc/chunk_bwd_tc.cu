@@ -67,8 +67,9 @@ using tct::mma_tiles;
 using tct::store_frag_bf16;
 
 // Decay of chunk n from its raw log_alpha tile (bf16, swizzled [64][D]):
-// seg[s][c] = sum of log_alpha[., c] over rows 4 s .. 4 s + 3 (lane = channel
-// quad, warp = segment, as in the token-level gradients), gamma[c] = e^{L_end};
+// seg[s][c] = sum of log_alpha[., c] over the rows before row 4 s (lane =
+// channel quad, warp = 4-row segment, as in the token-level gradients),
+// gamma[c] = e^{L_end};
 // true (and L in lam_ws, [64][D] fp32) when the chunk decays by more than
 // e^{-kSpanGuard} in some channel.  Tokens past T read as zeros.
 __device__ bool decay_sums(const bf16 *la, float (*seg)[D], float *gamma, int *slow_flag, float *lam_ws, int tid) {
@@ -84,13 +85,16 @@ __device__ bool decay_sums(const bf16 *la, float (*seg)[D], float *gamma, int *s
     }
     *reinterpret_cast<float4 *>(&seg[s4][c4]) = make_float4(s0.x, s0.y, s1.x, s1.y);
     __syncthreads();
-    if (s4 == P4 - 1) {  // the last segment's warp: the chunk totals L_end
+    if (s4 == P4 - 1) {  // the last segment's warp: exclusive prefix sums in place, and L_end
+        float4 t[P4];
+#pragma unroll
+        for (int s = 0; s < P4; ++s) t[s] = *reinterpret_cast<const float4 *>(&seg[s][c4]);
         float2 t0 = make_float2(0.f, 0.f), t1 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int s = 0; s < P4; ++s) {
-            const float4 t = *reinterpret_cast<const float4 *>(&seg[s][c4]);
-            t0 = __fadd2_rn(t0, make_float2(t.x, t.y));
-            t1 = __fadd2_rn(t1, make_float2(t.z, t.w));
+            *reinterpret_cast<float4 *>(&seg[s][c4]) = make_float4(t0.x, t0.y, t1.x, t1.y);
+            t0 = __fadd2_rn(t0, make_float2(t[s].x, t[s].y));
+            t1 = __fadd2_rn(t1, make_float2(t[s].z, t[s].w));
         }
         *reinterpret_cast<float4 *>(gamma + c4) = make_float4(__expf(t0.x), __expf(t0.y), __expf(t1.x), __expf(t1.y));
         if (fminf(fminf(t0.x, t0.y), fminf(t1.x, t1.y)) < -kSpanGuard) *slow_flag = 1;
