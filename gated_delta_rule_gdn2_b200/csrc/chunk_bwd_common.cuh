@@ -553,6 +553,7 @@ struct BwdChunk {
         __syncthreads();
         rows_done();
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+#pragma unroll 4
         for (int s = s4 + 1; s < P4; ++s) {
             const float4 t = *reinterpret_cast<const float4 *>(&dseg[s][c4]);
             acc0 = __fadd2_rn(acc0, make_float2(t.x, t.y));
