@@ -292,29 +292,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
             mma_tiles<false, false>(tmem + COL_S, st.q, 64, x.dO16, 64, 4, ID128x128_MN_MN, true);
         }
         mma_done();
-        // ---- E1: dU -> bf16 (all warps, column quarters) ; dM = strict_lower(dO U^T)
-        // with its diagonal kept aside in fp32 (warps with qc < 2)
+        // ---- E1: dU -> bf16 (all warps, column quarters)
         {
             Frag<4> f;
             ld_frag(tmem + lane_base + COL_C + 32 * qc, f);
             tc::wait_ld();
             store_frag_bf16<D, 4>(f, x.dU16, 16 * p, 32 * qc, lane, 1.f);
-            if (qc < 2) {
-                ld_frag(tmem + lane_base + COL_A + 32 * qc, f);
-                tc::wait_ld();
-                const int r0 = 16 * p + (lane >> 2);
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        // The diagonal of M carries no decay factor: its gradient goes
-                        // straight to dq and dk in fp32 and stays out of the Gram products.
-                        const int r = r0 + (e >> 1) * 8, i = 32 * qc + 8 * nt + 2 * (lane & 3) + (e & 1);
-                        if (i == r) s_dmd[r] = f[0][nt][e];
-                        if (i >= r) f[0][nt][e] = 0.f;
-                    }
-                store_frag_bf16<64, 4>(f, x.dM16, 16 * p, 32 * qc, lane, 1.f);
-            }
         }
         handoff();
         if (abort_flag) break;
@@ -341,19 +324,28 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
             mma_tiles<false, false>(tmem + COL_S, st.b, 64, x.nR16, 64, 4, ID128x128_MN_MN, true);
             tc::commit(&mbar);
         }
-        x.dvdw<32>(n, Cn);  // while the tensor cores run (warps 1..15): dv, dw from nR and the global v, w
-        mma_wait();
-        // ---- row sums of dSigma . Sigma for chunk n - 1: dSigma is now its
-        // chunk-end gradient and Sigma = this chunk's start state S
-        if (n > 0) {
-            float v[32];
-            tc::ld_32x32b_x32(t_srow, v);
+        // While the tensor cores run: dM = strict_lower(dO U^T) from M1's columns,
+        // with its diagonal kept aside in fp32 (warps 8..15; M3 writes other
+        // columns) -- the diagonal of M carries no decay factor, so its gradient
+        // goes straight to dq and dk and stays out of the Gram products -- and
+        // dv, dw from nR and the global v, w (warps 1..15).
+        if (qc >= 2) {
+            Frag<4> f;
+            ld_frag(tmem + lane_base + COL_A + 32 * (qc - 2), f);
             tc::wait_ld();
-            float rs = 0.f;
+            const int r0 = 16 * p + (lane >> 2);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) rs += dot8(v + 8 * i, *reinterpret_cast<const uint4 *>(tile_row(x.S16, i)));
-            s_rs[(n - 1) & 1][qc][c] = rs;
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = r0 + (e >> 1) * 8, i = 32 * (qc - 2) + 8 * nt + 2 * (lane & 3) + (e & 1);
+                    if (i == r) s_dmd[r] = f[0][nt][e];
+                    if (i >= r) f[0][nt][e] = 0.f;
+                }
+            store_frag_bf16<64, 4>(f, x.dM16, 16 * p, 32 * (qc - 2), lane, 1.f);
         }
+        x.dvdw<32>(n, Cn);
+        mma_wait();
         // ---- E3: dA = strict_lower(nR U^T) -> bf16 (warps with qc < 2)
         if (qc < 2) {
             Frag<4> f;
@@ -385,6 +377,18 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         }
         Chunk::RawRows4 raw;
         x.load_rows4(raw, n, Cn);  // while the tensor cores run
+        // ---- row sums of dSigma . Sigma for chunk n - 1 (dSigma is now its
+        // chunk-end gradient, Sigma = this chunk's start state S), also inside M4
+        if (n > 0) {
+            float v[32];
+            tc::ld_32x32b_x32(t_srow, v);
+            tc::wait_ld();
+            float rs = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rs += dot8(v + 8 * i, *reinterpret_cast<const uint4 *>(tile_row(x.S16, i)));
+            s_rs[(n - 1) & 1][qc][c] = rs;
+        }
+        __syncthreads();  // every read of S16 is done before E4 stages dQt over it
         mma_wait();
         // ---- E4: dQt, dGt, dKb -> fp32 staging (the S, D and T/M/dU regions are dead)
         {
