@@ -285,13 +285,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         if (abort_flag) break;
 
         // ---- M1: dU = M^T dO + Kx D ; dO U^T ; dSigma += Qt^T dO
+        // (dU is committed first: dO U^T and Qt^T dO run under E1, and M2's
+        // commit covers them)
         if (tid == 0) {
             mma_tiles<false, false>(tmem + COL_C, x.M16, 64, x.dO16, 64, 4, ID64x128_MN_MN, false);
             mma_tiles<true, false>(tmem + COL_C, st.la, 64, x.D16, D, 8, ID64x128_K_MN, true);
+            tc::commit(&mbar);
             mma_tiles<true, true>(tmem + COL_A, x.dO16, 64, x.U16, 64, 8, ID64x64_K_K, false);
             mma_tiles<false, false>(tmem + COL_S, st.q, 64, x.dO16, 64, 4, ID128x128_MN_MN, true);
         }
-        mma_done();
+        mma_wait();
         // ---- E1: dU -> bf16 (all warps, column quarters)
         {
             Frag<4> f;
