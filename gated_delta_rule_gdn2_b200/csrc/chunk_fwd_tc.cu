@@ -382,13 +382,15 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 GB::sync();
                 tc::fence_after();
             }
-            // ---- S += Kx^T U ; O += M U
+            // ---- O += M U (committed first: the O epilogue runs under the state
+            // update) ; S += Kx^T U
             if (tb == 0) {
-                mma_tiles<false, false>(tmem + COL_S, st.la, 64, U16, 64, 4, IDESC_S, true);
                 if (with_o) mma_tiles<true, false>(tmem + COL_O, M16, 64, U16, 64, 4, ID64x128_K_MN, true);
+                tc::commit(&sm.mbar_o);
+                mma_tiles<false, false>(tmem + COL_S, st.la, 64, U16, 64, 4, IDESC_S, true);
                 tc::commit(&sm.mbar_b);
             }
-            wait_on(&sm.mbar_b, ph_b);
+            wait_on(&sm.mbar_o, ph_o);
             gm_owed = slow ? 1.f : gm;  // a fast chunk's Diag(gam) is applied with the next bf16 copy
             if (with_o) {  // O -> its bf16 image in the k slot (free since U), stored by the TMA
                 Frag<8> f;
@@ -397,6 +399,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 store_frag_bf16<D, 8>(f, st.k, 16 * p, 64 * hc, lane, 1.f);
                 tc::fence_async_smem();
             }
+            wait_on(&sm.mbar_b, ph_b);  // S (and with it every read of the stage's tiles)
             tc::fence_before();
             GB::sync();
             if (tb == 0) {
