@@ -7,7 +7,8 @@ shape of the pages: gdn2_chunk_fwd_save (the forward that keeps its
 chunk-boundary states) + gdn2_chunk_bwd_saved (the gate-aware backward using
 them).  The plain forward (prefill, gdn2_chunk_fwd) and the decode step
 (B=256, H=16, fp32 state of 268 MB updated in place) are timed in the same
-run and reported under "prefill" and "decode".  Inputs are seeded synthetic data of the
+run and reported under "prefill" and "decode", and the long-sequence forward
+(B=1, T=32768, H=16) under "long".  Inputs are seeded synthetic data of the
 pages' distributions (gated_delta_rule_gdn2_b200.inputs); they are larger
 than L2 (about 1 GB per step), so no separate flush is needed.
 
@@ -33,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 B, T, H, D = 8, 4096, 16, 128  # B can be lowered with --batch for profiling captures
 DEC_B, DEC_H = 256, 16
+LONG_T = 32768  # the long-sequence forward leg (B1 H16)
 WORKLOAD = "train fwd+bwd B8 T4096 H16 dk=dv=128 bf16 (prefill and decode B256 H16 alongside)"
 METRIC = "GDN-2 chunk fwd+bwd tokens/s & TFLOP/s (H16 dk=dv=128); decode state GB/s"
 # algorithmic work per (token, head), d = 128, C = 64: dense-counted products and bytes read + written once
@@ -242,6 +244,33 @@ def run_gpu(args):
     torch.cuda.synchronize()
     pre_ms = p0.elapsed_time(p1) / args.steps
 
+    # ---- long-sequence forward (B1 T32768 H16: 16 sequences, so 16 CTAs)
+    from gated_delta_rule_gdn2_b200.inputs import WORKLOADS, make_workload
+    xl = make_workload(WORKLOADS["long"], T=LONG_T)
+    tl = [torch.from_numpy(xl[n]).to(device=dev, dtype=torch.bfloat16)
+          for n in ("q", "k", "v", "log_alpha", "b", "w")]
+    S0l = torch.from_numpy(xl["S0"]).to(dev)
+    ol = torch.empty((1, LONG_T, H, D), dtype=torch.bfloat16, device=dev)
+    STl = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
+    nlw = g.gdn2_chunk_fwd_workspace(1, LONG_T, H, D, D, g.GDN2_BF16)
+    wsl = torch.empty(max(nlw, 16), dtype=torch.uint8, device=dev)
+
+    def long_fwd():
+        st = g.gdn2_chunk_fwd(*tl, S0l, ol, STl, 1, LONG_T, H, D, D, g.GDN2_BF16, wsl, nlw, sh)
+        assert st == 0, st
+
+    for _ in range(3):
+        long_fwd()
+    torch.cuda.synchronize()
+    l0, l1 = ev(), ev()
+    l0.record(stream)
+    for _ in range(args.steps):
+        long_fwd()
+    l1.record(stream)
+    torch.cuda.synchronize()
+    long_ms = l0.elapsed_time(l1) / args.steps
+    del tl, ol, wsl
+
     # ---- decode step, state of B256 H16 d128 resident and updated in place
     from gated_delta_rule_gdn2_b200.inputs import decode_initial_state, decode_step_inputs
     Sdec = torch.from_numpy(decode_initial_state(DEC_B, DEC_H, D, D, seed=1002)).to(dev)
@@ -368,6 +397,10 @@ def run_gpu(args):
             "bwd_tflops": th * FLOP_BWD / (bwd_ms * 1e-3) / 1e12,
             "bwd_gbs": bwd_gbs, "bwd_hbm_frac": bwd_gbs / hbm,
         },
+        "long": {"workload": "B1 T%d H16 dk=dv=128 forward (gdn2_chunk_fwd; 16 sequences)" % LONG_T,
+                 "ms": long_ms, "tokens_per_s": LONG_T / (long_ms * 1e-3),
+                 "gbs": (LONG_T * H * BYTES_FWD + 2 * H * STATE_BYTES) / (long_ms * 1e-3) / 1e9,
+                 "hbm_frac": (LONG_T * H * BYTES_FWD + 2 * H * STATE_BYTES) / (long_ms * 1e-3) / 1e9 / hbm},
         "prefill": {"workload": "B8 T4096 H16 dk=dv=128 forward (gdn2_chunk_fwd)", "ms": pre_ms,
                     "tokens_per_s": B * T / (pre_ms * 1e-3), "tflops": th * FLOP_FWD / (pre_ms * 1e-3) / 1e12,
                     "gbs": pre_gbs, "hbm_frac": pre_gbs / hbm,
