@@ -5,6 +5,8 @@
 
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "launch.h"
 
 namespace gdn2 {
@@ -99,7 +101,9 @@ int gdn2_get_device_status(cudaStream_t stream) {
 size_t gdn2_chunk_fwd_workspace(int B, int T, int H, int dk, int dv, int dtype) {
     if (check_sizes(B, T, H, dk, dv, dtype) != GDN2_OK) return 0;
     if (B == 0 || H == 0 || T == 0 || dtype != GDN2_BF16) return 0;
-    return chunk_fwd_ws_bytes(B, H, dk);
+    const size_t plain = chunk_fwd_ws_bytes(B, H, dk);
+    const int P = segment_count(B, T, H, dk, dv);
+    return P > 1 ? std::max(plain, segments_ws_bytes(B, T, H, dk, dv, P)) : plain;
 }
 
 int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_alpha,
@@ -114,11 +118,16 @@ int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) ||
         !ok_ptr(o))
         return GDN2_ERR_INVALID_ARG;
-    const size_t need = gdn2_chunk_fwd_workspace(B, T, H, dk, dv, dtype);
+    // the one-CTA-per-sequence path needs the plain size; the workspace size
+    // query's larger figure, where it applies, enables sequence segments
+    const size_t need = dtype == GDN2_BF16 ? chunk_fwd_ws_bytes(B, H, dk) : 0;
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return GDN2_ERR_WORKSPACE;
     if (dtype == GDN2_BF16) {
         ChunkFwdArgs a{q, k, v, log_alpha, b, w, S0, o, S_T, static_cast<float *>(ws),
                        (size_t)64 * dk, nullptr, nullptr, nullptr, status_ptr(), B, T, H};
+        const int P = segment_count(B, T, H, dk, dv);
+        if (P > 1 && ws_bytes >= segments_ws_bytes(B, T, H, dk, dv, P))
+            return launch_status(launch_chunk_fwd_segments(a, dk, dv, P, ws, stream));
         return launch_status(launch_chunk_fwd(a, dk, dv, stream));
     }
     // fp32 precision mode: the recurrence token by token in fp32
@@ -222,7 +231,7 @@ int gdn2_chunk_fwd_save(const void *q, const void *k, const void *v, const void 
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) ||
         !ok_ptr(o))
         return GDN2_ERR_INVALID_ARG;
-    const size_t need = gdn2_chunk_fwd_workspace(B, T, H, dk, dv, dtype);
+    const size_t need = chunk_fwd_ws_bytes(B, H, dk);  // (the training forward is never segmented)
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return GDN2_ERR_WORKSPACE;
     ChunkFwdArgs a{q, k, v, log_alpha, b, w, S0, o, S_T, static_cast<float *>(ws), (size_t)64 * dk, states,
                    static_cast<char *>(states) + states_region_bytes(B, T, H, dk, dv),

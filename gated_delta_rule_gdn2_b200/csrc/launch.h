@@ -49,6 +49,14 @@ cudaError_t launch_chunk_fwd(const ChunkFwdArgs &a, int dk, int dv, cudaStream_t
 cudaError_t launch_chunk_fwd_tc(const ChunkFwdArgs &a, cudaStream_t s);  // dk = dv = 128, tcgen05
 size_t chunk_fwd_ws_bytes(int B, int H, int dk);
 
+// The plain forward for few long sequences as P sequence segments side by
+// side (segments.cu): segment_count gives P (1 = not worth it), the
+// workspace it needs, and the launch (S_T, o, status as in ChunkFwdArgs; the
+// args' ws is ignored, `ws` of segments_ws_bytes holds everything).
+int segment_count(int B, int T, int H, int dk, int dv);
+size_t segments_ws_bytes(int B, int T, int H, int dk, int dv, int P);
+cudaError_t launch_chunk_fwd_segments(const ChunkFwdArgs &a, int dk, int dv, int P, void *ws, cudaStream_t s);
+
 // Chunk-parallel gate-aware backward (bf16 tokens): a state pass (the
 // forward writing bf16 chunk-boundary states to `states`) and a reverse chunk
 // pass.  scratch: per-CTA fp32 work area of scr_stride floats.

@@ -63,7 +63,13 @@ typedef enum {
     GDN2_FP32 = 1   /* token tensors in fp32; fp32 arithmetic throughout */
 } gdn2_dtype;
 
-/* Bytes of device workspace gdn2_chunk_fwd needs for these sizes (may be 0). */
+/*
+ * Bytes of device workspace for gdn2_chunk_fwd at these sizes (may be 0).
+ * For bf16 with dk = dv and too few sequences to fill the GPU (B*H*4 <= the
+ * SM count) with T a multiple of 4 segments of at least 8 chunks, this is the
+ * size of the sequence-segmented forward (below); otherwise, and always for
+ * fp32, it is the one-CTA-per-sequence forward's B*H*64*dk*4 bytes.
+ */
 size_t gdn2_chunk_fwd_workspace(int B, int T, int H, int dk, int dv, int dtype);
 
 /*
@@ -71,8 +77,17 @@ size_t gdn2_chunk_fwd_workspace(int B, int T, int H, int dk, int dv, int dtype);
  * be a multiple of 64).  Computes o [B,T,H,dv] and, when S_T is non-null, the
  * final state S_T [B,H,dk,dv].  S0 may be null (zero initial state).
  * T = 0 is valid: it copies S0 (or zeros) to S_T.  B = 0 or H = 0 is a no-op.
- * ws/ws_bytes: caller-owned device workspace of at least
- * gdn2_chunk_fwd_workspace(...) bytes (ws may be null when that is 0).
+ * ws/ws_bytes: caller-owned device workspace of at least B*H*64*dk*4 bytes
+ * for bf16 (0 for fp32); ws may be null when that is 0.
+ * With ws_bytes >= gdn2_chunk_fwd_workspace(...) where that figure is the
+ * segmented one, each sequence runs as P equal segments side by side
+ * (P = 4..16, up to the SM count): the state update of a chunk is affine in
+ * the state (Gated Delta Rule-2 section of "Why NVIDIA Gated DeltaNet-2
+ * separates erase and write gates"), so every segment's local end state and
+ * dk x dk transition come from two forwards over the segments, an fp32 scan
+ * over the segments gives their start states, and a third forward gives o and
+ * S_T.  Same results to bf16 rounding; about three forwards of work on P times
+ * as many SMs.
  */
 int gdn2_chunk_fwd(const void *q, const void *k, const void *v, const void *log_alpha,
                    const void *b, const void *w, const float *S0, void *o, float *S_T,

@@ -77,6 +77,13 @@ def test_decode_and_bwd_reject_bad_arguments():
 
 def test_workspace_sizes():
     assert g.gdn2_chunk_fwd_workspace(8, 4096, 16, 128, 128, g.GDN2_BF16) == 8 * 16 * 64 * 128 * 4
+    # few long sequences: the segmented forward's workspace (P = 8 segments of
+    # B1 H16 T32768 on 148 SMs: per-CTA scratch of 8*16 CTAs, bf16 zeros of
+    # the token tensor, and four fp32 [8*16][128][128] state arrays)
+    seg = 8 * 16 * 64 * 128 * 4 + 32768 * 16 * 128 * 2 + 4 * 8 * 16 * 128 * 128 * 4
+    assert g.gdn2_chunk_fwd_workspace(1, 32768, 16, 128, 128, g.GDN2_BF16) == seg
+    # too short to split into four segments of 8 chunks: the plain size
+    assert g.gdn2_chunk_fwd_workspace(1, 1024, 16, 128, 128, g.GDN2_BF16) == 16 * 64 * 128 * 4
     assert g.gdn2_chunk_fwd_workspace(8, 4096, 16, 128, 128, g.GDN2_FP32) == 0
     assert g.gdn2_chunk_fwd_workspace(0, 4096, 16, 128, 128, g.GDN2_BF16) == 0
     assert g.gdn2_chunk_bwd_workspace(8, 4096, 16, 128, 128, g.GDN2_BF16) > 0
