@@ -69,3 +69,29 @@ def test_chunk_backward_bf16_error_budget():
     for n in ref:
         assert rel(got[n], ref[n]) < 8e-3, n
         assert np.max(np.abs(got[n] - ref[n])) < 5e-2, n
+
+
+def test_segment_composition_exact():
+    """The state update is affine in the state, so a sequence cut into segments
+    composes from each segment's end state from a zero start (S_loc) and from
+    an identity start with the write term w . v removed (the transition Phi):
+    S_start(p) = Phi(p-1) S_start(p-1) + S_loc(p-1), and each segment's o from
+    its true start state equals the whole sequence's o (the sequence-segmented
+    forward's algebra, checked on the oracle in fp64)."""
+    B, T, H, dk, dv, P = 1, 48, 2, 8, 8, 4
+    x = make_inputs(B, T, H, dk, dv, seed=21, dtype="fp32")
+    o_full, S_full = oracle.fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"], x["S0"])
+    L = T // P
+    seg = lambda a, p: a[:, p * L:(p + 1) * L]
+    eye = np.broadcast_to(np.eye(dk), (B, H, dk, dk)).copy()
+    S = x["S0"].astype(np.float64)
+    for p in range(P):
+        toks = [seg(x[n], p) for n in ("q", "k", "v", "log_alpha", "b", "w")]
+        _, S_loc = oracle.fwd(*toks, None)
+        zeros = np.zeros_like(toks[2])
+        _, Phi = oracle.fwd(toks[0], toks[1], zeros, toks[3], toks[4], zeros, eye)
+        o_seg, S_end = oracle.fwd(*toks, S)
+        np.testing.assert_allclose(o_seg, seg(o_full, p), rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(S_end, np.einsum("bhij,bhjk->bhik", Phi, S) + S_loc, rtol=1e-11, atol=1e-12)
+        S = S_end
+    np.testing.assert_allclose(S, S_full, rtol=1e-11, atol=1e-12)

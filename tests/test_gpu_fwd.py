@@ -137,3 +137,35 @@ def test_prefill_full_size_sampled_heads():
 @pytest.mark.parametrize("T", [8192, 32768, 131072])
 def test_long_sequence_sampled_heads(T):
     _sampled_full(WORKLOADS["long"], T=T, heads=((0, 0), (0, 11)))
+
+
+@pytest.mark.parametrize("dk", [128, 64])
+def test_segmented_and_one_cta_per_sequence(dk):
+    """B1 H4 T4096: with the workspace gdn2_chunk_fwd_workspace asks for, the
+    forward runs four sequence segments side by side; given only the plain
+    B*H*64*dk*4 bytes it runs one CTA per sequence.  Both against the oracle,
+    and against each other."""
+    import torch
+    import gated_delta_rule_gdn2_b200 as g
+    B, T, H = 1, 4096, 4
+    x = make_inputs(B, T, H, dk, dk, seed=404 + dk, dtype="bf16")
+    toks = tokens(x, "bf16")
+    S0 = dev_state(x["S0"])
+    plain = B * H * 64 * dk * 4
+    full = g.gdn2_chunk_fwd_workspace(B, T, H, dk, dk, g.GDN2_BF16)
+    assert full > plain
+    outs = []
+    for nbytes in (full, plain):
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        o = torch.empty((B, T, H, dk), dtype=torch.bfloat16, device="cuda")
+        ST = torch.empty((B, H, dk, dk), dtype=torch.float32, device="cuda")
+        st = g.gdn2_chunk_fwd(*toks, S0, o, ST, B, T, H, dk, dk, g.GDN2_BF16, ws, nbytes,
+                              torch.cuda.current_stream().cuda_stream)
+        assert st == 0
+        assert g.gdn2_get_device_status() == 0
+        outs.append((host(o), host(ST)))
+    o_ref, ST_ref = oracle_fwd(x)
+    for o, ST in outs:
+        check("o", o, o_ref, TOL_BF16)
+        check("S_T", ST, ST_ref, TOL_BF16)
+    check("o segmented vs one CTA per sequence", outs[0][0], outs[1][0], TOL_BF16)
