@@ -19,6 +19,7 @@ the data path); the time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import tempfile
 import hashlib
 import json
 import os
@@ -71,7 +72,9 @@ class ClockSampler:
     def __init__(self, bus_id):
         self.bus_id = bus_id
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_%d.csv" % os.getpid())
+        # the samples go to a file of their own (GDN2_CLOCKS_DIR, else the temp directory)
+        self.path = os.path.join(os.environ.get("GDN2_CLOCKS_DIR", tempfile.gettempdir()),
+                                 "gdn2_clocks_%d.csv" % os.getpid())
 
     def __enter__(self):
         try:
