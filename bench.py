@@ -60,6 +60,19 @@ def dist_env():
         int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def max_over_ranks(ms, world, device=None):
+    """The slowest rank's time (every rank calls this at the same point; one
+    rank returns its own).  The data path has no collective: this is the only
+    exchange, on the host side of the timing."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 
@@ -229,10 +242,7 @@ def run_gpu(args):
     total_ms = t_start.elapsed_time(t_end)
     fwd_ms = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
     bwd_ms = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_step = total_ms / args.steps
 
     # ---- prefill forward (gdn2_chunk_fwd, no states kept)
@@ -360,10 +370,7 @@ def run_gpu(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
     hbm, tf_burst, tf_sus, src = peaks()
     tokens = B * T * world
