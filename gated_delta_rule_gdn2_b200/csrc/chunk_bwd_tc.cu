@@ -15,16 +15,19 @@
 // read the results back (16x256b shape for the 64-row products, which lands
 // in the register layout of a warp-level m16n8 fragment; 32x32b rows for
 // dSigma), form the next bf16 operands in shared memory, and hand over:
-//   M1  dU = M^T dO + Kx D ;  dO U^T ;  dSigma += Qt^T dO      (D = g . dSigma)
+//   M1  dU = M^T dO + Kx D (committed first) ; dO U^T ; dSigma += Qt^T dO
+//       (D = g . dSigma)
 //   M2  T^T dU
 //   M3  nR U^T ;  dGt = nR S^T ;  dKb = U D^T ;  dSigma += Gt^T nR
 //   M4  dQt = dO S^T (+ dM Kb) ;  dGt += dA Kb ;  dKb += dA^T Gt + dM^T Qt
 // (the Gram terms in M4 only on a fast chunk; a slow chunk takes them term by
-// term in fp32, as in chunk_bwd.cu).  dQt, dGt and dKb then go to the fp32
-// staging tiles and the token-level gradients follow (chunk_bwd_common.cuh).
-// Every wait on the MMA completion barrier is bounded: on expiry the kernel
-// records GDN2_ERR_TIMEOUT in the device status word, frees its tensor memory
-// and returns.
+// term in fp32, as in chunk_bwd.cu).  Work off the chain runs inside the
+// products: dM and dv, dw during M3, the raw token rows and the dSigma.Sigma
+// row sums during M4.  dQt, dGt and dKb then go to the fp32 staging tiles and
+// the token-level gradients follow, four key channels per thread
+// (chunk_bwd_common.cuh token_grads4).  Every wait on an mbarrier is bounded:
+// on expiry the kernel records GDN2_ERR_TIMEOUT in the device status word,
+// frees its tensor memory and returns.
 #include "chunk_bwd_common.cuh"
 #include "gdn2.h"
 #include "tc_tiles.cuh"

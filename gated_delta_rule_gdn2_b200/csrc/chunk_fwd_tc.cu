@@ -7,21 +7,26 @@
 //   A = Gt Kb^T, M = Qt Kb^T,  T = (I + A)^{-1},
 //   U = T (w . v) - (T Gt) S,   O = Qt S + M U,   S <- Diag(gam) (S + Kb^T U).
 // The fp32 state S lives in TMEM (128 lanes = key channels x 128 columns)
-// for the whole sequence.  Per chunk one thread issues four MMA groups:
-//   the two Grams (M = N = 64, K = 128);
-//   T (w . v) into U's columns and T Gt (M = 64, N = 128, K = 64);
-//   U += (-W) S and O = Qt S (K = 128, bf16 S copy in shared memory as B);
-//   S += Kb^T U (M = 128) and O += M U,
-// and between them the warps read the results back with the 16x256b TMEM
-// load shape (the register layout of a warp-level m16n8 fragment) to form
-// the next bf16 operands: A in fp32 for the WY solve (TF32 tensor-core levels
-// on fp32 16x16 diagonal blocks, chunk_common.cuh), M, -W and U in bf16.  S is
-// scaled by gam in TMEM (32x32b load/store) and copied to bf16 for the next
-// chunk.  A chunk whose decay spans more than e^{-64} takes its Grams term by
-// term in fp32 inside the shared intra-chunk stage.  Tiles arrive by TMA and
-// the tiles kept for the backward leave as bulk stores.  Every wait on an
-// mbarrier is bounded: on expiry the kernel records GDN2_ERR_TIMEOUT in the
-// device status word, frees its tensor memory and returns.
+// for the whole sequence.  Two warp groups of 8 warps share the work: group
+// A forms chunk m's decay prefix and operands Qt, Gt, Kb and w . v, issues the
+// two Grams (M = N = 64, K = 128) and reads back A (fp32, for the WY solve)
+// and M (bf16); group B runs chunk m - 1's state chain: the WY solve (TF32
+// tensor-core levels on fp32 16x16 diagonal blocks, chunk_common.cuh), then
+//   T Gt (M = 64, N = 128, K = 64) and O = Qt S (K = 128, bf16 S copy in
+//   shared memory as B);
+//   U = T (w . v) + (-W) S;
+//   O += M U (committed first: the O epilogue runs under the next one) and
+//   S += Kb^T U (M = 128),
+// reading results back with the 16x256b TMEM load shape (the register layout
+// of a warp-level m16n8 fragment) to form -W and U in bf16.  S is scaled by
+// gam in TMEM (32x32b load/store) and copied to bf16 for the next chunk.  A
+// chunk whose decay spans more than e^{-64} takes its Grams term by term in
+// fp32 inside the shared intra-chunk stage (group A, with its own solve).
+// Tiles arrive by TMA into two stages, the pipeline's buffers; the tiles kept
+// for the backward leave as bulk stores and O as a TMA tensor store of its
+// bf16 image.  Every wait on an mbarrier is bounded: on expiry the kernel
+// records GDN2_ERR_TIMEOUT in the device status word, frees its tensor memory
+// and returns.
 #include "chunk_common.cuh"
 #include "gdn2.h"
 #include "launch.h"
