@@ -95,3 +95,41 @@ def test_segment_composition_exact():
         np.testing.assert_allclose(S_end, np.einsum("bhij,bhjk->bhik", Phi, S) + S_loc, rtol=1e-11, atol=1e-12)
         S = S_end
     np.testing.assert_allclose(S, S_full, rtol=1e-11, atol=1e-12)
+
+
+def test_backward_segment_composition_exact():
+    """The reverse chain composes over segments with the transpose of the
+    forward's segment transition: the state gradient at a segment's start is
+    Phi^T (its gradient at the segment's end) + the segment's own contribution
+    (its dS0 for a zero end gradient), and each segment's backward from its true
+    start state and end gradient gives the whole sequence's gradients on that
+    segment (the algebra a segmented backward would rest on, on the oracle in
+    fp64)."""
+    B, T, H, dk, dv, P = 1, 48, 2, 8, 8, 4
+    x = make_inputs(B, T, H, dk, dv, seed=23, dtype="fp32", with_do=True)
+    rng = np.random.default_rng(9)
+    dST = rng.standard_normal((B, H, dk, dv))
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    full = oracle.bwd(*[x[n] for n in names], x["S0"], x["dO"], dST)
+    L = T // P
+    seg = lambda a, p: a[:, p * L:(p + 1) * L]
+    eye = np.broadcast_to(np.eye(dk), (B, H, dk, dk)).copy()
+    # start states of the segments (forward) and their transitions
+    starts, phis = [x["S0"].astype(np.float64)], []
+    for p in range(P):
+        toks = [seg(x[n], p) for n in names]
+        zeros = np.zeros_like(toks[2])
+        phis.append(oracle.fwd(toks[0], toks[1], zeros, toks[3], toks[4], zeros, eye)[1])
+        starts.append(oracle.fwd(*toks, starts[-1])[1])
+    # the reverse scan over segments, then each segment's gradients
+    dS_end = dST
+    for p in reversed(range(P)):
+        toks = [seg(x[n], p) for n in names]
+        loc = oracle.bwd(*toks, starts[p], seg(x["dO"], p), np.zeros_like(dST))["dS0"]
+        dS_start = np.einsum("bhji,bhjk->bhik", phis[p], dS_end) + loc
+        g = oracle.bwd(*toks, starts[p], seg(x["dO"], p), dS_end)
+        np.testing.assert_allclose(g["dS0"], dS_start, rtol=1e-10, atol=1e-11)
+        for n in ("dq", "dk", "dv", "dlog_alpha", "db", "dw"):
+            np.testing.assert_allclose(g[n], seg(full[n], p), rtol=1e-10, atol=1e-11)
+        dS_end = dS_start
+    np.testing.assert_allclose(dS_end, full["dS0"], rtol=1e-10, atol=1e-11)
