@@ -293,7 +293,7 @@ def run_gpu(args):
         dec_inputs.append([torch.from_numpy(xs[n]).to(device=dev, dtype=torch.bfloat16)
                            for n in ("q", "k", "v", "log_alpha", "b", "w")])
     odec = torch.empty((DEC_B, DEC_H, D), dtype=torch.bfloat16, device=dev)
-    ndec = 256
+    ndec = 1024  # one timed block of 1024 steps (four pre-staged token sets in turn)
 
     def dec(i):
         st = g.gdn2_decode_step(*dec_inputs[i % 4], Sdec, odec, DEC_B, DEC_H, D, D, g.GDN2_BF16, sh)
