@@ -35,16 +35,20 @@ __global__ void identity_kernel(float *m, size_t count, int d) {
 }
 
 // Start states of the segments.  Block (b*H + h, column group g) owns 16
-// value columns of one sequence and walks its P segments in order.
+// value columns of one sequence and walks its P segments in order; each
+// segment's transition is staged in shared memory (coalesced) before use.
 constexpr int SCAN_COLS = 16, SCAN_THREADS = 256;
 template <int DK>
 __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(const float *S0, const float *Phi, const float *Sloc,
                                                            float *Sstart, int B, int H, int P, int dv) {
-    __shared__ float prev[DK][SCAN_COLS];
+    extern __shared__ __align__(16) float sm[];
+    // the transition with rows padded to DK + 1 floats: a warp's 32 rows fall in 32 banks
+    float (*phi_s)[DK + 1] = reinterpret_cast<float (*)[DK + 1]>(sm);                         // [DK][DK + 1]
+    float (*prev)[SCAN_COLS] = reinterpret_cast<float (*)[SCAN_COLS]>(sm + DK * (DK + 1));  // [DK][16]
     const int bh = blockIdx.x, b = bh / H, h = bh % H, c0 = blockIdx.y * SCAN_COLS;
     const int tid = threadIdx.x;
     constexpr int CPT = DK * SCAN_COLS / SCAN_THREADS;  // outputs per thread: CPT columns of one row
-    const int r = tid / (SCAN_COLS / CPT), cc = (tid % (SCAN_COLS / CPT)) * CPT;
+    const int r = tid % DK, cc = (tid / DK) * CPT;
     auto at = [&](int p) {  // offset of the [DK][dv] matrix of segment p of (b, h)
         return (((size_t)b * P + p) * H + h) * DK * dv;
     };
@@ -54,30 +58,39 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(const float *S0, con
         prev[rr][c] = v;
         Sstart[at(0) + (size_t)rr * dv + c0 + c] = v;
     }
-    __syncthreads();
     for (int p = 1; p < P; ++p) {
-        const float *phi = Phi + (((size_t)b * P + p - 1) * H + h) * DK * DK + (size_t)r * DK;
+        const float4 *src = reinterpret_cast<const float4 *>(Phi + (((size_t)b * P + p - 1) * H + h) * DK * DK);
+        for (int i = tid; i < DK * DK / 4; i += SCAN_THREADS) {
+            const float4 t = src[i];
+            const int rr = (4 * i) / DK, k = (4 * i) % DK;
+            phi_s[rr][k] = t.x;
+            phi_s[rr][k + 1] = t.y;
+            phi_s[rr][k + 2] = t.z;
+            phi_s[rr][k + 3] = t.w;
+        }
+        __syncthreads();  // the transition and prev are in place
         const float *loc = Sloc + at(p - 1) + (size_t)r * dv + c0 + cc;
         float acc[CPT];
 #pragma unroll
         for (int j = 0; j < CPT; ++j) acc[j] = loc[j];
-        for (int k = 0; k < DK; k += 4) {
-            const float4 a = *reinterpret_cast<const float4 *>(phi + k);
+#pragma unroll 4
+        for (int k = 0; k < DK; ++k) {
+            const float a = phi_s[r][k];
 #pragma unroll
-            for (int j = 0; j < CPT; ++j)
-                acc[j] += a.x * prev[k][cc + j] + a.y * prev[k + 1][cc + j] + a.z * prev[k + 2][cc + j] +
-                          a.w * prev[k + 3][cc + j];
+            for (int j = 0; j < CPT; ++j) acc[j] += a * prev[k][cc + j];
         }
-        __syncthreads();  // every thread is done reading prev
+        __syncthreads();  // every thread is done reading the transition and prev
         float *out = Sstart + at(p) + (size_t)r * dv + c0 + cc;
 #pragma unroll
         for (int j = 0; j < CPT; ++j) {
             prev[r][cc + j] = acc[j];
             out[j] = acc[j];
         }
-        __syncthreads();
     }
 }
+
+template <int DK>
+constexpr int scan_smem_bytes() { return (DK * (DK + 1) + DK * SCAN_COLS) * (int)sizeof(float); }
 
 using chunk::bf16;
 
@@ -158,10 +171,16 @@ cudaError_t launch_chunk_fwd_segments(const ChunkFwdArgs &a, int dk, int dv, int
     if ((e = launch_chunk_fwd(phi, dk, dk, s)) != cudaSuccess) return e;
     // 2. the segments' start states
     const dim3 grid((unsigned)(a.B * a.H), (unsigned)(dv / seg::SCAN_COLS));
-    if (dk == 128)
-        seg::scan_kernel<128><<<grid, seg::SCAN_THREADS, 0, s>>>(a.S0, c.phi, c.sloc, c.sstart, a.B, a.H, P, dv);
-    else
-        seg::scan_kernel<64><<<grid, seg::SCAN_THREADS, 0, s>>>(a.S0, c.phi, c.sloc, c.sstart, a.B, a.H, P, dv);
+    if (dk == 128) {
+        constexpr int bytes = seg::scan_smem_bytes<128>();
+        if ((e = cudaFuncSetAttribute(seg::scan_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) !=
+            cudaSuccess)
+            return e;
+        seg::scan_kernel<128><<<grid, seg::SCAN_THREADS, bytes, s>>>(a.S0, c.phi, c.sloc, c.sstart, a.B, a.H, P, dv);
+    } else {
+        constexpr int bytes = seg::scan_smem_bytes<64>();
+        seg::scan_kernel<64><<<grid, seg::SCAN_THREADS, bytes, s>>>(a.S0, c.phi, c.sloc, c.sstart, a.B, a.H, P, dv);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // 3. o and the segments' end states from the true start states
     ChunkFwdArgs fin{a.q, a.k, a.v, a.log_alpha, a.b, a.w, c.sstart, a.o, c.sloc, c.fwd_ws, wstride,
