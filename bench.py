@@ -60,6 +60,13 @@ def dist_env():
         int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def run_config(world):
+    """The workload as both arms report it."""
+    return {"workload": WORKLOAD, "global_batch": B * world, "seq_len": T, "heads": H, "dk": D, "dv": D,
+            "chunk": 64, "parallelism": "dp%d (independent batches)" % world,
+            "l2": "inputs larger than L2 (about 1 GB per step)"}
+
+
 def max_over_ranks(ms, world, device=None):
     """The slowest rank's time (every rank calls this at the same point; one
     rank returns its own).  The data path has no collective: this is the only
@@ -396,9 +403,7 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded normals of the pages' distributions; no dataset)",
-        "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": T, "heads": H,
-                   "dk": D, "dv": D, "chunk": 64, "parallelism": "dp%d (independent batches)" % world,
-                   "l2": "inputs larger than L2 (about 1 GB per step)"},
+        "config": run_config(world),
         "tflops": th * world * (FLOP_FWD + FLOP_BWD) / (ms_step * 1e-3) / 1e12,
         "breakdown": {
             "fwd_save_ms": fwd_ms, "bwd_saved_ms": bwd_ms,
@@ -459,7 +464,7 @@ def cpu_baseline(x, target_s=12.0):
             break
     tok = reps * n * T / H  # head-tokens / H = tokens of the batch
     return {"value": tok / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": "%d whole heads (T=%d) of the B8 H16 batch, fwd+bwd, %d rep(s), %.1f s" % (n, T, reps, el)}
+            "sample": "%d whole heads (T=%d) of the B%d H%d batch, fwd+bwd, %d rep(s), %.1f s" % (n, T, B, H, reps, el)}
 
 
 def run_reference(args):
@@ -467,7 +472,8 @@ def run_reference(args):
     if rank != 0:
         return
     from gated_delta_rule_gdn2_b200.inputs import WORKLOADS, make_workload
-    x = make_workload(WORKLOADS["train"])
+    w = WORKLOADS["train"]
+    x = make_workload(type(w)(**{**w.__dict__, "B": B}))
     vals = []
     cb = None
     per_step = max(1.0, min(5.0, 150.0 / max(1, args.steps)))
@@ -479,7 +485,7 @@ def run_reference(args):
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": B * T / v * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "config": {"workload": WORKLOAD, "global_batch": B, "seq_len": T},
+           "data": "synthetic", "config": run_config(world),
            "cpu_baseline": cb,
            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
