@@ -26,12 +26,14 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile gdn2_oracle.c into liboracle.so (gcc, -O2, OpenMP)."""
+    """Compile gdn2_oracle.c into liboracle.so (gcc, -O2, OpenMP), and the
+    layer oracle (gdn2_layer_oracle.c) beside it."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + ".tmp%d" % os.getpid()
         subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
                                "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
+    _load_layer()
     return _LIB
 
 
@@ -162,3 +164,93 @@ def decode(*a, **kw):
 
 def bwd(*a, **kw):
     return _default().bwd(*a, **kw)
+
+
+# ---------------------------------------------------------------------------
+# The layer prologue and epilogue (gdn2_layer_oracle.c): short causal
+# convolution + SiLU (+ L2 norm) of the q/k/v paths, the gate activations and
+# the RMS-normalised, SiLU-gated output, with their backward passes.
+
+_LAYER_SRC = os.path.join(_HERE, "gdn2_layer_oracle.c")
+_LAYER_LIB = os.path.join(_HERE, "liblayer_oracle.so")
+_layer = None
+
+
+def _load_layer():
+    global _layer
+    if _layer is None:
+        if not os.path.exists(_LAYER_LIB) or os.path.getmtime(_LAYER_LIB) < os.path.getmtime(_LAYER_SRC):
+            tmp = _LAYER_LIB + ".tmp%d" % os.getpid()
+            subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c99", "-o", tmp, _LAYER_SRC, "-lm"])
+            os.replace(tmp, _LAYER_LIB)
+        lib = ctypes.CDLL(_LAYER_LIB)
+        P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        lib.oracle_prologue_path.argtypes = [P, P, I, P, I, I, I, I, I, P, P]
+        lib.oracle_prologue_path_bwd.argtypes = [P, P, I, P, P, P, I, I, I, I, I, P, P, P]
+        lib.oracle_gate.argtypes = [P, P, Z, I]
+        lib.oracle_gate_bwd.argtypes = [P, P, P, Z, I]
+        lib.oracle_epilogue.argtypes = [P, P, P, P, I, I, I, I]
+        lib.oracle_epilogue_bwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I]
+        for f in ("oracle_prologue_path", "oracle_prologue_path_bwd", "oracle_gate", "oracle_gate_bwd",
+                  "oracle_epilogue", "oracle_epilogue_bwd"):
+            getattr(lib, f).restype = None
+        _layer = lib
+    return _layer
+
+
+def prologue_path(x, W, l2):
+    """One input path: depthwise causal conv (W [H*D][K]) + SiLU, and for the
+    query/key paths (l2=True) the L2 norm over the head dim.  x [B,T,H,D]."""
+    x, W = _f64(x), _f64(W)
+    B, T, H, D = x.shape
+    K = W.shape[-1]
+    assert W.shape == (H * D, K)
+    out, yw, sw = np.zeros(x.shape), np.zeros(x.shape), np.zeros(x.shape)
+    _load_layer().oracle_prologue_path(_ptr(x), _ptr(W), K, _ptr(out), B, T, H, D, int(bool(l2)), _ptr(yw), _ptr(sw))
+    return out
+
+
+def prologue_path_bwd(x, W, dout, l2):
+    """Backward of prologue_path: (dx [B,T,H,D], dW [H*D][K])."""
+    x, W, dout = _f64(x), _f64(W), _f64(dout)
+    B, T, H, D = x.shape
+    K = W.shape[-1]
+    dx, dW = np.zeros(x.shape), np.zeros(W.shape)
+    work = [np.zeros(x.shape) for _ in range(3)]
+    _load_layer().oracle_prologue_path_bwd(_ptr(x), _ptr(W), K, _ptr(dout), _ptr(dx), _ptr(dW), B, T, H, D,
+                                           int(bool(l2)), *[_ptr(w) for w in work])
+    return dx, dW
+
+
+def gate(x, kind):
+    """kind 'log_alpha': log sigmoid(x); 'sigmoid': sigmoid(x)."""
+    x = _f64(x)
+    out = np.zeros(x.shape)
+    _load_layer().oracle_gate(_ptr(x), _ptr(out), x.size, 0 if kind == "log_alpha" else 1)
+    return out
+
+
+def gate_bwd(x, dout, kind):
+    x, dout = _f64(x), _f64(dout)
+    dx = np.zeros(x.shape)
+    _load_layer().oracle_gate_bwd(_ptr(x), _ptr(dout), _ptr(dx), x.size, 0 if kind == "log_alpha" else 1)
+    return dx
+
+
+def epilogue(o, g, gamma):
+    """z = o / rms(o) * gamma * silu(g) per token and head; o, g [B,T,H,D], gamma [D]."""
+    o, g, gamma = _f64(o), _f64(g), _f64(gamma)
+    B, T, H, D = o.shape
+    z = np.zeros(o.shape)
+    _load_layer().oracle_epilogue(_ptr(o), _ptr(g), _ptr(gamma), _ptr(z), B, T, H, D)
+    return z
+
+
+def epilogue_bwd(o, g, gamma, dz):
+    """Backward of epilogue: (do, dg, dgamma)."""
+    o, g, gamma, dz = _f64(o), _f64(g), _f64(gamma), _f64(dz)
+    B, T, H, D = o.shape
+    dO, dg, dgamma = np.zeros(o.shape), np.zeros(o.shape), np.zeros(D)
+    _load_layer().oracle_epilogue_bwd(_ptr(o), _ptr(g), _ptr(gamma), _ptr(dz), _ptr(dO), _ptr(dg), _ptr(dgamma),
+                                      B, T, H, D)
+    return dO, dg, dgamma
