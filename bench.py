@@ -8,9 +8,12 @@ chunk-boundary states) + gdn2_chunk_bwd_saved (the gate-aware backward using
 them).  The plain forward (prefill, gdn2_chunk_fwd) and the decode step
 (B=256, H=16, fp32 state of 268 MB updated in place) are timed in the same
 run and reported under "prefill" and "decode", and the long-sequence forward
-(B=1, T=32768, H=16) under "long".  Inputs are seeded synthetic data of the
-pages' distributions (gated_delta_rule_gdn2_b200.inputs); they are larger
-than L2 (about 1 GB per step), so no separate flush is needed.
+(B=1, H=16, T = 8192, 32768 and 131072) under "long".  Inputs are seeded
+synthetic data of the pages' distributions (gated_delta_rule_gdn2_b200.inputs;
+the long-sequence inputs are drawn on the GPU from the same distributions);
+they are larger than L2 (about 1 GB per step), so no separate flush is needed.
+After the K timed steps, "sustained" repeats the step for at least a second
+with the clocks sampled throughout.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 Under torchrun each rank runs its own batch (weak scaling, no collective on
@@ -35,7 +38,8 @@ sys.path.insert(0, ROOT)
 
 B, T, H, D = 8, 4096, 16, 128  # B can be lowered with --batch for profiling captures
 DEC_B, DEC_H = 256, 16
-LONG_T = 32768  # the long-sequence forward leg (B1 H16)
+LONG_TS = (8192, 32768, 131072)  # the long-sequence forward legs (B1 H16)
+SUSTAINED_S = 1.0  # seconds of back-to-back steps after the timed ones
 WORKLOAD = "train fwd+bwd B8 T4096 H16 dk=dv=128 bf16 (prefill and decode B256 H16 alongside)"
 METRIC = "GDN-2 chunk fwd+bwd tokens/s & TFLOP/s (H16 dk=dv=128); decode state GB/s"
 # algorithmic work per (token, head), d = 128, C = 64: dense-counted products and bytes read + written once
@@ -43,7 +47,8 @@ FLOP_FWD = 6 * D * D + 10 * 64 * D          # 180,224
 FLOP_BWD = 524288 - (4 * D * D + 8 * 64 * D)  # 393,216: backward without the state recompute
 BYTES_FWD = 7 * D * 2                        # q,k,v,log_alpha,b,w in + o out, bf16
 BYTES_BWD = 13 * D * 2                       # 6 inputs + dO in, 6 gradients out, bf16
-BYTES_STATES = D * D * 2 // 64               # bf16 chunk-boundary state per token (written once, read once)
+# (the chunk-boundary states and per-chunk tiles the training forward keeps
+# for the backward are intermediates: counted in the ncu traffic, not here)
 STATE_BYTES = D * D * 4
 
 
@@ -100,7 +105,7 @@ class ClockSampler:
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
-            cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "200"]
+            cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "100"]
             if self.bus_id:
                 cmd[1:1] = ["-i", self.bus_id]
             self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
@@ -242,6 +247,20 @@ def run_gpu(args):
             m[2].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
+        # ---- sustained: the same step back to back for at least SUSTAINED_S
+        # seconds (the clocks are sampled across both regions)
+        n_sus = 0
+        s0, s1 = ev(), ev()
+        s0.record(stream)
+        t_wall = time.perf_counter()
+        while time.perf_counter() - t_wall < SUSTAINED_S:
+            for _ in range(50):
+                fwd()
+                bwd()
+            n_sus += 50
+            s1.record(stream)
+            s1.synchronize()
+        sus_ms = s0.elapsed_time(s1) / n_sus
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -250,6 +269,7 @@ def run_gpu(args):
     fwd_ms = statistics.mean(m[0].elapsed_time(m[1]) for m in marks)
     bwd_ms = statistics.mean(m[1].elapsed_time(m[2]) for m in marks)
     total_ms = max_over_ranks(total_ms, world, dev)
+    sus_ms = max_over_ranks(sus_ms, world, dev)
     ms_step = total_ms / args.steps
 
     # ---- prefill forward (gdn2_chunk_fwd, no states kept)
@@ -264,32 +284,40 @@ def run_gpu(args):
     torch.cuda.synchronize()
     pre_ms = p0.elapsed_time(p1) / args.steps
 
-    # ---- long-sequence forward (B1 T32768 H16: 16 sequences, so 16 CTAs)
-    from gated_delta_rule_gdn2_b200.inputs import WORKLOADS, make_workload
-    xl = make_workload(WORKLOADS["long"], T=LONG_T)
-    tl = [torch.from_numpy(xl[n]).to(device=dev, dtype=torch.bfloat16)
-          for n in ("q", "k", "v", "log_alpha", "b", "w")]
-    S0l = torch.from_numpy(xl["S0"]).to(dev)
-    ol = torch.empty((1, LONG_T, H, D), dtype=torch.bfloat16, device=dev)
-    STl = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
-    nlw = g.gdn2_chunk_fwd_workspace(1, LONG_T, H, D, D, g.GDN2_BF16)
-    wsl = torch.empty(max(nlw, 16), dtype=torch.uint8, device=dev)
+    # ---- long-sequence forward (B1 H16: 16 sequences) at T = 8192, 32768, 131072;
+    # inputs drawn on the device (the same distributions as the host recipe)
+    from gated_delta_rule_gdn2_b200.inputs import WORKLOADS, make_inputs_device
+    wl = WORKLOADS["long"]
+    xl = make_inputs_device(1, max(LONG_TS), H, D, D, seed=wl.seed, device=dev, alpha_mu=wl.alpha_mu)
+    long_legs = []
+    for TL in LONG_TS:
+        tl = [xl[n][:, :TL].contiguous() for n in ("q", "k", "v", "log_alpha", "b", "w")]
+        ol = torch.empty((1, TL, H, D), dtype=torch.bfloat16, device=dev)
+        STl = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
+        nlw = g.gdn2_chunk_fwd_workspace(1, TL, H, D, D, g.GDN2_BF16)
+        wsl = torch.empty(max(nlw, 16), dtype=torch.uint8, device=dev)
 
-    def long_fwd():
-        st = g.gdn2_chunk_fwd(*tl, S0l, ol, STl, 1, LONG_T, H, D, D, g.GDN2_BF16, wsl, nlw, sh)
-        assert st == 0, st
+        def long_fwd():
+            st = g.gdn2_chunk_fwd(*tl, xl["S0"], ol, STl, 1, TL, H, D, D, g.GDN2_BF16, wsl, nlw, sh)
+            assert st == 0, st
 
-    for _ in range(3):
-        long_fwd()
-    torch.cuda.synchronize()
-    l0, l1 = ev(), ev()
-    l0.record(stream)
-    for _ in range(args.steps):
-        long_fwd()
-    l1.record(stream)
-    torch.cuda.synchronize()
-    long_ms = l0.elapsed_time(l1) / args.steps
-    del tl, ol, wsl
+        for _ in range(3):
+            long_fwd()
+        torch.cuda.synchronize()
+        reps = max(3, min(args.steps, int(2e6 // TL)))
+        l0, l1 = ev(), ev()
+        l0.record(stream)
+        for _ in range(reps):
+            long_fwd()
+        l1.record(stream)
+        torch.cuda.synchronize()
+        ms = l0.elapsed_time(l1) / reps
+        nbytes = TL * H * BYTES_FWD + 2 * H * STATE_BYTES
+        long_legs.append({"T": TL, "ms": ms, "tokens_per_s": TL / (ms * 1e-3), "gbs": nbytes / (ms * 1e-3) / 1e9,
+                          "reps": reps})
+        del tl, ol, wsl
+    del xl
+    assert g.gdn2_get_device_status() == 0
 
     # ---- decode step, state of B256 H16 d128 resident and updated in place
     from gated_delta_rule_gdn2_b200.inputs import decode_initial_state, decode_step_inputs
@@ -382,14 +410,24 @@ def run_gpu(args):
     hbm, tf_burst, tf_sus, src = peaks()
     tokens = B * T * world
     th = B * T * H
-    fwd_gbs = (th * (BYTES_FWD + BYTES_STATES) + 2 * B * H * STATE_BYTES) / (fwd_ms * 1e-3) / 1e9
-    bwd_gbs = (th * (BYTES_BWD + BYTES_STATES) + 2 * B * H * STATE_BYTES) / (bwd_ms * 1e-3) / 1e9
+    # algorithmic bytes: token tensors in and out once, the fp32 S0 read and S_T
+    # (or dS0) written once; the states kept between the passes are not counted
+    fwd_gbs = (th * BYTES_FWD + 2 * B * H * STATE_BYTES) / (fwd_ms * 1e-3) / 1e9
+    bwd_gbs = (th * BYTES_BWD + 2 * B * H * STATE_BYTES) / (bwd_ms * 1e-3) / 1e9
     pre_gbs = (th * BYTES_FWD + 2 * B * H * STATE_BYTES) / (pre_ms * 1e-3) / 1e9
+    for leg in long_legs:
+        leg["hbm_frac"] = leg["gbs"] / hbm
+        leg["tflops"] = leg["T"] * H * FLOP_FWD / (leg["ms"] * 1e-3) / 1e12
+        leg["tensor_frac_of_bf16"] = leg["tflops"] / tf_burst
     dom = "bwd" if bwd_ms >= fwd_ms else "fwd"
     kname = {"fwd": "chunk_fwd_tc_kernel (with state output)", "bwd": "chunk_bwd_tc_kernel"}[dom]
     achieved = bwd_gbs if dom == "bwd" else fwd_gbs
     traffic = kernel_traffic("chunk_fwd_tc_kernel" if dom == "fwd" else "chunk_bwd_tc_kernel")
+    if traffic is not None:
+        traffic = traffic * B / 8  # the committed figure is per launch at B = 8
     clocks = clk.summary()
+    fwd_tf = th * FLOP_FWD / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = th * FLOP_BWD / (bwd_ms * 1e-3) / 1e12
     out = {
         "metric": METRIC,
         "value": tokens / (ms_step * 1e-3),
@@ -405,17 +443,20 @@ def run_gpu(args):
         "data": "synthetic (seeded normals of the pages' distributions; no dataset)",
         "config": run_config(world),
         "tflops": th * world * (FLOP_FWD + FLOP_BWD) / (ms_step * 1e-3) / 1e12,
+        # every tensor fraction below is against the measured bf16 burst peak
+        # (each leg is timed over well under a second); HBM fractions against
+        # the measured copy bandwidth
+        "peaks": {"hbm_gbs": hbm, "bf16_tflops": tf_burst, "source": src},
         "breakdown": {
             "fwd_save_ms": fwd_ms, "bwd_saved_ms": bwd_ms,
-            "fwd_tflops": th * FLOP_FWD / (fwd_ms * 1e-3) / 1e12,
+            "fwd_tflops": fwd_tf, "fwd_tensor_frac": fwd_tf / tf_burst,
             "fwd_gbs": fwd_gbs, "fwd_hbm_frac": fwd_gbs / hbm,
-            "bwd_tflops": th * FLOP_BWD / (bwd_ms * 1e-3) / 1e12,
+            "bwd_tflops": bwd_tf, "bwd_tensor_frac": bwd_tf / tf_burst,
             "bwd_gbs": bwd_gbs, "bwd_hbm_frac": bwd_gbs / hbm,
         },
-        "long": {"workload": "B1 T%d H16 dk=dv=128 forward (gdn2_chunk_fwd; 16 sequences)" % LONG_T,
-                 "ms": long_ms, "tokens_per_s": LONG_T / (long_ms * 1e-3),
-                 "gbs": (LONG_T * H * BYTES_FWD + 2 * H * STATE_BYTES) / (long_ms * 1e-3) / 1e9,
-                 "hbm_frac": (LONG_T * H * BYTES_FWD + 2 * H * STATE_BYTES) / (long_ms * 1e-3) / 1e9 / hbm},
+        "sustained": {"ms_per_step": sus_ms, "steps": n_sus, "seconds": sus_ms * n_sus / 1e3,
+                      "tokens_per_s": tokens / (sus_ms * 1e-3)},
+        "long": long_legs,
         "prefill": {"workload": "B8 T4096 H16 dk=dv=128 forward (gdn2_chunk_fwd)", "ms": pre_ms,
                     "tokens_per_s": B * T / (pre_ms * 1e-3), "tflops": th * FLOP_FWD / (pre_ms * 1e-3) / 1e12,
                     "gbs": pre_gbs, "hbm_frac": pre_gbs / hbm,
@@ -426,8 +467,7 @@ def run_gpu(args):
         "roofline": {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic,
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs, copy)" % src,
-                     "tensor_frac_of_bf16": (th * (FLOP_FWD if dom == "fwd" else FLOP_BWD)
-                                             / ((fwd_ms if dom == "fwd" else bwd_ms) * 1e-3) / 1e12) / tf_sus},
+                     "tensor_frac_of_bf16": (fwd_tf if dom == "fwd" else bwd_tf) / tf_burst},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,  # chunk_fwd_tc_kernel (with states) + chunk_bwd_tc_kernel per step

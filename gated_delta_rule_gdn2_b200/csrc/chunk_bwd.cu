@@ -35,6 +35,7 @@
 // then; the per-CTA fp32 scratch of the caller's workspace (L2-resident) holds
 // the slow-path partial gradients and a few row sums.
 #include "chunk_bwd_common.cuh"
+#include "gdn2.h"
 
 namespace gdn2 {
 namespace cbwd {
@@ -54,10 +55,18 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
     __shared__ float s_rs[2][DK];
     BwdChunk<DK, DV> x(a, smem, &sh, s_dpart, s_dmd, s_rs);
     const int warp = x.warp, lane = x.lane, bh = blockIdx.x;
-    const int T = a.T, nchunks = x.nchunks;
+    if (!x.sv.ok) {  // packed-sequence offsets out of range: nothing of this sequence is touched
+        if (x.tid == 0) record_status(a.status, GDN2_ERR_INVALID_ARG);
+        return;
+    }
+    const int T = x.len, nchunks = x.nchunks;
     const ChunkTiles st = x.st;
     bf16 *dO16 = x.dO16, *S16 = x.S16, *D16 = x.D16, *T16 = x.T16, *M16 = x.M16, *dU16 = x.dU16, *U16 = x.U16;
     bf16 *nR16 = x.nR16, *dM16 = x.dM16, *dA16 = x.dA16;
+    // dM's entries reach tens: its products take it as two bf16 tiles, the
+    // rounding dM16 and the remainder dMlo16 (about 16 significant bits)
+    bf16 *dMlo16 = reinterpret_cast<bf16 *>(smem + BSmem<DK, DV>::OMLO);
+    x.dMlo16 = dMlo16;
     float *A32 = x.A32, *T32 = x.T32, *LAM = x.LAM, *DQT = x.DQT, *DGT = x.DGT, *DKB = x.DKB;
     const bf16 *states = x.states;
 
@@ -143,6 +152,12 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
                     if (i >= r) acc[0][nt][e] = 0.f;
                 }
             store_tile_bf16<8, 64>(acc, dM16, 16 * (warp & 3), lane, 1.f);
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc[0][nt][e] -= __bfloat162float(__float2bfloat16_rn(acc[0][nt][e]));
+            store_tile_bf16<8, 64>(acc, dMlo16, 16 * (warp & 3), lane, 1.f);
         }
         __syncthreads();
 
@@ -182,6 +197,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
             store_stage<DK, NTK>(accK, DGT, 16 * warp, 0, lane);  // the WY-solve area is dead
         } else if (!slow) {
             warp_gemm<1, NTK, true, false, 64, DK, C, C, KU>(accK, dM16, 16 * (warp & 3), st.la, 0, C, lane);
+            warp_gemm<1, NTK, true, false, 64, DK, C, C, KU>(accK, dMlo16, 16 * (warp & 3), st.la, 0, C, lane);
         }
         __syncthreads();  // S is no longer read: its region takes dQt
 
@@ -194,6 +210,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_bwd_kernel(ChunkBwdArgs a) {
             if (!slow) {
                 warp_gemm<1, NTK, false, false, 64, DK, C, C, KU>(accK, dA16, m0, st.b, 0, C, lane);
                 warp_gemm<1, NTK, false, false, 64, DK, C, C, KU>(accK, dM16, m0, st.q, 0, C, lane);
+                warp_gemm<1, NTK, false, false, 64, DK, C, C, KU>(accK, dMlo16, m0, st.q, 0, C, lane);
             }
             asm volatile("bar.sync 1, 128;\n" ::: "memory");  // warps 4..7 are done reading Dh
             store_stage<DK, NTK>(accK, DKB, m0, 0, lane);
@@ -239,7 +256,8 @@ cudaError_t launch_t(const ChunkBwdArgs &a, cudaStream_t s) {
     cudaError_t e = cudaSuccess;
     if (!a.states_given) {
         ChunkFwdArgs f{a.q, a.k, a.v, a.log_alpha, a.b, a.w, a.S0, nullptr, nullptr, a.scratch, a.scr_stride,
-                       a.states, a.intra, a.ops, a.status, a.B, a.T, a.H};
+                       a.states, a.intra, a.ops, a.status, a.B, a.T, a.H, a.cu_seqlens};
+        f.gates = a.gates;
         e = launch_chunk_fwd(f, DK, DV, s);
         if (e != cudaSuccess) return e;
     }
@@ -256,9 +274,9 @@ cudaError_t launch_t(const ChunkBwdArgs &a, cudaStream_t s) {
 }
 
 template <int DK, int DV>
-size_t ws_t(int B, int T, int H, size_t *scr_stride, size_t *states_bytes) {
-    const size_t sb = states_region_bytes(B, T, H, DK, DV) + intra_region_bytes(B, T, H, DV) +
-                      ops_region_bytes(B, T, H, DK, DV);
+size_t ws_t(int B, int T, int H, size_t *scr_stride, size_t *states_bytes, bool varlen) {
+    const size_t sb = states_region_bytes(B, T, H, DK, DV, varlen) + intra_region_bytes(B, T, H, DV, varlen) +
+                      ops_region_bytes(B, T, H, DK, DV, varlen);
     const size_t stride = (Scratch<DK>::FLOATS + 63) / 64 * 64;
     if (scr_stride) *scr_stride = stride;
     if (states_bytes) *states_bytes = sb;
@@ -267,11 +285,12 @@ size_t ws_t(int B, int T, int H, size_t *scr_stride, size_t *states_bytes) {
 
 }  // namespace cbwd
 
-size_t chunk_bwd_ws_bytes(int B, int T, int H, int dk, int dv, size_t *scr_stride, size_t *states_bytes) {
-    if (dk == 128 && dv == 128) return cbwd::ws_t<128, 128>(B, T, H, scr_stride, states_bytes);
-    if (dk == 128 && dv == 64) return cbwd::ws_t<128, 64>(B, T, H, scr_stride, states_bytes);
-    if (dk == 64 && dv == 128) return cbwd::ws_t<64, 128>(B, T, H, scr_stride, states_bytes);
-    return cbwd::ws_t<64, 64>(B, T, H, scr_stride, states_bytes);
+size_t chunk_bwd_ws_bytes(int B, int T, int H, int dk, int dv, size_t *scr_stride, size_t *states_bytes,
+                          bool varlen) {
+    if (dk == 128 && dv == 128) return cbwd::ws_t<128, 128>(B, T, H, scr_stride, states_bytes, varlen);
+    if (dk == 128 && dv == 64) return cbwd::ws_t<128, 64>(B, T, H, scr_stride, states_bytes, varlen);
+    if (dk == 64 && dv == 128) return cbwd::ws_t<64, 128>(B, T, H, scr_stride, states_bytes, varlen);
+    return cbwd::ws_t<64, 64>(B, T, H, scr_stride, states_bytes, varlen);
 }
 
 cudaError_t launch_chunk_bwd(const ChunkBwdArgs &a, int dk, int dv, cudaStream_t s) {

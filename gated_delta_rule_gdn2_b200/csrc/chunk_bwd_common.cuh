@@ -34,7 +34,11 @@ struct BSmem {
     static constexpr bool STAGE_REUSE = (DK == 128 && DV == 128);
     static constexpr bool STAGE_DED = (DK == 64);
     static constexpr int OSTG = OAM + (AM_IN_K ? 0 : 16384);
-    static constexpr int BYTES = OSTG + (STAGE_DED ? 3 * C * DK * 4 : 0);
+    // the low-order part dM - bf16(dM) of dM (64x64 bf16): a region of its own
+    // for the warp-level kernel (the tensor-memory kernel reuses the U slot)
+    static constexpr bool MLO_DED = !(DK == 128 && DV == 128);
+    static constexpr int OMLO = OSTG + (STAGE_DED ? 3 * C * DK * 4 : 0);
+    static constexpr int BYTES = OMLO + (MLO_DED ? C * C * 2 : 0);
 };
 
 template <int DK>
@@ -80,10 +84,17 @@ struct BwdChunk {
     IntraShared<DK, NT> *sh;  // decay sums of the two-channel token pass (token_grads)
     float (*s_dpart)[DK];     // [NT / (DK / 2)][DK] segment sums of dL (token_grads)
     float *s_dmd;          // [C] diagonal of dO U^T
+    float *s_dbw = nullptr;  // [C] scalar gates: per token, the sum of dw over the value channels
     float (*s_rs)[DK];     // [NRS][DK] row sums of dSigma . Sigma over NRS column parts
-    int tid, warp, lane, b, h, T, H, nchunks;
+    int tid, warp, lane, b, h, H, nchunks;
+    SeqView sv;   // the sequence's token rows and saved-tile slots
+    size_t row0;  // its first token row
+    int len;      // its tokens
     ChunkTiles st;
     bf16 *dO16, *S16, *D16, *T16, *M16, *dU16, *U16, *nR16, *dM16, *dA16;
+    // optional: the low-order bf16 part dM - bf16(dM) of the masked dO U^T (a
+    // kernel that keeps it sets this; a slow chunk's Gram gradients add it)
+    const bf16 *dMlo16 = nullptr;
     float *A32, *T32;
     float *LAM, *DQT, *DGT, *DKB, *PQ, *PG, *PK, *PL;
     const bf16 *states, *gq, *gk, *gb, *gv, *gw;
@@ -94,8 +105,11 @@ struct BwdChunk {
         : a(args), sh(sh_), s_dpart(dpart), s_dmd(dmd), s_rs(rs) {
         tid = threadIdx.x; warp = tid >> 5; lane = tid & 31;
         const int bh = blockIdx.x;
-        b = bh / a.H; h = bh % a.H; T = a.T; H = a.H;
-        nchunks = (T + C - 1) / C;
+        b = bh / a.H; h = bh % a.H; H = a.H;
+        sv = seq_view(a.cu_seqlens, b, h, a.B, a.T, a.H);
+        row0 = sv.row0;
+        len = sv.len;
+        nchunks = sv.nchunks;
         st = ChunkTiles{reinterpret_cast<bf16 *>(smem + L::OQ), reinterpret_cast<bf16 *>(smem + L::OK),
                         reinterpret_cast<bf16 *>(smem + L::OLA), reinterpret_cast<bf16 *>(smem + L::OB),
                         reinterpret_cast<bf16 *>(smem + L::OV), reinterpret_cast<bf16 *>(smem + L::OW)};
@@ -125,8 +139,8 @@ struct BwdChunk {
             DKB = DQT + C * DK;
             DGT = DKB + C * DK;
         }
-        states = static_cast<const bf16 *>(a.states) + (size_t)bh * (nchunks + 1) * DK * DV;
-        intra = static_cast<const unsigned char *>(a.intra) + (size_t)bh * nchunks * I_BYTES;
+        states = static_cast<const bf16 *>(a.states) + sv.sslot * DK * DV;
+        intra = static_cast<const unsigned char *>(a.intra) + sv.cslot * I_BYTES;
         gq = static_cast<const bf16 *>(a.q); gk = static_cast<const bf16 *>(a.k);
         gb = static_cast<const bf16 *>(a.b); gv = static_cast<const bf16 *>(a.v);
         gw = static_cast<const bf16 *>(a.w);
@@ -137,11 +151,11 @@ struct BwdChunk {
     // group B = the chunk-start state and the forward's T, M (into the WY-solve
     // area).  The forward's tiles are stored as their shared-memory images.
     __device__ void issue_a(int n) {
-        load_token_tile<DK, NT>(st.q, gq, b, h, n, T, H);
-        load_token_tile<DK, NT>(st.k, gk, b, h, n, T, H);
-        load_token_tile<DK, NT>(st.la, static_cast<const bf16 *>(a.log_alpha), b, h, n, T, H);
-        load_token_tile<DK, NT>(st.b, gb, b, h, n, T, H);
-        load_token_tile<DV, NT>(dO16, static_cast<const bf16 *>(a.dO), b, h, n, T, H);
+        load_token_tile<DK, NT>(st.q, gq, row0, len, h, n, H);
+        load_token_tile<DK, NT>(st.k, gk, row0, len, h, n, H);
+        load_token_tile<DK, NT>(st.la, static_cast<const bf16 *>(a.log_alpha), row0, len, h, n, H);
+        load_token_tile<DK, NT>(st.b, gb, row0, len, h, n, H);
+        load_token_tile<DV, NT>(dO16, static_cast<const bf16 *>(a.dO), row0, len, h, n, H);
         const unsigned char *it = intra + (size_t)n * I_BYTES + TM_BYTES;
         for (int id = tid; id < U_BYTES / 16; id += NT)
             cp_async16(reinterpret_cast<unsigned char *>(U16) + 16 * id, it + 16 * id, true);
@@ -163,16 +177,16 @@ struct BwdChunk {
         if (tid >= 256) return;
         const int slot = tid & 63, grp = tid >> 6;
         if (grp == 0) {
-            prefetch_token_rows_l2<DK>(gq, b, h, n, T, H, slot, 64);
-            prefetch_token_rows_l2<DK>(gk, b, h, n, T, H, slot, 64);
+            prefetch_token_rows_l2<DK>(gq, row0, len, h, n, H, slot, 64);
+            prefetch_token_rows_l2<DK>(gk, row0, len, h, n, H, slot, 64);
         } else if (grp == 1) {
-            prefetch_token_rows_l2<DK>(static_cast<const bf16 *>(a.log_alpha), b, h, n, T, H, slot, 64);
-            prefetch_token_rows_l2<DK>(gb, b, h, n, T, H, slot, 64);
+            prefetch_token_rows_l2<DK>(static_cast<const bf16 *>(a.log_alpha), row0, len, h, n, H, slot, 64);
+            prefetch_token_rows_l2<DK>(gb, row0, len, h, n, H, slot, 64);
         } else if (grp == 2) {
-            prefetch_token_rows_l2<DV>(gv, b, h, n, T, H, slot, 64);
-            prefetch_token_rows_l2<DV>(gw, b, h, n, T, H, slot, 64);
+            prefetch_token_rows_l2<DV>(gv, row0, len, h, n, H, slot, 64);
+            prefetch_token_rows_l2<DV>(gw, row0, len, h, n, H, slot, 64);
         } else {
-            prefetch_token_rows_l2<DV>(static_cast<const bf16 *>(a.dO), b, h, n, T, H, slot, 64);
+            prefetch_token_rows_l2<DV>(static_cast<const bf16 *>(a.dO), row0, len, h, n, H, slot, 64);
             if (slot < 16) {
                 const bf16 *sp = states + (size_t)n * DK * DV + (size_t)slot * (DK * DV / 16);
                 asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(sp), "r"(DK * DV * 2 / 16)
@@ -188,9 +202,9 @@ struct BwdChunk {
     // straight from global memory (one 128-byte line per thread).
     __device__ void prefetch_vw_l2(int n) {
         const int t = n * C + ((tid >> 1) & (C - 1));
-        if (tid >= 4 * C || t >= T) return;
+        if (tid >= 4 * C || t >= len) return;
         const bf16 *src = (tid < 2 * C) ? gv : gw;
-        const bf16 *row = src + (((size_t)b * T + t) * H + h) * DV;
+        const bf16 *row = src + ((row0 + t) * H + h) * DV;
         if ((tid & 1) * 64 < DV)
             asm volatile("prefetch.global.L2 [%0];\n" ::"l"(row + (tid & 1) * 64) : "memory");
     }
@@ -213,17 +227,21 @@ struct BwdChunk {
                 PQ[r * DK + ch] = 0.f; PG[r * DK + ch] = 0.f; PK[r * DK + ch] = 0.f; PL[r * DK + ch] = 0.f;
             }
             for (int r = 0; r < Cn; ++r) {
-                const size_t orr = (((size_t)b * T + n * C + r) * H + h) * DK + ch;
+                const size_t orr = ((row0 + n * C + r) * H + h) * DK + ch;
                 const float qr = __bfloat162float(gq[orr]);
-                const float gr = __bfloat162float(gb[orr]) * __bfloat162float(gk[orr]);
+                const float br = a.gates == kGatesFull ? __bfloat162float(gb[orr])
+                                                       : __bfloat162float(gb[(row0 + n * C + r) * H + h]);
+                const float gr = br * __bfloat162float(gk[orr]);
                 const float lr = LAM[r * DK + ch];
                 float pq = 0.f, pg = 0.f, pl = 0.f;
                 for (int i = 0; i <= r; ++i) {
-                    const size_t oi = (((size_t)b * T + n * C + i) * H + h) * DK + ch;
+                    const size_t oi = ((row0 + n * C + i) * H + h) * DK + ch;
                     const float ki = __bfloat162float(gk[oi]);
                     const float e = __expf(lr - LAM[i * DK + ch]);
                     const float wA = i < r ? __bfloat162float(dA16[swz<64>(r, i)]) * e : 0.f;
-                    const float wM = __bfloat162float(dM16[swz<64>(r, i)]) * e;
+                    const float dm = __bfloat162float(dM16[swz<64>(r, i)]) +
+                                     (dMlo16 ? __bfloat162float(dMlo16[swz<64>(r, i)]) : 0.f);
+                    const float wM = dm * e;
                     pg += wA * ki;
                     pq += wM * ki;
                     const float tk = wA * gr + wM * qr;
@@ -247,21 +265,50 @@ struct BwdChunk {
     template <int T0 = 0>
     __device__ void dvdw(int n, int Cn) {
         constexpr int ITEMS = C * DV / 8, NV = (ITEMS + NT - T0 - 1) / (NT - T0);
+        // scalar gates (the tensor-memory kernel only): a row's 16 items on a half-warp
+        constexpr bool kScalarOK = T0 % 16 == 0 && (NT - T0) % 16 == 0 && DV == 128;
         const int t = tid - T0;
         if (t < 0) return;
+        const bool scalar = kScalarOK && a.gates != kGatesFull;  // w = beta 1: w from beta, the sum of dw per token
         uint4 v8[NV], w8[NV];
 #pragma unroll
         for (int it = 0; it < NV; ++it) {
             const int id = min(t + it * (NT - T0), ITEMS - 1), r = id / (DV / 8), j = (id % (DV / 8)) * 8;
-            const size_t o = (((size_t)b * T + n * C + min(r, Cn - 1)) * H + h) * DV + j;
+            const size_t o = ((row0 + n * C + min(r, Cn - 1)) * H + h) * DV + j;
             v8[it] = *reinterpret_cast<const uint4 *>(gv + o);
-            w8[it] = *reinterpret_cast<const uint4 *>(gw + o);
+            if (!scalar) {
+                w8[it] = *reinterpret_cast<const uint4 *>(gw + o);
+            } else {
+                uint32_t x = reinterpret_cast<const unsigned short *>(gw)[(row0 + n * C + min(r, Cn - 1)) * H + h];
+                x |= x << 16;
+                w8[it] = make_uint4(x, x, x, x);
+            }
+        }
+        if constexpr (kScalarOK) if (scalar) {
+#pragma unroll
+            for (int it = 0; it < NV; ++it) {
+                const int id = t + it * (NT - T0), r = id / (DV / 8);
+                float part = 0.f;
+                if (id < ITEMS && r < Cn) {
+                    uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, (id % (DV / 8)) * 8));
+                    const __nv_bfloat162 *n2 = reinterpret_cast<const __nv_bfloat162 *>(&nr);
+                    const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&v8[it]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 nn = __bfloat1622float2(n2[e]), vv = __bfloat1622float2(v2[e]);
+                        part -= nn.x * vv.x + nn.y * vv.y;  // dRHS = -nR
+                    }
+                }
+#pragma unroll
+                for (int off = 8; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+                if (id < ITEMS && r < Cn && (id & 15) == 0) s_dbw[r] = part;
+            }
         }
 #pragma unroll
         for (int it = 0; it < NV; ++it) {
             const int id = t + it * (NT - T0), r = id / (DV / 8), j = (id % (DV / 8)) * 8;
             if (id < ITEMS && r < Cn) {
-                const size_t o = (((size_t)b * T + n * C + r) * H + h) * DV + j;
+                const size_t o = ((row0 + n * C + r) * H + h) * DV + j;
                 uint4 nr = *reinterpret_cast<const uint4 *>(nR16 + swz<DV>(r, j));
                 nr.x ^= 0x80008000u; nr.y ^= 0x80008000u; nr.z ^= 0x80008000u; nr.w ^= 0x80008000u;  // dRHS = -nR
                 const __nv_bfloat162 *n2 = reinterpret_cast<const __nv_bfloat162 *>(&nr);
@@ -276,7 +323,7 @@ struct BwdChunk {
                     dwp[e] = __hmul2(n2[e], v2[e]);
                 }
                 *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dv) + o) = dv8;
-                *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dw) + o) = dw8;
+                if (!scalar) *reinterpret_cast<uint4 *>(static_cast<bf16 *>(a.dw) + o) = dw8;
             }
         }
     }
@@ -293,7 +340,7 @@ struct BwdChunk {
 #pragma unroll
         for (int i = 0; i < RS2; ++i) {
             const int r = min(s2 * RS2 + i, Cn - 1);
-            const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c2;
+            const size_t o = ((row0 + n * C + r) * H + h) * DK + c2;
             raw.q[i] = *reinterpret_cast<const __nv_bfloat162 *>(gq + o);
             raw.k[i] = *reinterpret_cast<const __nv_bfloat162 *>(gk + o);
             raw.b[i] = *reinterpret_cast<const __nv_bfloat162 *>(gb + o);
@@ -343,7 +390,7 @@ struct BwdChunk {
                 dla_r[i] = 0.f;
                 dlb_r[i] = 0.f;
                 if (r < Cn) {
-                    const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c2;
+                    const size_t o = ((row0 + n * C + r) * H + h) * DK + c2;
                     const float2 q = __bfloat1622float2(raw.q[i]);
                     const float2 kk = __bfloat1622float2(raw.k[i]);
                     const float2 bb = __bfloat1622float2(raw.b[i]);
@@ -403,7 +450,7 @@ struct BwdChunk {
                     acca += dla_r[i];
                     accb += dlb_r[i];
                     *reinterpret_cast<uint32_t *>(static_cast<bf16 *>(a.dlog_alpha) +
-                                                  (((size_t)b * T + n * C + r) * H + h) * DK + c2) =
+                                                  ((row0 + n * C + r) * H + h) * DK + c2) =
                         pack_bf16(acca, accb);
                 }
             }
@@ -421,14 +468,27 @@ struct BwdChunk {
     __device__ void load_rows4(RawRows4 &raw, int n, int Cn) const {
         const int c4 = 4 * (tid % NQ), s4 = tid / NQ;
         const bf16 *gla = static_cast<const bf16 *>(a.log_alpha);
+        const unsigned short *sb = reinterpret_cast<const unsigned short *>(gb);
+        const unsigned short *sla = reinterpret_cast<const unsigned short *>(gla);
 #pragma unroll
         for (int i = 0; i < R4; ++i) {
             const int r = min(s4 * R4 + i, Cn - 1);
-            const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c4;
+            const size_t o = ((row0 + n * C + r) * H + h) * DK + c4;
+            const size_t os = (row0 + n * C + r) * H + h;  // a scalar gate's element
             raw.q[i] = *reinterpret_cast<const uint2 *>(gq + o);
             raw.k[i] = *reinterpret_cast<const uint2 *>(gk + o);
-            raw.b[i] = *reinterpret_cast<const uint2 *>(gb + o);
-            raw.la[i] = *reinterpret_cast<const uint2 *>(gla + o);
+            if (a.gates == kGatesFull) {
+                raw.b[i] = *reinterpret_cast<const uint2 *>(gb + o);
+            } else {
+                const uint32_t x = sb[os] | ((uint32_t)sb[os] << 16);
+                raw.b[i] = make_uint2(x, x);
+            }
+            if (a.gates != kGatesGDN) {
+                raw.la[i] = *reinterpret_cast<const uint2 *>(gla + o);
+            } else {
+                const uint32_t x = sla[os] | ((uint32_t)sla[os] << 16);
+                raw.la[i] = make_uint2(x, x);
+            }
         }
     }
     // One channel pair of a fast chunk: dq, dk, db before the diagonal-of-M
@@ -496,7 +556,7 @@ struct BwdChunk {
             dl0[i] = make_float2(0.f, 0.f);
             dl1[i] = make_float2(0.f, 0.f);
             if (r < Cn) {
-                const size_t o = (((size_t)b * T + n * C + r) * H + h) * DK + c4;
+                const size_t o = ((row0 + n * C + r) * H + h) * DK + c4;
                 const float2 q0 = unpack_bf16(raw.q[i].x), q1 = unpack_bf16(raw.q[i].y);
                 const float2 k0 = unpack_bf16(raw.k[i].x), k1 = unpack_bf16(raw.k[i].y);
                 const float2 b0 = unpack_bf16(raw.b[i].x), b1 = unpack_bf16(raw.b[i].y);
@@ -540,7 +600,13 @@ struct BwdChunk {
                 const float2 db0 = __fmul2_rn(p0.dg, k0), db1 = __fmul2_rn(p1.dg, k1);
                 *reinterpret_cast<uint2 *>(gdq + o) = make_uint2(pack_bf16(p0.dq.x, p0.dq.y), pack_bf16(p1.dq.x, p1.dq.y));
                 *reinterpret_cast<uint2 *>(gdk + o) = make_uint2(pack_bf16(dk0.x, dk0.y), pack_bf16(dk1.x, dk1.y));
-                *reinterpret_cast<uint2 *>(gdb + o) = make_uint2(pack_bf16(db0.x, db0.y), pack_bf16(db1.x, db1.y));
+                if (a.gates == kGatesFull) {
+                    *reinterpret_cast<uint2 *>(gdb + o) =
+                        make_uint2(pack_bf16(db0.x, db0.y), pack_bf16(db1.x, db1.y));
+                } else {  // dbeta = sum over the key channels of db, plus that of dw
+                    const float sdb = warp_sum(db0.x + db0.y + db1.x + db1.y);
+                    if (lane == 0) gdb[(row0 + n * C + r) * H + h] = __float2bfloat16_rn(sdb + s_dbw[r]);
+                }
                 dl0[i] = p0.dl;
                 dl1[i] = p1.dl;
                 ps0 = __fadd2_rn(ps0, p0.dl);
@@ -566,8 +632,13 @@ struct BwdChunk {
             if (r < Cn) {
                 acc0 = __fadd2_rn(acc0, dl0[i]);
                 acc1 = __fadd2_rn(acc1, dl1[i]);
-                *reinterpret_cast<uint2 *>(gdl + (((size_t)b * T + n * C + r) * H + h) * DK + c4) =
-                    make_uint2(pack_bf16(acc0.x, acc0.y), pack_bf16(acc1.x, acc1.y));
+                if (a.gates != kGatesGDN) {
+                    *reinterpret_cast<uint2 *>(gdl + ((row0 + n * C + r) * H + h) * DK + c4) =
+                        make_uint2(pack_bf16(acc0.x, acc0.y), pack_bf16(acc1.x, acc1.y));
+                } else {  // a scalar decay: the sum over the key channels
+                    const float sdl = warp_sum(acc0.x + acc0.y + acc1.x + acc1.y);
+                    if (lane == 0) gdl[(row0 + n * C + r) * H + h] = __float2bfloat16_rn(sdl);
+                }
             }
         }
     }

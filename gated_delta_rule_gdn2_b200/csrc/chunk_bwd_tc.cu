@@ -20,6 +20,7 @@
 //   M2  T^T dU
 //   M3  nR U^T ;  dGt = nR S^T ;  dKb = U D^T ;  dSigma += Gt^T nR
 //   M4  dQt = dO S^T (+ dM Kb) ;  dGt += dA Kb ;  dKb += dA^T Gt + dM^T Qt
+//       (dM as the sum of two bf16 tiles, its rounding and the remainder)
 // (the Gram terms in M4 only on a fast chunk; a slow chunk takes them term by
 // term in fp32, as in chunk_bwd.cu).  Work off the chain runs inside the
 // products: dM and dv, dw during M3, the raw token rows and the dSigma.Sigma
@@ -124,15 +125,24 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
     __shared__ __align__(16) float s_gamma[D];            // e^{L_end} of the chunk
     __shared__ int s_slow;
     __shared__ float s_dmd[C];
+    __shared__ float s_dbw[C];  // scalar gates: per token, the sum of dw over the value channels
     __shared__ __align__(16) float s_rs[2][Chunk::NRS][D];  // by chunk parity: row sums of dSigma . Sigma (column quarters)
     __shared__ uint64_t mbar;
     __shared__ uint64_t mbar_ld[3];  // load groups A, B and the state image
+    __shared__ uint64_t mbar_fin;    // the issuing thread's last tensor-core work, at the end
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
     Chunk x(a, smem, nullptr, nullptr, s_dmd, s_rs[0]);
+    x.dMlo16 = x.U16;  // dM's low-order part goes to the U slot after M3 (E3)
+    x.s_dbw = s_dbw;
     const int tid = x.tid, warp = x.warp, lane = x.lane, bh = blockIdx.x;
     const ChunkTiles st = x.st;
+    if (!x.sv.ok) {  // packed-sequence offsets out of range: nothing of this sequence is touched
+        if (tid == 0) record_status(a.status, GDN2_ERR_INVALID_ARG);
+        return;
+    }
+    const bool packed = a.cu_seqlens != nullptr;
 
     if (warp == 0) tc::tmem_alloc(&tmem_slot, kTmemCols);
     if (tid == 0) {
@@ -140,6 +150,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         tc::mbar_init(&mbar_ld[0], 1);
         tc::mbar_init(&mbar_ld[1], 1);
         tc::mbar_init(&mbar_ld[2], 1);
+        tc::mbar_init(&mbar_fin, 1);
         tc::fence_mbar_init();
         abort_flag = 0;
     }
@@ -173,9 +184,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
     }
 
     uint32_t phase = 0;
+    const uint32_t wait_limit = a.wait_limit ? a.wait_limit : tc::kWaitLimit;
     // Wait for the MMAs committed last (all threads) ...
     auto mma_wait = [&]() {
-        if (!tc::mbar_wait(&mbar, phase)) {
+        if (!tc::mbar_wait(&mbar, phase, wait_limit)) {
             abort_flag = 1;
             record_status(a.status, GDN2_ERR_TIMEOUT);
         }
@@ -206,44 +218,74 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
     // token-level gradients are formed, group B and the state while chunk
     // n - 1's decay sums, E0 and first products run.
     uint32_t ph_ld[3] = {0, 0, 0};
+    int ld_issued[3] = {0, 0, 0}, ld_landed[3] = {0, 0, 0};  // (thread 0: its loads, for the drain at the end)
+    const bool scalar_la = a.gates == kGatesGDN;  // a scalar decay: its tile is filled after the loads
     auto issue_a = [&](int m) {
-        tc::mbar_expect_tx(&mbar_ld[0], 6 * TILE_BYTES);
+        tc::mbar_expect_tx(&mbar_ld[0], (scalar_la ? 5 : 6) * TILE_BYTES);
         const unsigned char *img = x.intra + (size_t)m * x.I_BYTES + TM_BYTES;
-        const unsigned char *op = static_cast<const unsigned char *>(a.ops) + ((size_t)bh * x.nchunks + m) * kOpsTileBytes;
+        const unsigned char *op = static_cast<const unsigned char *>(a.ops) + (x.sv.cslot + m) * kOpsTileBytes;
+        const int t = x.sv.map_t0 + m * C, mb = x.sv.map_b;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             const int cx = 64 * half, off = half * C * 64;
-            tc::tma_load_4d(st.k + off, &maps.la, cx, x.h, m * C, x.b, &mbar_ld[0]);
-            tc::tma_load_4d(x.dO16 + off, &maps.dO, cx, x.h, m * C, x.b, &mbar_ld[0]);
+            if (!scalar_la) tc::tma_load_4d(st.k + off, &maps.la, cx, x.h, t, mb, &mbar_ld[0]);
+            tc::tma_load_4d(x.dO16 + off, &maps.dO, cx, x.h, t, mb, &mbar_ld[0]);
         }
         tc::bulk_load(st.q, op, TILE_BYTES, &mbar_ld[0]);
         tc::bulk_load(st.b, op + TILE_BYTES, TILE_BYTES, &mbar_ld[0]);
         tc::bulk_load(st.la, op + 2 * TILE_BYTES, TILE_BYTES, &mbar_ld[0]);
         tc::bulk_load(x.U16, img, TILE_BYTES, &mbar_ld[0]);
+        ++ld_issued[0];
     };
     auto issue_b = [&](int m) {
         tc::mbar_expect_tx(&mbar_ld[1], TM_BYTES);
         tc::bulk_load(x.T16, x.intra + (size_t)m * x.I_BYTES, TM_BYTES, &mbar_ld[1]);
         tc::mbar_expect_tx(&mbar_ld[2], D * D * 2);
         tc::bulk_load(x.S16, x.states + (size_t)m * D * D, D * D * 2, &mbar_ld[2]);
+        ++ld_issued[1];
+        ++ld_issued[2];
     };
     auto wait_loads = [&](int g) {
-        if (!tc::mbar_wait(&mbar_ld[g], ph_ld[g])) {
+        if (!tc::mbar_wait(&mbar_ld[g], ph_ld[g], wait_limit)) {
             abort_flag = 1;
             record_status(a.status, GDN2_ERR_TIMEOUT);
+        } else {
+            ++ld_landed[g];
         }
         ph_ld[g] ^= 1;
     };
 
-    if (tid == 0) {
+    if (tid == 0 && x.nchunks > 0) {
         issue_a(x.nchunks - 1);
         issue_b(x.nchunks - 1);
     }
     for (int n = x.nchunks - 1; n >= 0; --n) {
-        const int Cn = min(C, a.T - n * C);
+        const int Cn = min(C, x.len - n * C);
         wait_loads(0);
         __syncthreads();
         if (abort_flag) break;
+        if (scalar_la) {
+            // the raw log_alpha tile from the scalar decay (zero past the sequence's end)
+            const unsigned short *lsc = static_cast<const unsigned short *>(a.log_alpha);
+            for (int id = tid; id < 2 * C * 8; id += NT) {
+                const int blk = id / (C * 8), r = (id % (C * 8)) / 8, ch = id % 8;
+                uint32_t v = r < Cn ? lsc[(x.row0 + (size_t)n * C + r) * a.H + x.h] : 0u;
+                v |= v << 16;
+                *reinterpret_cast<uint4 *>(st.k + blk * (C * 64) + r * 64 + ch * 8) = make_uint4(v, v, v, v);
+            }
+            __syncthreads();
+        }
+        if (packed && Cn < C) {
+            // the last chunk of a packed sequence: the log_alpha and dO boxes reach
+            // into the next sequence; its rows read as zero tokens
+            for (int id = tid; id < 2 * 2 * (C - Cn) * 8; id += NT) {
+                const int tl = id / (2 * (C - Cn) * 8), rem = id % (2 * (C - Cn) * 8);
+                const int blk = rem / ((C - Cn) * 8), r = Cn + (rem % ((C - Cn) * 8)) / 8, ch = rem % 8;
+                *reinterpret_cast<uint4 *>((tl ? x.dO16 : st.k) + blk * (C * 64) + r * 64 + ch * 8) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            __syncthreads();
+        }
         if (n > 0) x.prefetch_vw_l2(n - 1);
         // gam, the decay segment sums and (slow chunk) L from the raw log_alpha in the k slot
         const bool slow = decay_sums(st.k, s_seg, s_gamma, &s_slow, x.LAM, tid);
@@ -352,20 +394,27 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
         }
         x.dvdw<32>(n, Cn);
         mma_wait();
-        // ---- E3: dA = strict_lower(nR U^T) -> bf16 (warps with qc < 2)
-        if (qc < 2) {
+        // ---- E3: dA = strict_lower(nR U^T) -> bf16 (warps with qc < 2); the
+        // low-order part dM - bf16(dM) of dM (still in M1's columns) -> bf16 in
+        // the U slot, which M3 was the last to read (warps with qc >= 2).  dM's
+        // entries reach tens, and its bf16 rounding alone would move the
+        // largest dq and dk entries by a few hundredths; with the second term
+        // dM Kb and dM^T Qt carry about 16 significant bits.
+        {
             Frag<4> f;
-            ld_frag(tmem + lane_base + COL_A + 64 + 32 * qc, f);
+            const int j = 32 * (qc & 1);
+            ld_frag(tmem + lane_base + COL_A + (qc < 2 ? 64 : 0) + j, f);
             tc::wait_ld();
             const int r0 = 16 * p + (lane >> 2);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int r = r0 + (e >> 1) * 8, i = 32 * qc + 8 * nt + 2 * (lane & 3) + (e & 1);
-                    if (i >= r) f[0][nt][e] = 0.f;
+                    const int r = r0 + (e >> 1) * 8, i = j + 8 * nt + 2 * (lane & 3) + (e & 1);
+                    const float y = f[0][nt][e];
+                    f[0][nt][e] = i >= r ? 0.f : (qc < 2 ? y : y - __bfloat162float(__float2bfloat16_rn(y)));
                 }
-            store_frag_bf16<64, 4>(f, x.dA16, 16 * p, 32 * qc, lane, 1.f);
+            store_frag_bf16<64, 4>(f, qc < 2 ? x.dA16 : x.U16, 16 * p, j, lane, 1.f);
         }
         handoff();
         if (abort_flag) break;
@@ -375,9 +424,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
             mma_tiles<true, true>(tmem + COL_A, x.dO16, 64, x.S16, D, 8, ID64x128_K_K, false);
             if (!slow) {
                 mma_tiles<true, false>(tmem + COL_A, x.dM16, 64, st.la, 64, 4, ID64x128_K_MN, true);
+                mma_tiles<true, false>(tmem + COL_A, x.U16, 64, st.la, 64, 4, ID64x128_K_MN, true);  // dM lo
                 mma_tiles<true, false>(tmem + COL_B, x.dA16, 64, st.la, 64, 4, ID64x128_K_MN, true);
                 mma_tiles<false, false>(tmem + COL_C, x.dA16, 64, st.b, 64, 4, ID64x128_MN_MN, true);
                 mma_tiles<false, false>(tmem + COL_C, x.dM16, 64, st.q, 64, 4, ID64x128_MN_MN, true);
+                mma_tiles<false, false>(tmem + COL_C, x.U16, 64, st.q, 64, 4, ID64x128_MN_MN, true);  // dM lo
             }
             tc::commit(&mbar);
         }
@@ -439,6 +490,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
 #pragma unroll
         for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
+    // Before the tensor memory is freed: the issuing thread's tensor-core work
+    // has finished (a commit tracks all of it; immediate after a normal pass)
+    // and, after an aborted pass, every tile load issued has landed (bounded).
+    if (tid == 0) {
+        tc::commit(&mbar_fin);
+        (void)tc::mbar_wait(&mbar_fin, 0, wait_limit);
+        for (int g = 0; g < 3; ++g)
+            for (; ld_landed[g] < ld_issued[g]; ++ld_landed[g])
+                (void)tc::mbar_wait(&mbar_ld[g], (uint32_t)(ld_landed[g] & 1), wait_limit);
+    }
     tc::fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -451,8 +512,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
 
 cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs &a, cudaStream_t s) {
     cbwd_tc::BwdMaps m;
-    if (!token_tensor_map(&m.la, a.log_alpha, a.B, a.T, a.H, cbwd_tc::D) ||
-        !token_tensor_map(&m.dO, a.dO, a.B, a.T, a.H, cbwd_tc::D))
+    const int MB = a.cu_seqlens ? 1 : a.B;  // a packed batch is one [T, H, D] sequence of rows
+    if ((a.gates != kGatesGDN && !token_tensor_map(&m.la, a.log_alpha, MB, a.T, a.H, cbwd_tc::D)) ||
+        !token_tensor_map(&m.dO, a.dO, MB, a.T, a.H, cbwd_tc::D))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(cbwd_tc::chunk_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          cbwd_tc::BYTES);

@@ -161,29 +161,32 @@ __device__ __forceinline__ void store_tile_bf16(const float (&acc)[1][NT][4], bf
     }
 }
 
-// cp.async of rows [n*C, n*C + C) of a token tensor [B,T,H,D] (head h of
-// batch b) into a swizzled [C][D] tile; rows past T are zero-filled.
+// cp.async of tokens [n*C, n*C + C) of one sequence (head h; its tokens are
+// the rows row0 .. row0 + len - 1 of a token tensor [rows][H][D]) into a
+// swizzled [C][D] tile; tokens past len are zero-filled.
 template <int D, int NT = NTHR>
-__device__ __forceinline__ void load_token_tile(bf16 *dst, const bf16 *src, int b, int h, int n, int T, int H) {
+__device__ __forceinline__ void load_token_tile(bf16 *dst, const bf16 *src, size_t row0, int len, int h, int n,
+                                                int H) {
     constexpr int CPR = D / 8;  // 16-byte chunks per row
     for (int id = threadIdx.x; id < C * CPR; id += NT) {
         const int r = id / CPR, ch = id % CPR;
         const int t = n * C + r;
-        const bool ok = t < T;
-        const bf16 *g = src + (ok ? ((((size_t)b * T + t) * H + h) * D + ch * 8) : 0);
+        const bool ok = t < len;
+        const bf16 *g = src + (ok ? (((row0 + t) * H + h) * D + ch * 8) : 0);
         cp_async16(dst + swz<D>(r, ch * 8), g, ok);
     }
 }
 
-// L2 prefetch (no shared-memory destination) of rows [n*C, n*C + C) of a
-// token tensor [B,T,H,D], one bulk request per row; thread `slot` of `nslots`.
+// L2 prefetch (no shared-memory destination) of tokens [n*C, n*C + C) of one
+// sequence (rows row0 .. of a token tensor [rows][H][D]), one bulk request per
+// row; thread `slot` of `nslots`.
 template <int D>
-__device__ __forceinline__ void prefetch_token_rows_l2(const bf16 *src, int b, int h, int n, int T, int H, int slot,
-                                                       int nslots) {
+__device__ __forceinline__ void prefetch_token_rows_l2(const bf16 *src, size_t row0, int len, int h, int n, int H,
+                                                       int slot, int nslots) {
     for (int r = slot; r < C; r += nslots) {
         const int t = n * C + r;
-        if (t < T) {
-            const bf16 *g = src + (((size_t)b * T + t) * H + h) * D;
+        if (t < len) {
+            const bf16 *g = src + ((row0 + t) * H + h) * D;
             asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(g), "r"(D * 2) : "memory");
         }
     }

@@ -35,6 +35,7 @@
 // into the second stage buffer while chunk n is computed; the derived operands
 // of a chunk overwrite its own raw inputs in place.
 #include "chunk_common.cuh"
+#include "gdn2.h"
 #include "launch.h"
 
 namespace gdn2 {
@@ -69,13 +70,13 @@ __device__ __forceinline__ ChunkTiles stage_tiles(unsigned char *smem, int s) {
 }
 
 template <int DK, int DV>
-__device__ __forceinline__ void issue_chunk(const ChunkFwdArgs &a, ChunkTiles st, int b, int h, int n) {
-    load_token_tile<DK>(st.q, static_cast<const bf16 *>(a.q), b, h, n, a.T, a.H);
-    load_token_tile<DK>(st.k, static_cast<const bf16 *>(a.k), b, h, n, a.T, a.H);
-    load_token_tile<DK>(st.la, static_cast<const bf16 *>(a.log_alpha), b, h, n, a.T, a.H);
-    load_token_tile<DK>(st.b, static_cast<const bf16 *>(a.b), b, h, n, a.T, a.H);
-    load_token_tile<DV>(st.v, static_cast<const bf16 *>(a.v), b, h, n, a.T, a.H);
-    load_token_tile<DV>(st.w, static_cast<const bf16 *>(a.w), b, h, n, a.T, a.H);
+__device__ __forceinline__ void issue_chunk(const ChunkFwdArgs &a, ChunkTiles st, const SeqView &sv, int h, int n) {
+    load_token_tile<DK>(st.q, static_cast<const bf16 *>(a.q), sv.row0, sv.len, h, n, a.H);
+    load_token_tile<DK>(st.k, static_cast<const bf16 *>(a.k), sv.row0, sv.len, h, n, a.H);
+    load_token_tile<DK>(st.la, static_cast<const bf16 *>(a.log_alpha), sv.row0, sv.len, h, n, a.H);
+    load_token_tile<DK>(st.b, static_cast<const bf16 *>(a.b), sv.row0, sv.len, h, n, a.H);
+    load_token_tile<DV>(st.v, static_cast<const bf16 *>(a.v), sv.row0, sv.len, h, n, a.H);
+    load_token_tile<DV>(st.w, static_cast<const bf16 *>(a.w), sv.row0, sv.len, h, n, a.H);
     cp_commit();
 }
 
@@ -94,12 +95,17 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
-    const int nchunks = (a.T + C - 1) / C;
+    const SeqView sv = seq_view(a.cu_seqlens, b, h, a.B, a.T, a.H);
+    if (!sv.ok) {  // packed-sequence offsets out of range: nothing of this sequence is touched
+        if (tid == 0) record_status(a.status, GDN2_ERR_INVALID_ARG);
+        return;
+    }
+    const int nchunks = sv.nchunks;
     bf16 *S16 = reinterpret_cast<bf16 *>(smem + L::OS16);
     float *lam_ws = a.ws ? a.ws + (size_t)bh * a.ws_stride : nullptr;
     const bool with_o = a.o != nullptr;
     auto keep_tile = [&](int n) {
-        return static_cast<unsigned char *>(a.intra) + ((size_t)bh * nchunks + n) * intra_tile_bytes(DV);
+        return static_cast<unsigned char *>(a.intra) + (sv.cslot + n) * intra_tile_bytes(DV);
     };
 
     // ---- state tile of this warp, fp32 in registers
@@ -117,7 +123,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
             }
     // bf16 copy of the state into shared memory (and to a.states[n] when set)
     auto write_S16 = [&](int n) {
-        bf16 *gs = a.states ? static_cast<bf16 *>(a.states) + ((size_t)bh * (nchunks + 1) + n) * DK * DV : nullptr;
+        bf16 *gs = a.states ? static_cast<bf16 *>(a.states) + (sv.sslot + n) * DK * DV : nullptr;
 #pragma unroll
         for (int mt = 0; mt < MTS; ++mt)
 #pragma unroll
@@ -136,8 +142,9 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
     };
     write_S16(0);
 
-    issue_chunk<DK, DV>(a, stage_tiles<DK, DV>(smem, 0), b, h, 0);
-    if (nchunks > 1) issue_chunk<DK, DV>(a, stage_tiles<DK, DV>(smem, 1), b, h, 1);
+    if (nchunks > 0) issue_chunk<DK, DV>(a, stage_tiles<DK, DV>(smem, 0), sv, h, 0);
+    else cp_commit();
+    if (nchunks > 1) issue_chunk<DK, DV>(a, stage_tiles<DK, DV>(smem, 1), sv, h, 1);
     else cp_commit();
 
     for (int n = 0; n < nchunks; ++n) {
@@ -193,8 +200,8 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const int t = n * C + rl + 8 * half;
-                if (t < a.T) {
-                    bf16 *orow = o + (((size_t)b * a.T + t) * a.H + h) * DV;
+                if (t < sv.len) {
+                    bf16 *orow = o + ((sv.row0 + t) * a.H + h) * DV;
 #pragma unroll
                     for (int nt = 0; nt < NTV; ++nt)
                         *reinterpret_cast<uint32_t *>(orow + 8 * nt + 2 * (lane & 3)) =
@@ -227,7 +234,7 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
         }
         write_S16(n + 1);
         __syncthreads();
-        if (n + 2 < nchunks) issue_chunk<DK, DV>(a, st, b, h, n + 2);
+        if (n + 2 < nchunks) issue_chunk<DK, DV>(a, st, sv, h, n + 2);
         else cp_commit();
     }
     cp_wait<0>();

@@ -60,6 +60,11 @@ struct Small {
     uint64_t mbar_o;      // MMA completion, group B's O = Qt S (a second barrier: each keeps one phase in flight)
     uint64_t mbar_ld[2];  // tile loads of stage 0 and 1
     uint64_t ready[2];    // stage s: its intra-chunk stage is done
+    uint64_t mbar_fin[2]; // the issuing threads' last tensor-core work (groups A, B), at the end
+    uint64_t mbar_g;      // the fused epilogue's output-gate tile
+    int ld_issued[2];     // per stage: tile loads issued (thread tb = 0) ...
+    int ld_waited[2];     // ... and waited for (group A)
+    int g_issued, g_landed;  // output-gate tiles issued and landed (group B)
     uint32_t tmem;
     int abort;
 };
@@ -89,22 +94,70 @@ __device__ __forceinline__ ChunkTiles stage_tiles(unsigned char *smem, int s) {
 
 // TMA tensor maps of the six token tensors and of the output o.
 struct FwdMaps {
-    CUtensorMap q, k, la, b, v, w, o;
+    CUtensorMap q, k, la, b, v, w, o, g;  // g: the output gate of the fused epilogue
+    CUtensorMap qphi;                     // segments: the transition pass's rows Phi_t^T q_t
 };
 
 // Chunk n's six token tiles into a stage (one thread; 64 x 64 boxes, two per
-// tile), completion counted in bytes on the stage's mbarrier.
-__device__ __forceinline__ void issue_chunk(const FwdMaps &m, ChunkTiles st, int b, int h, int n, uint64_t *mbar) {
-    tc::mbar_expect_tx(mbar, 6 * TILE);
+// tile), completion counted in bytes on the stage's mbarrier.  Rows past the
+// end of the tensor read as zeros.
+// With scalar gates (KDA / GDN) the b and w tiles (and, for GDN, the
+// log_alpha tile) are not loaded: expand_gates fills them from the scalars.
+// A transition pass (no_vw) reads no v and w either.
+__device__ __forceinline__ void issue_chunk(const FwdMaps &m, ChunkTiles st, const SeqView &sv, int h, int n,
+                                            uint64_t *mbar, int gates, bool no_vw = false) {
+    const int ntiles = no_vw ? 4 : (gates == kGatesFull ? 6 : (gates == kGatesKDA ? 4 : 3));
+    tc::mbar_expect_tx(mbar, ntiles * TILE);
+    const int t = sv.map_t0 + n * C, b = sv.map_b;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         const int cx = 64 * half, off = half * C * 64;
-        tc::tma_load_4d(st.q + off, &m.q, cx, h, n * C, b, mbar);
-        tc::tma_load_4d(st.k + off, &m.k, cx, h, n * C, b, mbar);
-        tc::tma_load_4d(st.la + off, &m.la, cx, h, n * C, b, mbar);
-        tc::tma_load_4d(st.b + off, &m.b, cx, h, n * C, b, mbar);
-        tc::tma_load_4d(st.v + off, &m.v, cx, h, n * C, b, mbar);
-        tc::tma_load_4d(st.w + off, &m.w, cx, h, n * C, b, mbar);
+        tc::tma_load_4d(st.q + off, &m.q, cx, h, t, b, mbar);
+        tc::tma_load_4d(st.k + off, &m.k, cx, h, t, b, mbar);
+        if (!no_vw) tc::tma_load_4d(st.v + off, &m.v, cx, h, t, b, mbar);
+        if (gates != kGatesGDN) tc::tma_load_4d(st.la + off, &m.la, cx, h, t, b, mbar);
+        if (no_vw) {
+            tc::tma_load_4d(st.b + off, &m.b, cx, h, t, b, mbar);
+        } else if (gates == kGatesFull) {
+            tc::tma_load_4d(st.b + off, &m.b, cx, h, t, b, mbar);
+            tc::tma_load_4d(st.w + off, &m.w, cx, h, t, b, mbar);
+        }
+    }
+}
+
+// Scalar gates into whole tiles: row r of the b and w tiles (and, for GDN, of
+// the log_alpha tile) holds the scalar of token n*C + r in every column; rows
+// past the sequence's end hold zeros (a zero token).  The NTG threads of G.
+template <class G, int NTG>
+__device__ __forceinline__ void expand_gates(ChunkTiles st, const ChunkFwdArgs &a, const SeqView &sv, int h, int n) {
+    const int ntiles = a.gates == kGatesGDN ? 3 : 2;
+    const int valid = min(C, sv.len - n * C);
+    const unsigned short *beta = static_cast<const unsigned short *>(a.b);
+    const unsigned short *lsc = static_cast<const unsigned short *>(a.log_alpha);
+    for (int id = G::tid(); id < ntiles * 2 * C * 8; id += NTG) {
+        const int t = id / (2 * C * 8), rem = id % (2 * C * 8);
+        const int blk = rem / (C * 8), r = (rem % (C * 8)) / 8, ch = rem % 8;
+        uint32_t x = 0;
+        if (r < valid) {
+            const size_t o = (sv.row0 + (size_t)n * C + r) * a.H + h;
+            x = t < 2 ? beta[o] : lsc[o];
+        }
+        x |= x << 16;
+        bf16 *tile = t == 0 ? st.b : (t == 1 ? st.w : st.la);
+        *reinterpret_cast<uint4 *>(tile + blk * (C * 64) + r * 64 + ch * 8) = make_uint4(x, x, x, x);
+    }
+}
+
+// Rows Cn .. 63 of the six tiles of a stage to zero (the last chunk of a
+// packed sequence, whose box reaches into the next sequence): zero tokens
+// leave the state and the other rows unchanged.  The NT threads of G.
+template <class G, int NTG>
+__device__ __forceinline__ void zero_tail_rows(ChunkTiles st, int Cn) {
+    const int rows = C - Cn;  // (the six tiles lie back to back from st.q, TILE bytes each)
+    for (int id = G::tid(); id < 6 * 2 * rows * 8; id += NTG) {
+        const int t = id / (2 * rows * 8), rem = id % (2 * rows * 8);
+        const int blk = rem / (rows * 8), r = Cn + (rem % (rows * 8)) / 8, ch = rem % 8;
+        *reinterpret_cast<uint4 *>(st.q + t * (C * D) + blk * (C * 64) + r * 64 + ch * 8) = make_uint4(0u, 0u, 0u, 0u);
     }
 }
 
@@ -116,8 +169,47 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         if (tid == 0) record_status(a.status, GDN2_ERR_CUDA);
         return;
     }
-    const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
-    const int nchunks = (a.T + C - 1) / C;
+    int b, h;
+    SeqView sv;
+    bool phi = false;  // a segment's transition pass
+    const float *S0p;  // this CTA's start state (nullptr: zero; a transition pass starts from I)
+    float *STp;        // and its end state (or nullptr)
+    void *op = a.o;    // its output rows
+    if (a.seg_P == 0) {
+        const int bh = blockIdx.x;
+        b = bh / a.H;
+        h = bh % a.H;
+        sv = seq_view(a.cu_seqlens, b, h, a.B, a.T, a.H);
+        S0p = a.S0 ? a.S0 + (size_t)bh * D * D : nullptr;
+        STp = a.S_T ? a.S_T + (size_t)bh * D * D : nullptr;
+    } else {
+        const int P = a.seg_P, nloc = a.B * P * a.H;
+        int i = blockIdx.x, p;
+        phi = i >= nloc;
+        if (phi) i -= nloc;
+        h = i % a.H;
+        const int bp = i / a.H;
+        b = phi ? bp / (P - 1) : bp / P;
+        p = phi ? bp % (P - 1) + 1 : bp % P;
+        const int nch = a.T / C, base = nch / P, rem = nch % P;
+        const int c0 = p * base + min(p, rem), cn = base + (p < rem ? 1 : 0);
+        sv.row0 = (size_t)b * a.T + (size_t)c0 * C;
+        sv.len = cn * C;
+        sv.nchunks = cn;
+        sv.cslot = sv.sslot = 0;
+        sv.map_b = b;
+        sv.map_t0 = c0 * C;
+        sv.ok = true;
+        S0p = (!phi && p == 0 && a.S0) ? a.S0 + ((size_t)b * a.H + h) * D * D : nullptr;
+        STp = (phi ? a.seg_phi : a.seg_loc) + (size_t)i * D * D;
+        if (phi) op = a.seg_qphi;
+    }
+    if (!sv.ok) {  // packed-sequence offsets out of range: nothing of this sequence is touched
+        if (tid == 0) record_status(a.status, GDN2_ERR_INVALID_ARG);
+        return;
+    }
+    const int nchunks = sv.nchunks;
+    const bool packed = a.cu_seqlens != nullptr;
 
     if (warp == 0) tc::tmem_alloc(&sm.tmem, kTmemCols);
     if (tid == 0) {
@@ -127,7 +219,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&sm.mbar_ld[i], 1);
             tc::mbar_init(&sm.ready[i], 1);
+            tc::mbar_init(&sm.mbar_fin[i], 1);
+            sm.ld_issued[i] = 0;
+            sm.ld_waited[i] = 0;
         }
+        tc::mbar_init(&sm.mbar_g, 1);
+        sm.g_issued = 0;
+        sm.g_landed = 0;
         tc::fence_mbar_init();
         sm.abort = 0;
     }
@@ -141,20 +239,23 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
     const int p = warp & 3, hc = (warp >> 2) & 1;
     const uint32_t lane_base = (uint32_t)(32 * p) << 16;
     // Bounded wait on an mbarrier phase; a timeout is recorded and ends the pass.
+    const uint32_t wait_limit = a.wait_limit ? a.wait_limit : tc::kWaitLimit;
     auto wait_on = [&](uint64_t *mbar, uint32_t &phase) {
-        if (!tc::mbar_wait(mbar, phase)) {
+        const bool ok = tc::mbar_wait(mbar, phase, wait_limit);
+        if (!ok) {
             sm.abort = 1;
             record_status(a.status, GDN2_ERR_TIMEOUT);
         }
         phase ^= 1;
         tc::fence_after();
+        return ok;
     };
 
     if (warp < 8) {
         // ================= group A: decay prep, Grams, A and M =================
         // (a fast chunk's WY solve runs in group B; a slow chunk takes its Grams
         // term by term and its solve in the intra-chunk stage here)
-        float *lam_ws = a.ws ? a.ws + (size_t)bh * a.ws_stride : nullptr;
+        float *lam_ws = a.ws ? a.ws + (size_t)blockIdx.x * a.ws_stride : nullptr;
         uint32_t ph_a = 0, ph_ld[2] = {0, 0};
         for (int m = 0; m < nchunks; ++m) {
             const int s = m & 1;
@@ -163,9 +264,22 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             float *T32 = reinterpret_cast<float *>(st.w);
             bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
 
-            wait_on(&sm.mbar_ld[s], ph_ld[s]);
+            if (wait_on(&sm.mbar_ld[s], ph_ld[s]) && tid == 0) ++sm.ld_waited[s];  // (landed)
             GA::sync();
             if (sm.abort) break;
+            if (packed && sv.len - m * C < C) {
+                zero_tail_rows<GA, NG>(st, sv.len - m * C);
+                GA::sync();
+            }
+            if (a.gates != kGatesFull) {
+                expand_gates<GA, NG>(st, a, sv, h, m);
+                GA::sync();
+            }
+            if (phi) {  // a transition pass: no write term (w . v = 0)
+                for (int id = tid; id < 2 * C * D / 8; id += NG)
+                    reinterpret_cast<uint4 *>(id < C * D / 8 ? st.v : st.w)[id % (C * D / 8)] = make_uint4(0, 0, 0, 0);
+                GA::sync();
+            }
             const IntraView<D> iv{sm.part, sm.gamma[s], &sm.slow[s]};
             // a slow chunk takes its Grams term by term, its WY solve and w . v in
             // here; a fast chunk forms w . v below, while its Grams run
@@ -219,22 +333,30 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             tc::fence_async_smem();
             tc::fence_before();
             GA::sync();
-            if (tid == 0) tc::mbar_arrive(&sm.ready[s]);
+            if (tid == 0 && m != a.withhold_ready) tc::mbar_arrive(&sm.ready[s]);
         }
     } else {
         // ================= group B: the state chain =================
         const int tb = tid - NG;
-        const bool with_o = a.o != nullptr;
+        const bool with_o = op != nullptr;
+        const CUtensorMap *omap = phi ? &maps.qphi : &maps.o;
+        // the fused output epilogue: the gate tile lands in the S16 area (free
+        // from U's completion to the next chunk's solve), the RMS partials of
+        // the two column halves beside it
+        const bool gated = with_o && a.out_gate != nullptr;
+        bf16 *G16 = reinterpret_cast<bf16 *>(smem + OS16);
+        float *rms_part = reinterpret_cast<float *>(smem + OS16 + TILE);  // [2][64]
+        uint32_t ph_g = 0;
         bf16 *S16 = reinterpret_cast<bf16 *>(smem + OS16);
         const int c = 32 * p + lane;  // this thread's state row; columns 64 hc .. 64 hc + 63
         const uint32_t t_row = tmem + lane_base + COL_S + 64 * hc;
         auto keep_tile = [&](int n) {
-            return static_cast<unsigned char *>(a.intra) + ((size_t)bh * nchunks + n) * intra_tile_bytes(D);
+            return static_cast<unsigned char *>(a.intra) + (sv.cslot + n) * intra_tile_bytes(D);
         };
         // the chunk-boundary state n (when requested) as the image of S16 (thread tb = 0)
         auto keep_state = [&](int n) {
             if (a.states) {
-                tc::bulk_store(static_cast<bf16 *>(a.states) + ((size_t)bh * (nchunks + 1) + n) * D * D, S16,
+                tc::bulk_store(static_cast<bf16 *>(a.states) + (sv.sslot + n) * D * D, S16,
                                D * D * 2);
                 tc::bulk_commit();
             }
@@ -273,16 +395,20 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             float v[32];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float4 x = a.S0 ? reinterpret_cast<const float4 *>(a.S0 + (size_t)bh * D * D + (size_t)c * D +
-                                                                         64 * hc + 32 * i)[j]
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 x = S0p ? reinterpret_cast<const float4 *>(S0p + (size_t)c * D + 64 * hc + 32 * i)[j]
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
                 v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+                if (phi)  // the identity: row c, column 64 hc + 32 i + 4 j + e
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) v[4 * j + e] = (c == 64 * hc + 32 * i + 4 * j + e) ? 1.f : 0.f;
             }
             store_half(i, v);
         }
         if (tb == 0) {
-            issue_chunk(maps, stage_tiles(smem, 0), b, h, 0, &sm.mbar_ld[0]);
-            if (nchunks > 1) issue_chunk(maps, stage_tiles(smem, 1), b, h, 1, &sm.mbar_ld[1]);
+            for (int i = 0; i < 2 && i < nchunks; ++i) {
+                issue_chunk(maps, stage_tiles(smem, i), sv, h, i, &sm.mbar_ld[i], a.gates, phi);
+                ++sm.ld_issued[i];
+            }
         }
 
         // gam of the previous chunk for this thread's row, when that chunk's
@@ -297,6 +423,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             bf16 *M16 = T16 + C * C;
             bf16 *U16 = st.v;  // after T (w . v)
 
+            if (gated && tb == 0) {  // the chunk's output-gate rows into L2 while the chain runs
+                tc::tma_prefetch_4d(&maps.g, 0, h, sv.map_t0 + n * C, sv.map_b);
+                tc::tma_prefetch_4d(&maps.g, 64, h, sv.map_t0 + n * C, sv.map_b);
+            }
             wait_on(&sm.ready[s], ph_rdy[s]);
             GB::sync();
             if (sm.abort) break;
@@ -315,7 +445,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             // operands Qt, Gt, Kb (or Kt) go out for the backward
             if (tb == 0) {
                 if (a.ops) {
-                    unsigned char *op = static_cast<unsigned char *>(a.ops) + ((size_t)bh * nchunks + n) * kOpsTileBytes;
+                    unsigned char *op = static_cast<unsigned char *>(a.ops) + (sv.cslot + n) * kOpsTileBytes;
                     tc::bulk_store(op, st.q, TILE);
                     tc::bulk_store(op + TILE, st.b, TILE);
                     tc::bulk_store(op + 2 * TILE, st.la, TILE);
@@ -374,6 +504,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 tc::bulk_store(keep_tile(n) + 2 * C * C * 2, U16, C * D * 2);
                 tc::bulk_commit();
             }
+            if (gated && tb == 0) {  // every product that reads S16 is complete
+                tc::mbar_expect_tx(&sm.mbar_g, TILE);
+                tc::tma_load_4d(G16, &maps.g, 0, h, sv.map_t0 + n * C, sv.map_b, &sm.mbar_g);
+                tc::tma_load_4d(G16 + C * 64, &maps.g, 64, h, sv.map_t0 + n * C, sv.map_b, &sm.mbar_g);
+                ++sm.g_issued;
+            }
             // ---- slow chunk: S <- Diag(gam) S before adding Kt^T U
             if (slow) {
                 for (int i = 0; i < 2; ++i) {
@@ -401,23 +537,75 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 Frag<8> f;
                 ld_frag(tmem + lane_base + COL_O + 64 * hc, f);
                 tc::wait_ld();
+                if (gated) {  // z = O / rms(O) * gamma * silu(g), row by row over both column halves
+                    const int r0 = 16 * p + (lane >> 2);
+                    float ss[2] = {0.f, 0.f};
+#pragma unroll
+                    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) ss[e >> 1] = fmaf(f[0][nt][e], f[0][nt][e], ss[e >> 1]);
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], 1);
+                        ss[i] += __shfl_xor_sync(0xffffffffu, ss[i], 2);
+                    }
+                    if ((lane & 3) == 0) {
+                        rms_part[hc * C + r0] = ss[0];
+                        rms_part[hc * C + r0 + 8] = ss[1];
+                    }
+                    if (wait_on(&sm.mbar_g, ph_g) && tb == 0) ++sm.g_landed;
+                    GB::sync();
+                    float rs[2];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+                        rs[i] = rsqrtf((rms_part[r0 + 8 * i] + rms_part[C + r0 + 8 * i]) * (1.f / D) + 1e-6f);
+#pragma unroll
+                    for (int nt = 0; nt < 8; ++nt) {
+                        const int col = 64 * hc + 8 * nt + 2 * (lane & 3);
+                        const float2 gmw = *reinterpret_cast<const float2 *>(a.gamma + col);
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const float2 gg = unpack_bf16(*reinterpret_cast<const uint32_t *>(G16 + swz<D>(r0 + 8 * i, col)));
+                            f[0][nt][2 * i] *= rs[i] * gmw.x * gg.x / (1.f + __expf(-gg.x));
+                            f[0][nt][2 * i + 1] *= rs[i] * gmw.y * gg.y / (1.f + __expf(-gg.y));
+                        }
+                    }
+                }
                 store_frag_bf16<D, 8>(f, st.k, 16 * p, 64 * hc, lane, 1.f);
                 tc::fence_async_smem();
             }
             wait_on(&sm.mbar_b, ph_b);  // S (and with it every read of the stage's tiles)
             tc::fence_before();
             GB::sync();
+            // the last chunk of a packed sequence: its rows of o by the threads
+            // (a box would reach into the next sequence's rows)
+            const int Cn = min(C, sv.len - n * C);
+            const bool o_rows = with_o && packed && Cn < C;
+            if (o_rows) {
+                bf16 *o = static_cast<bf16 *>(op);
+                for (int id = tb; id < Cn * 16; id += NG) {
+                    const int r = id >> 4, j = id & 15;
+                    const uint4 val = *reinterpret_cast<const uint4 *>(st.k + (j >> 3) * (C * 64) + r * 64 +
+                                                                       (((j & 7) ^ (r & 7)) << 3));
+                    *reinterpret_cast<uint4 *>(o + ((sv.row0 + n * C + r) * a.H + h) * D + 8 * j) = val;
+                }
+                tc::fence_async_smem();
+                GB::sync();
+            }
             if (tb == 0) {
-                if (with_o) {  // (tokens past T are clipped)
-                    tc::tma_store_4d(&maps.o, st.k, 0, h, n * C, b);
-                    tc::tma_store_4d(&maps.o, st.k + C * 64, 64, h, n * C, b);
+                if (with_o && !o_rows) {  // (tokens past the tensor's end are clipped)
+                    tc::tma_store_4d(omap, st.k, 0, h, sv.map_t0 + n * C, sv.map_b);
+                    tc::tma_store_4d(omap, st.k + C * 64, 64, h, sv.map_t0 + n * C, sv.map_b);
                     tc::bulk_commit();
                 }
                 // the stage's T, M, U and O images and the state image are out
                 // before the stage is refilled (and before S16 is rewritten, which
                 // follows this thread's next MMA issue)
                 tc::bulk_wait_read();
-                if (n + 2 < nchunks) issue_chunk(maps, st, b, h, n + 2, &sm.mbar_ld[s]);
+                if (n + 2 < nchunks) {
+                    issue_chunk(maps, st, sv, h, n + 2, &sm.mbar_ld[s], a.gates, phi);
+                    ++sm.ld_issued[s];
+                }
             }
         }
         GB::sync();
@@ -428,8 +616,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 load_half(i, v);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] *= gm_owed;
-                if (a.S_T) {
-                    float4 *dst = reinterpret_cast<float4 *>(a.S_T + (size_t)bh * D * D + (size_t)c * D + 64 * hc +
+                if (STp) {
+                    float4 *dst = reinterpret_cast<float4 *>(STp + (size_t)c * D + 64 * hc +
                                                              32 * i);
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
@@ -445,7 +633,23 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         }
         if (tb == 0) tc::bulk_wait();
     }
+    // Before the tensor memory is freed: each issuing thread's tensor-core work
+    // has finished (a commit tracks all of it; immediate after a normal pass)
+    // and, after an aborted pass, every tile load issued has landed (bounded).
+    if (tid == 0 || tid == NG) {
+        uint64_t *fin = &sm.mbar_fin[tid == 0 ? 0 : 1];
+        tc::commit(fin);
+        (void)tc::mbar_wait(fin, 0, wait_limit);
+    }
     tc::fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i)
+            for (; sm.ld_waited[i] < sm.ld_issued[i]; ++sm.ld_waited[i])
+                (void)tc::mbar_wait(&sm.mbar_ld[i], (uint32_t)(sm.ld_waited[i] & 1), wait_limit);
+        for (; sm.g_landed < sm.g_issued; ++sm.g_landed)
+            (void)tc::mbar_wait(&sm.mbar_g, (uint32_t)(sm.g_landed & 1), wait_limit);
+    }
     __syncthreads();
     if (warp == 0) {
         tc::fence_after();
@@ -458,15 +662,25 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
 cudaError_t launch_chunk_fwd_tc(const ChunkFwdArgs &a, cudaStream_t s) {
     cfwd_tc::FwdMaps m{};
     const int D = cfwd_tc::D;
-    if (!token_tensor_map(&m.q, a.q, a.B, a.T, a.H, D) || !token_tensor_map(&m.k, a.k, a.B, a.T, a.H, D) ||
-        !token_tensor_map(&m.la, a.log_alpha, a.B, a.T, a.H, D) || !token_tensor_map(&m.b, a.b, a.B, a.T, a.H, D) ||
-        !token_tensor_map(&m.v, a.v, a.B, a.T, a.H, D) || !token_tensor_map(&m.w, a.w, a.B, a.T, a.H, D) ||
-        (a.o && !token_tensor_map(&m.o, a.o, a.B, a.T, a.H, D)))
+    const int MB = a.cu_seqlens ? 1 : a.B;  // a packed batch is one [T, H, D] sequence of rows
+    const bool vec_la = a.gates != kGatesGDN, vec_bw = a.gates == kGatesFull;  // (scalar gates: no maps)
+    if (!token_tensor_map(&m.q, a.q, MB, a.T, a.H, D) || !token_tensor_map(&m.k, a.k, MB, a.T, a.H, D) ||
+        (vec_la && !token_tensor_map(&m.la, a.log_alpha, MB, a.T, a.H, D)) ||
+        (vec_bw && !token_tensor_map(&m.b, a.b, MB, a.T, a.H, D)) || !token_tensor_map(&m.v, a.v, MB, a.T, a.H, D) ||
+        (vec_bw && !token_tensor_map(&m.w, a.w, MB, a.T, a.H, D)) ||
+        (a.o && !token_tensor_map(&m.o, a.o, MB, a.T, a.H, D)) ||
+        (a.out_gate && !token_tensor_map(&m.g, a.out_gate, MB, a.T, a.H, D)) ||
+        (a.seg_P && !token_tensor_map(&m.qphi, a.seg_qphi, a.B, a.T, a.H, D)))
         return cudaErrorInvalidValue;
+    if (a.seg_P && (a.seg_P < 2 || a.T % cfwd_tc::C || a.T / cfwd_tc::C < a.seg_P || a.cu_seqlens || a.states ||
+                    a.gates != kGatesFull || !a.seg_loc || !a.seg_phi || !a.seg_qphi))
+        return cudaErrorInvalidValue;
+    if (a.out_gate && (a.states || !a.o || !a.gamma)) return cudaErrorInvalidValue;  // (inference path only)
     cudaError_t e = cudaFuncSetAttribute(cfwd_tc::chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          cfwd_tc::BYTES);
     if (e != cudaSuccess) return e;
-    cfwd_tc::chunk_fwd_tc_kernel<<<(unsigned)(a.B * a.H), cfwd_tc::NT, cfwd_tc::BYTES, s>>>(a, m);
+    const unsigned ctas = (unsigned)(a.B * a.H) * (a.seg_P ? 2u * a.seg_P - 1u : 1u);
+    cfwd_tc::chunk_fwd_tc_kernel<<<ctas, cfwd_tc::NT, cfwd_tc::BYTES, s>>>(a, m);
     return cudaGetLastError();
 }
 

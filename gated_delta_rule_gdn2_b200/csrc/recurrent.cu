@@ -46,25 +46,30 @@ __device__ __forceinline__ float row_sum(float x) {
     return x;
 }
 
-__device__ __forceinline__ size_t tok_off(int b, int t, int T, int H, int h, int D) {
-    return (((size_t)b * T + t) * H + h) * (size_t)D;
+// Element offset of token t of a sequence whose tokens are the rows row0 .. of
+// a token tensor [rows][H][D] (head h).
+__device__ __forceinline__ size_t tok_off(size_t row0, int t, int H, int h, int D) {
+    return ((row0 + t) * H + h) * (size_t)D;
 }
 
 // Loads one token's gates into shared memory.  Key side: alpha, (b.k).alpha,
 // q.alpha, k, b.k; value side: w.v, v, w.  Returns q.k in *qk (valid after the
 // caller's next __syncthreads through s_qkp).
 template <typename Tin, int DK, int DV>
-__device__ __forceinline__ void load_token(const RecurrentArgs &a, int b, int t, int h,
+__device__ __forceinline__ void load_token(const RecurrentArgs &a, size_t row0, int t, int h,
                                            float *s_a, float *s_ga, float *s_qa, float *s_k,
                                            float *s_g, float *s_wv, float *s_v, float *s_w,
                                            float *s_qkp) {
     const int tid = threadIdx.x;
+    // a scalar gate (KDA: beta for b and w; GDN: also the decay) is one
+    // element per token and head
+    const size_t os = (row0 + t) * a.H + h;
     if (tid < DK) {
-        const size_t o = tok_off(b, t, a.T, a.H, h, DK);
+        const size_t o = tok_off(row0, t, a.H, h, DK);
         const float q = to_f32(static_cast<const Tin *>(a.q)[o + tid]);
         const float k = to_f32(static_cast<const Tin *>(a.k)[o + tid]);
-        const float la = to_f32(static_cast<const Tin *>(a.log_alpha)[o + tid]);
-        const float bg = to_f32(static_cast<const Tin *>(a.b)[o + tid]);
+        const float la = to_f32(static_cast<const Tin *>(a.log_alpha)[a.gates == kGatesGDN ? os : o + tid]);
+        const float bg = to_f32(static_cast<const Tin *>(a.b)[a.gates == kGatesFull ? o + tid : os]);
         const float al = expf(la);
         const float g = bg * k;
         s_a[tid] = al;
@@ -76,9 +81,9 @@ __device__ __forceinline__ void load_token(const RecurrentArgs &a, int b, int t,
         if ((tid & 31) == 0) s_qkp[tid >> 5] = qk;
     } else if (tid < DK + DV) {
         const int j = tid - DK;
-        const size_t o = tok_off(b, t, a.T, a.H, h, DV);
+        const size_t o = tok_off(row0, t, a.H, h, DV);
         const float v = to_f32(static_cast<const Tin *>(a.v)[o + j]);
-        const float w = to_f32(static_cast<const Tin *>(a.w)[o + j]);
+        const float w = to_f32(static_cast<const Tin *>(a.w)[a.gates == kGatesFull ? o + j : os]);
         s_wv[j] = w * v;
         if (s_v) s_v[j] = v;
         if (s_w) s_w[j] = w;
@@ -91,6 +96,8 @@ __global__ void __launch_bounds__(kThreads) recurrent_fwd_kernel(RecurrentArgs a
     const int bh = blockIdx.x;
     const int b = bh / a.H, h = bh % a.H;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, cg = L::cg(lane);
+    const SeqView sv = seq_view(a.cu_seqlens, b, h, a.B, a.T, a.H);
+    if (!sv.ok) return;  // packed-sequence offsets out of range
 
     __shared__ float s_a[DK], s_ga[DK], s_qa[DK], s_k[DK], s_wv[DV], s_u[DV];
     __shared__ float s_red[2][kWarps][DV];
@@ -105,8 +112,8 @@ __global__ void __launch_bounds__(kThreads) recurrent_fwd_kernel(RecurrentArgs a
                       : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
-    for (int t = 0; t < a.T; ++t) {
-        load_token<Tin, DK, DV>(a, b, t, h, s_a, s_ga, s_qa, s_k, nullptr, s_wv, nullptr, nullptr, s_qkp);
+    for (int t = 0; t < sv.len; ++t) {
+        load_token<Tin, DK, DV>(a, sv.row0, t, h, s_a, s_ga, s_qa, s_k, nullptr, s_wv, nullptr, nullptr, s_qkp);
         __syncthreads();
         float4 p = make_float4(0.f, 0.f, 0.f, 0.f), r = p;
 #pragma unroll
@@ -136,7 +143,7 @@ __global__ void __launch_bounds__(kThreads) recurrent_fwd_kernel(RecurrentArgs a
             for (int w = 0; w < DK / 32; ++w) qk += s_qkp[w];
             const float u = s_wv[j] - pj;
             s_u[j] = u;
-            static_cast<Tin *>(a.o)[tok_off(b, t, a.T, a.H, h, DV) + j] = from_f32<Tin>(rj + qk * u);
+            static_cast<Tin *>(a.o)[tok_off(sv.row0, t, a.H, h, DV) + j] = from_f32<Tin>(rj + qk * u);
         }
         __syncthreads();
         const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[4 * cg]);
@@ -161,14 +168,17 @@ __global__ void __launch_bounds__(kThreads) recurrent_fwd_kernel(RecurrentArgs a
 // ---------------------------------------------------------------------------
 // Reverse-time backward (fp32 precision mode).
 //
-// Workspace per (b,h): NSEG checkpoints [DK x DV], then one 64-token segment
-// of decayed states S'_t [64][DK x DV] and edits u_t [64][DV].
+// Workspace: the checkpoints [DK x DV] at every 64-token segment start, one
+// slot per segment as the chunk path lays out its per-chunk tiles (SeqView),
+// then per (b,h) one 64-token segment of decayed states S'_t [64][DK x DV]
+// and edits u_t [64][DV].
 
 constexpr int kSeg = 64;
+static_assert(kSeg == 64, "checkpoint slots follow the 64-token chunk slots");
 
 template <int DK, int DV>
-__host__ __device__ constexpr size_t bwd_ws_floats_per_head(int T) {
-    return (size_t)((T + kSeg - 1) / kSeg) * DK * DV + (size_t)kSeg * DK * DV + (size_t)kSeg * DV;
+__host__ __device__ constexpr size_t bwd_seg_floats() {
+    return (size_t)kSeg * DK * DV + (size_t)kSeg * DV;
 }
 
 template <typename Tin, int DK, int DV>
@@ -177,7 +187,9 @@ __global__ void __launch_bounds__(kThreads) recurrent_bwd_kernel(RecurrentBwdArg
     const int bh = blockIdx.x;
     const int b = bh / a.H, h = bh % a.H;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, cg = L::cg(lane);
-    const int T = a.T, nseg = (T + kSeg - 1) / kSeg;
+    const SeqView sv = seq_view(a.cu_seqlens, b, h, a.B, a.T, a.H);
+    if (!sv.ok) return;  // packed-sequence offsets out of range
+    const int T = sv.len, nseg = sv.nchunks;
 
     __shared__ float s_a[DK], s_ga[DK], s_qa[DK], s_k[DK], s_g[DK], s_q[DK], s_b[DK];
     __shared__ float s_wv[DV], s_v[DV], s_w[DV], s_u[DV], s_do[DV], s_du[DV];
@@ -185,12 +197,12 @@ __global__ void __launch_bounds__(kThreads) recurrent_bwd_kernel(RecurrentBwdArg
     __shared__ float s_qkp[kWarps];
     __shared__ float s_udo;
 
-    float *ws = a.ws + (size_t)bh * bwd_ws_floats_per_head<DK, DV>(T);
-    float *ckpt = ws;
-    float *segSp = ws + (size_t)nseg * DK * DV;
+    const size_t nslots = chunk_slots(a.B, a.T, a.H, a.cu_seqlens != nullptr);
+    float *ckpt = a.ws + sv.cslot * DK * DV;
+    float *segSp = a.ws + nslots * DK * DV + (size_t)bh * bwd_seg_floats<DK, DV>();
     float *segU = segSp + (size_t)kSeg * DK * DV;
     const size_t sbase = (size_t)bh * DK * DV;
-    RecurrentArgs fa{a.q, a.k, a.v, a.log_alpha, a.b, a.w, nullptr, nullptr, nullptr, a.B, a.T, a.H};
+    RecurrentArgs fa{a.q, a.k, a.v, a.log_alpha, a.b, a.w, nullptr, nullptr, nullptr, a.B, a.T, a.H, a.cu_seqlens};
 
     // 1. forward pass, checkpoint at every segment start
     float4 S[L::RT];
@@ -208,7 +220,7 @@ __global__ void __launch_bounds__(kThreads) recurrent_bwd_kernel(RecurrentBwdArg
                 reinterpret_cast<float4 *>(ckpt + (size_t)(t / kSeg) * DK * DV + (size_t)row * DV)[cg] = S[i];
             }
         }
-        load_token<Tin, DK, DV>(fa, b, t, h, s_a, s_ga, s_qa, s_k, nullptr, s_wv, nullptr, nullptr, s_qkp);
+        load_token<Tin, DK, DV>(fa, sv.row0, t, h, s_a, s_ga, s_qa, s_k, nullptr, s_wv, nullptr, nullptr, s_qkp);
         __syncthreads();
         float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -257,7 +269,7 @@ __global__ void __launch_bounds__(kThreads) recurrent_bwd_kernel(RecurrentBwdArg
             S[i] = reinterpret_cast<const float4 *>(ckpt + (size_t)seg * DK * DV + (size_t)row * DV)[cg];
         }
         for (int t = t0; t < t1; ++t) {
-            load_token<Tin, DK, DV>(fa, b, t, h, s_a, s_ga, s_qa, s_k, nullptr, s_wv, nullptr, nullptr, s_qkp);
+            load_token<Tin, DK, DV>(fa, sv.row0, t, h, s_a, s_ga, s_qa, s_k, nullptr, s_wv, nullptr, nullptr, s_qkp);
             __syncthreads();
             float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
             float *Sp = segSp + (size_t)(t - t0) * DK * DV;
@@ -296,7 +308,7 @@ __global__ void __launch_bounds__(kThreads) recurrent_bwd_kernel(RecurrentBwdArg
         for (int t = t1 - 1; t >= t0; --t) {
             const int tid = threadIdx.x;
             if (tid < DK) {
-                const size_t o = tok_off(b, t, T, a.H, h, DK);
+                const size_t o = tok_off(sv.row0, t, a.H, h, DK);
                 const float q = to_f32(static_cast<const Tin *>(a.q)[o + tid]);
                 const float k = to_f32(static_cast<const Tin *>(a.k)[o + tid]);
                 const float la = to_f32(static_cast<const Tin *>(a.log_alpha)[o + tid]);
@@ -304,7 +316,7 @@ __global__ void __launch_bounds__(kThreads) recurrent_bwd_kernel(RecurrentBwdArg
                 s_q[tid] = q; s_k[tid] = k; s_b[tid] = bg; s_g[tid] = bg * k; s_a[tid] = expf(la);
             } else if (tid < DK + DV) {
                 const int j = tid - DK;
-                const size_t o = tok_off(b, t, T, a.H, h, DV);
+                const size_t o = tok_off(sv.row0, t, a.H, h, DV);
                 s_v[j] = to_f32(static_cast<const Tin *>(a.v)[o + j]);
                 s_w[j] = to_f32(static_cast<const Tin *>(a.w)[o + j]);
                 s_do[j] = to_f32(static_cast<const Tin *>(a.dO)[o + j]);
@@ -347,14 +359,14 @@ __global__ void __launch_bounds__(kThreads) recurrent_bwd_kernel(RecurrentBwdArg
                 float x = 0.f;
                 for (int w = 0; w < kWarps; ++w) x += s_red[w][tid];
                 s_du[tid] = x;
-                const size_t o = tok_off(b, t, T, a.H, h, DV);
+                const size_t o = tok_off(sv.row0, t, a.H, h, DV);
                 static_cast<Tin *>(a.dw)[o + tid] = from_f32<Tin>(x * s_v[tid]);
                 static_cast<Tin *>(a.dv)[o + tid] = from_f32<Tin>(x * s_w[tid]);
             }
             __syncthreads();
             const float4 du4 = *reinterpret_cast<const float4 *>(&s_du[4 * cg]);
             const float udo = s_udo;
-            const size_t ok = tok_off(b, t, T, a.H, h, DK);
+            const size_t ok = tok_off(sv.row0, t, a.H, h, DK);
 #pragma unroll
             for (int i = 0; i < L::RT; ++i) {
                 const int row = L::row(i, warp, lane);
@@ -427,9 +439,8 @@ cudaError_t launch_recurrent_bwd(const RecurrentBwdArgs &a, int dk, int dv, bool
     return bf16 ? dispatch_bwd<__nv_bfloat16>(a, dk, dv, s) : dispatch_bwd<float>(a, dk, dv, s);
 }
 
-size_t recurrent_bwd_ws_bytes(int B, int T, int H, int dk, int dv) {
-    const size_t nseg = (size_t)((T + kSeg - 1) / kSeg);
-    return (size_t)B * H * 4 * (nseg * dk * dv + (size_t)kSeg * dk * dv + (size_t)kSeg * dv);
+size_t recurrent_bwd_ws_bytes(int B, int T, int H, int dk, int dv, bool varlen) {
+    return 4 * (chunk_slots(B, T, H, varlen) * dk * dv + (size_t)B * H * ((size_t)kSeg * dk * dv + (size_t)kSeg * dv));
 }
 
 }  // namespace gdn2

@@ -30,7 +30,7 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 // MN-major = 64-element x 8-row atoms, `lbo` bytes between 64-element groups
 // along M/N and `sbo` bytes between 8-row groups along K).  Start addresses
 // are in bytes; the atoms must sit on 1 KB boundaries.
-__device__ __forceinline__ uint64_t sdesc(uint32_t start, uint32_t lbo, uint32_t sbo) {
+__host__ __device__ __forceinline__ uint64_t sdesc(uint32_t start, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;
     d |= (uint64_t)((start >> 4) & 0x3FFFu);
     d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
@@ -76,8 +76,11 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *mbar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(mbar)) : "memory");
 }
 
+// Iterations of a bounded wait before it gives up (a few seconds at most).
+constexpr uint32_t kWaitLimit = 1u << 22;
+
 // Bounded wait for the phase `parity` of `mbar`; false when it ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint32_t max_iter = 1u << 22) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint32_t max_iter = kWaitLimit) {
     const uint32_t a = smem_addr(mbar);
     for (uint32_t i = 0; i < max_iter; ++i) {
         uint32_t done;
@@ -105,6 +108,12 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *map, int x, i
         "%5}], [%6];\n" ::"r"(smem_addr(dst)),
         "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(mbar))
         : "memory");
+}
+// L2 prefetch of a tiled box of a 4-D tensor map (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_4d(const void *map, int x, int y, int z, int w) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];\n" ::"l"(map), "r"(x),
+                 "r"(y), "r"(z), "r"(w)
+                 : "memory");
 }
 // Contiguous copy (addresses 16-byte aligned, bytes a multiple of 16).
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *mbar) {

@@ -13,20 +13,28 @@ namespace tct {
 
 using namespace chunk;
 
-// k-step s (16 elements) of a K-major operand in an [R][.] tile (rows = M or N,
-// columns = K) ...
-__device__ __forceinline__ uint64_t kmaj(const void *tile, int R, int s) {
-    return tc::sdesc(tc::smem_addr(tile) + (uint32_t)((s >> 2) * (R * 128) + (s & 3) * 32), 16, 1024);
-}
-// ... and of an MN-major operand (rows = K, columns = M or N).
-__device__ __forceinline__ uint64_t mnmaj(const void *tile, int R, int s) {
-    return tc::sdesc(tc::smem_addr(tile) + (uint32_t)(s * 2048), (uint32_t)(R * 128), 1024);
-}
-
-// Byte offset of k-step s from k-step 0 of an operand in an [R][.] tile.
+// Byte offset of k-step s (16 elements) from k-step 0 of an operand in an
+// [R][.] tile: K-major (rows = M or N, columns = K; four k-steps per 128-byte
+// swizzle row, then the next 64-column block R * 128 bytes on) or MN-major
+// (rows = K: 16 rows of 128 bytes per k-step).
 template <bool K_MAJOR>
-__device__ __forceinline__ uint32_t kstep_bytes(int R, int s) {
+__host__ __device__ __forceinline__ uint32_t kstep_bytes(int R, int s) {
     return K_MAJOR ? (uint32_t)((s >> 2) * (R * 128) + (s & 3) * 32) : (uint32_t)(s * 2048);
+}
+// Descriptor of k-step s of such an operand whose tile starts at shared
+// address `start`: K-major atoms of 8 rows x 128 bytes stacked every 1024
+// bytes along M/N; MN-major atoms of 64 elements x 8 rows, the next 64
+// elements R * 128 bytes on, the next 8 K rows 1024 bytes on.
+template <bool K_MAJOR>
+__host__ __device__ __forceinline__ uint64_t operand_desc(uint32_t start, int R, int s) {
+    return K_MAJOR ? tc::sdesc(start + kstep_bytes<true>(R, s), 16, 1024)
+                   : tc::sdesc(start + kstep_bytes<false>(R, s), (uint32_t)(R * 128), 1024);
+}
+__device__ __forceinline__ uint64_t kmaj(const void *tile, int R, int s) {
+    return operand_desc<true>(tc::smem_addr(tile), R, s);
+}
+__device__ __forceinline__ uint64_t mnmaj(const void *tile, int R, int s) {
+    return operand_desc<false>(tc::smem_addr(tile), R, s);
 }
 
 // D (+)= A B over K = 16 ks, issued by one thread.  A_K / B_K: K-major operand.

@@ -63,6 +63,13 @@ WORKLOADS = {
 def round_bf16(x: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even), kept as float32."""
     x = np.ascontiguousarray(x, dtype=np.float32)
+    if x.ndim > 0 and x.size > (1 << 22):
+        return _blockwise(_round_bf16, x)
+    return _round_bf16(x)
+
+
+def _round_bf16(x):
+    x = np.ascontiguousarray(x, dtype=np.float32)
     u = x.view(np.uint32).astype(np.uint64)
     nan = np.isnan(x)
     lsb = (u >> 16) & 1
@@ -74,17 +81,34 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
     return out
 
 
+def _blockwise(f, x, rows=1 << 14):
+    """f applied to blocks of rows of x (last axis kept whole): the same
+    values as f(x), with temporaries that stay in cache on long inputs."""
+    x = np.ascontiguousarray(x)
+    if x.ndim == 0 or x.size <= rows * x.shape[-1]:
+        return f(x)
+    flat = x.reshape(-1, x.shape[-1])
+    out = np.empty(flat.shape, dtype=np.float32)
+    for i in range(0, flat.shape[0], rows):
+        out[i:i + rows] = f(flat[i:i + rows])
+    return out.reshape(x.shape)
+
+
 def _sigmoid(x):
-    return (1.0 / (1.0 + np.exp(-x.astype(np.float64)))).astype(np.float32)
+    return _blockwise(lambda y: (1.0 / (1.0 + np.exp(-y.astype(np.float64)))).astype(np.float32), x)
 
 
 def _log_sigmoid(x):
-    return (-np.logaddexp(0.0, -x.astype(np.float64))).astype(np.float32)
+    return _blockwise(lambda y: (-np.logaddexp(0.0, -y.astype(np.float64))).astype(np.float32), x)
+
+
+def _unit_rows(x):
+    n = np.sqrt(np.sum(x.astype(np.float64) ** 2, axis=-1, keepdims=True))
+    return (x / np.maximum(n, 1e-30)).astype(np.float32)
 
 
 def _unit(x):
-    n = np.sqrt(np.sum(x.astype(np.float64) ** 2, axis=-1, keepdims=True))
-    return (x / np.maximum(n, 1e-30)).astype(np.float32)
+    return _blockwise(_unit_rows, x)
 
 
 def draw_tokens(rng: np.random.Generator, lead: tuple, dk: int, dv: int, alpha_mu: float,
@@ -135,3 +159,29 @@ def decode_initial_state(B: int, H: int, dk: int, dv: int, *, seed: int,
                          s0_std: float = 0.02) -> np.ndarray:
     rng = np.random.Generator(np.random.PCG64([seed, 1 << 30]))
     return np.float32(s0_std) * rng.standard_normal((B, H, dk, dv), dtype=np.float32)
+
+
+def make_inputs_device(B: int, T: int, H: int, dk: int, dv: int, *, seed: int, device,
+                       alpha_mu: float = 3.0, s0_std: float = 0.02):
+    """The same distributions as make_inputs, drawn on the GPU with torch's
+    seeded generator (for benchmark inputs of hundreds of millions of values,
+    which the host generator takes minutes to draw).  Token tensors bf16
+    [B,T,H,D], S0 fp32 [B,H,dk,dv].  Not the values make_inputs gives: the
+    parity tests use make_inputs."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    lead = (B, T, H)
+
+    def n(*shape):
+        return torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+
+    q = torch.nn.functional.normalize(n(*lead, dk), dim=-1)
+    k = torch.nn.functional.normalize(n(*lead, dk), dim=-1)
+    v = n(*lead, dv)
+    la = torch.nn.functional.logsigmoid(n(*lead, dk) + alpha_mu)
+    b = torch.sigmoid(n(*lead, dk))
+    w = torch.sigmoid(n(*lead, dv))
+    out = {name: t.to(torch.bfloat16) for name, t in zip(TOKEN_NAMES, (q, k, v, la, b, w))}
+    out["S0"] = s0_std * n(B, H, dk, dv)
+    return out

@@ -1,15 +1,13 @@
 """Helpers of the GPU parity tests: device copies of seeded inputs and the
 error measures of the tolerance (relative L2 over the whole tensor, max-abs)."""
+import os
+
 import numpy as np
 
 NAMES = ("q", "k", "v", "log_alpha", "b", "w")
-# bf16 tokens with an fp32 state: rel-L2 <= 1e-2 and max-abs <= 5e-2; fp32
-# tokens: rel-L2 <= 1e-4.  For gradients the absolute bound is taken in units
-# of the reference tensor's RMS when that exceeds 1 (with do ~ N(0,1) the
-# dq/dk RMS is ~1.5 and single entries reach ~12, where bf16 operands alone
-# give ~0.5% element errors); o, S_T and unit-scale gradients keep 5e-2.
+# bf16 tokens with an fp32 state: rel-L2 <= 1e-2 and max-abs <= 5e-2 on o,
+# S_T and every gradient; fp32 tokens: rel-L2 <= 1e-4.
 TOL_BF16 = dict(rel=1e-2, abs=5e-2)
-TOL_BF16_GRAD = dict(rel=1e-2, abs=5e-2, abs_scale="rms")
 TOL_FP32 = dict(rel=1e-4, abs=1e-3)
 
 
@@ -28,8 +26,8 @@ def check(name, x, ref, tol):
     r, m = rel_l2(x, ref), max_abs(x, ref)
     assert np.all(np.isfinite(x)), "%s: non-finite values" % name
     bound = tol["abs"]
-    if tol.get("abs_scale") == "rms" and np.size(ref):
-        bound *= max(1.0, float(np.sqrt(np.mean(np.asarray(ref, np.float64) ** 2))))
+    if os.environ.get("GDN2_REPORT"):
+        print("parity %-28s rel-L2 %.3e (<= %.0e)  max-abs %.4f (<= %.3g)" % (name, r, tol["rel"], m, bound))
     assert r <= tol["rel"] and m <= bound, "%s: rel-L2 %.3e max-abs %.3e (bound %.3e, tol %s)" % (
         name, r, m, bound, tol)
     return r, m

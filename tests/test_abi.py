@@ -77,13 +77,20 @@ def test_decode_and_bwd_reject_bad_arguments():
 
 def test_workspace_sizes():
     assert g.gdn2_chunk_fwd_workspace(8, 4096, 16, 128, 128, g.GDN2_BF16) == 8 * 16 * 64 * 128 * 4
-    # few long sequences: the segmented forward's workspace (P = 8 segments of
-    # B1 H16 T32768 on 148 SMs: per-CTA scratch of 8*16 CTAs, bf16 zeros of
-    # the token tensor, and four fp32 [8*16][128][128] state arrays)
-    seg = 8 * 16 * 64 * 128 * 4 + 32768 * 16 * 128 * 2 + 4 * 8 * 16 * 128 * 128 * 4
+    # few long sequences: the segmented forward's workspace (P = 5 segments of
+    # B1 H16 T32768 on 148 SMs, 16 * (2 * 5 - 1) = 144 CTAs: their per-CTA
+    # scratch, the bf16 rows Phi_t^T q_t like the token tensor, and the fp32
+    # [128][128] end states of 5 segments, transitions and start states of 4)
+    r = lambda x: (x + 255) // 256 * 256
+    seg = (r(144 * 64 * 128 * 4) + r(32768 * 16 * 128 * 2) + r(5 * 16 * 128 * 128 * 4)
+           + 2 * r(4 * 16 * 128 * 128 * 4))
     assert g.gdn2_chunk_fwd_workspace(1, 32768, 16, 128, 128, g.GDN2_BF16) == seg
-    # too short to split into four segments of 8 chunks: the plain size
-    assert g.gdn2_chunk_fwd_workspace(1, 1024, 16, 128, 128, g.GDN2_BF16) == 16 * 64 * 128 * 4
+    # too short for two segments of 8 chunks: the plain size
+    assert g.gdn2_chunk_fwd_workspace(1, 960, 16, 128, 128, g.GDN2_BF16) == 16 * 64 * 128 * 4
+    # too many sequences to split (3 * 64 CTAs > 148): the plain size
+    assert g.gdn2_chunk_fwd_workspace(4, 32768, 16, 128, 128, g.GDN2_BF16) == 4 * 16 * 64 * 128 * 4
+    # a ragged length never splits
+    assert g.gdn2_chunk_fwd_workspace(1, 32767, 16, 128, 128, g.GDN2_BF16) == 16 * 64 * 128 * 4
     assert g.gdn2_chunk_fwd_workspace(8, 4096, 16, 128, 128, g.GDN2_FP32) == 0
     assert g.gdn2_chunk_fwd_workspace(0, 4096, 16, 128, 128, g.GDN2_BF16) == 0
     assert g.gdn2_chunk_bwd_workspace(8, 4096, 16, 128, 128, g.GDN2_BF16) > 0
@@ -111,3 +118,32 @@ def test_saved_state_entry_points_validate():
     assert g.gdn2_chunk_bwd_saved(*args, B, T, H, 128, 128, 0, 16, 1 << 40, 0) == -1
     assert g.gdn2_chunk_fwd_save(16, 16, 16, 16, 16, 16, None, 16, None, None, B, T, H, 128, 128, 0, 16,
                                  1 << 40, 0) == -1
+
+
+def test_varlen_rejects_missing_or_misaligned_offsets():
+    args = [16] * 6 + [None, 16, None]
+    assert g.gdn2_chunk_fwd_varlen(*args, None, 2, 100, 1, 128, 128, g.GDN2_BF16, 16, 1 << 30, 0) == -1
+    assert g.gdn2_chunk_fwd_varlen(*args, 18, 2, 100, 1, 128, 128, g.GDN2_BF16, 16, 1 << 30, 0) == -1
+    assert g.gdn2_chunk_fwd_varlen(*args, 16, 2, 100, 1, 96, 128, g.GDN2_BF16, 16, 1 << 30, 0) == -2
+    assert g.gdn2_chunk_fwd_varlen(*args, 16, 2, 100, 1, 128, 128, g.GDN2_BF16, 16, 0, 0) == -5
+    # N = 0 is a no-op; total_T = 0 only copies the states (none here)
+    assert g.gdn2_chunk_fwd_varlen(*args, 16, 0, 100, 1, 128, 128, g.GDN2_BF16, None, 0, 0) == 0
+    assert g.gdn2_chunk_fwd_varlen(*args, 16, 2, 0, 1, 128, 128, g.GDN2_BF16, None, 0, 0) == 0
+    gargs = [16] * 6 + [None, 16, None] + [16] * 6 + [None]
+    assert g.gdn2_chunk_bwd_varlen(*gargs, None, 2, 100, 1, 128, 128, g.GDN2_BF16, 16, 1 << 40, 0) == -1
+    assert g.gdn2_chunk_bwd_varlen(*gargs, 16, 2, 100, 1, 128, 128, g.GDN2_BF16, 16, 16, 0) == -5
+
+
+def test_varlen_buffer_sizes_depend_on_totals_only():
+    # the saved-state buffer of a packed batch: per head floor(T/64) + 2N
+    # state slots and floor(T/64) + N chunk slots, whatever the lengths
+    N, T, H = 5, 1000, 2
+    st = g.gdn2_chunk_states_varlen_bytes(N, T, H, 128, 128, g.GDN2_BF16)
+    states = H * (T // 64 + 2 * N) * 128 * 128 * 2
+    chunks = H * (T // 64 + N)
+    intra = chunks * (2 * 64 * 64 * 2 + 64 * 128 * 2)
+    ops = chunks * 3 * 64 * 128 * 2
+    r = lambda x: (x + 255) // 256 * 256
+    assert st == r(states) + r(intra) + ops
+    assert g.gdn2_chunk_fwd_varlen_workspace(N, T, H, 128, 128, g.GDN2_BF16) == N * H * 64 * 128 * 4
+    assert g.gdn2_chunk_states_varlen_bytes(N, T, H, 128, 128, g.GDN2_FP32) == 0

@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 
 import oracle
-from gpu_util import TOL_BF16, TOL_BF16_GRAD, TOL_FP32, NAMES, check, dev, dev_state, host, sub_heads, tokens
+from gpu_util import TOL_BF16, TOL_FP32, NAMES, check, dev, dev_state, host, sub_heads, tokens
 from gated_delta_rule_gdn2_b200.inputs import WORKLOADS, make_inputs, make_workload
 
 pytestmark = pytest.mark.gpu
@@ -18,7 +18,7 @@ def run_bwd(x, dtype, dST=None):
     return {n: host(v) for n, v in out.items()}
 
 
-@pytest.mark.parametrize("dtype,tol", [("bf16", TOL_BF16_GRAD), ("fp32", TOL_FP32)])
+@pytest.mark.parametrize("dtype,tol", [("bf16", TOL_BF16), ("fp32", TOL_FP32)])
 @pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (128, 64), (64, 128)])
 @pytest.mark.parametrize("T", [1, 64, 150])
 def test_bwd_matches_oracle(dtype, tol, dk, dv, T):
@@ -33,18 +33,19 @@ def test_bwd_matches_oracle(dtype, tol, dk, dv, T):
 
 def test_bwd_train_full_size_sampled_heads():
     """B=8, T=4096, H=16, d=128, do ~ N(0,1), dS_T = 0: every gradient of three
-    whole heads against the oracle."""
+    whole heads (first, middle and last batch) against the oracle, at the
+    stated bf16 bound (rel-L2 <= 1e-2, max-abs <= 5e-2)."""
     w = WORKLOADS["train"]
     x = make_workload(w)
     g = run_bwd(x, "bf16")
-    heads = [(0, 0), (5, 9)]
+    heads = [(0, 0), (5, 9), (7, 15)]
     xs = sub_heads(x, heads)
     ref = oracle.bwd(*[xs[n] for n in NAMES], xs["S0"], xs["dO"], None)
     for i, (b, h) in enumerate(heads):
         for n in GRADS:
             got = g[n][b, h] if n == "dS0" else g[n][b, :, h]
             exp = ref[n][i, 0] if n == "dS0" else ref[n][i, :, 0]
-            check("%s head %s" % (n, (b, h)), got, exp, TOL_BF16_GRAD)
+            check("%s head %s" % (n, (b, h)), got, exp, TOL_BF16)
 
 
 @pytest.mark.parametrize("scale", [8.0, 40.0, 800.0])
@@ -65,7 +66,7 @@ def test_bwd_fast_decay_and_reset(scale):
     g = run_bwd(x, "bf16", dST)
     ref = oracle.bwd(*[x[n] for n in NAMES], x["S0"], x["dO"], dST)
     for n in GRADS:
-        check(n, g[n], ref[n], TOL_BF16_GRAD)
+        check(n, g[n], ref[n], TOL_BF16)
 
 
 def test_bwd_deterministic():

@@ -169,3 +169,37 @@ def test_segmented_and_one_cta_per_sequence(dk):
         check("o", o, o_ref, TOL_BF16)
         check("S_T", ST, ST_ref, TOL_BF16)
     check("o segmented vs one CTA per sequence", outs[0][0], outs[1][0], TOL_BF16)
+
+
+@pytest.mark.parametrize("B,T,H", [(2, 1088, 16), (1, 3264, 16), (1, 4096, 3)])
+def test_segmented_uneven_segments(B, T, H):
+    """The segment path at shapes whose chunk count does not divide evenly
+    (17 chunks in 2 segments; 51 in 5; 64 in 8 with three heads), with a
+    nonzero S0 (the first segment starts from it, the others are corrected
+    from their scanned start states): against the oracle and against the
+    one-CTA-per-sequence path."""
+    import torch
+    import gated_delta_rule_gdn2_b200 as g
+    x = make_inputs(B, T, H, 128, 128, seed=T + B + H, dtype="bf16")
+    toks = tokens(x, "bf16")
+    S0 = dev_state(x["S0"])
+    plain = B * H * 64 * 128 * 4
+    full = g.gdn2_chunk_fwd_workspace(B, T, H, 128, 128, g.GDN2_BF16)
+    assert full > plain
+    outs = []
+    for nbytes in (full, plain):
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        o = torch.empty((B, T, H, 128), dtype=torch.bfloat16, device="cuda")
+        ST = torch.empty((B, H, 128, 128), dtype=torch.float32, device="cuda")
+        assert g.gdn2_chunk_fwd(*toks, S0, o, ST, B, T, H, 128, 128, g.GDN2_BF16, ws, nbytes) == 0
+        assert g.gdn2_get_device_status() == 0
+        outs.append((host(o), host(ST)))
+    heads = [(0, 0), (B - 1, H - 1)]
+    xs = sub_heads(x, heads)
+    o_ref, ST_ref = oracle_fwd(xs)
+    for o, ST in outs:
+        for i, (b, h) in enumerate(heads):
+            check("o[%d,:,%d]" % (b, h), o[b, :, h], o_ref[i, :, 0], TOL_BF16)
+            check("S_T[%d,%d]" % (b, h), ST[b, h], ST_ref[i, 0], TOL_BF16)
+    check("o segmented vs one CTA per sequence", outs[0][0], outs[1][0], TOL_BF16)
+    check("S_T segmented vs one CTA per sequence", outs[0][1], outs[1][1], TOL_BF16)

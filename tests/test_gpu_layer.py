@@ -1,0 +1,190 @@
+"""The layer prologue (short causal conv + SiLU + L2 norm of q/k, conv + SiLU
+of v, gate activations) and the output epilogue (RMS norm with a SiLU output
+gate), forward and backward, against the fp64 layer oracle through the C ABI:
+fixed-length and packed batches (ragged, with an empty sequence), filter
+widths 1..4, head sizes 64 and 128, bf16 and fp32.
+
+Tolerance: every output that leaves in the token dtype is one rounding of an
+fp32 computation on values of order one, so the mixer's bound applies as
+stated (bf16: rel-L2 <= 1e-2, max-abs <= 5e-2; fp32: rel-L2 <= 1e-4).  The
+filter and gamma gradients leave in fp32 as sums over every token; their
+bound is relative: rel-L2 <= 1e-3 (fp32 sums of bf16-rounded products)."""
+import numpy as np
+import pytest
+
+import oracle
+from gpu_util import TOL_BF16, TOL_FP32, check, host
+from gated_delta_rule_gdn2_b200.inputs import round_bf16
+
+pytestmark = pytest.mark.gpu
+TOL_SUM = dict(rel=1e-3, abs=np.inf)
+
+
+def _t(x, dtype):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda().to(
+        torch.bfloat16 if dtype == "bf16" else torch.float32)
+
+
+def _draw(shape, dtype, rng, scale=1.0):
+    x = (scale * rng.standard_normal(shape)).astype(np.float32)
+    return round_bf16(x) if dtype == "bf16" else x
+
+
+def _segments(lens):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    return list(zip(cu[:-1], cu[1:])), cu
+
+
+def oracle_prologue(x, W, lens=None):
+    """Oracle outputs and the (dx, dW) backward for rows [rows, H, D] packed by lens."""
+    out = {}
+    if lens is None:
+        out["q"] = oracle.prologue_path(x["xq"], W["Wq"], True)
+        out["k"] = oracle.prologue_path(x["xk"], W["Wk"], True)
+        out["v"] = oracle.prologue_path(x["xv"], W["Wv"], False)
+    else:
+        segs, _ = _segments(lens)
+        for n, l2 in (("q", True), ("k", True), ("v", False)):
+            xx = x["x" + n]
+            o = np.zeros(xx.shape)
+            for r0, r1 in segs:
+                if r1 > r0:
+                    o[r0:r1] = oracle.prologue_path(xx[None, r0:r1], W["W" + n], l2)[0]
+            out[n] = o
+    out["log_alpha"] = oracle.gate(x["xa"], "log_alpha")
+    out["b"] = oracle.gate(x["xb"], "sigmoid")
+    out["w"] = oracle.gate(x["xw"], "sigmoid")
+    return out
+
+
+def oracle_prologue_bwd(x, W, g, lens=None):
+    out = {}
+    for n, l2 in (("q", True), ("k", True), ("v", False)):
+        xx, dd = x["x" + n], g["d" + n]
+        if lens is None:
+            out["dx" + n], out["dW" + n] = oracle.prologue_path_bwd(xx, W["W" + n], dd, l2)
+        else:
+            dx, dW = np.zeros(xx.shape), np.zeros(W["W" + n].shape)
+            for r0, r1 in _segments(lens)[0]:
+                if r1 > r0:
+                    a, b = oracle.prologue_path_bwd(xx[None, r0:r1], W["W" + n], dd[None, r0:r1], l2)
+                    dx[r0:r1] = a[0]
+                    dW += b
+            out["dx" + n], out["dW" + n] = dx, dW
+    out["dxa"] = oracle.gate_bwd(x["xa"], g["dlog_alpha"], "log_alpha")
+    out["dxb"] = oracle.gate_bwd(x["xb"], g["db"], "sigmoid")
+    out["dxw"] = oracle.gate_bwd(x["xw"], g["dw"], "sigmoid")
+    return out
+
+
+def _case(shape_k, shape_v, dtype, K, H, seed):
+    rng = np.random.default_rng(seed)
+    dk, dv = shape_k[-1], shape_v[-1]
+    x = {"xq": _draw(shape_k, dtype, rng), "xk": _draw(shape_k, dtype, rng), "xv": _draw(shape_v, dtype, rng),
+         "xa": _draw(shape_k, dtype, rng, 2.0), "xb": _draw(shape_k, dtype, rng), "xw": _draw(shape_v, dtype, rng)}
+    W = {"Wq": (0.5 * rng.standard_normal((H * dk, K))).astype(np.float32),
+         "Wk": (0.5 * rng.standard_normal((H * dk, K))).astype(np.float32),
+         "Wv": (0.5 * rng.standard_normal((H * dv, K))).astype(np.float32)}
+    g = {"dq": _draw(shape_k, dtype, rng), "dk": _draw(shape_k, dtype, rng), "dv": _draw(shape_v, dtype, rng),
+         "dlog_alpha": _draw(shape_k, dtype, rng), "db": _draw(shape_k, dtype, rng), "dw": _draw(shape_v, dtype, rng)}
+    return x, W, g
+
+
+def _run_and_check(x, W, g, dtype, lens=None):
+    import torch
+    import gated_delta_rule_gdn2_b200 as gg
+    cu = None if lens is None else torch.from_numpy(_segments(lens)[1].astype(np.int32)).cuda()
+    dev = {n: _t(v, dtype) for n, v in x.items()}
+    Wd = {n: torch.from_numpy(v).cuda() for n, v in W.items()}
+    out = gg.prologue(dev["xq"], dev["xk"], dev["xv"], Wd["Wq"], Wd["Wk"], Wd["Wv"], dev["xa"], dev["xb"], dev["xw"],
+                      cu_seqlens=cu)
+    gr = gg.prologue_bwd(dev["xq"], dev["xk"], dev["xv"], Wd["Wq"], Wd["Wk"], Wd["Wv"], dev["xa"], dev["xb"],
+                         dev["xw"], {n: _t(v, dtype) for n, v in g.items()}, cu_seqlens=cu)
+    assert gg.gdn2_get_device_status() == 0
+    tol = TOL_BF16 if dtype == "bf16" else TOL_FP32
+    ref = oracle_prologue(x, W, lens)
+    for n in ("q", "k", "v", "log_alpha", "b", "w"):
+        check(n, host(out[n]), ref[n], tol)
+    rb = oracle_prologue_bwd(x, W, g, lens)
+    for n in ("dxq", "dxk", "dxv", "dxa", "dxb", "dxw"):
+        check(n, host(gr[n]), rb[n], tol)
+    for n in ("dWq", "dWk", "dWv"):
+        check(n, host(gr[n]), rb[n], TOL_SUM if dtype == "bf16" else TOL_FP32)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("K,dk,dv", [(4, 128, 128), (1, 64, 128), (3, 128, 64), (2, 64, 64)])
+def test_prologue_fixed_length(dtype, K, dk, dv):
+    B, T, H = 2, 100, 2
+    x, W, g = _case((B, T, H, dk), (B, T, H, dv), dtype, K, H, seed=K + dk + dv)
+    _run_and_check(x, W, g, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_prologue_packed(dtype):
+    lens = (5, 0, 64, 1, 31, 19)
+    H, dk, dv, K = 2, 128, 128, 4
+    T = sum(lens)
+    x, W, g = _case((T, H, dk), (T, H, dv), dtype, K, H, seed=3)
+    _run_and_check(x, W, g, dtype, lens)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("dv", [128, 64])
+def test_output_gate(dtype, dv):
+    import torch
+    import gated_delta_rule_gdn2_b200 as gg
+    rng = np.random.default_rng(dv)
+    B, T, H = 2, 77, 3
+    o, g, dz = (_draw((B, T, H, dv), dtype, rng) for _ in range(3))
+    gamma = (1.0 + 0.1 * rng.standard_normal(dv)).astype(np.float32)
+    z = gg.output_gate(_t(o, dtype), _t(g, dtype), torch.from_numpy(gamma).cuda())
+    dO, dg, dgamma = gg.output_gate_bwd(_t(o, dtype), _t(g, dtype), torch.from_numpy(gamma).cuda(), _t(dz, dtype))
+    assert gg.gdn2_get_device_status() == 0
+    tol = TOL_BF16 if dtype == "bf16" else TOL_FP32
+    check("z", host(z), oracle.epilogue(o, g, gamma), tol)
+    rO, rg, rgamma = oracle.epilogue_bwd(o, g, gamma, dz)
+    check("do", host(dO), rO, tol)
+    check("dg", host(dg), rg, tol)
+    check("dgamma", host(dgamma), rgamma, TOL_SUM if dtype == "bf16" else TOL_FP32)
+
+
+def test_layer_deterministic():
+    """The filter and gamma gradients are fixed-order sums: bit-identical runs."""
+    import torch
+    import gated_delta_rule_gdn2_b200 as gg
+    x, W, g = _case((2, 300, 2, 128), (2, 300, 2, 128), "bf16", 4, 2, seed=11)
+    dev = {n: _t(v, "bf16") for n, v in x.items()}
+    Wd = {n: torch.from_numpy(v).cuda() for n, v in W.items()}
+    gd = {n: _t(v, "bf16") for n, v in g.items()}
+    r1 = gg.prologue_bwd(*(dev[n] for n in ("xq", "xk", "xv")), *(Wd[n] for n in ("Wq", "Wk", "Wv")),
+                         *(dev[n] for n in ("xa", "xb", "xw")), gd)
+    r2 = gg.prologue_bwd(*(dev[n] for n in ("xq", "xk", "xv")), *(Wd[n] for n in ("Wq", "Wk", "Wv")),
+                         *(dev[n] for n in ("xa", "xb", "xw")), gd)
+    for n in r1:
+        np.testing.assert_array_equal(host(r1[n]), host(r2[n]))
+
+
+@pytest.mark.parametrize("B,T,H,dk,dv,dtype", [(2, 200, 3, 128, 128, "bf16"), (2, 130, 2, 64, 128, "bf16"),
+                                               (1, 4096, 1, 128, 128, "bf16"), (2, 100, 2, 128, 64, "fp32")])
+def test_forward_with_output_gate(B, T, H, dk, dv, dtype):
+    """gdn2_chunk_fwd_gated: the forward with the RMS-norm / SiLU-gate epilogue
+    (inside the O epilogue for bf16 d = 128, after the forward otherwise; the
+    B1 H1 T4096 case takes the sequence-segmented forward) against the oracle
+    forward followed by the oracle epilogue."""
+    import torch
+    import gated_delta_rule_gdn2_b200 as gg
+    from gated_delta_rule_gdn2_b200.inputs import make_inputs
+    from gpu_util import NAMES, dev_state, tokens
+    x = make_inputs(B, T, H, dk, dv, seed=T + dk, dtype=dtype)
+    rng = np.random.default_rng(T)
+    g = _draw((B, T, H, dv), dtype, rng)
+    gamma = (1.0 + 0.1 * rng.standard_normal(dv)).astype(np.float32)
+    z, ST = gg.chunk_fwd_gated(*tokens(x, dtype), _t(g, dtype), torch.from_numpy(gamma).cuda(),
+                               S0=dev_state(x["S0"]))
+    assert gg.gdn2_get_device_status() == 0
+    o_ref, ST_ref = oracle.fwd(*[x[n] for n in NAMES], x["S0"])
+    tol = TOL_BF16 if dtype == "bf16" else TOL_FP32
+    check("z", host(z), oracle.epilogue(o_ref, g, gamma), tol)
+    check("S_T", host(ST), ST_ref, tol)
