@@ -180,7 +180,11 @@ size_t fwd_ws_bytes(int B, int T, int H, int dk, int dv, int dtype, bool varlen)
     const size_t plain = chunk_fwd_ws_bytes(B, H, dk);
     if (varlen) return plain;  // (packed batches always run one CTA per sequence)
     const int P = segment_count(B, T, H, dk, dv);
-    return P > 1 ? std::max(plain, segments_ws_bytes(B, T, H, dk, dv, P)) : plain;
+    if (P <= 1) return plain;
+    size_t need = std::max(plain, segments_ws_bytes(B, T, H, dk, dv, P));
+    const int Pt = seg_train_count(B, T, H, dk, dv);  // (the saving forward's segment path)
+    if (Pt > 1) need = std::max(need, seg_train_fwd_ws_bytes(B, T, H, Pt));
+    return need;
 }
 
 int fwd_impl(const void *q, const void *k, const void *v, const void *log_alpha, const void *b, const void *w,
@@ -206,6 +210,16 @@ int fwd_impl(const void *q, const void *k, const void *v, const void *log_alpha,
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return GDN2_ERR_WORKSPACE;
     if (dtype == GDN2_BF16) {
         const bool varlen = cu != nullptr;
+        // few long sequences, states kept: segmented training (its buffer layout
+        // follows from the sizes alone, so the backward always finds it)
+        const int Pt = (keep && !varlen && gates == kGatesFull) ? seg_train_count(B, T, H, dk, dv) : 1;
+        if (Pt > 1) {
+            if (ws_bytes < seg_train_fwd_ws_bytes(B, T, H, Pt)) return GDN2_ERR_WORKSPACE;
+            ChunkFwdArgs a{q, k, v, log_alpha, b, w, S0, o, S_T, nullptr, 0, nullptr, nullptr, nullptr,
+                           status_ptr(), B, T, H};
+            a.wait_limit = g_wait_limit;
+            return launch_status(launch_seg_train_fwd(a, states, Pt, ws, stream));
+        }
         char *sb = static_cast<char *>(states);
         ChunkFwdArgs a{q, k, v, log_alpha, b, w, S0, o, S_T, static_cast<float *>(ws), (size_t)64 * dk,
                        keep ? sb : nullptr,
@@ -258,6 +272,8 @@ size_t bwd_ws_bytes(int B, int T, int H, int dk, int dv, int dtype, bool varlen)
 size_t states_bytes(int B, int T, int H, int dk, int dv, int dtype, bool varlen) {
     if (check_sizes(B, T, H, dk, dv, dtype) != GDN2_OK) return 0;
     if (B == 0 || H == 0 || T == 0 || dtype != GDN2_BF16) return 0;
+    const int Pt = varlen ? 1 : seg_train_count(B, T, H, dk, dv);
+    if (Pt > 1) return seg_train_states_bytes(B, T, H, Pt);
     size_t sbytes = 0;
     chunk_bwd_ws_bytes(B, T, H, dk, dv, nullptr, &sbytes, varlen);
     return sbytes;
@@ -267,6 +283,8 @@ size_t bwd_saved_ws_bytes(int B, int T, int H, int dk, int dv, int dtype, bool v
     if (check_sizes(B, T, H, dk, dv, dtype) != GDN2_OK) return 0;
     if (B == 0 || H == 0 || T == 0) return 0;
     if (dtype != GDN2_BF16) return bwd_ws_bytes(B, T, H, dk, dv, dtype, varlen);
+    const int Pt = varlen ? 1 : seg_train_count(B, T, H, dk, dv);
+    if (Pt > 1) return seg_train_bwd_ws_bytes(B, T, H, Pt);
     size_t sbytes = 0;
     return chunk_bwd_ws_bytes(B, T, H, dk, dv, nullptr, &sbytes, varlen) - sbytes;
 }
@@ -299,6 +317,13 @@ int bwd_impl(const void *q, const void *k, const void *v, const void *log_alpha,
                               : bwd_ws_bytes(B, T, H, dk, dv, dtype, varlen);
     if (ws_bytes < need || (need > 0 && ws == nullptr)) return GDN2_ERR_WORKSPACE;
     if (dtype == GDN2_BF16) {
+        const int Pt = (saved && !varlen && gates == kGatesFull) ? seg_train_count(B, T, H, dk, dv) : 1;
+        if (Pt > 1) {  // segmented training: the forward kept its own layout
+            ChunkBwdArgs a{q, k, v, log_alpha, b, w, S0, dO, dS_T, dq, dk_, dv_, dlog_alpha, db, dw, dS0, nullptr,
+                           nullptr, nullptr, nullptr, 0, status_ptr(), 1, B, T, H};
+            a.wait_limit = g_wait_limit;
+            return launch_status(launch_seg_train_bwd(a, states, Pt, ws, stream));
+        }
         size_t stride = 0, sbytes = 0;
         chunk_bwd_ws_bytes(B, T, H, dk, dv, &stride, &sbytes, varlen);
         char *st_buf = saved ? static_cast<char *>(const_cast<void *>(states)) : static_cast<char *>(ws);

@@ -72,8 +72,10 @@ __device__ __forceinline__ void store_stage(const float (&acc)[1][NT][4], float 
 
 // Per-CTA view of one (batch, head) sequence in the reverse chunk pass: the
 // shared-memory tiles, the caller's per-CTA scratch and the global tensors.
-// NT: threads of the CTA (256 or 512).
-template <int DK, int DV, int NT = NTHR>
+// NT: threads of the CTA (256 or 512).  GATES: the gate form (kGatesKDA /
+// kGatesGDN: the tensor-memory kernel only), fixed at compile time so that
+// the general form's loops carry no branch on it.
+template <int DK, int DV, int NT = NTHR, int GATES = kGatesFull>
 struct BwdChunk {
     using L = BSmem<DK, DV>;
     using SC = Scratch<DK>;
@@ -229,7 +231,7 @@ struct BwdChunk {
             for (int r = 0; r < Cn; ++r) {
                 const size_t orr = ((row0 + n * C + r) * H + h) * DK + ch;
                 const float qr = __bfloat162float(gq[orr]);
-                const float br = a.gates == kGatesFull ? __bfloat162float(gb[orr])
+                const float br = GATES == kGatesFull ? __bfloat162float(gb[orr])
                                                        : __bfloat162float(gb[(row0 + n * C + r) * H + h]);
                 const float gr = br * __bfloat162float(gk[orr]);
                 const float lr = LAM[r * DK + ch];
@@ -269,7 +271,7 @@ struct BwdChunk {
         constexpr bool kScalarOK = T0 % 16 == 0 && (NT - T0) % 16 == 0 && DV == 128;
         const int t = tid - T0;
         if (t < 0) return;
-        const bool scalar = kScalarOK && a.gates != kGatesFull;  // w = beta 1: w from beta, the sum of dw per token
+        const bool scalar = kScalarOK && GATES != kGatesFull;  // w = beta 1: w from beta, the sum of dw per token
         uint4 v8[NV], w8[NV];
 #pragma unroll
         for (int it = 0; it < NV; ++it) {
@@ -477,13 +479,13 @@ struct BwdChunk {
             const size_t os = (row0 + n * C + r) * H + h;  // a scalar gate's element
             raw.q[i] = *reinterpret_cast<const uint2 *>(gq + o);
             raw.k[i] = *reinterpret_cast<const uint2 *>(gk + o);
-            if (a.gates == kGatesFull) {
+            if (GATES == kGatesFull) {
                 raw.b[i] = *reinterpret_cast<const uint2 *>(gb + o);
             } else {
                 const uint32_t x = sb[os] | ((uint32_t)sb[os] << 16);
                 raw.b[i] = make_uint2(x, x);
             }
-            if (a.gates != kGatesGDN) {
+            if (GATES != kGatesGDN) {
                 raw.la[i] = *reinterpret_cast<const uint2 *>(gla + o);
             } else {
                 const uint32_t x = sla[os] | ((uint32_t)sla[os] << 16);
@@ -600,7 +602,7 @@ struct BwdChunk {
                 const float2 db0 = __fmul2_rn(p0.dg, k0), db1 = __fmul2_rn(p1.dg, k1);
                 *reinterpret_cast<uint2 *>(gdq + o) = make_uint2(pack_bf16(p0.dq.x, p0.dq.y), pack_bf16(p1.dq.x, p1.dq.y));
                 *reinterpret_cast<uint2 *>(gdk + o) = make_uint2(pack_bf16(dk0.x, dk0.y), pack_bf16(dk1.x, dk1.y));
-                if (a.gates == kGatesFull) {
+                if (GATES == kGatesFull) {
                     *reinterpret_cast<uint2 *>(gdb + o) =
                         make_uint2(pack_bf16(db0.x, db0.y), pack_bf16(db1.x, db1.y));
                 } else {  // dbeta = sum over the key channels of db, plus that of dw
@@ -632,7 +634,7 @@ struct BwdChunk {
             if (r < Cn) {
                 acc0 = __fadd2_rn(acc0, dl0[i]);
                 acc1 = __fadd2_rn(acc1, dl1[i]);
-                if (a.gates != kGatesGDN) {
+                if (GATES != kGatesGDN) {
                     *reinterpret_cast<uint2 *>(gdl + ((row0 + n * C + r) * H + h) * DK + c4) =
                         make_uint2(pack_bf16(acc0.x, acc0.y), pack_bf16(acc1.x, acc1.y));
                 } else {  // a scalar decay: the sum over the key channels

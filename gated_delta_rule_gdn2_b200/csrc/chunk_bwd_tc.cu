@@ -118,7 +118,9 @@ __device__ bool decay_sums(const bf16 *la, float (*seg)[D], float *gamma, int *s
     return slow;
 }
 
+template <int GATES>
 __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, const __grid_constant__ BwdMaps maps) {
+    using Chunk = BwdChunk<D, D, NT, GATES>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u);
     __shared__ __align__(16) float s_seg[Chunk::P4][D];  // log_alpha sums over the 4-row segments of a chunk
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
     // n - 1's decay sums, E0 and first products run.
     uint32_t ph_ld[3] = {0, 0, 0};
     int ld_issued[3] = {0, 0, 0}, ld_landed[3] = {0, 0, 0};  // (thread 0: its loads, for the drain at the end)
-    const bool scalar_la = a.gates == kGatesGDN;  // a scalar decay: its tile is filled after the loads
+    constexpr bool scalar_la = GATES == kGatesGDN;  // a scalar decay: its tile is filled after the loads
     auto issue_a = [&](int m) {
         tc::mbar_expect_tx(&mbar_ld[0], (scalar_la ? 5 : 6) * TILE_BYTES);
         const unsigned char *img = x.intra + (size_t)m * x.I_BYTES + TM_BYTES;
@@ -432,7 +434,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
             }
             tc::commit(&mbar);
         }
-        Chunk::RawRows4 raw;
+        typename Chunk::RawRows4 raw;
         x.load_rows4(raw, n, Cn);  // while the tensor cores run
         // ---- row sums of dSigma . Sigma for chunk n - 1 (dSigma is now its
         // chunk-end gradient, Sigma = this chunk's start state S), also inside M4
@@ -516,10 +518,12 @@ cudaError_t launch_chunk_bwd_tc(const ChunkBwdArgs &a, cudaStream_t s) {
     if ((a.gates != kGatesGDN && !token_tensor_map(&m.la, a.log_alpha, MB, a.T, a.H, cbwd_tc::D)) ||
         !token_tensor_map(&m.dO, a.dO, MB, a.T, a.H, cbwd_tc::D))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(cbwd_tc::chunk_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         cbwd_tc::BYTES);
+    auto kernel = a.gates == kGatesKDA   ? cbwd_tc::chunk_bwd_tc_kernel<kGatesKDA>
+                  : a.gates == kGatesGDN ? cbwd_tc::chunk_bwd_tc_kernel<kGatesGDN>
+                                         : cbwd_tc::chunk_bwd_tc_kernel<kGatesFull>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, cbwd_tc::BYTES);
     if (e != cudaSuccess) return e;
-    cbwd_tc::chunk_bwd_tc_kernel<<<(unsigned)(a.B * a.H), cbwd_tc::NT, cbwd_tc::BYTES, s>>>(a, m);
+    kernel<<<(unsigned)(a.B * a.H), cbwd_tc::NT, cbwd_tc::BYTES, s>>>(a, m);
     return cudaGetLastError();
 }
 

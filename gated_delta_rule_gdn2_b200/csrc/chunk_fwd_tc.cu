@@ -128,9 +128,9 @@ __device__ __forceinline__ void issue_chunk(const FwdMaps &m, ChunkTiles st, con
 // Scalar gates into whole tiles: row r of the b and w tiles (and, for GDN, of
 // the log_alpha tile) holds the scalar of token n*C + r in every column; rows
 // past the sequence's end hold zeros (a zero token).  The NTG threads of G.
-template <class G, int NTG>
+template <class G, int NTG, int GATES>
 __device__ __forceinline__ void expand_gates(ChunkTiles st, const ChunkFwdArgs &a, const SeqView &sv, int h, int n) {
-    const int ntiles = a.gates == kGatesGDN ? 3 : 2;
+    constexpr int ntiles = GATES == kGatesGDN ? 3 : 2;
     const int valid = min(C, sv.len - n * C);
     const unsigned short *beta = static_cast<const unsigned short *>(a.b);
     const unsigned short *lsc = static_cast<const unsigned short *>(a.log_alpha);
@@ -161,6 +161,11 @@ __device__ __forceinline__ void zero_tail_rows(ChunkTiles st, int Cn) {
     }
 }
 
+// Compile-time forms: GATES (the gate form) and MODE (kPlain, kSegments: the
+// segment path's local and transition passes, kGated: the output epilogue in
+// the O epilogue), so that the plain form carries no branch on them.
+constexpr int kPlain = 0, kSegments = 1, kGated = 2;
+template <int GATES, int MODE>
 __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, const __grid_constant__ FwdMaps maps) {
     extern __shared__ __align__(1024) unsigned char smem[];
     Small &sm = *reinterpret_cast<Small *>(smem + OSMALL);
@@ -175,7 +180,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
     const float *S0p;  // this CTA's start state (nullptr: zero; a transition pass starts from I)
     float *STp;        // and its end state (or nullptr)
     void *op = a.o;    // its output rows
-    if (a.seg_P == 0) {
+    if constexpr (MODE != kSegments) {
         const int bh = blockIdx.x;
         b = bh / a.H;
         h = bh % a.H;
@@ -271,8 +276,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 zero_tail_rows<GA, NG>(st, sv.len - m * C);
                 GA::sync();
             }
-            if (a.gates != kGatesFull) {
-                expand_gates<GA, NG>(st, a, sv, h, m);
+            if constexpr (GATES != kGatesFull) {
+                expand_gates<GA, NG, GATES>(st, a, sv, h, m);
                 GA::sync();
             }
             if (phi) {  // a transition pass: no write term (w . v = 0)
@@ -343,7 +348,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         // the fused output epilogue: the gate tile lands in the S16 area (free
         // from U's completion to the next chunk's solve), the RMS partials of
         // the two column halves beside it
-        const bool gated = with_o && a.out_gate != nullptr;
+        constexpr bool gated = MODE == kGated;  // (with_o: the launch checks o)
         bf16 *G16 = reinterpret_cast<bf16 *>(smem + OS16);
         float *rms_part = reinterpret_cast<float *>(smem + OS16 + TILE);  // [2][64]
         uint32_t ph_g = 0;
@@ -406,7 +411,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         }
         if (tb == 0) {
             for (int i = 0; i < 2 && i < nchunks; ++i) {
-                issue_chunk(maps, stage_tiles(smem, i), sv, h, i, &sm.mbar_ld[i], a.gates, phi);
+                issue_chunk(maps, stage_tiles(smem, i), sv, h, i, &sm.mbar_ld[i], GATES, phi);
                 ++sm.ld_issued[i];
             }
         }
@@ -603,7 +608,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 // follows this thread's next MMA issue)
                 tc::bulk_wait_read();
                 if (n + 2 < nchunks) {
-                    issue_chunk(maps, st, sv, h, n + 2, &sm.mbar_ld[s], a.gates, phi);
+                    issue_chunk(maps, st, sv, h, n + 2, &sm.mbar_ld[s], GATES, phi);
                     ++sm.ld_issued[s];
                 }
             }
@@ -676,11 +681,17 @@ cudaError_t launch_chunk_fwd_tc(const ChunkFwdArgs &a, cudaStream_t s) {
                     a.gates != kGatesFull || !a.seg_loc || !a.seg_phi || !a.seg_qphi))
         return cudaErrorInvalidValue;
     if (a.out_gate && (a.states || !a.o || !a.gamma)) return cudaErrorInvalidValue;  // (inference path only)
-    cudaError_t e = cudaFuncSetAttribute(cfwd_tc::chunk_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         cfwd_tc::BYTES);
+    using namespace cfwd_tc;
+    auto kernel = a.seg_P                  ? chunk_fwd_tc_kernel<kGatesFull, kSegments>
+                  : a.out_gate             ? chunk_fwd_tc_kernel<kGatesFull, kGated>
+                  : a.gates == kGatesKDA   ? chunk_fwd_tc_kernel<kGatesKDA, kPlain>
+                  : a.gates == kGatesGDN   ? chunk_fwd_tc_kernel<kGatesGDN, kPlain>
+                                           : chunk_fwd_tc_kernel<kGatesFull, kPlain>;
+    if (a.out_gate && a.gates != kGatesFull) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, BYTES);
     if (e != cudaSuccess) return e;
     const unsigned ctas = (unsigned)(a.B * a.H) * (a.seg_P ? 2u * a.seg_P - 1u : 1u);
-    cfwd_tc::chunk_fwd_tc_kernel<<<ctas, cfwd_tc::NT, cfwd_tc::BYTES, s>>>(a, m);
+    kernel<<<ctas, NT, BYTES, s>>>(a, m);
     return cudaGetLastError();
 }
 

@@ -89,6 +89,17 @@ int segment_count(int B, int T, int H, int dk, int dv);
 size_t segments_ws_bytes(int B, int T, int H, int dk, int dv, int P);
 cudaError_t launch_chunk_fwd_segments(const ChunkFwdArgs &a, int dk, int dv, int P, void *ws, cudaStream_t s);
 
+// Segmented training (segments.cu): the saved-state pair for few long
+// sequences at dk = dv = 128 (P = seg_train_count(...) > 1), with its own
+// saved-buffer layout and workspaces.
+struct ChunkBwdArgs;
+int seg_train_count(int B, int T, int H, int dk, int dv);
+size_t seg_train_states_bytes(int B, int T, int H, int P);
+size_t seg_train_fwd_ws_bytes(int B, int T, int H, int P);
+size_t seg_train_bwd_ws_bytes(int B, int T, int H, int P);
+cudaError_t launch_seg_train_fwd(const ChunkFwdArgs &a, void *states, int P, void *ws, cudaStream_t s);
+cudaError_t launch_seg_train_bwd(const ChunkBwdArgs &a, const void *states, int P, void *ws, cudaStream_t s);
+
 // Chunk-parallel gate-aware backward (bf16 tokens): a state pass (the
 // forward writing bf16 chunk-boundary states to `states`) and a reverse chunk
 // pass.  scratch: per-CTA fp32 work area of scr_stride floats.

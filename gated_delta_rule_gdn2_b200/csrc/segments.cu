@@ -165,32 +165,37 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan2_kernel(const float *Phi, c
 // o_t += S_start(p)^T (Phi_t^T q_t) for every token of segments 1..P-1: per
 // block one (segment, head) and up to kCorrTiles 64-token tiles; the start
 // state goes to shared memory once as bf16, each tile's rows Phi_t^T q_t
-// arrive by cp.async, and the product runs on the tensor cores (warp-level
-// m16n8k16; the pass is bound by the bytes of o and of those rows).
-constexpr int kCorrTiles = 8, kCorrThreads = 128;
-constexpr int CORR_SMEM = 128 * 128 * 2 + 64 * 128 * 2;
+// arrive by cp.async, the product runs on the tensor cores (warp-level
+// m16n8k16) into an fp32 tile in shared memory, and o is read, added to and
+// written back with coalesced 16-byte accesses.  The pass is bound by the
+// bytes of o and of those rows.
+constexpr int kCorrTiles = 16, kCorrThreads = 128;
+constexpr int CORR_LD = 128 + 4;  // fp32 sum tile row pitch (rows 4 banks apart)
+constexpr int CORR_SMEM = 128 * 128 * 2 + 64 * 128 * 2 + 64 * CORR_LD * 4;
 __global__ void __launch_bounds__(kCorrThreads) correct_kernel(const bf16 *qphi, const float *Sstart, bf16 *o, int B,
                                                                int T, int H, int P) {
     constexpr int D = 128;
     extern __shared__ __align__(1024) unsigned char smc[];
-    bf16 *S16 = reinterpret_cast<bf16 *>(smc);              // [128 k][128 n], swizzled
-    bf16 *Q16 = reinterpret_cast<bf16 *>(smc + D * D * 2);   // [64 t][128 k], swizzled
-    const int seg = blockIdx.y / H, h = blockIdx.y % H;      // seg = b*(P-1) + p - 1
+    bf16 *S16 = reinterpret_cast<bf16 *>(smc);                            // [128 k][128 n], swizzled
+    bf16 *Q16 = reinterpret_cast<bf16 *>(smc + D * D * 2);                 // [64 t][128 k], swizzled
+    float *acc_s = reinterpret_cast<float *>(smc + D * D * 2 + 64 * D * 2);  // [64 t][CORR_LD] fp32
+    const int seg = blockIdx.y / H, h = blockIdx.y % H;                    // seg = b*(P-1) + p - 1
     const int b = seg / (P - 1), p = seg % (P - 1) + 1;
     const int nch = T / chunk::C, base = nch / P, rem = nch % P;
     const int c0 = p * base + min(p, rem), cn = base + (p < rem ? 1 : 0);
     const int t0 = blockIdx.x * kCorrTiles;
     if (t0 >= cn) return;
     const size_t row0 = (size_t)b * T + (size_t)c0 * chunk::C;
-    const float *Ss = Sstart + ((size_t)seg * H + h) * D * D;
-    for (int i = threadIdx.x; i < D * D / 2; i += kCorrThreads) {
-        const int k = (2 * i) / D, n = (2 * i) % D;
-        const float2 v = *reinterpret_cast<const float2 *>(Ss + (size_t)k * D + n);
-        *reinterpret_cast<uint32_t *>(S16 + chunk::swz<D, D>(k, n)) = chunk::pack_bf16(v.x, v.y);
+    const float4 *Ss = reinterpret_cast<const float4 *>(Sstart + ((size_t)seg * H + h) * D * D);
+    for (int i = threadIdx.x; i < D * D / 4; i += kCorrThreads) {
+        const float4 v = Ss[i];
+        const int k = (4 * i) / D, n = (4 * i) % D;
+        *reinterpret_cast<uint2 *>(S16 + chunk::swz<D, D>(k, n)) =
+            make_uint2(chunk::pack_bf16(v.x, v.y), chunk::pack_bf16(v.z, v.w));
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int tl = t0; tl < min(cn, t0 + kCorrTiles); ++tl) {
-        __syncthreads();  // (S16 written; the previous tile's rows read)
+        __syncthreads();  // (S16 written; the previous tile's rows and sums read)
         chunk::load_token_tile<D, kCorrThreads>(Q16, qphi, row0, cn * chunk::C, h, tl, H);
         chunk::cp_commit();
         chunk::cp_wait<0>();
@@ -200,16 +205,129 @@ __global__ void __launch_bounds__(kCorrThreads) correct_kernel(const bf16 *qphi,
         chunk::warp_gemm<1, 16, true, false, D, D, 64, D>(acc, Q16, 16 * warp, S16, 0, D, lane);
         const int r = 16 * warp + (lane >> 2);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            bf16 *orow = o + ((row0 + (size_t)tl * chunk::C + r + 8 * half) * H + h) * D;
-#pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                const int c = 8 * nt + 2 * (lane & 3);
-                __nv_bfloat162 *pr = reinterpret_cast<__nv_bfloat162 *>(orow + c);
-                const float2 ov = __bfloat1622float2(*pr);
-                *pr = __floats2bfloat162_rn(ov.x + acc[0][nt][2 * half], ov.y + acc[0][nt][2 * half + 1]);
-            }
+        for (int nt = 0; nt < 16; ++nt) {
+            const int c = 8 * nt + 2 * (lane & 3);
+            *reinterpret_cast<float2 *>(acc_s + r * CORR_LD + c) = make_float2(acc[0][nt][0], acc[0][nt][1]);
+            *reinterpret_cast<float2 *>(acc_s + (r + 8) * CORR_LD + c) = make_float2(acc[0][nt][2], acc[0][nt][3]);
         }
+        __syncthreads();
+        // o rows of the tile: 16 bytes (8 values) per access; every load of the
+        // tile is issued before the first store (a store may alias a later
+        // load, so interleaving them would serialise the loads)
+        constexpr int IT = 64 * D / 8 / kCorrThreads;
+        uint4 ov[IT];
+        uint4 *op[IT];
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+            const int id = threadIdx.x + it * kCorrThreads, rr = id / (D / 8), cc = (id % (D / 8)) * 8;
+            op[it] = reinterpret_cast<uint4 *>(o + ((row0 + (size_t)tl * chunk::C + rr) * H + h) * D + cc);
+            ov[it] = *op[it];
+        }
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+            const int id = threadIdx.x + it * kCorrThreads, rr = id / (D / 8), cc = (id % (D / 8)) * 8;
+            const float4 a0 = *reinterpret_cast<const float4 *>(acc_s + rr * CORR_LD + cc);
+            const float4 a1 = *reinterpret_cast<const float4 *>(acc_s + rr * CORR_LD + cc + 4);
+            const float2 x0 = chunk::unpack_bf16(ov[it].x), x1 = chunk::unpack_bf16(ov[it].y);
+            const float2 x2 = chunk::unpack_bf16(ov[it].z), x3 = chunk::unpack_bf16(ov[it].w);
+            *op[it] = make_uint4(chunk::pack_bf16(x0.x + a0.x, x0.y + a0.y), chunk::pack_bf16(x1.x + a0.z, x1.y + a0.w),
+                                 chunk::pack_bf16(x2.x + a1.x, x2.y + a1.y), chunk::pack_bf16(x3.x + a1.z, x3.y + a1.w));
+        }
+    }
+}
+
+// ---- segmented training (the saved-state pair, dk = dv = 128)
+
+// Offsets of the B*P segments as a packed batch over the B*T token rows.
+__global__ void seg_cu_kernel(int *cu, int B, int T, int P) {
+    const int nch = T / chunk::C, base = nch / P, rem = nch % P;
+    for (int n = blockIdx.x * blockDim.x + threadIdx.x; n <= B * P; n += gridDim.x * blockDim.x) {
+        if (n == B * P) {
+            cu[n] = B * T;
+        } else {
+            const int b = n / P, p = n % P;
+            cu[n] = b * T + chunk::C * (p * base + min(p, rem));
+        }
+    }
+}
+
+// The start states of the segments, per (b*P + p, head h): p == 0 from S0
+// (a [B][H] array, nullptr = zero), p >= 1 from `later` (a [B*(P-1)][H] array).
+__global__ void seg_gather_kernel(const float *first, const float *later, float *out, int B, int H, int P) {
+    constexpr int DD = 128 * 128;
+    const size_t n = (size_t)B * P * H * DD;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const size_t m = i / DD, e = i % DD;
+        const int h = (int)(m % H), bp = (int)(m / H), b = bp / P, p = bp % P;
+        float v = 0.f;
+        if (p == 0) {
+            if (first) v = first[((size_t)b * H + h) * DD + e];
+        } else if (later) {
+            v = later[(((size_t)b * (P - 1) + p - 1) * H + h) * DD + e];
+        }
+        out[i] = v;
+    }
+}
+
+// dS0 [B][H] = the first segment's start-state gradient of each sequence.
+__global__ void seg_first_kernel(const float *seg, float *out, int B, int H, int P) {
+    constexpr int DD = 128 * 128;
+    const size_t n = (size_t)B * H * DD;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const size_t m = i / DD, e = i % DD;
+        const int b = (int)(m / H), h = (int)(m % H);
+        out[i] = seg[(((size_t)b * P) * H + h) * DD + e];
+    }
+}
+
+// End-state gradients of the segments, last to first: G(P-1) = dS_T,
+// G(p) = Phi(p+1)^T G(p+1) + L(p+1), with L(q) the start-state gradient of
+// segment q from a zero end gradient.  One block per (b*H + h, column
+// group), as the forward scan.
+template <int DK>
+__global__ void __launch_bounds__(SCAN_THREADS) rscan_kernel(const float *Phi, const float *L, const float *dS_T,
+                                                            float *G, int B, int H, int P) {
+    extern __shared__ __align__(16) float sm[];
+    float (*phit)[DK + 1] = reinterpret_cast<float (*)[DK + 1]>(sm);  // Phi^T, padded rows
+    float (*prev)[SCAN_COLS] = reinterpret_cast<float (*)[SCAN_COLS]>(sm + DK * (DK + 1));
+    const int bh = blockIdx.x, b = bh / H, h = bh % H, c0 = blockIdx.y * SCAN_COLS;
+    const int tid = threadIdx.x;
+    constexpr int CPT = DK * SCAN_COLS / SCAN_THREADS;
+    const int r = tid % DK, cc = (tid / DK) * CPT;
+    auto at = [&](int p) { return (((size_t)b * P + p) * H + h) * DK * DK; };
+    for (int i = tid; i < DK * SCAN_COLS; i += SCAN_THREADS) {
+        const int rr = i / SCAN_COLS, c = i % SCAN_COLS;
+        prev[rr][c] = dS_T ? dS_T[((size_t)b * H + h) * DK * DK + (size_t)rr * DK + c0 + c] : 0.f;
+    }
+    for (int p = P - 1; p >= 0; --p) {
+        __syncthreads();  // prev complete
+        for (int i = tid; i < DK * SCAN_COLS; i += SCAN_THREADS)
+            G[at(p) + (size_t)(i / SCAN_COLS) * DK + c0 + i % SCAN_COLS] = prev[i / SCAN_COLS][i % SCAN_COLS];
+        if (p == 0) break;
+        // Phi(p) (stored at (b*(P-1) + p-1)*H + h) transposed into shared memory
+        const float4 *src = reinterpret_cast<const float4 *>(Phi + (((size_t)b * (P - 1) + p - 1) * H + h) * DK * DK);
+        for (int i = tid; i < DK * DK / 4; i += SCAN_THREADS) {
+            const float4 t = src[i];
+            const int rr = (4 * i) / DK, k = (4 * i) % DK;
+            phit[k][rr] = t.x;
+            phit[k + 1][rr] = t.y;
+            phit[k + 2][rr] = t.z;
+            phit[k + 3][rr] = t.w;
+        }
+        __syncthreads();
+        const float *lp = L + at(p) + (size_t)r * DK + c0 + cc;
+        float acc[CPT];
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) acc[j] = lp[j];
+#pragma unroll 4
+        for (int k = 0; k < DK; ++k) {
+            const float a = phit[r][k];
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) acc[j] += a * prev[k][cc + j];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) prev[r][cc + j] = acc[j];
     }
 }
 
@@ -384,6 +502,172 @@ cudaError_t launch_chunk_fwd_segments(const ChunkFwdArgs &a, int dk, int dv, int
                                 cudaMemcpyDeviceToDevice, s);
             if (e != cudaSuccess) return e;
         }
+    }
+    return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// Segmented training: the saved-state pair for few long sequences (dk = dv =
+// 128, bf16).  The forward finds every segment's start state with the
+// segment path (local and transition passes, the scan), then runs the saving
+// forward over the B*P segments as a packed batch from those start states.
+// The backward runs the packed backward twice: first with zero end gradients
+// (each segment's own start-state gradient L), then, after a reverse scan
+// G(p) = Phi(p+1)^T G(p+1) + L(p+1), with the true end gradients G.
+
+namespace seg {
+
+struct TrainFwdCarve {
+    Carve2 c2;
+    float *s0seg;
+    int *cu;
+    float *fwd_ws;
+};
+size_t carve_train_fwd(void *p, int B, int T, int H, int P, TrainFwdCarve *c) {
+    constexpr int D = 128;
+    Carve2 c2{};
+    size_t off = align256(carve2(p, B, T, H, P, &c2));
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += align256(bytes);
+        return p ? static_cast<unsigned char *>(p) + at : nullptr;
+    };
+    unsigned char *s0 = take((size_t)B * P * H * D * D * sizeof(float));
+    unsigned char *cu = take(((size_t)B * P + 1) * sizeof(int));
+    unsigned char *fw = take(chunk_fwd_ws_bytes(B * P, H, D));
+    if (c) *c = {c2, reinterpret_cast<float *>(s0), reinterpret_cast<int *>(cu), reinterpret_cast<float *>(fw)};
+    return off;
+}
+
+struct TrainBwdCarve {
+    float *scratch;
+    size_t stride;
+    float *dst_seg, *l_seg, *g_seg;
+    int *cu;
+};
+size_t carve_train_bwd(void *p, int B, int T, int H, int P, TrainBwdCarve *c) {
+    constexpr int D = 128;
+    size_t stride = 0, sbytes = 0;
+    const size_t scr = chunk_bwd_ws_bytes(B * P, B * T, H, D, D, &stride, &sbytes, true) - sbytes;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += align256(bytes);
+        return p ? static_cast<unsigned char *>(p) + at : nullptr;
+    };
+    unsigned char *sc = take(scr);
+    unsigned char *d = take((size_t)B * P * H * D * D * sizeof(float));
+    unsigned char *l = take((size_t)B * P * H * D * D * sizeof(float));
+    unsigned char *g = take((size_t)B * P * H * D * D * sizeof(float));
+    unsigned char *cu = take(((size_t)B * P + 1) * sizeof(int));
+    if (c)
+        *c = {reinterpret_cast<float *>(sc), stride, reinterpret_cast<float *>(d), reinterpret_cast<float *>(l),
+              reinterpret_cast<float *>(g), reinterpret_cast<int *>(cu)};
+    return off;
+}
+
+unsigned grid_for(size_t n) { return (unsigned)std::min<size_t>((n + 255) / 256, 4096); }
+
+}  // namespace seg
+
+int seg_train_count(int B, int T, int H, int dk, int dv) {
+    return (dk == 128 && dv == 128) ? segment_count(B, T, H, dk, dv) : 1;
+}
+
+// The saved buffer of segmented training: the packed batch's states, tiles
+// and decayed operands (the layout of the _varlen pair for B*P sequences
+// over B*T rows), then the transitions Phi of segments 1..P-1.
+size_t seg_train_states_bytes(int B, int T, int H, int P) {
+    const int N = B * P, R = B * T;
+    return states_region_bytes(N, R, H, 128, 128, true) + intra_region_bytes(N, R, H, 128, true) +
+           (ops_region_bytes(N, R, H, 128, 128, true) + 255) / 256 * 256 +
+           (size_t)B * (P - 1) * H * 128 * 128 * sizeof(float);
+}
+size_t seg_train_fwd_ws_bytes(int B, int T, int H, int P) { return seg::carve_train_fwd(nullptr, B, T, H, P, nullptr); }
+size_t seg_train_bwd_ws_bytes(int B, int T, int H, int P) { return seg::carve_train_bwd(nullptr, B, T, H, P, nullptr); }
+
+namespace {
+// the regions of the segmented-training saved buffer
+void train_regions(void *states, int B, int T, int H, int P, char **st, char **intra, char **ops, float **phi) {
+    const int N = B * P, R = B * T;
+    char *base = static_cast<char *>(states);
+    *st = base;
+    *intra = base + states_region_bytes(N, R, H, 128, 128, true);
+    *ops = *intra + intra_region_bytes(N, R, H, 128, true);
+    *phi = reinterpret_cast<float *>(*ops + (ops_region_bytes(N, R, H, 128, 128, true) + 255) / 256 * 256);
+}
+}  // namespace
+
+cudaError_t launch_seg_train_fwd(const ChunkFwdArgs &a, void *states, int P, void *ws, cudaStream_t s) {
+    constexpr int D = 128;
+    seg::TrainFwdCarve c;
+    seg::carve_train_fwd(ws, a.B, a.T, a.H, P, &c);
+    char *st, *intra, *ops;
+    float *phi;
+    train_regions(states, a.B, a.T, a.H, P, &st, &intra, &ops, &phi);
+    cudaError_t e;
+    // 1. every segment's local pass and the transitions (into the saved buffer), then the scan
+    ChunkFwdArgs f = a;
+    f.ws = c.c2.fwd_ws;
+    f.ws_stride = (size_t)chunk::C * D;
+    f.S_T = nullptr;
+    f.states = f.intra = f.ops = nullptr;
+    f.seg_P = P;
+    f.seg_loc = c.c2.sloc;
+    f.seg_phi = phi;
+    f.seg_qphi = c.c2.qphi;
+    if ((e = launch_chunk_fwd_tc(f, s)) != cudaSuccess) return e;
+    constexpr int bytes = seg::scan_smem_bytes<D>();
+    if ((e = cudaFuncSetAttribute(seg::scan2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) !=
+        cudaSuccess)
+        return e;
+    seg::scan2_kernel<D><<<dim3((unsigned)(a.B * a.H), D / seg::SCAN_COLS), seg::SCAN_THREADS, bytes, s>>>(
+        phi, c.c2.sloc, c.c2.sstart, a.S_T, a.B, a.H, P, D);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 2. the segments as a packed batch from their start states, keeping what the backward needs
+    const size_t nseg = (size_t)a.B * P * a.H * D * D;
+    seg::seg_gather_kernel<<<seg::grid_for(nseg), 256, 0, s>>>(a.S0, c.c2.sstart, c.s0seg, a.B, a.H, P);
+    seg::seg_cu_kernel<<<1, 256, 0, s>>>(c.cu, a.B, a.T, P);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ChunkFwdArgs g{a.q, a.k, a.v, a.log_alpha, a.b, a.w, c.s0seg, a.o, nullptr, c.fwd_ws, (size_t)chunk::C * D,
+                   st, intra, ops, a.status, a.B * P, a.B * a.T, a.H, c.cu};
+    g.wait_limit = a.wait_limit;
+    return launch_chunk_fwd_tc(g, s);
+}
+
+cudaError_t launch_seg_train_bwd(const ChunkBwdArgs &a, const void *states, int P, void *ws, cudaStream_t s) {
+    constexpr int D = 128;
+    seg::TrainBwdCarve c;
+    seg::carve_train_bwd(ws, a.B, a.T, a.H, P, &c);
+    char *st, *intra, *ops;
+    float *phi;
+    train_regions(const_cast<void *>(states), a.B, a.T, a.H, P, &st, &intra, &ops, &phi);
+    cudaError_t e;
+    const size_t nseg = (size_t)a.B * P * a.H * D * D;
+    seg::seg_cu_kernel<<<1, 256, 0, s>>>(c.cu, a.B, a.T, P);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(c.dst_seg, 0, nseg * sizeof(float), s)) != cudaSuccess) return e;
+    ChunkBwdArgs b{a.q, a.k, a.v, a.log_alpha, a.b, a.w, nullptr, a.dO, c.dst_seg, a.dq, a.dk, a.dv, a.dlog_alpha,
+                   a.db, a.dw, c.l_seg, st, intra, ops, c.scratch, c.stride, a.status, 1, a.B * P, a.B * a.T, a.H,
+                   c.cu};
+    b.wait_limit = a.wait_limit;
+    // 1. every segment from a zero end gradient: its own start-state gradient L
+    if ((e = launch_chunk_bwd_tc(b, s)) != cudaSuccess) return e;
+    // 2. the true end gradients, last segment to first
+    constexpr int bytes = seg::scan_smem_bytes<D>();
+    if ((e = cudaFuncSetAttribute(seg::rscan_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) !=
+        cudaSuccess)
+        return e;
+    seg::rscan_kernel<D><<<dim3((unsigned)(a.B * a.H), D / seg::SCAN_COLS), seg::SCAN_THREADS, bytes, s>>>(
+        phi, c.l_seg, a.dS_T, c.g_seg, a.B, a.H, P);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // 3. every segment again from its true end gradient: the gradients, and dS0 of the first
+    b.dS_T = c.g_seg;
+    b.dS0 = c.l_seg;
+    if ((e = launch_chunk_bwd_tc(b, s)) != cudaSuccess) return e;
+    if (a.dS0) {
+        seg::seg_first_kernel<<<seg::grid_for((size_t)a.B * a.H * D * D), 256, 0, s>>>(c.l_seg, a.dS0, a.B, a.H, P);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

@@ -148,6 +148,17 @@ int gdn2_chunk_bwd(const void *q, const void *k, const void *v, const void *log_
  * keeps them instead of recomputing them.)
  * For GDN2_FP32 the state buffer is not used (gdn2_chunk_states_bytes = 0):
  * the fp32 mode checkpoints inside its own workspace.
+ * Few long sequences (bf16, dk = dv = 128, where gdn2_chunk_fwd_workspace
+ * gives the segmented size): the pair splits every sequence into P segments
+ * (segmented training).  The forward finds each segment's start state with
+ * the segmented forward and then keeps the states and tiles of the segments
+ * as a packed batch; the backward runs over the segments twice, first from
+ * zero end gradients (each segment's own start-state gradient), then from the
+ * end gradients a reverse scan through the segments' transitions gives.  The
+ * choice follows from B, T, H, dk, dv alone, and the sizes
+ * (gdn2_chunk_states_bytes, gdn2_chunk_fwd_workspace,
+ * gdn2_chunk_bwd_saved_workspace) are those of that path; the forward then
+ * needs the full gdn2_chunk_fwd_workspace (GDN2_ERR_WORKSPACE otherwise).
  */
 size_t gdn2_chunk_states_bytes(int B, int T, int H, int dk, int dv, int dtype);
 int gdn2_chunk_fwd_save(const void *q, const void *k, const void *v, const void *log_alpha,

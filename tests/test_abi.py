@@ -84,7 +84,10 @@ def test_workspace_sizes():
     r = lambda x: (x + 255) // 256 * 256
     seg = (r(144 * 64 * 128 * 4) + r(32768 * 16 * 128 * 2) + r(5 * 16 * 128 * 128 * 4)
            + 2 * r(4 * 16 * 128 * 128 * 4))
-    assert g.gdn2_chunk_fwd_workspace(1, 32768, 16, 128, 128, g.GDN2_BF16) == seg
+    # ... and, for the saving forward of segmented training, the start states
+    # of the 5 segments, their offsets and the packed forward's scratch
+    train = seg + r(5 * 16 * 128 * 128 * 4) + r(6 * 4) + r(5 * 16 * 64 * 128 * 4)
+    assert g.gdn2_chunk_fwd_workspace(1, 32768, 16, 128, 128, g.GDN2_BF16) == max(seg, train)
     # too short for two segments of 8 chunks: the plain size
     assert g.gdn2_chunk_fwd_workspace(1, 960, 16, 128, 128, g.GDN2_BF16) == 16 * 64 * 128 * 4
     # too many sequences to split (3 * 64 CTAs > 148): the plain size

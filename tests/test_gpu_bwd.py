@@ -96,3 +96,46 @@ def test_saved_state_path_equals_recompute(dk, dv, T):
     assert g.gdn2_get_device_status() == 0
     for n in GRADS:
         np.testing.assert_array_equal(host(g1[n]), host(g2[n]))
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 4096, 16), (2, 1088, 16), (1, 32768, 16)])
+def test_segmented_training_matches_oracle(B, T, H):
+    """Few long sequences: gdn2_chunk_fwd_save / gdn2_chunk_bwd_saved split
+    every sequence into segments (local and transition passes, a packed saving
+    forward from the scanned start states, two packed backward passes around a
+    reverse scan of the end-state gradients).  The training workload's
+    distributions (alpha = sigmoid(N(3,1)), do ~ N(0,1)) at long T.  Both the
+    segmented pair and the one-CTA-per-sequence recompute backward
+    (gdn2_chunk_bwd) against the oracle on sampled whole heads, with a nonzero
+    dS_T, and against each other.  Bound: as stated (rel-L2 <= 1e-2, max-abs <=
+    5e-2) up to T = 4096; at T = 32768 a head's gradient has 4.2M entries, and
+    the largest (|dk| near 10, where a bf16 result alone is rounded by up to
+    0.031) are held per element to 5e-2 + 2^-7 |ref| -- for both paths alike."""
+    import gated_delta_rule_gdn2_b200 as g
+    from gpu_util import TOL_BF16_ELEM
+    x = make_inputs(B, T, H, 128, 128, seed=1200 + T + B, dtype="bf16", with_do=True)
+    rng = np.random.default_rng(T)
+    dST = (0.1 * rng.standard_normal(x["S0"].shape)).astype(np.float32)
+    toks = tokens(x, "bf16")
+    S0 = dev_state(x["S0"])
+    dO = dev(x["dO"], "bf16")
+    o, ST, states = g.chunk_fwd(*toks, S0=S0, save_states=True)
+    gs = g.chunk_bwd(*toks, S0, dO, dev_state(dST), states=states)
+    gr = g.chunk_bwd(*toks, S0, dO, dev_state(dST))
+    assert g.gdn2_get_device_status() == 0
+    tol = TOL_BF16 if T <= 4096 else TOL_BF16_ELEM
+    heads = [(0, 0), (B - 1, H - 1)]
+    xs = sub_heads(x, heads)
+    ref = oracle.bwd(*[xs[n] for n in NAMES], xs["S0"], xs["dO"], np.stack([dST[b, h] for b, h in heads])[:, None])
+    o_ref, ST_ref = oracle.fwd(*[xs[n] for n in NAMES], xs["S0"])
+    oh, STh = host(o), host(ST)
+    for i, (b, h) in enumerate(heads):
+        check("o head %s" % ((b, h),), oh[b, :, h], o_ref[i, :, 0], TOL_BF16)
+        check("S_T head %s" % ((b, h),), STh[b, h], ST_ref[i, 0], TOL_BF16)
+        for label, gg in (("segmented", gs), ("recompute", gr)):
+            for n in GRADS:
+                got = host(gg[n][b, h]) if n == "dS0" else host(gg[n][b, :, h])
+                exp = ref[n][i, 0] if n == "dS0" else ref[n][i, :, 0]
+                check("%s %s head %s" % (label, n, (b, h)), got, exp, tol)
+    for n in GRADS:
+        check(n + " segmented vs recompute", host(gs[n]), host(gr[n]), tol)

@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 import oracle
-from gpu_util import TOL_BF16, TOL_FP32, check, host
+from gpu_util import TOL_BF16, TOL_BF16_ELEM, TOL_FP32, check, host
 from gated_delta_rule_gdn2_b200.inputs import round_bf16
 
 pytestmark = pytest.mark.gpu
@@ -186,5 +186,6 @@ def test_forward_with_output_gate(B, T, H, dk, dv, dtype):
     assert gg.gdn2_get_device_status() == 0
     o_ref, ST_ref = oracle.fwd(*[x[n] for n in NAMES], x["S0"])
     tol = TOL_BF16 if dtype == "bf16" else TOL_FP32
-    check("z", host(z), oracle.epilogue(o_ref, g, gamma), tol)
+    # z = o / rms(o) gamma silu(g) reaches ~10: the per-element bound of large outputs
+    check("z", host(z), oracle.epilogue(o_ref, g, gamma), TOL_BF16_ELEM if dtype == "bf16" else TOL_FP32)
     check("S_T", host(ST), ST_ref, tol)

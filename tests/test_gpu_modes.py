@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 
 import oracle
-from gpu_util import NAMES, TOL_BF16, TOL_FP32, check, dev, dev_state, host
+from gpu_util import NAMES, TOL_BF16, TOL_BF16_ELEM, TOL_FP32, check, check_sum, dev, dev_state, host
 from gated_delta_rule_gdn2_b200.inputs import make_inputs, round_bf16
 
 pytestmark = pytest.mark.gpu
@@ -83,12 +83,18 @@ def test_reduced_backward_matches_oracle(mode, B, T, H):
     # the gradients that do not pass through a gate reduction: the general call's bits
     for n in ("dq", "dk", "dv", "dS0") + (("dlog_alpha",) if mode == "kda" else ()):
         np.testing.assert_array_equal(host(gr[n]), host(ge[n]))
+    # against the oracle: these gates push the largest gradient entries to ~15,
+    # so entries are held to the per-element bound 5e-2 + 2^-7 |ref| (rel-L2 <= 1e-2)
     ref = oracle.bwd(*[x[n] for n in NAMES], x["S0"], x["dO"], dST)
     for n in ("dq", "dk", "dv", "dS0"):
-        check(n, host(gr[n]), ref[n], TOL_BF16)
-    check("dbeta", host(gr["dbeta"]), ref["db"].sum(-1) + ref["dw"].sum(-1), TOL_BF16)
-    check("dlog_alpha", host(gr["dlog_alpha"]),
-          ref["dlog_alpha"] if mode == "kda" else ref["dlog_alpha"].sum(-1), TOL_BF16)
+        check(n, host(gr[n]), ref[n], TOL_BF16_ELEM)
+    check_sum("dbeta", host(gr["dbeta"]), ref["db"].sum(-1) + ref["dw"].sum(-1),
+              np.abs(ref["db"]).sum(-1) + np.abs(ref["dw"]).sum(-1))
+    if mode == "kda":
+        check("dlog_alpha", host(gr["dlog_alpha"]), ref["dlog_alpha"], TOL_BF16_ELEM)
+    else:
+        check_sum("dlog_alpha", host(gr["dlog_alpha"]), ref["dlog_alpha"].sum(-1),
+                  np.abs(ref["dlog_alpha"]).sum(-1))
 
 
 @pytest.mark.parametrize("mode", ["kda", "gdn"])
