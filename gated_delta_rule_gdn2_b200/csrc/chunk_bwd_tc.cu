@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_tc_kernel(ChunkBwdArgs a, con
                 }
             store_frag_bf16<64, 4>(f, x.dM16, 16 * p, 32 * (qc - 2), lane, 1.f);
         }
-        x.dvdw<32>(n, Cn);
+        x.template dvdw<32>(n, Cn);
         mma_wait();
         // ---- E3: dA = strict_lower(nR U^T) -> bf16 (warps with qc < 2); the
         // low-order part dM - bf16(dM) of dM (still in M1's columns) -> bf16 in

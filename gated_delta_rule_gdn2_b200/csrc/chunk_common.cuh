@@ -233,6 +233,12 @@ struct Grp {
     static __device__ __forceinline__ int tid() { return (int)threadIdx.x - BASE; }
 };
 
+// The fp32 [64][64] work arrays of the WY solve (A, T) are row-major with the
+// 16-byte column group of row r XORed with r & 7: the eight rows that one
+// access of a warp touches (a TF32 A fragment, a fragment write-back) then lie
+// in distinct banks instead of all in the same four.
+__device__ __forceinline__ int fsw(int r, int c) { return r * C + (c ^ ((r & 7) << 2)); }
+
 __device__ __forceinline__ uint32_t to_tf32(float x) {
     uint32_t r;
     asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
@@ -247,28 +253,29 @@ __device__ __forceinline__ void mma1688_tf32(float (&d)[4], const uint32_t (&a)[
 }
 
 // One 16x16 block product on the tensor cores in TF32, operands read from
-// row-major fp32 [.][64] arrays: acc += X[r0.., k0..k0+16) * Y[k0.., c0..c0+16).
+// fp32 [64][64] work arrays (fsw layout): acc += X[r0.., k0..k0+16) * Y[k0.., c0..c0+16).
 __device__ __forceinline__ void block16_tf32(float (&acc)[2][4], const float *X, int r0, int k0, const float *Y,
                                              int c0, int lane) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int kk = 0; kk < 16; kk += 8) {
         uint32_t a[4];
-        a[0] = to_tf32(X[(r0 + g) * C + k0 + kk + t]);
-        a[1] = to_tf32(X[(r0 + g + 8) * C + k0 + kk + t]);
-        a[2] = to_tf32(X[(r0 + g) * C + k0 + kk + t + 4]);
-        a[3] = to_tf32(X[(r0 + g + 8) * C + k0 + kk + t + 4]);
+        a[0] = to_tf32(X[fsw(r0 + g, k0 + kk + t)]);
+        a[1] = to_tf32(X[fsw(r0 + g + 8, k0 + kk + t)]);
+        a[2] = to_tf32(X[fsw(r0 + g, k0 + kk + t + 4)]);
+        a[3] = to_tf32(X[fsw(r0 + g + 8, k0 + kk + t + 4)]);
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-            const uint32_t b0 = to_tf32(Y[(k0 + kk + t) * C + c0 + 8 * nt + g]);
-            const uint32_t b1 = to_tf32(Y[(k0 + kk + t + 4) * C + c0 + 8 * nt + g]);
+            const uint32_t b0 = to_tf32(Y[fsw(k0 + kk + t, c0 + 8 * nt + g)]);
+            const uint32_t b1 = to_tf32(Y[fsw(k0 + kk + t + 4, c0 + 8 * nt + g)]);
             mma1688_tf32(acc[nt], a, b0, b1);
         }
     }
 }
 
 // WY solve: T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 area
-// A32, in the fp32 work area T32 and then as T16 = bf16 T (swizzled [64][64];
+// A32 (fsw layout), in the fp32 work area T32 (fsw layout) and then as T16 =
+// bf16 T (swizzled [64][64];
 // T16 may be the first half of the T32 area).  All NT threads of G; on return
 // the T32 area past T16 may be written, and T16 is complete after the
 // caller's next barrier.
@@ -280,22 +287,24 @@ __device__ void wy_solve(const float *A32, float *T32, bf16 *T16) {
         // column j of the inverse of unit lower-triangular block R, column by
         // column: once x_r is final, every later row takes its update at once
         const int R = tid >> 4, j = tid & 15;
-        const float *Ablk = A32 + (16 * R) * C + 16 * R;
+        // (rows 16 R + s2 have r & 7 = s2 & 7, so column 16 R + r of row s2 sits
+        // at 16 R ^ (r ^ 4 (s2 & 7)) in the row)
+        const float *Ablk = A32 + (16 * R) * C;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
         for (int r = 0; r < 15; ++r)
 #pragma unroll
-            for (int s2 = r + 1; s2 < 16; ++s2) x[s2] -= Ablk[s2 * C + r] * x[r];
+            for (int s2 = r + 1; s2 < 16; ++s2) x[s2] -= Ablk[s2 * C + ((16 * R) ^ (r ^ ((s2 & 7) << 2)))] * x[r];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) T32[(16 * R + r) * C + 16 * R + j] = x[r];
+        for (int r = 0; r < 16; ++r) T32[fsw(16 * R + r, 16 * R + j)] = x[r];
     } else {
         for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
             const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
             const int R = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
             const int Q = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            T32[(16 * R + r) * C + 16 * Q + c] = 0.f;
+            T32[fsw(16 * R + r, 16 * Q + c)] = 0.f;
         }
     }
     G::sync();
@@ -309,8 +318,8 @@ __device__ void wy_solve(const float *A32, float *T32, bf16 *T16) {
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
             const int c = 16 * Q + 8 * nt + 2 * t;
-            *reinterpret_cast<float2 *>(T32 + (16 * R + g) * C + c) = make_float2(sc * x[nt][0], sc * x[nt][1]);
-            *reinterpret_cast<float2 *>(T32 + (16 * R + g + 8) * C + c) = make_float2(sc * x[nt][2], sc * x[nt][3]);
+            *reinterpret_cast<float2 *>(T32 + fsw(16 * R + g, c)) = make_float2(sc * x[nt][0], sc * x[nt][1]);
+            *reinterpret_cast<float2 *>(T32 + fsw(16 * R + g + 8, c)) = make_float2(sc * x[nt][2], sc * x[nt][3]);
         }
     };
     float x[2][4] = {};
@@ -347,12 +356,16 @@ __device__ void wy_solve(const float *A32, float *T32, bf16 *T16) {
     G::sync();
     // T32 -> T16 (bf16, swizzled [64][64], the first half of the T32 area)
     {
-        constexpr int EPT = C * C / NT;  // elements per thread
+        constexpr int EPT = C * C / NT;  // elements per thread (row r, columns cb ..)
+        static_assert(EPT % 4 == 0, "whole column groups");
+        const int r = tid / (C / EPT), cb = (tid % (C / EPT)) * EPT;
         float tv[EPT];
 #pragma unroll
-        for (int s = 0; s < EPT; ++s) tv[s] = T32[tid * EPT + s];
+        for (int s = 0; s < EPT; s += 4) {
+            const float4 v4 = *reinterpret_cast<const float4 *>(T32 + fsw(r, cb + s));
+            tv[s] = v4.x; tv[s + 1] = v4.y; tv[s + 2] = v4.z; tv[s + 3] = v4.w;
+        }
         G::sync();
-        const int r = tid / (C / EPT), cb = (tid % (C / EPT)) * EPT;
 #pragma unroll
         for (int s = 0; s < EPT; s += 2)
             *reinterpret_cast<uint32_t *>(T16 + swz<64>(r, cb + s)) = pack_bf16(tv[s], tv[s + 1]);
@@ -410,10 +423,13 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK>
     constexpr int NP = DK / 2, P2 = NT / NP, RS2 = C / P2;
     const int cp = tid % NP, s2 = tid / NP, c2 = 2 * cp;
     if (!prep_only && wv_here) form_wv<DV, NT, G>(st);
+    // this thread's rows s2 RS2 .. of its channel pair stay in registers for pass 2
+    __nv_bfloat162 la2[RS2];
+#pragma unroll
+    for (int i = 0; i < RS2; ++i) la2[i] = *reinterpret_cast<const __nv_bfloat162 *>(st.la + swz<DK>(s2 * RS2 + i, c2));
     float2 psum = make_float2(0.f, 0.f);
-#pragma unroll 4
-    for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r)
-        psum = __fadd2_rn(psum, __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.la + swz<DK>(r, c2))));
+#pragma unroll
+    for (int i = 0; i < RS2; ++i) psum = __fadd2_rn(psum, __bfloat1622float2(la2[i]));
     const float pa = psum.x, pb = psum.y;
     if (s2 < P2 - 1) {
         sh.part[s2][c2] = pa;
@@ -450,22 +466,38 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK>
     if (!slow) {
         // ---- pass 2 (fast): Qt, Gt, Kb in place of q, b, log_alpha (two channels per thread)
         // (both channels of a thread on the packed fp32x2 pipe)
+        // the loads of a batch of the thread's rows are issued before its first
+        // store: the in-place stores would otherwise order each row's loads
+        // behind the previous row's stores (the tiles are separate arrays, but
+        // the compiler cannot tell)
         float2 lam = make_float2(la0, lb0);
-#pragma unroll 4
-        for (int r = s2 * RS2; r < (s2 + 1) * RS2; ++r) {
-            const int o = swz<DK>(r, c2);
-            const float2 l = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.la + o));
-            const float2 q2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.q + o));
-            const float2 k2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.k + o));
-            const float2 b2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(st.b + o));
-            lam = __fadd2_rn(lam, l);
-            if (keep_lam) *reinterpret_cast<float2 *>(lam_ws + r * DK + c2) = lam;
-            const float2 e = make_float2(__expf(lam.x), __expf(lam.y));
-            const float2 ie = make_float2(__expf(-lam.x), __expf(-lam.y));
-            const float2 qt = __fmul2_rn(q2, e), gt = __fmul2_rn(__fmul2_rn(b2, k2), e), kb = __fmul2_rn(k2, ie);
-            *reinterpret_cast<uint32_t *>(st.q + o) = pack_bf16(qt.x, qt.y);
-            *reinterpret_cast<uint32_t *>(st.b + o) = pack_bf16(gt.x, gt.y);
-            *reinterpret_cast<uint32_t *>(st.la + o) = pack_bf16(kb.x, kb.y);
+        constexpr int RB = RS2 > 8 ? 8 : RS2;  // rows per batch
+#pragma unroll
+        for (int i0 = 0; i0 < RS2; i0 += RB) {
+            __nv_bfloat162 qr[RB], kr[RB], br[RB];
+#pragma unroll
+            for (int j = 0; j < RB; ++j) {
+                const int o = swz<DK>(s2 * RS2 + i0 + j, c2);
+                qr[j] = *reinterpret_cast<const __nv_bfloat162 *>(st.q + o);
+                kr[j] = *reinterpret_cast<const __nv_bfloat162 *>(st.k + o);
+                br[j] = *reinterpret_cast<const __nv_bfloat162 *>(st.b + o);
+            }
+#pragma unroll
+            for (int j = 0; j < RB; ++j) {
+                const int i = i0 + j, r = s2 * RS2 + i, o = swz<DK>(r, c2);
+                const float2 l = __bfloat1622float2(la2[i]);
+                const float2 q2 = __bfloat1622float2(qr[j]);
+                const float2 k2 = __bfloat1622float2(kr[j]);
+                const float2 b2 = __bfloat1622float2(br[j]);
+                lam = __fadd2_rn(lam, l);
+                if (keep_lam) *reinterpret_cast<float2 *>(lam_ws + r * DK + c2) = lam;
+                const float2 e = make_float2(__expf(lam.x), __expf(lam.y));
+                const float2 ie = make_float2(__expf(-lam.x), __expf(-lam.y));
+                const float2 qt = __fmul2_rn(q2, e), gt = __fmul2_rn(__fmul2_rn(b2, k2), e), kb = __fmul2_rn(k2, ie);
+                *reinterpret_cast<uint32_t *>(st.q + o) = pack_bf16(qt.x, qt.y);
+                *reinterpret_cast<uint32_t *>(st.b + o) = pack_bf16(gt.x, gt.y);
+                *reinterpret_cast<uint32_t *>(st.la + o) = pack_bf16(kb.x, kb.y);
+            }
         }
         G::sync();
         if (prep_only || grams_ext) return false;
@@ -481,7 +513,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK>
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = r0 + (e >> 1) * 8, i = 8 * nt + 2 * (lane & 3) + (e & 1);
-                    if (warp < 4) A32[r * C + i] = i < r ? acc[0][nt][e] : 0.f;
+                    if (warp < 4) A32[fsw(r, i)] = i < r ? acc[0][nt][e] : 0.f;
                     else accM[0][nt][e] = i <= r ? acc[0][nt][e] : 0.f;
                 }
         }
@@ -549,8 +581,8 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK>
                 while ((r + 1) * (r + 2) / 2 <= p) ++r;
                 while (r * (r + 1) / 2 > p) --r;
                 const int i = p - r * (r + 1) / 2;
-                if (i < r) A32[r * C + i] = pa[s];
-                T32[r * C + i] = pm[s];  // M parked in the T region
+                if (i < r) A32[fsw(r, i)] = pa[s];
+                T32[fsw(r, i)] = pm[s];  // M parked in the T region
             }
         }
         G::sync();
@@ -560,7 +592,7 @@ __device__ bool intra_chunk(ChunkTiles st, float *A32, float *T32, IntraView<DK>
             for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    accM[0][nt][e] = T32[(r0 + (e >> 1) * 8) * C + 8 * nt + 2 * (lane & 3) + (e & 1)];
+                    accM[0][nt][e] = T32[fsw(r0 + (e >> 1) * 8, 8 * nt + 2 * (lane & 3) + (e & 1))];
         }
     }
     G::sync();

@@ -125,6 +125,22 @@ __device__ __forceinline__ void issue_chunk(const FwdMaps &m, ChunkTiles st, con
     }
 }
 
+// The same tiles into L2 ahead of their load (one thread).
+__device__ __forceinline__ void prefetch_chunk(const FwdMaps &m, const SeqView &sv, int h, int n, int gates,
+                                               bool no_vw) {
+    const int t = sv.map_t0 + n * C, b = sv.map_b;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int cx = 64 * half;
+        tc::tma_prefetch_4d(&m.q, cx, h, t, b);
+        tc::tma_prefetch_4d(&m.k, cx, h, t, b);
+        if (!no_vw) tc::tma_prefetch_4d(&m.v, cx, h, t, b);
+        if (gates != kGatesGDN) tc::tma_prefetch_4d(&m.la, cx, h, t, b);
+        if (no_vw || gates == kGatesFull) tc::tma_prefetch_4d(&m.b, cx, h, t, b);
+        if (!no_vw && gates == kGatesFull) tc::tma_prefetch_4d(&m.w, cx, h, t, b);
+    }
+}
+
 // Scalar gates into whole tiles: row r of the b and w tiles (and, for GDN, of
 // the log_alpha tile) holds the scalar of token n*C + r in every column; rows
 // past the sequence's end hold zeros (a zero token).  The NTG threads of G.
@@ -255,13 +271,20 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         tc::fence_after();
         return ok;
     };
+    // ... on the barrier of stage s, whose phase is bit s of a per-thread word
+    // (a phase array indexed by the stage would live in local memory)
+    auto wait_stage = [&](uint64_t *mbar, uint32_t &bits, int s) {
+        uint32_t ph = (bits >> s) & 1u;
+        bits ^= 1u << s;
+        return wait_on(mbar, ph);
+    };
 
     if (warp < 8) {
         // ================= group A: decay prep, Grams, A and M =================
         // (a fast chunk's WY solve runs in group B; a slow chunk takes its Grams
         // term by term and its solve in the intra-chunk stage here)
         float *lam_ws = a.ws ? a.ws + (size_t)blockIdx.x * a.ws_stride : nullptr;
-        uint32_t ph_a = 0, ph_ld[2] = {0, 0};
+        uint32_t ph_a = 0, ph_ld = 0;
         for (int m = 0; m < nchunks; ++m) {
             const int s = m & 1;
             ChunkTiles st = stage_tiles(smem, s);
@@ -269,7 +292,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             float *T32 = reinterpret_cast<float *>(st.w);
             bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
 
-            if (wait_on(&sm.mbar_ld[s], ph_ld[s]) && tid == 0) ++sm.ld_waited[s];  // (landed)
+            if (wait_stage(&sm.mbar_ld[s], ph_ld, s) && tid == 0) ++sm.ld_waited[s];  // (landed)
             GA::sync();
             if (sm.abort) break;
             if (packed && sv.len - m * C < C) {
@@ -313,7 +336,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
 #pragma unroll
                         for (int h2 = 0; h2 < 2; ++h2) {
                             const int r = r0 + 8 * h2, i = 32 * hc + 8 * nt + 2 * (lane & 3);
-                            *reinterpret_cast<float2 *>(A32 + r * C + i) = make_float2(
+                            *reinterpret_cast<float2 *>(A32 + fsw(r, i)) = make_float2(
                                 i < r ? f[0][nt][2 * h2] : 0.f, i + 1 < r ? f[0][nt][2 * h2 + 1] : 0.f);
                         }
                 }
@@ -345,14 +368,15 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         const int tb = tid - NG;
         const bool with_o = op != nullptr;
         const CUtensorMap *omap = phi ? &maps.qphi : &maps.o;
-        // the fused output epilogue: the gate tile lands in the S16 area (free
-        // from U's completion to the next chunk's solve), the RMS partials of
-        // the two column halves beside it
+        // The S16 area is free from U's completion to the next chunk's state
+        // copy: the chunk's O image goes out from its first half (so that the
+        // stage can be refilled without waiting for that store), and the fused
+        // output epilogue's gate tile lands in its second half.
         constexpr bool gated = MODE == kGated;  // (with_o: the launch checks o)
-        bf16 *G16 = reinterpret_cast<bf16 *>(smem + OS16);
-        float *rms_part = reinterpret_cast<float *>(smem + OS16 + TILE);  // [2][64]
-        uint32_t ph_g = 0;
         bf16 *S16 = reinterpret_cast<bf16 *>(smem + OS16);
+        bf16 *O16 = S16;
+        bf16 *G16 = reinterpret_cast<bf16 *>(smem + OS16 + TILE);
+        uint32_t ph_g = 0;
         const int c = 32 * p + lane;  // this thread's state row; columns 64 hc .. 64 hc + 63
         const uint32_t t_row = tmem + lane_base + COL_S + 64 * hc;
         auto keep_tile = [&](int n) {
@@ -419,7 +443,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         // gam of the previous chunk for this thread's row, when that chunk's
         // state update still owes the Diag(gam) (a fast chunk)
         float gm_owed = 1.f;
-        uint32_t ph_b = 0, ph_o = 0, ph_rdy[2] = {0, 0};
+        uint32_t ph_b = 0, ph_o = 0, ph_rdy = 0;
         for (int n = 0; n < nchunks; ++n) {
             const int s = n & 1;
             ChunkTiles st = stage_tiles(smem, s);
@@ -428,23 +452,29 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             bf16 *M16 = T16 + C * C;
             bf16 *U16 = st.v;  // after T (w . v)
 
+            if (tb == 0 && n + 2 < nchunks)  // the tiles that refill this stage into L2
+                prefetch_chunk(maps, sv, h, n + 2, GATES, phi);
             if (gated && tb == 0) {  // the chunk's output-gate rows into L2 while the chain runs
                 tc::tma_prefetch_4d(&maps.g, 0, h, sv.map_t0 + n * C, sv.map_b);
                 tc::tma_prefetch_4d(&maps.g, 64, h, sv.map_t0 + n * C, sv.map_b);
             }
-            wait_on(&sm.ready[s], ph_rdy[s]);
+            wait_stage(&sm.ready[s], ph_rdy, s);
             GB::sync();
             if (sm.abort) break;
             const bool slow = sm.slow[s] != 0;
             const float gm = sm.gamma[s][c];
             if (!slow) {
                 // ---- WY solve of a fast chunk: A (k slot) -> T16 (first half of the
-                // w tile), with the fp32 work area in the S16 area, free until the
-                // state's bf16 copy below (the previous state image is out)
-                wy_solve<NG, GB>(reinterpret_cast<const float *>(st.k), reinterpret_cast<float *>(S16), T16);
+                // w tile), with the fp32 work area in the second half of the S16
+                // area (the previous chunk's O image may still be going out from
+                // the first half)
+                wy_solve<NG, GB>(reinterpret_cast<const float *>(st.k), reinterpret_cast<float *>(G16), T16);
                 tc::fence_async_smem();
-                GB::sync();
             }
+            // (the solve's work area and the state copy below take the S16
+            // area: the previous chunk's O image has been read by now)
+            if (tb == 0) tc::bulk_wait_read();
+            GB::sync();
 
             // ---- T Gt (M = 64, N = 128, K = 64) on the tensor cores; the decayed
             // operands Qt, Gt, Kb (or Kt) go out for the backward
@@ -460,7 +490,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 tc::commit(&sm.mbar_b);
             }
             // ---- meanwhile the chunk-start state: the owed Diag(gam) of the
-            // previous chunk, and its bf16 copy (the S16 area is free again)
+            // previous chunk, and its bf16 copy
             for (int i = 0; i < 2; ++i) {
                 float v[32];
                 load_half(i, v);
@@ -538,11 +568,22 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             }
             wait_on(&sm.mbar_o, ph_o);
             gm_owed = slow ? 1.f : gm;  // a fast chunk's Diag(gam) is applied with the next bf16 copy
-            if (with_o) {  // O -> its bf16 image in the k slot (free since U), stored by the TMA
+            if (a.states && with_o) {  // the state image (the S16 area) has gone out
+                if (tb == 0) {
+                    if (a.intra) tc::bulk_wait_read_but<1>();  // (all but the U tile's store)
+                    else tc::bulk_wait_read();
+                }
+                GB::sync();
+            }
+            if (with_o) {  // O -> its bf16 image in the first half of the S16 area, stored by the TMA
                 Frag<8> f;
                 ld_frag(tmem + lane_base + COL_O + 64 * hc, f);
                 tc::wait_ld();
                 if (gated) {  // z = O / rms(O) * gamma * silu(g), row by row over both column halves
+                    // (the RMS partials of the two column halves [2][64] in the q slot,
+                    // whose last reader, O = Qt S, is complete; the fused epilogue
+                    // keeps nothing for a backward pass)
+                    float *rms_part = reinterpret_cast<float *>(st.q);
                     const int r0 = 16 * p + (lane >> 2);
                     float ss[2] = {0.f, 0.f};
 #pragma unroll
@@ -576,7 +617,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                         }
                     }
                 }
-                store_frag_bf16<D, 8>(f, st.k, 16 * p, 64 * hc, lane, 1.f);
+                store_frag_bf16<D, 8>(f, O16, 16 * p, 64 * hc, lane, 1.f);
                 tc::fence_async_smem();
             }
             wait_on(&sm.mbar_b, ph_b);  // S (and with it every read of the stage's tiles)
@@ -590,7 +631,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 bf16 *o = static_cast<bf16 *>(op);
                 for (int id = tb; id < Cn * 16; id += NG) {
                     const int r = id >> 4, j = id & 15;
-                    const uint4 val = *reinterpret_cast<const uint4 *>(st.k + (j >> 3) * (C * 64) + r * 64 +
+                    const uint4 val = *reinterpret_cast<const uint4 *>(O16 + (j >> 3) * (C * 64) + r * 64 +
                                                                        (((j & 7) ^ (r & 7)) << 3));
                     *reinterpret_cast<uint4 *>(o + ((sv.row0 + n * C + r) * a.H + h) * D + 8 * j) = val;
                 }
@@ -599,20 +640,21 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             }
             if (tb == 0) {
                 if (with_o && !o_rows) {  // (tokens past the tensor's end are clipped)
-                    tc::tma_store_4d(omap, st.k, 0, h, sv.map_t0 + n * C, sv.map_b);
-                    tc::tma_store_4d(omap, st.k + C * 64, 64, h, sv.map_t0 + n * C, sv.map_b);
-                    tc::bulk_commit();
+                    tc::tma_store_4d(omap, O16, 0, h, sv.map_t0 + n * C, sv.map_b);
+                    tc::tma_store_4d(omap, O16 + C * 64, 64, h, sv.map_t0 + n * C, sv.map_b);
                 }
-                // the stage's T, M, U and O images and the state image are out
-                // before the stage is refilled (and before S16 is rewritten, which
-                // follows this thread's next MMA issue)
-                tc::bulk_wait_read();
+                tc::bulk_commit();  // (one group, possibly empty, so that the wait below skips exactly it)
+                // the stage's T, M, U and operand images are out before the stage
+                // is refilled; the O image may still be in flight (its area is
+                // waited for before the next state copy)
+                tc::bulk_wait_read_but<1>();
                 if (n + 2 < nchunks) {
                     issue_chunk(maps, st, sv, h, n + 2, &sm.mbar_ld[s], GATES, phi);
                     ++sm.ld_issued[s];
                 }
             }
         }
+        if (tb == 0) tc::bulk_wait_read();  // (the last O image, in the S16 area)
         GB::sync();
         if (!sm.abort) {  // the final state: S_T and (when requested) its bf16 image
             tc::fence_after();

@@ -144,6 +144,11 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // Until the sources of every committed bulk store have been read (the shared
 // memory may then be overwritten) ...
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+// ... of every committed bulk store but the N most recent groups ...
+template <int N>
+__device__ __forceinline__ void bulk_wait_read_but() {
+    asm volatile("cp.async.bulk.wait_group.read %0;\n" ::"n"(N) : "memory");
+}
 // ... or until the stores are complete.
 __device__ __forceinline__ void bulk_wait() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 
