@@ -239,11 +239,13 @@ struct Grp {
 // in distinct banks instead of all in the same four.
 __device__ __forceinline__ int fsw(int r, int c) { return r * C + (c ^ ((r & 7) << 2)); }
 
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
-    return r;
-}
+// TF32 operand from fp32 bits: the tensor cores read the sign, the exponent and
+// the top 10 mantissa bits, so adding half a unit of the 10th bit (2^12 to the
+// bit pattern) rounds the magnitude to nearest with ties away from zero (a
+// carry into the exponent is the correct rounding up a binade), with one
+// integer add instead of a conversion.
+__device__ __forceinline__ uint32_t tf32_round(uint32_t bits) { return bits + 0x1000u; }
+__device__ __forceinline__ uint32_t to_tf32(float x) { return tf32_round(__float_as_uint(x)); }
 __device__ __forceinline__ void mma1688_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -257,13 +259,16 @@ __device__ __forceinline__ void mma1688_tf32(float (&d)[4], const uint32_t (&a)[
 __device__ __forceinline__ void block16_tf32(float (&acc)[2][4], const float *X, int r0, int k0, const float *Y,
                                              int c0, int lane) {
     const int g = lane >> 2, t = lane & 3;
+    // A fragments by ldmatrix (four 8-row x 16-byte matrices of 32-bit words):
+    // lane l addresses row r0 + (l & 7) + 8 ((l >> 3) & 1) at column group
+    // (l >> 4) of the k-step; fsw keeps each 16-byte group whole
+    const int lr = r0 + (lane & 7) + 8 * ((lane >> 3) & 1), lc = 4 * (lane >> 4);
 #pragma unroll
     for (int kk = 0; kk < 16; kk += 8) {
         uint32_t a[4];
-        a[0] = to_tf32(X[fsw(r0 + g, k0 + kk + t)]);
-        a[1] = to_tf32(X[fsw(r0 + g + 8, k0 + kk + t)]);
-        a[2] = to_tf32(X[fsw(r0 + g, k0 + kk + t + 4)]);
-        a[3] = to_tf32(X[fsw(r0 + g + 8, k0 + kk + t + 4)]);
+        ldsm4(smem_u32(X + fsw(lr, k0 + kk + lc)), a);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = tf32_round(a[i]);
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
             const uint32_t b0 = to_tf32(Y[fsw(k0 + kk + t, c0 + 8 * nt + g)]);
@@ -273,30 +278,72 @@ __device__ __forceinline__ void block16_tf32(float (&acc)[2][4], const float *X,
     }
 }
 
+// Column j of the inverse of the unit lower-triangular 16x16 diagonal block R
+// of I + A (A: fp32 [64][64], fsw layout), row by row: x_s = [s == j] -
+// sum_{r < s} A[s][r] x_r.  Row s of the block is read as 16-byte groups
+// (rows 16 R + s have r & 7 = s & 7, so column group q of the block sits at
+// (16 R + 4 q) ^ 4 (s & 7)), the same address for all 16 threads of a block.
+__device__ __forceinline__ void diag_column(const float *A32, int R, int j, float (&x)[16]) {
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+        const float *row = A32 + (16 * R + s) * C;
+        float acc = s == j ? 1.f : 0.f;
+#pragma unroll
+        for (int q = 0; 4 * q < s; ++q) {
+            const float4 a4 = *reinterpret_cast<const float4 *>(row + ((16 * R + 4 * q) ^ ((s & 7) << 2)));
+            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (4 * q + e < s) acc = fmaf(-av[e], x[4 * q + e], acc);
+        }
+        x[s] = acc;
+    }
+}
+
+// The four diagonal-block inverses into Tdiag ([4][16][16] fp32, row-major
+// blocks): threads 0..63 of G, one column each; no barrier.
+template <class G>
+__device__ __forceinline__ void wy_diag(const float *A32, float *Tdiag) {
+    const int tid = G::tid();
+    if (tid < 64) {
+        const int R = tid >> 4, j = tid & 15;
+        float x[16];
+        diag_column(A32, R, j, x);
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tdiag[R * 256 + r * 16 + j] = x[r];
+    }
+}
+
 // WY solve: T = (I + A)^{-1} for the strictly lower 64x64 A in the fp32 area
 // A32 (fsw layout), in the fp32 work area T32 (fsw layout) and then as T16 =
-// bf16 T (swizzled [64][64];
-// T16 may be the first half of the T32 area).  All NT threads of G; on return
-// the T32 area past T16 may be written, and T16 is complete after the
-// caller's next barrier.
+// bf16 T (swizzled [64][64]; T16 may be the first half of the T32 area).  All
+// NT threads of G; on return the T32 area past T16 may be written, and T16 is
+// complete after the caller's next barrier.  With Tdiag the four diagonal-block
+// inverses come ready-made (wy_diag, [4][16][16] fp32); else they are formed here.
 template <int NT, class G = Grp<0, NT, 0>>
-__device__ void wy_solve(const float *A32, float *T32, bf16 *T16) {
+__device__ void wy_solve(const float *A32, float *T32, bf16 *T16, const float *Tdiag = nullptr) {
     const int tid = G::tid(), warp = tid >> 5, lane = tid & 31;
-    // 16x16 diagonal blocks by substitution in fp32.
-    if (tid < 64) {
-        // column j of the inverse of unit lower-triangular block R, column by
-        // column: once x_r is final, every later row takes its update at once
+    // 16x16 diagonal blocks (fp32), the blocks above them zero
+    if (Tdiag) {  // (every load before the first store, which would order the later loads)
+        static_assert(1024 % NT == 0, "whole blocks");
+        constexpr int ND = 1024 / NT;
+        float dv[ND];
+#pragma unroll
+        for (int i = 0; i < ND; ++i) dv[i] = Tdiag[tid + NT * i];
+#pragma unroll
+        for (int i = 0; i < ND; ++i) {
+            const int e = tid + NT * i, blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            T32[fsw(16 * blk + r, 16 * blk + c)] = dv[i];
+        }
+        for (int e = tid; e < 6 * 256; e += NT) {
+            const int u = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            const int R = u < 3 ? 0 : (u < 5 ? 1 : 2), Q = u < 3 ? u + 1 : (u < 5 ? u - 1 : 3);
+            T32[fsw(16 * R + r, 16 * Q + c)] = 0.f;
+        }
+    } else if (tid < 64) {
         const int R = tid >> 4, j = tid & 15;
-        // (rows 16 R + s2 have r & 7 = s2 & 7, so column 16 R + r of row s2 sits
-        // at 16 R ^ (r ^ 4 (s2 & 7)) in the row)
-        const float *Ablk = A32 + (16 * R) * C;
         float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
-#pragma unroll
-        for (int r = 0; r < 15; ++r)
-#pragma unroll
-            for (int s2 = r + 1; s2 < 16; ++s2) x[s2] -= Ablk[s2 * C + ((16 * R) ^ (r ^ ((s2 & 7) << 2)))] * x[r];
+        diag_column(A32, R, j, x);
 #pragma unroll
         for (int r = 0; r < 16; ++r) T32[fsw(16 * R + r, 16 * R + j)] = x[r];
     } else {

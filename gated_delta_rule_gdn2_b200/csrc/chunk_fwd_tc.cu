@@ -9,9 +9,10 @@
 // The fp32 state S lives in TMEM (128 lanes = key channels x 128 columns)
 // for the whole sequence.  Two warp groups of 8 warps share the work: group
 // A forms chunk m's decay prefix and operands Qt, Gt, Kb and w . v, issues the
-// two Grams (M = N = 64, K = 128) and reads back A (fp32, for the WY solve)
-// and M (bf16); group B runs chunk m - 1's state chain: the WY solve (TF32
-// tensor-core levels on fp32 16x16 diagonal blocks, chunk_common.cuh), then
+// two Grams (M = N = 64, K = 128), reads back A (fp32, for the WY solve) and
+// M (bf16) and inverts A's four 16x16 diagonal blocks; group B runs chunk
+// m - 1's state chain: the rest of the WY solve (TF32 tensor-core levels on
+// the diagonal-block inverses, chunk_common.cuh), then
 //   T Gt (M = 64, N = 128, K = 64) and O = Qt S (K = 128, bf16 S copy in
 //   shared memory as B);
 //   U = T (w . v) + (-W) S;
@@ -60,9 +61,11 @@ struct Small {
     uint64_t mbar_o;      // MMA completion, group B's O = Qt S (a second barrier: each keeps one phase in flight)
     uint64_t mbar_ld[2];  // tile loads of stage 0 and 1
     uint64_t ready[2];    // stage s: its intra-chunk stage is done
+    uint64_t freed[2];    // stage s: group B is done with its chunk (the refill may be issued): two
+                          // arrivals, its last tensor-core reads and its issuing thread
     uint64_t mbar_fin[2]; // the issuing threads' last tensor-core work (groups A, B), at the end
     uint64_t mbar_g;      // the fused epilogue's output-gate tile
-    int ld_issued[2];     // per stage: tile loads issued (thread tb = 0) ...
+    int ld_issued[2];     // per stage: tile loads issued (chunks 0, 1: B's thread 0; then A's) ...
     int ld_waited[2];     // ... and waited for (group A)
     int g_issued, g_landed;  // output-gate tiles issued and landed (group B)
     uint32_t tmem;
@@ -92,15 +95,16 @@ __device__ __forceinline__ ChunkTiles stage_tiles(unsigned char *smem, int s) {
             reinterpret_cast<bf16 *>(p + 5 * TILE)};
 }
 
-// TMA tensor maps of the six token tensors and of the output o.
+// TMA tensor maps of the six token tensors (whole-tile boxes, token_tile_map)
+// and of the output o (64 x 64 boxes).
 struct FwdMaps {
     CUtensorMap q, k, la, b, v, w, o, g;  // g: the output gate of the fused epilogue
     CUtensorMap qphi;                     // segments: the transition pass's rows Phi_t^T q_t
 };
 
-// Chunk n's six token tiles into a stage (one thread; 64 x 64 boxes, two per
-// tile), completion counted in bytes on the stage's mbarrier.  Rows past the
-// end of the tensor read as zeros.
+// Chunk n's six token tiles into a stage (one thread; one box per tile),
+// completion counted in bytes on the stage's mbarrier.  Rows past the end of
+// the tensor read as zeros.
 // With scalar gates (KDA / GDN) the b and w tiles (and, for GDN, the
 // log_alpha tile) are not loaded: expand_gates fills them from the scalars.
 // A transition pass (no_vw) reads no v and w either.
@@ -109,36 +113,12 @@ __device__ __forceinline__ void issue_chunk(const FwdMaps &m, ChunkTiles st, con
     const int ntiles = no_vw ? 4 : (gates == kGatesFull ? 6 : (gates == kGatesKDA ? 4 : 3));
     tc::mbar_expect_tx(mbar, ntiles * TILE);
     const int t = sv.map_t0 + n * C, b = sv.map_b;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const int cx = 64 * half, off = half * C * 64;
-        tc::tma_load_4d(st.q + off, &m.q, cx, h, t, b, mbar);
-        tc::tma_load_4d(st.k + off, &m.k, cx, h, t, b, mbar);
-        if (!no_vw) tc::tma_load_4d(st.v + off, &m.v, cx, h, t, b, mbar);
-        if (gates != kGatesGDN) tc::tma_load_4d(st.la + off, &m.la, cx, h, t, b, mbar);
-        if (no_vw) {
-            tc::tma_load_4d(st.b + off, &m.b, cx, h, t, b, mbar);
-        } else if (gates == kGatesFull) {
-            tc::tma_load_4d(st.b + off, &m.b, cx, h, t, b, mbar);
-            tc::tma_load_4d(st.w + off, &m.w, cx, h, t, b, mbar);
-        }
-    }
-}
-
-// The same tiles into L2 ahead of their load (one thread).
-__device__ __forceinline__ void prefetch_chunk(const FwdMaps &m, const SeqView &sv, int h, int n, int gates,
-                                               bool no_vw) {
-    const int t = sv.map_t0 + n * C, b = sv.map_b;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const int cx = 64 * half;
-        tc::tma_prefetch_4d(&m.q, cx, h, t, b);
-        tc::tma_prefetch_4d(&m.k, cx, h, t, b);
-        if (!no_vw) tc::tma_prefetch_4d(&m.v, cx, h, t, b);
-        if (gates != kGatesGDN) tc::tma_prefetch_4d(&m.la, cx, h, t, b);
-        if (no_vw || gates == kGatesFull) tc::tma_prefetch_4d(&m.b, cx, h, t, b);
-        if (!no_vw && gates == kGatesFull) tc::tma_prefetch_4d(&m.w, cx, h, t, b);
-    }
+    if (gates != kGatesGDN) tc::tma_load_5d(st.la, &m.la, 0, t, 0, h, b, mbar);
+    tc::tma_load_5d(st.q, &m.q, 0, t, 0, h, b, mbar);
+    tc::tma_load_5d(st.k, &m.k, 0, t, 0, h, b, mbar);
+    if (no_vw || gates == kGatesFull) tc::tma_load_5d(st.b, &m.b, 0, t, 0, h, b, mbar);
+    if (!no_vw) tc::tma_load_5d(st.v, &m.v, 0, t, 0, h, b, mbar);
+    if (!no_vw && gates == kGatesFull) tc::tma_load_5d(st.w, &m.w, 0, t, 0, h, b, mbar);
 }
 
 // Scalar gates into whole tiles: row r of the b and w tiles (and, for GDN, of
@@ -240,6 +220,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&sm.mbar_ld[i], 1);
             tc::mbar_init(&sm.ready[i], 1);
+            tc::mbar_init(&sm.freed[i], 2);
             tc::mbar_init(&sm.mbar_fin[i], 1);
             sm.ld_issued[i] = 0;
             sm.ld_waited[i] = 0;
@@ -284,7 +265,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         // (a fast chunk's WY solve runs in group B; a slow chunk takes its Grams
         // term by term and its solve in the intra-chunk stage here)
         float *lam_ws = a.ws ? a.ws + (size_t)blockIdx.x * a.ws_stride : nullptr;
-        uint32_t ph_a = 0, ph_ld = 0;
+        uint32_t ph_a = 0, ph_ld = 0, ph_free = 0;
         for (int m = 0; m < nchunks; ++m) {
             const int s = m & 1;
             ChunkTiles st = stage_tiles(smem, s);
@@ -292,6 +273,14 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             float *T32 = reinterpret_cast<float *>(st.w);
             bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
 
+            // the stage's refill: once group B is done with chunk m - 2, this
+            // thread (idle until the tiles land anyway) issues chunk m's loads, so
+            // that their issue stays off B's chain
+            if (m >= 2 && tid == 0 && wait_stage(&sm.freed[s], ph_free, s)) {
+                tc::fence_async_smem();
+                issue_chunk(maps, st, sv, h, m, &sm.mbar_ld[s], GATES, phi);
+                ++sm.ld_issued[s];
+            }
             if (wait_stage(&sm.mbar_ld[s], ph_ld, s) && tid == 0) ++sm.ld_waited[s];  // (landed)
             GA::sync();
             if (sm.abort) break;
@@ -340,7 +329,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                                 i < r ? f[0][nt][2 * h2] : 0.f, i + 1 < r ? f[0][nt][2 * h2 + 1] : 0.f);
                         }
                 }
-                GA::sync();  // every thread is done reading w for w . v
+                GA::sync();  // every thread is done reading w for w . v; A is complete
+                // the WY solve's diagonal-block inverses (fp32, in the w tile's first
+                // half, which B's T16 takes only after reading them)
+                wy_diag<GA>(A32, reinterpret_cast<float *>(st.w));
                 {  // M (lower with the diagonal) -> bf16 in the second half of the w tile
                     Frag<4> f;
                     ld_frag(tmem + lane_base + COL_G + 64 + 32 * hc, f);
@@ -373,6 +365,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         // stage can be refilled without waiting for that store), and the fused
         // output epilogue's gate tile lands in its second half.
         constexpr bool gated = MODE == kGated;  // (with_o: the launch checks o)
+        // the stage is free once its last products complete, unless bulk stores
+        // read it (the tiles kept for the backward) or the fused epilogue keeps
+        // its partial sums in it
+        const bool early_free = !gated && !a.ops && !a.intra;
         bf16 *S16 = reinterpret_cast<bf16 *>(smem + OS16);
         bf16 *O16 = S16;
         bf16 *G16 = reinterpret_cast<bf16 *>(smem + OS16 + TILE);
@@ -452,8 +448,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             bf16 *M16 = T16 + C * C;
             bf16 *U16 = st.v;  // after T (w . v)
 
-            if (tb == 0 && n + 2 < nchunks)  // the tiles that refill this stage into L2
-                prefetch_chunk(maps, sv, h, n + 2, GATES, phi);
             if (gated && tb == 0) {  // the chunk's output-gate rows into L2 while the chain runs
                 tc::tma_prefetch_4d(&maps.g, 0, h, sv.map_t0 + n * C, sv.map_b);
                 tc::tma_prefetch_4d(&maps.g, 64, h, sv.map_t0 + n * C, sv.map_b);
@@ -464,11 +458,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             const bool slow = sm.slow[s] != 0;
             const float gm = sm.gamma[s][c];
             if (!slow) {
-                // ---- WY solve of a fast chunk: A (k slot) -> T16 (first half of the
-                // w tile), with the fp32 work area in the second half of the S16
-                // area (the previous chunk's O image may still be going out from
-                // the first half)
-                wy_solve<NG, GB>(reinterpret_cast<const float *>(st.k), reinterpret_cast<float *>(G16), T16);
+                // ---- WY solve of a fast chunk: A (k slot) and group A's diagonal-block
+                // inverses (w slot) -> T16 (first half of the w tile), with the fp32
+                // work area in the second half of the S16 area (the previous chunk's
+                // O image may still be going out from the first half)
+                wy_solve<NG, GB>(reinterpret_cast<const float *>(st.k), reinterpret_cast<float *>(G16), T16,
+                                 reinterpret_cast<const float *>(st.w));
                 tc::fence_async_smem();
             }
             // (the solve's work area and the state copy below take the S16
@@ -565,6 +560,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 tc::commit(&sm.mbar_o);
                 mma_tiles<false, false>(tmem + COL_S, st.la, 64, U16, 64, 4, IDESC_S, true);
                 tc::commit(&sm.mbar_b);
+                // these are the stage's last readers: their completion releases it
+                // for the refill, and so does this thread's arrival -- here, when no
+                // bulk store reads the stage, else once those stores have read it
+                if (n + 2 < nchunks) {
+                    tc::commit(&sm.freed[s]);
+                    if (early_free) tc::mbar_arrive(&sm.freed[s]);
+                }
             }
             wait_on(&sm.mbar_o, ph_o);
             gm_owed = slow ? 1.f : gm;  // a fast chunk's Diag(gam) is applied with the next bf16 copy
@@ -645,13 +647,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 }
                 tc::bulk_commit();  // (one group, possibly empty, so that the wait below skips exactly it)
                 // the stage's T, M, U and operand images are out before the stage
-                // is refilled; the O image may still be in flight (its area is
-                // waited for before the next state copy)
+                // is refilled (by group A, on this arrival); the O image may still
+                // be in flight (its area is waited for before the next state copy)
                 tc::bulk_wait_read_but<1>();
-                if (n + 2 < nchunks) {
-                    issue_chunk(maps, st, sv, h, n + 2, &sm.mbar_ld[s], GATES, phi);
-                    ++sm.ld_issued[s];
-                }
+                if (n + 2 < nchunks && !early_free) tc::mbar_arrive(&sm.freed[s]);
             }
         }
         if (tb == 0) tc::bulk_wait_read();  // (the last O image, in the S16 area)
@@ -711,10 +710,10 @@ cudaError_t launch_chunk_fwd_tc(const ChunkFwdArgs &a, cudaStream_t s) {
     const int D = cfwd_tc::D;
     const int MB = a.cu_seqlens ? 1 : a.B;  // a packed batch is one [T, H, D] sequence of rows
     const bool vec_la = a.gates != kGatesGDN, vec_bw = a.gates == kGatesFull;  // (scalar gates: no maps)
-    if (!token_tensor_map(&m.q, a.q, MB, a.T, a.H, D) || !token_tensor_map(&m.k, a.k, MB, a.T, a.H, D) ||
-        (vec_la && !token_tensor_map(&m.la, a.log_alpha, MB, a.T, a.H, D)) ||
-        (vec_bw && !token_tensor_map(&m.b, a.b, MB, a.T, a.H, D)) || !token_tensor_map(&m.v, a.v, MB, a.T, a.H, D) ||
-        (vec_bw && !token_tensor_map(&m.w, a.w, MB, a.T, a.H, D)) ||
+    if (!token_tile_map(&m.q, a.q, MB, a.T, a.H, D) || !token_tile_map(&m.k, a.k, MB, a.T, a.H, D) ||
+        (vec_la && !token_tile_map(&m.la, a.log_alpha, MB, a.T, a.H, D)) ||
+        (vec_bw && !token_tile_map(&m.b, a.b, MB, a.T, a.H, D)) || !token_tile_map(&m.v, a.v, MB, a.T, a.H, D) ||
+        (vec_bw && !token_tile_map(&m.w, a.w, MB, a.T, a.H, D)) ||
         (a.o && !token_tensor_map(&m.o, a.o, MB, a.T, a.H, D)) ||
         (a.out_gate && !token_tensor_map(&m.g, a.out_gate, MB, a.T, a.H, D)) ||
         (a.seg_P && !token_tensor_map(&m.qphi, a.seg_qphi, a.B, a.T, a.H, D)))

@@ -102,6 +102,14 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *mbar, uint32_t bytes) {
                  : "memory");
 }
 // Tiled box of a 4-D tensor map at coordinates (x, y, z, w), x innermost.
+__device__ __forceinline__ void tma_load_5d(void *dst, const void *map, int x, int y, int z, int w, int v,
+                                            uint64_t *mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+        "%5, %6}], [%7];\n" ::"r"(smem_addr(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(v), "r"(smem_addr(mbar))
+        : "memory");
+}
 __device__ __forceinline__ void tma_load_4d(void *dst, const void *map, int x, int y, int z, int w, uint64_t *mbar) {
     asm volatile(
         "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "

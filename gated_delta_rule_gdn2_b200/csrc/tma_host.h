@@ -37,4 +37,21 @@ inline bool token_tensor_map(CUtensorMap *m, const void *base, int B, int T, int
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same tensor read as whole [64 tokens][128 channels] tiles in one box:
+// a 5D view (64 channels, token, channel half, head, batch) whose box {64, 64,
+// 2, 1, 1} lands as the kernels' tile layout, two [64][64] swizzled blocks
+// (channel halves) one after the other.  The channel-half stride (128 bytes)
+// lies below the token stride: the dimensions need not be ordered by stride.
+inline bool token_tile_map(CUtensorMap *m, const void *base, int B, int T, int H, int D) {
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc || D != 128) return false;
+    const cuuint64_t dims[5] = {64, (cuuint64_t)T, 2, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t strides[4] = {(cuuint64_t)H * D * 2, 128, (cuuint64_t)D * 2, (cuuint64_t)T * H * D * 2};
+    const cuuint32_t box[5] = {64, 64, 2, 1, 1};
+    const cuuint32_t unit[5] = {1, 1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, unit,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace gdn2

@@ -103,3 +103,24 @@ def test_operand_descriptors(probe):
         assert val == base + (off >> 4)
         seen += 1
     assert seen == 2 * 4 * 2 * 8
+
+
+def test_tf32_rounding_by_integer_add():
+    """The WY solve's TF32 operands are rounded by adding 2^12 to the fp32 bit
+    pattern (the tensor cores then ignore the low 13 bits).  That is rounding
+    of the magnitude to 10 fractional mantissa bits, ties away from zero: checked
+    against the rounding computed in fp64 from the value's binary exponent, on
+    random values over many binades, on exact ties and at binade edges."""
+    import numpy as np
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal(200000) * np.exp2(rng.integers(-60, 60, 200000))).astype(np.float32)
+    m, e = np.frexp(x.astype(np.float64))  # x = m 2^e, 0.5 <= |m| < 1
+    ties = (np.float64(1.0) + (2 * rng.integers(0, 1 << 10, 1000) + 1) * 2.0 ** -11).astype(np.float32)
+    edge = np.float32(2.0) - np.float32(2.0 ** -23) * np.arange(1, 600, dtype=np.float32)
+    x = np.concatenate([x, ties, -ties, edge, -edge])
+    m, e = np.frexp(x.astype(np.float64))
+    scaled = np.abs(m) * 2.0 ** 11                       # 11 significant bits kept
+    want = np.sign(m) * np.floor(scaled + 0.5) * 2.0 ** (e - 11)
+    bits = x.view(np.uint32).astype(np.uint64)
+    got = (((bits + 0x1000) & 0xFFFFE000) & 0xFFFFFFFF).astype(np.uint32).view(np.float32).astype(np.float64)
+    assert np.array_equal(got, want)
