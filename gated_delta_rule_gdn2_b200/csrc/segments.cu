@@ -107,7 +107,9 @@ constexpr int scan_smem_bytes() { return (DK * (DK + 1) + DK * SCAN_COLS) * (int
 // Start states of the segments of the tensor-memory path (one block per
 // (b*H + h, column group)): S_start(1) = S_loc(0), S_start(p+1) = Phi(p)
 // S_start(p) + S_loc(p); S_start(1..P-1) to Sstart[(b*(P-1) + p-1)*H + h] and
-// S_start(P) = S_T.
+// S_start(P) = S_T.  The steps are sequential; each one's global loads (the
+// next transition, the next S_loc columns) are issued into registers before
+// the current step's product, so that their latency hides behind it.
 template <int DK>
 __global__ void __launch_bounds__(SCAN_THREADS) scan2_kernel(const float *Phi, const float *Sloc, float *Sstart,
                                                             float *S_T, int B, int H, int P, int dv) {
@@ -117,14 +119,29 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan2_kernel(const float *Phi, c
     const int bh = blockIdx.x, b = bh / H, h = bh % H, c0 = blockIdx.y * SCAN_COLS;
     const int tid = threadIdx.x;
     constexpr int CPT = DK * SCAN_COLS / SCAN_THREADS;
+    constexpr int NPHI = DK * DK / 4 / SCAN_THREADS;  // float4 of a transition per thread
     const int r = tid % DK, cc = (tid / DK) * CPT;
     auto loc = [&](int p) { return Sloc + (((size_t)b * P + p) * H + h) * DK * dv; };
+    auto phi = [&](int p) {
+        return reinterpret_cast<const float4 *>(Phi + (((size_t)b * (P - 1) + p - 1) * H + h) * DK * DK);
+    };
+    float4 nphi[NPHI];  // the next transition
+    float nloc[CPT];    // the next S_loc columns of this thread
+    auto fetch = [&](int p) {  // (1 <= p < P)
+        const float4 *src = phi(p);
+#pragma unroll
+        for (int j = 0; j < NPHI; ++j) nphi[j] = src[tid + j * SCAN_THREADS];
+        const float *lp = loc(p) + (size_t)r * dv + c0 + cc;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) nloc[j] = lp[j];
+    };
+    if (P > 1) fetch(1);
     for (int i = tid; i < DK * SCAN_COLS; i += SCAN_THREADS) {
         const int rr = i / SCAN_COLS, c = i % SCAN_COLS;
         prev[rr][c] = loc(0)[(size_t)rr * dv + c0 + c];
     }
     for (int p = 1; p <= P; ++p) {
-        __syncthreads();  // prev complete
+        __syncthreads();  // prev complete; every thread is done reading phi_s
         if (p < P) {
             float *out = Sstart + (((size_t)b * (P - 1) + p - 1) * H + h) * DK * dv;
             for (int i = tid; i < DK * SCAN_COLS; i += SCAN_THREADS)
@@ -136,55 +153,59 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan2_kernel(const float *Phi, c
                         prev[i / SCAN_COLS][i % SCAN_COLS];
             break;
         }
-        const float4 *src = reinterpret_cast<const float4 *>(Phi + (((size_t)b * (P - 1) + p - 1) * H + h) * DK * DK);
-        for (int i = tid; i < DK * DK / 4; i += SCAN_THREADS) {
-            const float4 t = src[i];
-            const int rr = (4 * i) / DK, k = (4 * i) % DK;
-            phi_s[rr][k] = t.x;
-            phi_s[rr][k + 1] = t.y;
-            phi_s[rr][k + 2] = t.z;
-            phi_s[rr][k + 3] = t.w;
+#pragma unroll
+        for (int j = 0; j < NPHI; ++j) {
+            const int i4 = tid + j * SCAN_THREADS, rr = (4 * i4) / DK, k = (4 * i4) % DK;
+            phi_s[rr][k] = nphi[j].x;
+            phi_s[rr][k + 1] = nphi[j].y;
+            phi_s[rr][k + 2] = nphi[j].z;
+            phi_s[rr][k + 3] = nphi[j].w;
         }
-        __syncthreads();
-        const float *lp = loc(p) + (size_t)r * dv + c0 + cc;
         float acc[CPT];
 #pragma unroll
-        for (int j = 0; j < CPT; ++j) acc[j] = lp[j];
+        for (int j = 0; j < CPT; ++j) acc[j] = nloc[j];
+        if (p + 1 < P) fetch(p + 1);  // in flight during this step's product
+        __syncthreads();
 #pragma unroll 4
         for (int k = 0; k < DK; ++k) {
             const float a = phi_s[r][k];
 #pragma unroll
             for (int j = 0; j < CPT; ++j) acc[j] += a * prev[k][cc + j];
         }
-        __syncthreads();  // every thread is done reading Phi and prev
+        __syncthreads();  // every thread is done reading prev
 #pragma unroll
         for (int j = 0; j < CPT; ++j) prev[r][cc + j] = acc[j];
     }
 }
 
 // o_t += S_start(p)^T (Phi_t^T q_t) for every token of segments 1..P-1: per
-// block one (segment, head) and up to kCorrTiles 64-token tiles; the start
-// state goes to shared memory once as bf16, each tile's rows Phi_t^T q_t
-// arrive by cp.async, the product runs on the tensor cores (warp-level
-// m16n8k16) into an fp32 tile in shared memory, and o is read, added to and
-// written back with coalesced 16-byte accesses.  The pass is bound by the
-// bytes of o and of those rows.
-constexpr int kCorrTiles = 16, kCorrThreads = 128;
+// block one (segment, head) and up to `tpb` 64-token tiles (chosen by the host
+// so that the grid fills the SMs a few times over); the start state goes to
+// shared memory once as bf16, each tile's rows Phi_t^T q_t arrive by cp.async
+// one tile ahead, the product runs on the tensor cores (warp-level m16n8k16)
+// into an fp32 tile in shared memory, and o is read (before the product, so
+// that the load latency hides behind it), added to and written back with
+// coalesced 16-byte accesses.  The pass is bound by the bytes of o and of
+// those rows.
+constexpr int kCorrMaxTiles = 16, kCorrThreads = 128;
 constexpr int CORR_LD = 128 + 4;  // fp32 sum tile row pitch (rows 4 banks apart)
-constexpr int CORR_SMEM = 128 * 128 * 2 + 64 * 128 * 2 + 64 * CORR_LD * 4;
+constexpr int CORR_SMEM = 128 * 128 * 2 + 2 * 64 * 128 * 2 + 64 * CORR_LD * 4;
 __global__ void __launch_bounds__(kCorrThreads) correct_kernel(const bf16 *qphi, const float *Sstart, bf16 *o, int B,
-                                                               int T, int H, int P) {
+                                                               int T, int H, int P, int tpb) {
     constexpr int D = 128;
     extern __shared__ __align__(1024) unsigned char smc[];
-    bf16 *S16 = reinterpret_cast<bf16 *>(smc);                            // [128 k][128 n], swizzled
-    bf16 *Q16 = reinterpret_cast<bf16 *>(smc + D * D * 2);                 // [64 t][128 k], swizzled
-    float *acc_s = reinterpret_cast<float *>(smc + D * D * 2 + 64 * D * 2);  // [64 t][CORR_LD] fp32
+    bf16 *S16 = reinterpret_cast<bf16 *>(smc);                                  // [128 k][128 n], swizzled
+    auto Qb = [&](int par) {  // [64 t][128 k], swizzled, by tile parity
+        return reinterpret_cast<bf16 *>(smc + D * D * 2 + par * (64 * D * 2));
+    };
+    float *acc_s = reinterpret_cast<float *>(smc + D * D * 2 + 2 * 64 * D * 2);  // [64 t][CORR_LD] fp32
     const int seg = blockIdx.y / H, h = blockIdx.y % H;                    // seg = b*(P-1) + p - 1
     const int b = seg / (P - 1), p = seg % (P - 1) + 1;
     const int nch = T / chunk::C, base = nch / P, rem = nch % P;
     const int c0 = p * base + min(p, rem), cn = base + (p < rem ? 1 : 0);
-    const int t0 = blockIdx.x * kCorrTiles;
+    const int t0 = blockIdx.x * tpb;
     if (t0 >= cn) return;
+    const int ntl = min(cn, t0 + tpb) - t0;
     const size_t row0 = (size_t)b * T + (size_t)c0 * chunk::C;
     const float4 *Ss = reinterpret_cast<const float4 *>(Sstart + ((size_t)seg * H + h) * D * D);
     for (int i = threadIdx.x; i < D * D / 4; i += kCorrThreads) {
@@ -194,27 +215,16 @@ __global__ void __launch_bounds__(kCorrThreads) correct_kernel(const bf16 *qphi,
             make_uint2(chunk::pack_bf16(v.x, v.y), chunk::pack_bf16(v.z, v.w));
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int tl = t0; tl < min(cn, t0 + kCorrTiles); ++tl) {
-        __syncthreads();  // (S16 written; the previous tile's rows and sums read)
-        chunk::load_token_tile<D, kCorrThreads>(Q16, qphi, row0, cn * chunk::C, h, tl, H);
+    constexpr int IT = 64 * D / 8 / kCorrThreads;
+    chunk::load_token_tile<D, kCorrThreads>(Qb(0), qphi, row0, cn * chunk::C, h, t0, H);
+    chunk::cp_commit();
+    for (int i = 0; i < ntl; ++i) {
+        const int tl = t0 + i;
+        // the next tile's rows into the other buffer (its last reader, the
+        // product two tiles back, is behind the barrier that ended that tile)
+        if (i + 1 < ntl) chunk::load_token_tile<D, kCorrThreads>(Qb((i + 1) & 1), qphi, row0, cn * chunk::C, h, tl + 1, H);
         chunk::cp_commit();
-        chunk::cp_wait<0>();
-        __syncthreads();
-        float acc[1][16][4];
-        chunk::zero(acc);
-        chunk::warp_gemm<1, 16, true, false, D, D, 64, D>(acc, Q16, 16 * warp, S16, 0, D, lane);
-        const int r = 16 * warp + (lane >> 2);
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const int c = 8 * nt + 2 * (lane & 3);
-            *reinterpret_cast<float2 *>(acc_s + r * CORR_LD + c) = make_float2(acc[0][nt][0], acc[0][nt][1]);
-            *reinterpret_cast<float2 *>(acc_s + (r + 8) * CORR_LD + c) = make_float2(acc[0][nt][2], acc[0][nt][3]);
-        }
-        __syncthreads();
-        // o rows of the tile: 16 bytes (8 values) per access; every load of the
-        // tile is issued before the first store (a store may alias a later
-        // load, so interleaving them would serialise the loads)
-        constexpr int IT = 64 * D / 8 / kCorrThreads;
+        // this tile's o rows (16 bytes per access), in flight during the product
         uint4 ov[IT];
         uint4 *op[IT];
 #pragma unroll
@@ -223,6 +233,19 @@ __global__ void __launch_bounds__(kCorrThreads) correct_kernel(const bf16 *qphi,
             op[it] = reinterpret_cast<uint4 *>(o + ((row0 + (size_t)tl * chunk::C + rr) * H + h) * D + cc);
             ov[it] = *op[it];
         }
+        chunk::cp_wait<1>();  // this tile's rows (the group before the one just committed)
+        __syncthreads();      // (and S16; the previous tile's sums read)
+        float acc[1][16][4];
+        chunk::zero(acc);
+        chunk::warp_gemm<1, 16, true, false, D, D, 64, D>(acc, Qb(i & 1), 16 * warp, S16, 0, D, lane);
+        const int r = 16 * warp + (lane >> 2);
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+            const int c = 8 * nt + 2 * (lane & 3);
+            *reinterpret_cast<float2 *>(acc_s + r * CORR_LD + c) = make_float2(acc[0][nt][0], acc[0][nt][1]);
+            *reinterpret_cast<float2 *>(acc_s + (r + 8) * CORR_LD + c) = make_float2(acc[0][nt][2], acc[0][nt][3]);
+        }
+        __syncthreads();
 #pragma unroll
         for (int it = 0; it < IT; ++it) {
             const int id = threadIdx.x + it * kCorrThreads, rr = id / (D / 8), cc = (id % (D / 8)) * 8;
@@ -452,10 +475,13 @@ cudaError_t launch_chunk_fwd_segments(const ChunkFwdArgs &a, int dk, int dv, int
             if ((e = cudaFuncSetAttribute(seg::correct_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           seg::CORR_SMEM)) != cudaSuccess)
                 return e;
-            seg::correct_kernel<<<dim3((unsigned)((longest + seg::kCorrTiles - 1) / seg::kCorrTiles),
-                                       (unsigned)(a.B * (P - 1) * a.H)),
+            // tiles per block: about four blocks per SM (two resident at a time)
+            const long long tiles = (long long)longest * a.B * (P - 1) * a.H;
+            const int tpb = (int)std::max(1LL, std::min<long long>(seg::kCorrMaxTiles,
+                                                                  (tiles + 4LL * seg::num_sms() - 1) / (4LL * seg::num_sms())));
+            seg::correct_kernel<<<dim3((unsigned)((longest + tpb - 1) / tpb), (unsigned)(a.B * (P - 1) * a.H)),
                                   seg::kCorrThreads, seg::CORR_SMEM, s>>>(
-                c.qphi, c.sstart, static_cast<seg::bf16 *>(a.o), a.B, a.T, a.H, P);
+                c.qphi, c.sstart, static_cast<seg::bf16 *>(a.o), a.B, a.T, a.H, P, tpb);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
         return cudaSuccess;
