@@ -75,8 +75,10 @@ __device__ __forceinline__ void issue_chunk(const ChunkFwdArgs &a, ChunkTiles st
     load_token_tile<DK>(st.k, static_cast<const bf16 *>(a.k), sv.row0, sv.len, h, n, a.H);
     load_token_tile<DK>(st.la, static_cast<const bf16 *>(a.log_alpha), sv.row0, sv.len, h, n, a.H);
     load_token_tile<DK>(st.b, static_cast<const bf16 *>(a.b), sv.row0, sv.len, h, n, a.H);
-    load_token_tile<DV>(st.v, static_cast<const bf16 *>(a.v), sv.row0, sv.len, h, n, a.H);
-    load_token_tile<DV>(st.w, static_cast<const bf16 *>(a.w), sv.row0, sv.len, h, n, a.H);
+    if (!a.transition) {  // (a transition pass has no write term: its v and w tiles are zeroed instead)
+        load_token_tile<DV>(st.v, static_cast<const bf16 *>(a.v), sv.row0, sv.len, h, n, a.H);
+        load_token_tile<DV>(st.w, static_cast<const bf16 *>(a.w), sv.row0, sv.len, h, n, a.H);
+    }
     cp_commit();
 }
 
@@ -119,7 +121,8 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
             for (int e = 0; e < 4; ++e) {
                 const int c = c0 + 16 * mt + (lane >> 2) + (e >> 1) * 8;
                 const int j = j0 + 8 * nt + 2 * (lane & 3) + (e & 1);
-                S[mt][nt][e] = a.S0 ? a.S0[(size_t)bh * DK * DV + (size_t)c * DV + j] : 0.f;
+                S[mt][nt][e] = a.transition ? (c == j ? 1.f : 0.f)
+                               : (a.S0 ? a.S0[(size_t)bh * DK * DV + (size_t)c * DV + j] : 0.f);
             }
     // bf16 copy of the state into shared memory (and to a.states[n] when set)
     auto write_S16 = [&](int n) {
@@ -161,6 +164,11 @@ __global__ void __launch_bounds__(NTHR, 1) chunk_fwd_kernel(ChunkFwdArgs a) {
 
         cp_wait<1>();
         __syncthreads();
+        if (a.transition) {  // no write term: w . v = 0 (the slots hold other tiles' data otherwise)
+            for (int id = threadIdx.x; id < 2 * C * DV / 8; id += NTHR)
+                reinterpret_cast<uint4 *>(id < C * DV / 8 ? st.v : st.w)[id % (C * DV / 8)] = make_uint4(0, 0, 0, 0);
+            __syncthreads();
+        }
         const bool slow = intra_chunk<DK, DV>(st, A32, T32, view(sh), lam_ws, false);
         // T and M (then U, below) for the backward, as their shared-memory images
         if (a.intra) copy_smem_to_global(keep_tile(n), T16, 2 * C * C * 2);

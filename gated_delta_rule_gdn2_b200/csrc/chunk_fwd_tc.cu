@@ -722,6 +722,7 @@ cudaError_t launch_chunk_fwd_tc(const ChunkFwdArgs &a, cudaStream_t s) {
                     a.gates != kGatesFull || !a.seg_loc || !a.seg_phi || !a.seg_qphi))
         return cudaErrorInvalidValue;
     if (a.out_gate && (a.states || !a.o || !a.gamma)) return cudaErrorInvalidValue;  // (inference path only)
+    if (a.transition) return cudaErrorInvalidValue;  // (this kernel takes its transition passes by seg_P)
     using namespace cfwd_tc;
     auto kernel = a.seg_P                  ? chunk_fwd_tc_kernel<kGatesFull, kSegments>
                   : a.out_gate             ? chunk_fwd_tc_kernel<kGatesFull, kGated>

@@ -75,6 +75,9 @@ struct ChunkFwdArgs {
     int seg_P = 0;
     float *seg_loc = nullptr, *seg_phi = nullptr;
     void *seg_qphi = nullptr;
+    // the warp-level kernel's transition pass (segments.cu, dk = dv): the state
+    // starts from the identity and there is no write term (v and w are not read)
+    bool transition = false;
 };
 
 cudaError_t launch_chunk_fwd(const ChunkFwdArgs &a, int dk, int dv, cudaStream_t s);

@@ -37,15 +37,6 @@ namespace seg {
 
 using chunk::bf16;
 
-// Identity matrices [count][d][d] (fp32).
-__global__ void identity_kernel(float *m, size_t count, int d) {
-    const size_t n = count * d * d;
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
-        const size_t e = i % ((size_t)d * d);
-        m[i] = (e / d == e % d) ? 1.f : 0.f;
-    }
-}
-
 // Start states of the segments.  Block (b*H + h, column group g) owns 16
 // value columns of one sequence and walks its P segments in order; each
 // segment's transition is staged in shared memory (coalesced) before use.
@@ -356,8 +347,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) rscan_kernel(const float *Phi, c
 
 struct Carve {
     float *fwd_ws;
-    bf16 *zeros;
-    float *ident, *phi, *sloc, *sstart;
+    float *phi, *sloc, *sstart;
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -372,13 +362,11 @@ size_t carve(void *p, int B, int T, int H, int dk, int dv, int P, Carve *c) {
         return p ? static_cast<unsigned char *>(p) + at : nullptr;
     };
     unsigned char *fw = take(chunk_fwd_ws_bytes((int)Bp, H, dk));
-    unsigned char *z = take((size_t)B * T * H * dk * sizeof(bf16));
-    unsigned char *id = take(Bp * H * dk * dk * sizeof(float));
     unsigned char *ph = take(Bp * H * dk * dk * sizeof(float));
     unsigned char *sl = take(Bp * H * dk * dv * sizeof(float));
     unsigned char *ss = take(Bp * H * dk * dv * sizeof(float));
-    if (c) *c = {reinterpret_cast<float *>(fw), reinterpret_cast<bf16 *>(z), reinterpret_cast<float *>(id),
-                 reinterpret_cast<float *>(ph), reinterpret_cast<float *>(sl), reinterpret_cast<float *>(ss)};
+    if (c) *c = {reinterpret_cast<float *>(fw), reinterpret_cast<float *>(ph), reinterpret_cast<float *>(sl),
+                 reinterpret_cast<float *>(ss)};
     return off;
 }
 
@@ -490,18 +478,14 @@ cudaError_t launch_chunk_fwd_segments(const ChunkFwdArgs &a, int dk, int dv, int
     seg::carve(ws, a.B, a.T, a.H, dk, dv, P, &c);
     const int Bp = a.B * P, Tp = a.T / P;
     const size_t wstride = (size_t)chunk::C * dk;
-    e = cudaMemsetAsync(c.zeros, 0, (size_t)a.B * a.T * a.H * dk * sizeof(seg::bf16), s);
-    if (e != cudaSuccess) return e;
-    const size_t nident = (size_t)Bp * a.H;
-    seg::identity_kernel<<<(unsigned)std::min<size_t>((nident * dk * dk + 255) / 256, 4096), 256, 0, s>>>(
-        c.ident, nident, dk);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // 1. every segment from a zero start (S_loc) and its transition (Phi: start I, no write term)
+    // 1. every segment from a zero start (S_loc) and its transition (Phi: start I,
+    // no write term; the kernel reads no v and w for it)
     ChunkFwdArgs loc{a.q, a.k, a.v, a.log_alpha, a.b, a.w, nullptr, nullptr, c.sloc, c.fwd_ws, wstride,
                      nullptr, nullptr, nullptr, a.status, Bp, Tp, a.H};
     if ((e = launch_chunk_fwd(loc, dk, dv, s)) != cudaSuccess) return e;
-    ChunkFwdArgs phi{a.q, a.k, c.zeros, a.log_alpha, a.b, c.zeros, c.ident, nullptr, c.phi, c.fwd_ws, wstride,
+    ChunkFwdArgs phi{a.q, a.k, a.v, a.log_alpha, a.b, a.w, nullptr, nullptr, c.phi, c.fwd_ws, wstride,
                      nullptr, nullptr, nullptr, a.status, Bp, Tp, a.H};
+    phi.transition = true;
     if ((e = launch_chunk_fwd(phi, dk, dk, s)) != cudaSuccess) return e;
     // 2. the segments' start states
     const dim3 grid((unsigned)(a.B * a.H), (unsigned)(dv / seg::SCAN_COLS));
