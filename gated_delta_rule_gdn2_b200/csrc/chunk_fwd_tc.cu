@@ -61,11 +61,9 @@ struct Small {
     uint64_t mbar_o;      // MMA completion, group B's O = Qt S (a second barrier: each keeps one phase in flight)
     uint64_t mbar_ld[2];  // tile loads of stage 0 and 1
     uint64_t ready[2];    // stage s: its intra-chunk stage is done
-    uint64_t freed[2];    // stage s: group B is done with its chunk (the refill may be issued): two
-                          // arrivals, its last tensor-core reads and its issuing thread
     uint64_t mbar_fin[2]; // the issuing threads' last tensor-core work (groups A, B), at the end
     uint64_t mbar_g;      // the fused epilogue's output-gate tile
-    int ld_issued[2];     // per stage: tile loads issued (chunks 0, 1: B's thread 0; then A's) ...
+    int ld_issued[2];     // per stage: tile loads issued (thread tb = 0) ...
     int ld_waited[2];     // ... and waited for (group A)
     int g_issued, g_landed;  // output-gate tiles issued and landed (group B)
     uint32_t tmem;
@@ -220,7 +218,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&sm.mbar_ld[i], 1);
             tc::mbar_init(&sm.ready[i], 1);
-            tc::mbar_init(&sm.freed[i], 2);
             tc::mbar_init(&sm.mbar_fin[i], 1);
             sm.ld_issued[i] = 0;
             sm.ld_waited[i] = 0;
@@ -265,7 +262,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         // (a fast chunk's WY solve runs in group B; a slow chunk takes its Grams
         // term by term and its solve in the intra-chunk stage here)
         float *lam_ws = a.ws ? a.ws + (size_t)blockIdx.x * a.ws_stride : nullptr;
-        uint32_t ph_a = 0, ph_ld = 0, ph_free = 0;
+        uint32_t ph_a = 0, ph_ld = 0;
         for (int m = 0; m < nchunks; ++m) {
             const int s = m & 1;
             ChunkTiles st = stage_tiles(smem, s);
@@ -273,14 +270,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             float *T32 = reinterpret_cast<float *>(st.w);
             bf16 *M16 = reinterpret_cast<bf16 *>(T32) + C * C;
 
-            // the stage's refill: once group B is done with chunk m - 2, this
-            // thread (idle until the tiles land anyway) issues chunk m's loads, so
-            // that their issue stays off B's chain
-            if (m >= 2 && tid == 0 && wait_stage(&sm.freed[s], ph_free, s)) {
-                tc::fence_async_smem();
-                issue_chunk(maps, st, sv, h, m, &sm.mbar_ld[s], GATES, phi);
-                ++sm.ld_issued[s];
-            }
             if (wait_stage(&sm.mbar_ld[s], ph_ld, s) && tid == 0) ++sm.ld_waited[s];  // (landed)
             GA::sync();
             if (sm.abort) break;
@@ -365,10 +354,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
         // stage can be refilled without waiting for that store), and the fused
         // output epilogue's gate tile lands in its second half.
         constexpr bool gated = MODE == kGated;  // (with_o: the launch checks o)
-        // the stage is free once its last products complete, unless bulk stores
-        // read it (the tiles kept for the backward) or the fused epilogue keeps
-        // its partial sums in it
-        const bool early_free = !gated && !a.ops && !a.intra;
         bf16 *S16 = reinterpret_cast<bf16 *>(smem + OS16);
         bf16 *O16 = S16;
         bf16 *G16 = reinterpret_cast<bf16 *>(smem + OS16 + TILE);
@@ -560,13 +545,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 tc::commit(&sm.mbar_o);
                 mma_tiles<false, false>(tmem + COL_S, st.la, 64, U16, 64, 4, IDESC_S, true);
                 tc::commit(&sm.mbar_b);
-                // these are the stage's last readers: their completion releases it
-                // for the refill, and so does this thread's arrival -- here, when no
-                // bulk store reads the stage, else once those stores have read it
-                if (n + 2 < nchunks) {
-                    tc::commit(&sm.freed[s]);
-                    if (early_free) tc::mbar_arrive(&sm.freed[s]);
-                }
             }
             wait_on(&sm.mbar_o, ph_o);
             gm_owed = slow ? 1.f : gm;  // a fast chunk's Diag(gam) is applied with the next bf16 copy
@@ -647,10 +625,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 }
                 tc::bulk_commit();  // (one group, possibly empty, so that the wait below skips exactly it)
                 // the stage's T, M, U and operand images are out before the stage
-                // is refilled (by group A, on this arrival); the O image may still
-                // be in flight (its area is waited for before the next state copy)
+                // is refilled; the O image may still be in flight (its area is
+                // waited for before the next state copy)
                 tc::bulk_wait_read_but<1>();
-                if (n + 2 < nchunks && !early_free) tc::mbar_arrive(&sm.freed[s]);
+                if (n + 2 < nchunks) {  // (six whole-tile boxes: a short issue)
+                    issue_chunk(maps, st, sv, h, n + 2, &sm.mbar_ld[s], GATES, phi);
+                    ++sm.ld_issued[s];
+                }
             }
         }
         if (tb == 0) tc::bulk_wait_read();  // (the last O image, in the S16 area)
