@@ -13,9 +13,10 @@
 // M (bf16) and inverts A's four 16x16 diagonal blocks; group B runs chunk
 // m - 1's state chain: the rest of the WY solve (TF32 tensor-core levels on
 // the diagonal-block inverses, chunk_common.cuh), then
-//   T Gt (M = 64, N = 128, K = 64) and O = Qt S (K = 128, bf16 S copy in
-//   shared memory as B);
-//   U = T (w . v) + (-W) S;
+//   T Gt (M = 64, N = 128, K = 64, into O's columns) and T (w . v), which
+//   need no state;
+//   U += (-W) S (K = 128, bf16 S copy in shared memory as B), then O = Qt S,
+//   so that U, which the chain waits for, completes first;
 //   O += M U (committed first: the O epilogue runs under the next one) and
 //   S += Kb^T U (M = 128),
 // reading results back with the 16x256b TMEM load shape (the register layout
@@ -58,7 +59,7 @@ struct Small {
     int slow[2];          // per stage: the chunk took the exact path
     uint64_t mbar_a;      // MMA completion, group A
     uint64_t mbar_b;      // MMA completion, group B
-    uint64_t mbar_o;      // MMA completion, group B's O = Qt S (a second barrier: each keeps one phase in flight)
+    uint64_t mbar_o;      // MMA completion, group B's O products (a second barrier: each keeps one phase in flight)
     uint64_t mbar_ld[2];  // tile loads of stage 0 and 1
     uint64_t ready[2];    // stage s: its intra-chunk stage is done
     uint64_t mbar_fin[2]; // the issuing threads' last tensor-core work (groups A, B), at the end
@@ -456,8 +457,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
             if (tb == 0) tc::bulk_wait_read();
             GB::sync();
 
-            // ---- T Gt (M = 64, N = 128, K = 64) on the tensor cores; the decayed
-            // operands Qt, Gt, Kb (or Kt) go out for the backward
+            // ---- the products that need no state (M = 64, N = 128, K = 64): T Gt
+            // into O's columns (free until O = Qt S, issued once -W is read back)
+            // and T (w . v) into U's; the decayed operands Qt, Gt, Kb (or Kt) go
+            // out for the backward
             if (tb == 0) {
                 if (a.ops) {
                     unsigned char *op = static_cast<unsigned char *>(a.ops) + (sv.cslot + n) * kOpsTileBytes;
@@ -466,7 +469,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                     tc::bulk_store(op + 2 * TILE, st.la, TILE);
                     tc::bulk_commit();
                 }
-                mma_tiles<true, false>(tmem + COL_U, T16, 64, st.b, 64, 4, ID64x128_K_MN, false);
+                mma_tiles<true, false>(tmem + COL_O, T16, 64, st.b, 64, 4, ID64x128_K_MN, false);
+                mma_tiles<true, false>(tmem + COL_U, T16, 64, st.v, 64, 4, ID64x128_K_MN, false);
                 tc::commit(&sm.mbar_b);
             }
             // ---- meanwhile the chunk-start state: the owed Diag(gam) of the
@@ -480,32 +484,30 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 put_half(i, v);
             }
             handoff();
-            // ---- O = Qt S; the state, T and M (and U, below) go out for the
-            // backward as their shared-memory images
+            // ---- the state, T and M (and U, below) go out for the backward as
+            // their shared-memory images
             if (tb == 0) {
                 keep_state(n);
                 if (a.intra) {
                     tc::bulk_store(keep_tile(n), T16, 2 * C * C * 2);
                     tc::bulk_commit();
                 }
-                if (with_o) mma_tiles<true, false>(tmem + COL_O, st.q, 64, S16, D, 8, ID64x128_K_MN, false);
-                tc::commit(&sm.mbar_o);
             }
-            wait_on(&sm.mbar_b, ph_b);  // T Gt
+            wait_on(&sm.mbar_b, ph_b);  // T Gt, T (w . v)
             {  // -W = -(T Gt) -> bf16 in the k slot
                 Frag<8> f;
-                ld_frag(tmem + lane_base + COL_U + 64 * hc, f);
+                ld_frag(tmem + lane_base + COL_O + 64 * hc, f);
                 tc::wait_ld();
                 store_frag_bf16<D, 8>(f, W16, 16 * p, 64 * hc, lane, -1.f);
             }
             handoff();
-            // ---- U = T (w . v) + (-W) S
+            // ---- U = T (w . v) + (-W) S first (the chain waits for it), then O = Qt S
             if (tb == 0) {
-                mma_tiles<true, false>(tmem + COL_U, T16, 64, st.v, 64, 4, ID64x128_K_MN, false);
                 mma_tiles<true, false>(tmem + COL_U, W16, 64, S16, D, 8, ID64x128_K_MN, true);
                 tc::commit(&sm.mbar_b);
+                if (with_o) mma_tiles<true, false>(tmem + COL_O, st.q, 64, S16, D, 8, ID64x128_K_MN, false);
+                if (gated) tc::commit(&sm.mbar_o);
             }
-            wait_on(&sm.mbar_o, ph_o);  // O
             wait_on(&sm.mbar_b, ph_b);  // U
             {  // U -> bf16 in the v slot (w . v is consumed)
                 Frag<8> f;
@@ -513,6 +515,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_tc_kernel(ChunkFwdArgs a, con
                 tc::wait_ld();
                 store_frag_bf16<D, 8>(f, U16, 16 * p, 64 * hc, lane, 1.f);
             }
+            if (gated) wait_on(&sm.mbar_o, ph_o);  // O = Qt S: the gate tile lands where S16 was
             handoff();
             if (sm.abort) break;
             if (tb == 0 && a.intra) {
