@@ -150,3 +150,54 @@ def test_varlen_buffer_sizes_depend_on_totals_only():
     assert st == r(states) + r(intra) + ops
     assert g.gdn2_chunk_fwd_varlen_workspace(N, T, H, 128, 128, g.GDN2_BF16) == N * H * 64 * 128 * 4
     assert g.gdn2_chunk_states_varlen_bytes(N, T, H, 128, 128, g.GDN2_FP32) == 0
+
+
+def test_reduced_gate_entry_points_validate():
+    """KDA / Gated DeltaNet calls: a missing or misaligned scalar gate, a missing
+    gradient and unsupported sizes are refused on the host."""
+    P = 16  # a 16-byte aligned stand-in address (never dereferenced: the calls fail first)
+    fwd = lambda **kw: g.gdn2_chunk_fwd_kda(*[kw.get(n, P) for n in ("q", "k", "v", "la", "beta")], None,
+                                            kw.get("o", P), None, 1, 64, 1, kw.get("dk", 128), 128,
+                                            g.GDN2_BF16, P, 1 << 30, 0)
+    assert fwd(beta=None) == -1
+    assert fwd(beta=17) == -1          # not even element-aligned for bf16
+    assert fwd(dk=96) == -2
+    assert g.gdn2_chunk_fwd_gdn(P, P, P, 17, P, None, P, None, 1, 64, 1, 128, 128, g.GDN2_BF16, P, 1 << 30, 0) == -1
+    assert g.gdn2_chunk_fwd_gdn(P, P, P, P, P, None, P, None, 0, 64, 1, 128, 128, g.GDN2_BF16, None, 0, 0) == 0
+    bwd = [P] * 5 + [None, P, None] + [P] * 4
+    assert g.gdn2_chunk_bwd_kda(*bwd, None, None, 1, 64, 1, 128, 128, g.GDN2_BF16, P, 1 << 40, 0) == -1  # no dbeta
+    assert g.gdn2_chunk_bwd_gdn(*bwd, P, None, 1, 64, 1, 96, 128, g.GDN2_BF16, P, 1 << 40, 0) == -2
+    assert g.gdn2_decode_step_kda(P, P, P, P, None, P, P, 1, 1, 128, 128, g.GDN2_BF16, 0) == -1
+    assert g.gdn2_decode_step_gdn(P, P, P, 19, P, P, P, 1, 1, 128, 128, g.GDN2_BF16, 0) == -1
+
+
+def test_gated_forward_and_layer_entry_points_validate():
+    P = 16
+    toks = [P] * 6
+    # the fused output gate needs g and gamma
+    assert g.gdn2_chunk_fwd_gated(*toks, None, None, P, P, None, 1, 64, 1, 128, 128, g.GDN2_BF16, P, 1 << 30, 0) == -1
+    assert g.gdn2_chunk_fwd_gated(*toks, None, P, None, P, None, 1, 64, 1, 128, 128, g.GDN2_BF16, P, 1 << 30, 0) == -1
+    # prologue: filter width 1..4, head sizes 64 / 128, 16-byte pointers; no tokens = no-op
+    pro = lambda K=4, B=1, T=64, dk=128, xq=P: g.gdn2_prologue_fwd(xq, P, P, P, P, P, K, P, P, P, P, P, P, P, P, P,
+                                                                  None, B, T, 2, dk, 128, g.GDN2_BF16, 0)
+    assert pro(K=0) == -2 and pro(K=5) == -2 and pro(dk=96) == -2
+    assert pro(B=-1) == -1 and pro(xq=24) == -1
+    assert pro(T=0) == 0 and pro(B=0) == 0
+    # its backward's workspace: one fp32 partial per 64-row block, head, filter tap and channel
+    assert g.gdn2_prologue_bwd_workspace(2, 100, 3, 128, 64, 4, 0) == 4 * 3 * (2 * 128 + 64) * 4 * 4
+    assert g.gdn2_prologue_bwd_workspace(2, 100, 3, 128, 64, 4, 1) == 2 * 3 * (2 * 128 + 64) * 4 * 4
+    assert g.gdn2_prologue_bwd_workspace(2, 100, 3, 128, 64, 5, 0) == 0
+    assert g.gdn2_prologue_bwd(*[P] * 6, 4, *[P] * 18, None, 1, 64, 2, 128, 128, g.GDN2_BF16, P, 16, 0) == -5
+    # output gate: rows >= 0, dv 64 / 128, aligned pointers, enough workspace
+    assert g.gdn2_output_gate_fwd(P, P, P, P, -1, 2, 128, g.GDN2_BF16, 0) == -1
+    assert g.gdn2_output_gate_fwd(P, P, P, P, 64, 2, 96, g.GDN2_BF16, 0) == -2
+    assert g.gdn2_output_gate_fwd(24, P, P, P, 64, 2, 128, g.GDN2_BF16, 0) == -1
+    assert g.gdn2_output_gate_fwd(P, P, P, P, 0, 2, 128, g.GDN2_BF16, 0) == 0
+    assert g.gdn2_output_gate_bwd_workspace(100, 3, 128) == 2 * 3 * 128 * 4
+    assert g.gdn2_output_gate_bwd(*[P] * 7, 100, 3, 128, g.GDN2_BF16, P, 16, 0) == -5
+
+
+def test_debug_knobs_reject_out_of_range_values():
+    assert g.gdn2_debug_set(7, 0) == -1
+    assert g.gdn2_debug_set(g.GDN2_DEBUG_WAIT_LIMIT if hasattr(g, "GDN2_DEBUG_WAIT_LIMIT") else 0, -1) == -1
+    assert g.gdn2_debug_set(1, -2) == -1
